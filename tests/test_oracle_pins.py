@@ -1,0 +1,355 @@
+"""Pins of the CPU oracle against things other than itself (CPU only).
+
+Each test ties one oracle step to a closed form, a library routine, brute
+force, a hand-derived example or an invariant of the method, so that a
+plausible mistake (a dropped term, a wrong sign or index, a transposed
+operand, an off-by-one in the schedule) fails at least one of them.
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+from scipy.spatial.distance import cdist
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _bf16_vals(rng, shape, scale=1.0):
+    """Random values that are exactly representable in bf16 (as float32)."""
+    x = (rng.standard_normal(shape) * scale).astype(np.float32)
+    return torch.from_numpy(x).to(torch.bfloat16).to(torch.float32).numpy()
+
+
+# --- reference schedule (paper summary page, "DeltaKV Framework Architecture";
+#     news page, "How ResidualKV Works": dynamic-stride scheduling) -------------------
+
+@pytest.mark.parametrize("n,s,R", [(2048, 16, 128), (32768, 16, 2048), (131072, 16, 8192), (1, 16, 1),
+                                   (16, 16, 1), (17, 16, 2)])
+def test_schedule_fixed_counts(n, s, R):
+    pos = oracle.schedule(n, s)
+    assert len(pos) == R
+    assert np.array_equal(pos, np.arange(R, dtype=np.int32) * s)
+
+
+def test_schedule_fixed_ceil_for_ragged_lengths():
+    rng = np.random.default_rng(1)
+    for n in list(rng.integers(16384, 32769, 50)) + [16384, 32768, 31, 32, 33]:
+        assert len(oracle.schedule(int(n), 32)) == math.ceil(n / 32)
+
+
+def test_schedule_dynamic_one_million():
+    # stride 16 doubling after every 1024 references: phase p starts at
+    # 1024*16*(2^p - 1) with stride 16*2^p; 6 full phases below 2^20 and 16 refs of the 7th
+    pos = oracle.schedule(1 << 20, 16, 1024)
+    assert len(pos) == 6 * 1024 + 16 == 6160
+    for p in range(7):
+        start = 1024 * 16 * (2 ** p - 1)
+        assert pos[1024 * p] == start
+        seg = pos[1024 * p: 1024 * (p + 1)]
+        assert np.all(np.diff(seg) == 16 * 2 ** p)
+    assert pos[-1] == 1032192 + 15 * 1024
+
+
+def test_schedule_dynamic_count_closed_form():
+    rng = np.random.default_rng(2)
+    for n in list(rng.integers(1, 3_000_000, 40)) + [16384, 16385, 49152, 49153]:
+        n = int(n)
+        want, start, p = 0, 0, 0
+        while start < n:
+            stride = 16 * 2 ** p
+            want += min(1024, -(-(n - start) // stride))
+            start += 1024 * stride
+            p += 1
+        assert len(oracle.schedule(n, 16, 1024)) == want
+
+
+# --- rounding helpers: against torch's bf16 and numpy's binary16 -----------------------
+
+def test_bf16_round_matches_torch():
+    rng = np.random.default_rng(3)
+    x = np.concatenate([rng.standard_normal(100000).astype(np.float32) * 3,
+                        # exact ties: bf16 value + half an ulp
+                        (_bf16_vals(rng, 1000) * np.float32(1 + 2 ** -8)).astype(np.float32)])
+    ours = oracle.bf16_round(x)
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, ref)
+
+
+def test_fp16_round_up_is_smallest_binary16_above():
+    rng = np.random.default_rng(4)
+    vals = np.concatenate([np.exp(rng.uniform(math.log(1e-9), math.log(6.5e4), 4000)),
+                           np.float16(rng.uniform(0, 100, 500)).astype(np.float64),  # exactly representable
+                           [2.0 ** -24, 2.0 ** -25, 2.0 ** -14, 65504.0, 1e-45]]).astype(np.float32)
+    for f in vals:
+        bits, ov = oracle.fp16_round_up(float(f))
+        assert ov == 0
+        h = np.array([bits], dtype=np.uint16).view(np.float16)[0]
+        assert float(h) == oracle.fp16_value(bits)
+        assert float(h) >= float(f)
+        below = np.nextafter(h, np.float16(0))
+        assert float(below) < float(f)
+    bits, ov = oracle.fp16_round_up(65505.0)
+    assert ov == 1 and bits == 0x7C00
+    assert oracle.fp16_round_up(0.0) == (0, 0)
+
+
+# --- L2 distance: the expanded form in long double -----------------------------------
+
+def test_l2_matches_expanded_form():
+    rng = np.random.default_rng(5)
+    for D in (4, 64, 128):
+        for _ in range(200):
+            a = (rng.standard_normal(D) * rng.uniform(0.1, 8)).astype(np.float32)
+            b = (a + rng.standard_normal(D) * rng.uniform(1e-3, 1)).astype(np.float32)
+            al = a.astype(np.longdouble)
+            bl = b.astype(np.longdouble)
+            exp = float(np.dot(al, al) - 2 * np.dot(al, bl) + np.dot(bl, bl))
+            got = oracle.l2(a, b)
+            assert abs(got - exp) <= 1e-12 * float(np.dot(al, al) + np.dot(bl, bl))
+
+
+# --- top-k selection ------------------------------------------------------------------
+
+def test_select_top_k_is_the_minimum_k_subset():
+    """Exhaustive: the chosen set minimises the summed distance over all k-subsets."""
+    rng = np.random.default_rng(6)
+    n, D, s = 64, 4, 4
+    for trial in range(6):
+        X = rng.standard_normal((n, D)).astype(np.float32)
+        ref_pos = oracle.schedule(n, s)
+        refK = oracle.build_refs(X, ref_pos)
+        rv = oracle.bf16_value(refK)
+        for k in (1, 2, 3, 4):
+            tok = np.arange(n, dtype=np.int32)
+            idx, keff, _ = oracle.select(X, tok, refK, ref_pos, k)
+            d = cdist(X.astype(np.float64), rv.astype(np.float64), "sqeuclidean")
+            for t in range(n):
+                cands = [j for j in range(len(ref_pos)) if ref_pos[j] <= t]
+                kk = min(k, len(cands))
+                assert keff[t] == kk
+                best = min(itertools.combinations(cands, kk), key=lambda S: sum(d[t, j] for j in S))
+                sums = sorted(sum(d[t, j] for j in S) for S in itertools.combinations(cands, kk))
+                if len(sums) > 1:
+                    assert sums[1] - sums[0] > 1e-9  # unique minimum on random data
+                assert list(idx[t, :kk]) == sorted(best)
+                assert all(v == oracle.SENTINEL for v in idx[t, kk:])
+
+
+def test_select_planted_copies_and_causality():
+    rng = np.random.default_rng(7)
+    n, D, s, k = 512, 16, 16, 4
+    X = _bf16_vals(rng, (n, D))
+    ref_pos = oracle.schedule(n, s)
+    # plant: token 300 is an exact copy of reference ordinal 5 (position 80),
+    # token 301 of reference 18 (position 288)
+    X[300] = X[80]
+    X[301] = X[288]
+    refK = oracle.build_refs(X, ref_pos)
+    tok = np.arange(n, dtype=np.int32)
+    idx, keff, dist = oracle.select(X, tok, refK, ref_pos, k)
+    assert 5 in idx[300] and dist[300, 0] == 0.0
+    assert 18 in idx[301] and dist[301, 0] == 0.0
+    for t in range(n):
+        ch = idx[t, :keff[t]]
+        assert np.all(np.diff(ch.astype(int)) > 0)           # ascending ordinals
+        assert np.all(ref_pos[ch] <= t)                      # only earlier (or same) positions
+        assert np.all(np.diff(dist[t][~np.isnan(dist[t])]) >= 0)
+
+
+def test_select_tie_break_lowest_ordinal():
+    D = 8
+    X = np.zeros((64, D), dtype=np.float32)
+    X[:, 0] = 1.0                                            # every token identical
+    ref_pos = oracle.schedule(64, 8)
+    refK = oracle.build_refs(X, ref_pos)
+    idx, keff, _ = oracle.select(X, np.array([63], dtype=np.int32), refK, ref_pos, 3)
+    assert list(idx[0]) == [0, 1, 2]
+
+
+# --- residual encoding ----------------------------------------------------------------
+
+def _load_golden():
+    vals = {}
+    with open(os.path.join(GOLDEN, "quantiser_worked_example.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, *rest = line.split()
+            vals[key] = rest
+    return vals
+
+
+def test_encode_matches_hand_derived_example():
+    g = _load_golden()
+    x = np.array([float(v) for v in g["x"]], dtype=np.float32)[None, :]
+    refs = np.array([[0x3F80] * 32, [0x3F00] * 32], dtype=np.uint16)
+    idx = np.array([[0, 1]], dtype=np.uint16)
+    e4 = oracle.encode(x, refs, idx, 4, want_detail=True)
+    assert np.array_equal(e4["mean"][0], np.full(32, 0.75, dtype=np.float32))
+    assert np.array_equal(e4["delta"][0], np.array([float(v) for v in g["delta"]], dtype=np.float32))
+    assert e4["scales"][0, 0] == int(g["int4_scale_bits"][0], 16)
+    assert list(e4["codes"][0]) == [int(b, 16) for b in g["int4_bytes"]]
+    assert list(oracle.unpack_codes(e4["codes"][0], 32, 4)) == [int(v) for v in g["int4_codes"]]
+    e8 = oracle.encode(x, refs, idx, 8)
+    assert e8["scales"][0, 0] == int(g["int8_scale_bits"][0], 16)
+    assert list(e8["codes"][0].view(np.int8)) == [int(v) for v in g["int8_codes"]]
+
+
+def _numpy_unpack(codes, D, bits):
+    """Independent unpacking: two's complement bytes / nibbles, even channel low."""
+    if bits == 8:
+        return codes.view(np.int8).astype(np.int64)
+    lo = (codes & 0xF).astype(np.int64)
+    hi = (codes >> 4).astype(np.int64)
+    out = np.empty(codes.shape[:-1] + (D,), dtype=np.int64)
+    out[..., 0::2] = lo
+    out[..., 1::2] = hi
+    return np.where(out >= 8, out - 16, out)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_quantiser_invariants(bits):
+    rng = np.random.default_rng(8 + bits)
+    n, D, R, k = 400, 128, 40, 4
+    qmax = 127 if bits == 8 else 7
+    refs = oracle.bf16_round(rng.standard_normal((R, D)))
+    idx = np.sort(np.stack([rng.choice(R, k, replace=False) for _ in range(n)]), axis=1).astype(np.uint16)
+    idx[:50, 2:] = oracle.SENTINEL                           # k_eff = 2 rows
+    idx[50:60, 1:] = oracle.SENTINEL                         # k_eff = 1 rows
+    x = (oracle.bf16_value(refs)[idx[:, 0]] + rng.standard_normal((n, D)) * 0.2).astype(np.float32)
+    x[60, :32] = 0.0                                         # (a group stays nonzero through the mean)
+    e = oracle.encode(x, refs, idx, bits, want_detail=True)
+    codes = _numpy_unpack(e["codes"], D, bits)
+    scales = e["scales"].view(np.float16).astype(np.float64)
+    delta = e["delta"].astype(np.float64)
+    # mean = plain mean of the selected reference rows
+    rv = oracle.bf16_value(refs).astype(np.float64)
+    for t in range(n):
+        sel = [j for j in idx[t] if j != oracle.SENTINEL]
+        np.testing.assert_allclose(e["mean"][t], rv[sel].mean(axis=0), rtol=4 * 2 ** -24, atol=1e-30)
+    np.testing.assert_array_equal(e["delta"], (x - e["mean"]).astype(np.float32))
+    for t in range(n):
+        for gi in range(D // 32):
+            sl = slice(32 * gi, 32 * gi + 32)
+            a = np.max(np.abs(delta[t, sl]))
+            s = scales[t, gi]
+            if a == 0:
+                assert s == 0 and np.all(codes[t, sl] == 0)
+                continue
+            assert s >= np.float32(np.float32(a) / np.float32(qmax))
+            assert float(np.nextafter(np.float16(s), np.float16(0))) < np.float32(np.float32(a) / np.float32(qmax))
+            assert np.max(np.abs(codes[t, sl])) == qmax
+            assert np.all(np.abs(delta[t, sl] - codes[t, sl] * s) <= s / 2 + 1e-12 * s)
+
+
+def test_quantiser_grid_roundtrip():
+    rng = np.random.default_rng(9)
+    D = 64
+    refs = oracle.bf16_round(np.zeros((1, D)))
+    for bits, qmax in ((4, 7), (8, 127)):
+        s = np.float32(0.125)                                # binary16-exact scale
+        codes = rng.integers(-qmax, qmax + 1, (50, D))
+        codes[:, ::32] = qmax                                # max|code| = qmax in every group
+        x = (codes * s).astype(np.float32)
+        e = oracle.encode(x, refs, np.zeros((50, 1), dtype=np.uint16), bits)
+        assert np.all(e["scales"].view(np.float16) == np.float16(s))
+        assert np.array_equal(_numpy_unpack(e["codes"], D, bits), codes)
+
+
+def test_k1_at_reference_position_gives_zero_residual():
+    rng = np.random.default_rng(10)
+    n, D = 256, 64
+    X = _bf16_vals(rng, (n, D))
+    ref_pos = oracle.schedule(n, 16)
+    refK = oracle.build_refs(X, ref_pos)
+    idx, keff, dist = oracle.select(X[ref_pos], ref_pos, refK, ref_pos, 1)
+    assert np.array_equal(idx[:, 0], np.arange(len(ref_pos)))
+    assert np.all(dist[:, 0] == 0)
+    for bits in (4, 8):
+        e = oracle.encode(X[ref_pos], refK, idx, bits)
+        assert np.all(e["codes"] == 0) and np.all(e["scales"] == 0)
+
+
+# --- reconstruction and attention -----------------------------------------------------
+
+def test_unquantised_reconstruction_is_exact():
+    rng = np.random.default_rng(11)
+    n, D = 1024, 64
+    X = (rng.standard_normal((n, D)) * 2).astype(np.float32)   # fp32 inputs: refs get rounded
+    c = oracle.compress_unit(X, X, 16, 0, 4, 4)
+    e = oracle.encode(X[c["pos"]], c["refK"], c["idx"], 0)
+    xh = oracle.reconstruct(c["refK"], c["idx"], None, None, 0, delta_exact=e["delta_exact"])
+    assert np.array_equal(xh, X[c["pos"]].astype(np.float64))
+
+
+def test_quantised_reconstruction_error_bound():
+    rng = np.random.default_rng(12)
+    n, D = 1024, 128
+    X = _bf16_vals(rng, (n, D))
+    for bits in (4, 8):
+        c = oracle.compress_unit(X, X, 16, 0, 4, bits)
+        xh = oracle.reconstruct(c["refK"], c["idx"], c["codesK"], c["scalesK"], bits)
+        s = np.repeat(c["scalesK"].view(np.float16).astype(np.float64), 32, axis=1)
+        err = np.abs(xh.astype(np.float64) - X[c["pos"]])
+        assert np.all(err <= s / 2 + 4 * 2 ** -24 * np.abs(X[c["pos"]]) + 1e-30)
+
+
+def _plain_attention(q, K, V):
+    q = torch.from_numpy(np.asarray(q, np.float64))
+    K = torch.from_numpy(np.asarray(K, np.float64))
+    V = torch.from_numpy(np.asarray(V, np.float64))
+    w = torch.softmax(q @ K.T / math.sqrt(K.shape[1]), dim=-1)
+    return (w @ V).numpy()
+
+
+def test_attention_matches_torch():
+    rng = np.random.default_rng(13)
+    for n in (1, 7, 300):
+        q = rng.standard_normal((4, 32))
+        K = rng.standard_normal((n, 32))
+        V = rng.standard_normal((n, 32))
+        np.testing.assert_allclose(oracle.attention(q, K, V), _plain_attention(q, K, V), rtol=1e-12, atol=1e-13)
+
+
+def test_attention_special_cases():
+    rng = np.random.default_rng(14)
+    V = rng.standard_normal((5, 16))
+    q = rng.standard_normal((2, 16))
+    np.testing.assert_array_equal(oracle.attention(q, rng.standard_normal((1, 16)), V[:1]), np.tile(V[0], (2, 1)))
+    K = np.tile(rng.standard_normal(16), (5, 1))
+    np.testing.assert_allclose(oracle.attention(q, K, V), np.tile(V.mean(axis=0), (2, 1)), rtol=1e-13)
+    assert np.all(oracle.attention(q, np.zeros((0, 16)), np.zeros((0, 16))) == 0)
+
+
+def test_unquantised_cache_attention_equals_uncompressed_attention():
+    rng = np.random.default_rng(15)
+    n, D, G = 700, 64, 3
+    Xk = _bf16_vals(rng, (n, D))
+    Xv = _bf16_vals(rng, (n, D))
+    c = oracle.compress_unit(Xk, Xv, 16, 0, 4, 4)
+    ek = oracle.encode(Xk[c["pos"]], c["refK"], c["idx"], 0)
+    ev = oracle.encode(Xv[c["pos"]], c["refV"], c["idx"], 0)
+    Kh = np.empty((n, D))
+    Vh = np.empty((n, D))
+    Kh[c["ref_pos"]] = oracle.bf16_value(c["refK"])
+    Vh[c["ref_pos"]] = oracle.bf16_value(c["refV"])
+    Kh[c["pos"]] = oracle.reconstruct(c["refK"], c["idx"], None, None, 0, delta_exact=ek["delta_exact"])
+    Vh[c["pos"]] = oracle.reconstruct(c["refV"], c["idx"], None, None, 0, delta_exact=ev["delta_exact"])
+    q = rng.standard_normal((G, D))
+    np.testing.assert_allclose(oracle.attention(q, Kh, Vh), _plain_attention(q, Xk, Xv), rtol=1e-12, atol=1e-13)
+
+
+def test_compress_unit_dynamic_stride_smoke():
+    rng = np.random.default_rng(16)
+    n, D = 3000, 16
+    X = _bf16_vals(rng, (n, D))
+    c = oracle.compress_unit(X, X, 2, 64, 2, 4)
+    assert len(c["ref_pos"]) == len(oracle.schedule(n, 2, 64))
+    assert len(c["pos"]) == n - len(c["ref_pos"])
+    assert c["overflow"] == 0
