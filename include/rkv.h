@@ -1,0 +1,259 @@
+/*
+ * rkv.h — C ABI of the residual KV-cache compression library (librkv.so).
+ *
+ * The method (ResidualKV / DeltaKV) keeps a strided set of tokens as
+ * uncompressed references and stores every other token as a quantised
+ * residual against the mean of its k nearest earlier references:
+ *   - paper summary page "ResidualKV: Residual-Based KV Cache Compression for
+ *     Efficient Long-Context Inference", section "DeltaKV Framework
+ *     Architecture": strided reference selection (reference set T, top-k
+ *     nearest by L2 distance, mean reference KV_R), residual computation, and
+ *     reconstruction KV = KV_delta + KV_R;
+ *   - same page, section "Practical Deployment via Sparse-vLLM": a batched L2
+ *     distance kernel for the reference search and a fused reconstruction
+ *     kernel (gather, mean, residual add in one launch);
+ *   - news page "New KV Cache Compression Method Cuts Long-Context Inference
+ *     Costs by 85%", section "How ResidualKV Works": quantized residual codes,
+ *     on-the-fly reconstruction when attention needs a token, and
+ *     dynamic-stride scheduling (roughly logarithmic reference growth).
+ * The learned compressor/decompressor of the pages is replaced by a stated
+ * stand-in: the identity plus a symmetric group quantiser (int8 or int4 codes,
+ * one binary16 scale per 32 channels).
+ *
+ * Conventions for every call
+ *   - Memory: the caller allocates every buffer (inputs, the cache, the
+ *     workspace, outputs) and keeps ownership.  The library allocates no
+ *     device memory, keeps no global state and never frees caller memory.
+ *   - Streams: `stream` is a cudaStream_t (NULL = legacy default stream).
+ *     Device work is enqueued asynchronously on it; calls that only touch
+ *     host memory ignore it.  Calls on distinct buffers may run concurrently.
+ *   - Errors: every call returns an rkv_status.  Invalid arguments are
+ *     rejected before anything is enqueued.  A failed launch returns
+ *     RKV_ERR_CUDA.  Kernels that meet a corrupted cache (an out-of-range
+ *     reference index, an impossible scale) or a bounded wait that ran out
+ *     record RKV_ERR_CORRUPT / RKV_ERR_TIMEOUT in the cache's device error
+ *     word and skip the affected work; rkv_read_device_error() returns it.
+ *     Nothing aborts, traps or throws across this boundary.
+ *   - Tensor layouts (row-major, contiguous, device memory unless stated):
+ *       K, V   [batch][n_kv_heads][max_len][head_dim]  in_dtype  (one layer)
+ *       q      [batch][n_q_heads][head_dim]            in_dtype
+ *       out    [batch][n_q_heads][head_dim]            out_dtype
+ *     Rows of sequence b past lengths[b] are never read.  Query head g
+ *     attends with kv head g / (n_q_heads / n_kv_heads).
+ *   - One cache describes one layer: bind one buffer per layer.
+ */
+#ifndef RKV_H
+#define RKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define RKV_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define RKV_API __attribute__((visibility("default")))
+#else
+#define RKV_API
+#endif
+
+#define RKV_DTYPE_BF16 0
+#define RKV_DTYPE_F32 1
+
+#define RKV_MAX_BATCH 256         /* sequences per cache */
+#define RKV_MAX_K 16              /* neighbours per token */
+#define RKV_MAX_REFS 65535        /* references per (sequence, kv-head): 16-bit ordinals, 0xFFFF = unused */
+#define RKV_IDX_UNUSED 0xFFFFu
+
+/* Optional algorithm choices (rkv_config.flags).  Results agree within the
+ * library's tolerances whichever is chosen; the defaults are the fast paths. */
+#define RKV_FLAG_SELECT_SIMT 0x1u    /* reference search on CUDA cores even for bf16 inputs */
+#define RKV_FLAG_DECODE_DIRECT 0x2u  /* decode by gathering and averaging reference rows per token */
+
+typedef enum rkv_status {
+    RKV_OK = 0,
+    RKV_ERR_INVALID_ARG = 1, /* NULL pointer, bad size, inconsistent shape */
+    RKV_ERR_UNSUPPORTED = 2, /* valid but not implemented: head_dim not 64/128, k > 16, > 65535 refs,
+                                not an sm_100 device, binary16 scale overflow */
+    RKV_ERR_WORKSPACE = 3,   /* cache or workspace buffer smaller than required */
+    RKV_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
+    RKV_ERR_CORRUPT = 5,     /* device-side: cache contents out of range */
+    RKV_ERR_TIMEOUT = 6      /* device-side: a bounded wait ran out */
+} rkv_status;
+
+/*
+ * Static description of one layer's cache.
+ *   head_dim        D, 64 or 128
+ *   n_kv_heads      key/value heads (Hkv)
+ *   n_q_heads       query heads, a multiple of n_kv_heads
+ *   k               neighbours per compressed token, 1..16
+ *   bits            residual code width, 4 or 8
+ *   group           channels per binary16 scale; must be 32
+ *   stride0         reference stride s (>= 2): positions 0, s, 2s, ... are references
+ *   refs_per_phase  0: fixed stride.  > 0: dynamic stride — the stride doubles
+ *                   after every refs_per_phase references (phase p has stride
+ *                   stride0 * 2^p and starts where phase p-1's references end)
+ *   in_dtype        RKV_DTYPE_BF16 or RKV_DTYPE_F32, for K, V and q
+ *   out_dtype       decode output dtype, RKV_DTYPE_BF16 or RKV_DTYPE_F32
+ *   batch           sequences, 1..RKV_MAX_BATCH
+ *   max_len         row pitch (tokens) of K and V, >= every length
+ *   flags           RKV_FLAG_* bits
+ */
+typedef struct rkv_config {
+    int32_t head_dim;
+    int32_t n_kv_heads;
+    int32_t n_q_heads;
+    int32_t k;
+    int32_t bits;
+    int32_t group;
+    int32_t stride0;
+    int32_t refs_per_phase;
+    int32_t in_dtype;
+    int32_t out_dtype;
+    int32_t batch;
+    int32_t max_len;
+    uint32_t flags;
+    int32_t reserved[3];
+} rkv_config;
+
+/* Host-side handle of a bound cache.  Caller-allocated, opaque, plain data:
+ * copying it with memcpy gives an equivalent handle. */
+#define RKV_CACHE_DESC_BYTES 32768
+typedef struct rkv_cache_desc {
+    uint64_t opaque[RKV_CACHE_DESC_BYTES / 8];
+} rkv_cache_desc;
+
+/* Device pointers and sizes of one (sequence, kv-head) unit of a bound cache.
+ * Layout of each array (rows contiguous):
+ *   ref_K, ref_V     [n_ref][head_dim] bf16   reference rows, reference ordinal order
+ *   ref_half_norm    [n_ref] float            0.5 * |ref_K row|^2 (fp32)
+ *   ref_pos          [n_ref] int32            position of each reference
+ *   codes_K, codes_V [n_cmp][code_bytes]      residual codes of the compressed tokens in
+ *                                             position order; int8: one byte per channel;
+ *                                             int4: two channels per byte, even channel in
+ *                                             the low nibble; two's complement
+ *   scale_K, scale_V [n_cmp][n_groups] binary16 bits
+ *   idx              [n_cmp][k] uint16        reference ordinals, ascending, 0xFFFF padding */
+typedef struct rkv_unit_view {
+    int32_t n;
+    int32_t n_ref;
+    int32_t n_cmp;
+    int32_t k;
+    int32_t code_bytes;
+    int32_t n_groups;
+    int32_t reserved[2];
+    void* ref_K;
+    void* ref_V;
+    float* ref_half_norm;
+    int32_t* ref_pos;
+    uint8_t* codes_K;
+    uint8_t* codes_V;
+    uint16_t* scale_K;
+    uint16_t* scale_V;
+    uint16_t* idx;
+} rkv_unit_view;
+
+/* ABI version of the loaded library (RKV_ABI_VERSION). */
+RKV_API int32_t rkv_abi_version(void);
+
+/* Static text for a status code. */
+RKV_API const char* rkv_status_string(rkv_status s);
+
+/*
+ * Reference positions of one sequence of length n under cfg's schedule
+ * (paper summary page, "DeltaKV Framework Architecture", strided reference
+ * set; news page, "How ResidualKV Works", dynamic stride).  Host only.
+ * Writes min(count, cap) ascending positions to pos (host memory; may be NULL)
+ * and the count to *n_ref.
+ */
+RKV_API rkv_status rkv_schedule(const rkv_config* cfg, int32_t n, int32_t* pos, int64_t cap, int32_t* n_ref);
+
+/*
+ * Bytes of the cache buffer and of the workspace that rkv_compress and
+ * rkv_decode_attn need for one layer with these sequence lengths
+ * (lengths: host array of cfg->batch entries, 0 <= length <= max_len).
+ * Host only.
+ */
+RKV_API rkv_status rkv_cache_size(const rkv_config* cfg, const int32_t* lengths, uint64_t* cache_bytes,
+                          uint64_t* workspace_bytes);
+
+/*
+ * Lays a cache out in dev_buf (device memory, >= rkv_cache_size bytes,
+ * 256-byte aligned) and fills *desc.  Writes the per-unit tables and clears
+ * the device error word with synchronous copies (returns after they finish);
+ * the rest of the buffer is left as is until rkv_build_refs/rkv_compress.
+ * Fails with RKV_ERR_UNSUPPORTED on a device other than sm_100.
+ */
+RKV_API rkv_status rkv_cache_bind(const rkv_config* cfg, const int32_t* lengths, void* dev_buf, uint64_t bytes,
+                          rkv_cache_desc* desc);
+
+/* Device pointers of one unit (host only; no device access). */
+RKV_API rkv_status rkv_unit_view_get(const rkv_cache_desc* desc, int32_t seq, int32_t kv_head, rkv_unit_view* out);
+
+/*
+ * Reference store (paper summary page, "DeltaKV Framework Architecture",
+ * strided reference selection: the reference set T is kept uncompressed).
+ * For every unit copies the K and V rows at the reference positions into
+ * ref_K / ref_V as bf16 (fp32 inputs rounded to nearest even), and writes
+ * ref_half_norm and ref_pos.  K, V: one layer, layout above.
+ */
+RKV_API rkv_status rkv_build_refs(const rkv_cache_desc* desc, const void* K, const void* V, void* stream);
+
+/*
+ * Compression of every non-reference token (paper summary page, "DeltaKV
+ * Framework Architecture": top-k nearest references by L2 distance on the key,
+ * mean reference, residual; news page, "How ResidualKV Works": quantized
+ * residual codes).  Needs rkv_build_refs on the same K first.  Candidates of
+ * position i are the references at positions < i; ranking is by (distance,
+ * ordinal); k_eff = min(k, candidates); the mean is an fp32 sum in ascending
+ * ordinal order divided by k_eff; per 32-channel group
+ * scale = smallest binary16 >= max|delta| / qmax and
+ * code = round-half-even(delta / scale) (qmax 127 or 7).
+ * Writes codes, scales and idx.  workspace: device, >= the size from
+ * rkv_cache_size; its contents are scratch.
+ */
+RKV_API rkv_status rkv_compress(const rkv_cache_desc* desc, const void* K, const void* V, void* workspace,
+                        uint64_t workspace_bytes, void* stream);
+
+/*
+ * One decode step of attention over the compressed cache (paper summary
+ * page, "Training and Inference Integration" and "Practical Deployment via
+ * Sparse-vLLM": reconstruction fused into attention; news page, "How
+ * ResidualKV Works": a token is rebuilt on the fly from its references and
+ * residual code when attention needs it).  For every query head g:
+ *   out[b][g] = sum_i softmax_i(q[b][g] . K_i / sqrt(D)) V_i
+ * over all lengths[b] cached positions, where reference rows are the stored
+ * bf16 rows and compressed rows are mean(references) + code * scale.  The
+ * reconstructed cache is never written to memory.  A sequence of length 0
+ * gives zeros.  workspace: device, scratch, >= rkv_cache_size's size.
+ */
+RKV_API rkv_status rkv_decode_attn(const rkv_cache_desc* desc, const void* q, void* out, void* workspace,
+                           uint64_t workspace_bytes, void* stream);
+
+/*
+ * Materialises reconstructed rows of one unit (paper summary page, "DeltaKV
+ * Framework Architecture", reconstruction KV = KV_delta + KV_R; "Training and
+ * Inference Integration", selective decompression of only the rows needed).
+ * positions: device int32[n_pos] in [0, length) or NULL for every position
+ * 0..length-1 (then n_pos must equal the length).  K_out, V_out: device
+ * [n_pos][head_dim] in out_dtype (either may be NULL).  Reference positions
+ * return the stored bf16 row; others m + code * scale computed in fp32.
+ */
+RKV_API rkv_status rkv_reconstruct(const rkv_cache_desc* desc, int32_t seq, int32_t kv_head, const int32_t* positions,
+                           int64_t n_pos, void* K_out, void* V_out, int32_t out_dtype, void* stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the cache's device error word.
+ * *device_status gets RKV_OK or the first RKV_ERR_* a kernel recorded since
+ * the last read.  Returns RKV_ERR_CUDA if the synchronisation failed.
+ */
+RKV_API rkv_status rkv_read_device_error(const rkv_cache_desc* desc, void* stream, int32_t* device_status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RKV_H */

@@ -1,0 +1,464 @@
+// C ABI of librkv: argument validation, cache layout and binding, kernel dispatch.
+// Every entry point returns an rkv_status and never throws; see include/rkv.h.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <climits>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "launchers.h"
+#include "rkv.h"
+#include "rkv_internal.h"
+
+using namespace rkv;
+
+namespace {
+
+uint64_t align_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// ---- reference schedule on the host ----------------------------------------------------
+
+rkv_status make_phases(const rkv_config& c, int64_t max_len, Phases& ph)
+{
+    std::memset(&ph, 0, sizeof(ph));
+    if (c.refs_per_phase <= 0) {
+        ph.n = 1;
+        ph.stride[0] = c.stride0;
+        return RKV_OK;
+    }
+    int64_t start = 0, stride = c.stride0, ord = 0;
+    int n = 0;
+    do {
+        if (n >= kMaxPhases || stride > INT32_MAX / 2 || start > INT32_MAX)
+            return RKV_ERR_UNSUPPORTED;
+        ph.start[n] = static_cast<int32_t>(start);
+        ph.stride[n] = static_cast<int32_t>(stride);
+        ph.first_ord[n] = static_cast<int32_t>(ord);
+        ph.first_slot[n] = static_cast<int32_t>(start - ord);
+        ++n;
+        start += static_cast<int64_t>(c.refs_per_phase) * stride;
+        ord += c.refs_per_phase;
+        stride *= 2;
+    } while (start < max_len);
+    ph.n = n;
+    return RKV_OK;
+}
+
+// references at positions <= p
+int64_t host_refs_upto(const Phases& ph, int64_t p)
+{
+    int q = 0;
+    for (int i = 1; i < ph.n; ++i)
+        if (p >= ph.start[i])
+            q = i;
+    return ph.first_ord[q] + (p - ph.start[q]) / ph.stride[q] + 1;
+}
+
+int64_t host_ref_count(const Phases& ph, int64_t n) { return n <= 0 ? 0 : host_refs_upto(ph, n - 1); }
+
+// ---- validation ---------------------------------------------------------------------
+
+rkv_status validate_config(const rkv_config* c)
+{
+    if (!c)
+        return RKV_ERR_INVALID_ARG;
+    if (c->n_kv_heads <= 0 || c->n_q_heads <= 0 || c->n_q_heads % c->n_kv_heads != 0 || c->batch <= 0 ||
+        c->max_len < 0 || c->k <= 0 || c->stride0 < 2 || c->refs_per_phase < 0 || c->group <= 0)
+        return RKV_ERR_INVALID_ARG;
+    if (c->in_dtype != RKV_DTYPE_BF16 && c->in_dtype != RKV_DTYPE_F32)
+        return RKV_ERR_INVALID_ARG;
+    if (c->out_dtype != RKV_DTYPE_BF16 && c->out_dtype != RKV_DTYPE_F32)
+        return RKV_ERR_INVALID_ARG;
+    if (c->bits != 4 && c->bits != 8)
+        return RKV_ERR_UNSUPPORTED;
+    if (c->head_dim != 64 && c->head_dim != 128)
+        return RKV_ERR_UNSUPPORTED;
+    if (c->group != 32 || c->k > RKV_MAX_K || c->batch > RKV_MAX_BATCH)
+        return RKV_ERR_UNSUPPORTED;
+    if (c->n_q_heads / c->n_kv_heads > 16)
+        return RKV_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(c->batch) * c->n_kv_heads > 65535)
+        return RKV_ERR_UNSUPPORTED;
+    return RKV_OK;
+}
+
+int decode_splits(int n_units, int max_tokens)
+{
+    int s = static_cast<int>(ceil_div(4 * 148, n_units));
+    s = std::max(1, std::min(s, 64));
+    s = std::min<int64_t>(s, std::max<int64_t>(1, ceil_div(max_tokens, 256)));
+    return s;
+}
+
+rkv_status compute_layout(const rkv_config* c, const int32_t* lengths, Desc& d)
+{
+    rkv_status st = validate_config(c);
+    if (st != RKV_OK)
+        return st;
+    if (!lengths)
+        return RKV_ERR_INVALID_ARG;
+    std::memset(&d, 0, sizeof(d));
+    d.magic = kDescMagic;
+    d.cfg = *c;
+    int max_n = 0;
+    for (int b = 0; b < c->batch; ++b) {
+        if (lengths[b] < 0 || lengths[b] > c->max_len)
+            return RKV_ERR_INVALID_ARG;
+        max_n = std::max(max_n, lengths[b]);
+    }
+    st = make_phases(*c, std::max(1, max_n), d.ph);
+    if (st != RKV_OK)
+        return st;
+    const int D = c->head_dim, Hkv = c->n_kv_heads, G = c->n_q_heads / c->n_kv_heads;
+    d.kc = search_width(c->k);
+    d.code_bytes = D * c->bits / 8;
+    d.n_groups = D / c->group;
+    d.n_units = c->batch * Hkv;
+    d.max_n = max_n;
+    int64_t ref_rows = 0, cmp_rows = 0, tiles = 0;
+    for (int b = 0; b < c->batch; ++b) {
+        const int64_t n = lengths[b];
+        const int64_t R = host_ref_count(d.ph, n);
+        if (R > RKV_MAX_REFS)
+            return RKV_ERR_UNSUPPORTED;
+        d.len[b] = static_cast<int32_t>(n);
+        d.R[b] = static_cast<int32_t>(R);
+        d.C[b] = static_cast<int32_t>(n - R);
+        d.Rpad[b] = static_cast<int32_t>(align_up(R, kRefPad));
+        d.Cpad[b] = static_cast<int32_t>(align_up(n - R, kCmpPad));
+        d.ref_seq_row[b] = ref_rows;
+        d.cmp_seq_row[b] = cmp_rows;
+        ref_rows += static_cast<int64_t>(Hkv) * d.Rpad[b];
+        cmp_rows += static_cast<int64_t>(Hkv) * d.Cpad[b];
+        tiles += static_cast<int64_t>(Hkv) * ceil_div(n, kPosTile);
+        d.max_R = std::max<int32_t>(d.max_R, d.R[b]);
+        d.max_C = std::max<int32_t>(d.max_C, d.C[b]);
+    }
+    if (tiles > INT32_MAX)
+        return RKV_ERR_UNSUPPORTED;
+    d.total_ref_rows = ref_rows;
+    d.total_cmp_rows = cmp_rows;
+    d.n_tiles = static_cast<int32_t>(tiles);
+    uint64_t off = 0;
+    auto take = [&](uint64_t bytes) {
+        const uint64_t o = off;
+        off = align_up(off + bytes, 256);
+        return o;
+    };
+    Sections& s = d.sec;
+    s.err = take(256);
+    s.units = take(sizeof(UnitMeta) * d.n_units);
+    s.tiles = take(sizeof(Tile) * std::max<int64_t>(1, tiles));
+    s.ref_K = take(2ull * ref_rows * D);
+    s.ref_V = take(2ull * ref_rows * D);
+    s.ref_hn = take(4ull * ref_rows);
+    s.ref_pos = take(4ull * ref_rows);
+    s.codes_K = take(static_cast<uint64_t>(cmp_rows) * d.code_bytes);
+    s.codes_V = take(static_cast<uint64_t>(cmp_rows) * d.code_bytes);
+    s.scale_K = take(2ull * cmp_rows * d.n_groups);
+    s.scale_V = take(2ull * cmp_rows * d.n_groups);
+    s.idx = take(2ull * cmp_rows * c->k);
+    s.end = off;
+    d.ws_select = align_up(2ull * cmp_rows * d.kc, 256) + align_up(4ull * cmp_rows * d.kc, 256);
+    const int splits = decode_splits(d.n_units, max_n);
+    d.ws_decode = align_up(4ull * d.n_units * splits * G * (D + 2), 256);
+    return RKV_OK;
+}
+
+const Desc* get_desc(const rkv_cache_desc* h)
+{
+    if (!h)
+        return nullptr;
+    const Desc* d = reinterpret_cast<const Desc*>(h->opaque);
+    return d->magic == kDescMagic ? d : nullptr;
+}
+
+CacheArgs make_args(const Desc& d)
+{
+    CacheArgs a;
+    std::memset(&a, 0, sizeof(a));
+    const rkv_config& c = d.cfg;
+    a.D = c.head_dim;
+    a.Hkv = c.n_kv_heads;
+    a.Hq = c.n_q_heads;
+    a.G = c.n_q_heads / c.n_kv_heads;
+    a.k = c.k;
+    a.bits = c.bits;
+    a.group = c.group;
+    a.in_dtype = c.in_dtype;
+    a.out_dtype = c.out_dtype;
+    a.n_units = d.n_units;
+    a.code_bytes = d.code_bytes;
+    a.n_groups = d.n_groups;
+    a.kc = d.kc;
+    a.max_len = c.max_len;
+    a.ph = d.ph;
+    char* base = static_cast<char*>(d.base);
+    a.err = reinterpret_cast<int32_t*>(base + d.sec.err);
+    a.units = reinterpret_cast<const UnitMeta*>(base + d.sec.units);
+    a.ref_K = reinterpret_cast<uint16_t*>(base + d.sec.ref_K);
+    a.ref_V = reinterpret_cast<uint16_t*>(base + d.sec.ref_V);
+    a.ref_hn = reinterpret_cast<float*>(base + d.sec.ref_hn);
+    a.ref_pos = reinterpret_cast<int32_t*>(base + d.sec.ref_pos);
+    a.codes_K = reinterpret_cast<uint8_t*>(base + d.sec.codes_K);
+    a.codes_V = reinterpret_cast<uint8_t*>(base + d.sec.codes_V);
+    a.scale_K = reinterpret_cast<uint16_t*>(base + d.sec.scale_K);
+    a.scale_V = reinterpret_cast<uint16_t*>(base + d.sec.scale_V);
+    a.idx = reinterpret_cast<uint16_t*>(base + d.sec.idx);
+    return a;
+}
+
+rkv_status cuda_status(cudaError_t e) { return e == cudaSuccess ? RKV_OK : RKV_ERR_CUDA; }
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+int32_t rkv_abi_version(void) { return RKV_ABI_VERSION; }
+
+const char* rkv_status_string(rkv_status s)
+{
+    switch (s) {
+    case RKV_OK: return "ok";
+    case RKV_ERR_INVALID_ARG: return "invalid argument";
+    case RKV_ERR_UNSUPPORTED: return "unsupported configuration";
+    case RKV_ERR_WORKSPACE: return "buffer too small";
+    case RKV_ERR_CUDA: return "CUDA error";
+    case RKV_ERR_CORRUPT: return "corrupted cache contents";
+    case RKV_ERR_TIMEOUT: return "device wait timed out";
+    }
+    return "unknown status";
+}
+
+rkv_status rkv_schedule(const rkv_config* cfg, int32_t n, int32_t* pos, int64_t cap, int32_t* n_ref)
+{
+    rkv_status st = validate_config(cfg);
+    if (st != RKV_OK)
+        return st;
+    if (n < 0 || !n_ref)
+        return RKV_ERR_INVALID_ARG;
+    Phases ph;
+    st = make_phases(*cfg, std::max(1, n), ph);
+    if (st != RKV_OK)
+        return st;
+    const int64_t R = host_ref_count(ph, n);
+    *n_ref = static_cast<int32_t>(R);
+    if (pos) {
+        int64_t w = 0;
+        for (int q = 0; q < ph.n && w < std::min<int64_t>(cap, R); ++q) {
+            const int64_t cnt = (q + 1 < ph.n) ? (ph.first_ord[q + 1] - ph.first_ord[q]) : R - ph.first_ord[q];
+            for (int64_t m = 0; m < cnt && w < std::min<int64_t>(cap, R); ++m)
+                pos[w++] = static_cast<int32_t>(ph.start[q] + m * ph.stride[q]);
+        }
+    }
+    return RKV_OK;
+}
+
+rkv_status rkv_cache_size(const rkv_config* cfg, const int32_t* lengths, uint64_t* cache_bytes,
+                          uint64_t* workspace_bytes)
+{
+    if (!cache_bytes || !workspace_bytes)
+        return RKV_ERR_INVALID_ARG;
+    Desc* d = new (std::nothrow) Desc;
+    if (!d)
+        return RKV_ERR_INVALID_ARG;
+    const rkv_status st = compute_layout(cfg, lengths, *d);
+    if (st == RKV_OK) {
+        *cache_bytes = d->sec.end;
+        *workspace_bytes = std::max(d->ws_select, d->ws_decode);
+    }
+    delete d;
+    return st;
+}
+
+rkv_status rkv_cache_bind(const rkv_config* cfg, const int32_t* lengths, void* dev_buf, uint64_t bytes,
+                          rkv_cache_desc* desc)
+{
+    if (!desc || !dev_buf || !aligned(dev_buf, 256))
+        return RKV_ERR_INVALID_ARG;
+    Desc* d = reinterpret_cast<Desc*>(desc->opaque);
+    std::memset(desc, 0, sizeof(*desc));
+    rkv_status st = compute_layout(cfg, lengths, *d);
+    if (st != RKV_OK) {
+        std::memset(desc, 0, sizeof(*desc));
+        return st;
+    }
+    if (bytes < d->sec.end) {
+        std::memset(desc, 0, sizeof(*desc));
+        return RKV_ERR_WORKSPACE;
+    }
+    int dev = 0, major = 0, minor = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+        std::memset(desc, 0, sizeof(*desc));
+        return RKV_ERR_CUDA;
+    }
+    if (major != 10 || minor != 0) {
+        std::memset(desc, 0, sizeof(*desc));
+        return RKV_ERR_UNSUPPORTED;
+    }
+    d->base = dev_buf;
+    d->bytes = bytes;
+    // unit table and the selection tiles, heaviest first
+    const int Hkv = cfg->n_kv_heads;
+    std::vector<UnitMeta> units(d->n_units);
+    std::vector<std::pair<int64_t, Tile>> work;
+    work.reserve(d->n_tiles);
+    for (int b = 0; b < cfg->batch; ++b)
+        for (int h = 0; h < Hkv; ++h) {
+            const int u = b * Hkv + h;
+            UnitMeta& m = units[u];
+            m.n = d->len[b];
+            m.R = d->R[b];
+            m.C = d->C[b];
+            m.seq = b;
+            m.ref_row = d->ref_seq_row[b] + static_cast<int64_t>(h) * d->Rpad[b];
+            m.cmp_row = d->cmp_seq_row[b] + static_cast<int64_t>(h) * d->Cpad[b];
+            const int nt = static_cast<int>(ceil_div(m.n, kPosTile));
+            for (int t = 0; t < nt; ++t) {
+                const int64_t last = std::min<int64_t>(static_cast<int64_t>(t + 1) * kPosTile, m.n) - 1;
+                work.push_back({host_refs_upto(d->ph, last), Tile{u, t}});
+            }
+        }
+    std::stable_sort(work.begin(), work.end(),
+                     [](const std::pair<int64_t, Tile>& x, const std::pair<int64_t, Tile>& y) { return x.first > y.first; });
+    std::vector<Tile> tiles(work.size());
+    for (size_t i = 0; i < work.size(); ++i)
+        tiles[i] = work[i].second;
+    char* base = static_cast<char*>(dev_buf);
+    cudaError_t e = cudaMemset(base + d->sec.err, 0, 256);
+    if (e == cudaSuccess)
+        e = cudaMemcpy(base + d->sec.units, units.data(), sizeof(UnitMeta) * units.size(), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && !tiles.empty())
+        e = cudaMemcpy(base + d->sec.tiles, tiles.data(), sizeof(Tile) * tiles.size(), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) {
+        std::memset(desc, 0, sizeof(*desc));
+        return RKV_ERR_CUDA;
+    }
+    return RKV_OK;
+}
+
+rkv_status rkv_unit_view_get(const rkv_cache_desc* desc, int32_t seq, int32_t kv_head, rkv_unit_view* out)
+{
+    const Desc* d = get_desc(desc);
+    if (!d || !out || seq < 0 || seq >= d->cfg.batch || kv_head < 0 || kv_head >= d->cfg.n_kv_heads)
+        return RKV_ERR_INVALID_ARG;
+    const CacheArgs a = make_args(*d);
+    const int64_t ref_row = d->ref_seq_row[seq] + static_cast<int64_t>(kv_head) * d->Rpad[seq];
+    const int64_t cmp_row = d->cmp_seq_row[seq] + static_cast<int64_t>(kv_head) * d->Cpad[seq];
+    std::memset(out, 0, sizeof(*out));
+    out->n = d->len[seq];
+    out->n_ref = d->R[seq];
+    out->n_cmp = d->C[seq];
+    out->k = d->cfg.k;
+    out->code_bytes = d->code_bytes;
+    out->n_groups = d->n_groups;
+    out->ref_K = a.ref_K + ref_row * a.D;
+    out->ref_V = a.ref_V + ref_row * a.D;
+    out->ref_half_norm = a.ref_hn + ref_row;
+    out->ref_pos = a.ref_pos + ref_row;
+    out->codes_K = a.codes_K + cmp_row * d->code_bytes;
+    out->codes_V = a.codes_V + cmp_row * d->code_bytes;
+    out->scale_K = a.scale_K + cmp_row * d->n_groups;
+    out->scale_V = a.scale_V + cmp_row * d->n_groups;
+    out->idx = a.idx + cmp_row * d->cfg.k;
+    return RKV_OK;
+}
+
+rkv_status rkv_build_refs(const rkv_cache_desc* desc, const void* K, const void* V, void* stream)
+{
+    const Desc* d = get_desc(desc);
+    if (!d || !K || !V || !aligned(K, 16) || !aligned(V, 16))
+        return RKV_ERR_INVALID_ARG;
+    const CacheArgs a = make_args(*d);
+    return cuda_status(launch_refs_copy(a, d->max_R, K, V, static_cast<cudaStream_t>(stream)));
+}
+
+rkv_status rkv_compress(const rkv_cache_desc* desc, const void* K, const void* V, void* workspace,
+                        uint64_t workspace_bytes, void* stream)
+{
+    const Desc* d = get_desc(desc);
+    if (!d || !K || !V || !aligned(K, 16) || !aligned(V, 16) || (!workspace && d->ws_select > 0) ||
+        !aligned(workspace, 256))
+        return RKV_ERR_INVALID_ARG;
+    if (workspace_bytes < d->ws_select)
+        return RKV_ERR_WORKSPACE;
+    const CacheArgs a = make_args(*d);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint16_t* cand_idx = static_cast<uint16_t*>(workspace);
+    float* cand_t = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                             align_up(2ull * d->total_cmp_rows * d->kc, 256));
+    const Tile* tiles = reinterpret_cast<const Tile*>(static_cast<char*>(d->base) + d->sec.tiles);
+    cudaError_t e = launch_select_simt(a, tiles, d->n_tiles, K, cand_idx, cand_t, st);
+    if (e == cudaSuccess)
+        e = launch_encode(a, d->max_C, K, V, cand_idx, cand_t, st);
+    return cuda_status(e);
+}
+
+rkv_status rkv_decode_attn(const rkv_cache_desc* desc, const void* q, void* out, void* workspace,
+                           uint64_t workspace_bytes, void* stream)
+{
+    const Desc* d = get_desc(desc);
+    if (!d || !q || !out || !workspace || !aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, 256))
+        return RKV_ERR_INVALID_ARG;
+    if (workspace_bytes < d->ws_decode)
+        return RKV_ERR_WORKSPACE;
+    const CacheArgs a = make_args(*d);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int splits = decode_splits(d->n_units, d->max_n);
+    float* part = static_cast<float*>(workspace);
+    cudaError_t e = launch_decode_direct(a, splits, q, part, st);
+    if (e == cudaSuccess)
+        e = launch_decode_combine(a, d->cfg.batch, splits, part, out, st);
+    return cuda_status(e);
+}
+
+rkv_status rkv_reconstruct(const rkv_cache_desc* desc, int32_t seq, int32_t kv_head, const int32_t* positions,
+                           int64_t n_pos, void* K_out, void* V_out, int32_t out_dtype, void* stream)
+{
+    const Desc* d = get_desc(desc);
+    if (!d || seq < 0 || seq >= d->cfg.batch || kv_head < 0 || kv_head >= d->cfg.n_kv_heads || n_pos < 0)
+        return RKV_ERR_INVALID_ARG;
+    if (out_dtype != RKV_DTYPE_BF16 && out_dtype != RKV_DTYPE_F32)
+        return RKV_ERR_INVALID_ARG;
+    if (!positions && n_pos != d->len[seq])
+        return RKV_ERR_INVALID_ARG;
+    if ((K_out && !aligned(K_out, 16)) || (V_out && !aligned(V_out, 16)) || (positions && !aligned(positions, 4)))
+        return RKV_ERR_INVALID_ARG;
+    if (n_pos == 0)
+        return RKV_OK;
+    if (!K_out && !V_out)
+        return RKV_ERR_INVALID_ARG;
+    const CacheArgs a = make_args(*d);
+    return cuda_status(launch_reconstruct(a, seq * d->cfg.n_kv_heads + kv_head, positions, n_pos, K_out, V_out,
+                                          out_dtype, static_cast<cudaStream_t>(stream)));
+}
+
+rkv_status rkv_read_device_error(const rkv_cache_desc* desc, void* stream, int32_t* device_status)
+{
+    const Desc* d = get_desc(desc);
+    if (!d || !device_status)
+        return RKV_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess)
+        return RKV_ERR_CUDA;
+    int32_t* err = reinterpret_cast<int32_t*>(static_cast<char*>(d->base) + d->sec.err);
+    int32_t v = 0;
+    if (cudaMemcpy(&v, err, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return RKV_ERR_CUDA;
+    if (v != 0 && cudaMemset(err, 0, sizeof(int32_t)) != cudaSuccess)
+        return RKV_ERR_CUDA;
+    if (cudaDeviceSynchronize() != cudaSuccess)
+        return RKV_ERR_CUDA;
+    *device_status = v;
+    return RKV_OK;
+}
+
+}  // extern "C"

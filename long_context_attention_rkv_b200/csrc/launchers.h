@@ -1,0 +1,28 @@
+// Host-side launchers of the librkv kernels (one translation unit each).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "rkv_internal.h"
+
+namespace rkv {
+
+cudaError_t launch_refs_copy(const CacheArgs& a, int max_R, const void* K, const void* V, cudaStream_t st);
+
+cudaError_t launch_select_simt(const CacheArgs& a, const Tile* tiles, int n_tiles, const void* K, uint16_t* cand_idx,
+                               float* cand_t, cudaStream_t st);
+
+cudaError_t launch_encode(const CacheArgs& a, int max_C, const void* K, const void* V, const uint16_t* cand_idx,
+                          const float* cand_t, cudaStream_t st);
+
+cudaError_t launch_reconstruct(const CacheArgs& a, int unit, const int32_t* positions, int64_t n_pos, void* K_out,
+                               void* V_out, int out_dtype, cudaStream_t st);
+
+// Literal decode: per token gather + mean of the reference rows, dequantise, add, attend.
+cudaError_t launch_decode_direct(const CacheArgs& a, int splits, const void* q, float* partials, cudaStream_t st);
+
+// Merge of per-split partial softmax states into the output.
+cudaError_t launch_decode_combine(const CacheArgs& a, int batch, int splits, const float* partials, void* out,
+                                  cudaStream_t st);
+
+}  // namespace rkv

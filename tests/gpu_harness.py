@@ -1,0 +1,243 @@
+"""Shared helpers of the GPU parity tests: run the library through its C ABI on
+seeded synthetic inputs and compare every stage with the CPU oracle."""
+from __future__ import annotations
+
+import ctypes
+import math
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+import torch
+
+import long_context_attention_rkv_b200 as rkv
+import oracle
+import synth
+
+# tolerances of the parity contract
+IDX_TIE_BAND = 1e-4         # relative gap between the k-th and (k+1)-th oracle distance
+CODE_LSB_FRACTION = 1e-3    # codes may differ by one step on at most this fraction of elements
+RECON_ABS = 1e-2            # reconstructed K/V
+ATTN_ABS = 2e-3             # decode output (fp32 output; bf16 output adds half a bf16 ulp)
+
+
+def to_dev(arr: np.ndarray) -> torch.Tensor:
+    a = np.ascontiguousarray(arr)
+    if a.dtype == np.uint16:
+        a = a.view(np.int16)
+    return torch.from_numpy(a).cuda()
+
+
+def config(wl: synth.Workload, lengths, max_len=None, out_dtype=rkv.RKV_DTYPE_F32, flags=0, batch=None):
+    return rkv.make_config(head_dim=wl.head_dim, n_kv_heads=wl.n_kv_heads, n_q_heads=wl.n_q_heads, k=wl.k,
+                           bits=wl.bits, stride0=wl.stride0, batch=len(lengths) if batch is None else batch,
+                           max_len=max(max(lengths), 1) if max_len is None else max_len,
+                           refs_per_phase=wl.refs_per_phase, in_dtype=wl.dtype_code, out_dtype=out_dtype,
+                           flags=flags)
+
+
+class GpuRun:
+    """One layer compressed on the GPU through the C ABI."""
+
+    def __init__(self, wl: synth.Workload, K: np.ndarray, V: np.ndarray, lengths, out_dtype=rkv.RKV_DTYPE_F32,
+                 flags=0):
+        self.wl = wl
+        self.lengths = list(lengths)
+        self.cfg = config(wl, lengths, max_len=K.shape[2], out_dtype=out_dtype, flags=flags)
+        self.layer = rkv.Layer(self.cfg, self.lengths)
+        self.Kd = to_dev(K)
+        self.Vd = to_dev(V)
+        self.layer.build_refs(self.Kd, self.Vd)
+        self.layer.compress(self.Kd, self.Vd)
+        torch.cuda.synchronize()
+        err = self.layer.device_error()
+        assert err == 0, f"device error {rkv.STATUS.get(err, err)}"
+
+    def _read(self, ptr, nbytes, dtype, shape):
+        if nbytes == 0:
+            return np.zeros(shape, dtype=dtype)
+        off = ptr - self.layer.cache.data_ptr()
+        assert 0 <= off and off + nbytes <= self.layer.cache.numel()
+        raw = self.layer.cache[off:off + nbytes].cpu().numpy()
+        return raw.view(dtype).reshape(shape)
+
+    def unit(self, b: int, h: int) -> dict:
+        v = self.layer.unit(b, h)
+        D, R, C, k = self.wl.head_dim, v.n_ref, v.n_cmp, v.k
+        return dict(
+            n=v.n, R=R, C=C,
+            refK=self._read(v.ref_K, 2 * R * D, np.uint16, (R, D)),
+            refV=self._read(v.ref_V, 2 * R * D, np.uint16, (R, D)),
+            hn=self._read(v.ref_half_norm, 4 * R, np.float32, (R,)),
+            pos=self._read(v.ref_pos, 4 * R, np.int32, (R,)),
+            codesK=self._read(v.codes_K, C * v.code_bytes, np.uint8, (C, v.code_bytes)),
+            codesV=self._read(v.codes_V, C * v.code_bytes, np.uint8, (C, v.code_bytes)),
+            scalesK=self._read(v.scale_K, 2 * C * v.n_groups, np.uint16, (C, v.n_groups)),
+            scalesV=self._read(v.scale_V, 2 * C * v.n_groups, np.uint16, (C, v.n_groups)),
+            idx=self._read(v.idx, 2 * C * k, np.uint16, (C, k)),
+        )
+
+    def decode(self, q: np.ndarray) -> np.ndarray:
+        qd = to_dev(q)
+        dt = torch.float32 if self.cfg.out_dtype == rkv.RKV_DTYPE_F32 else torch.bfloat16
+        out = torch.empty((len(self.lengths), self.wl.n_q_heads, self.wl.head_dim), dtype=dt, device="cuda")
+        self.layer.decode(qd, out)
+        torch.cuda.synchronize()
+        err = self.layer.device_error()
+        assert err == 0, f"device error {rkv.STATUS.get(err, err)}"
+        return out.float().cpu().numpy()
+
+    def reconstruct(self, b: int, h: int, positions=None):
+        n = self.lengths[b]
+        npos = n if positions is None else len(positions)
+        K = torch.empty((max(npos, 1), self.wl.head_dim), dtype=torch.float32, device="cuda")
+        V = torch.empty_like(K)
+        pd = None if positions is None else to_dev(np.asarray(positions, dtype=np.int32))
+        self.layer.reconstruct(b, h, pd, npos, K, V, rkv.RKV_DTYPE_F32)
+        torch.cuda.synchronize()
+        assert self.layer.device_error() == 0
+        return K[:npos].cpu().numpy(), V[:npos].cpu().numpy()
+
+
+# --- oracle-side comparisons --------------------------------------------------------------
+
+def unit_rows(wl: synth.Workload, K: np.ndarray, V: np.ndarray, b: int, h: int, n: int):
+    """Float rows (exact input values) of one unit."""
+    return synth.as_f32(wl, K[b, h, :n]), synth.as_f32(wl, V[b, h, :n])
+
+
+def slots_of(positions: np.ndarray, ref_pos: np.ndarray) -> np.ndarray:
+    return positions - np.searchsorted(ref_pos, positions, side="right")
+
+
+def _unpack(codes: np.ndarray, D: int, bits: int) -> np.ndarray:
+    if bits == 8:
+        return codes.view(np.int8).astype(np.int64)
+    lo = (codes & 0xF).astype(np.int64)
+    hi = (codes >> 4).astype(np.int64)
+    out = np.empty(codes.shape[:-1] + (D,), dtype=np.int64)
+    out[..., 0::2] = lo
+    out[..., 1::2] = hi
+    return np.where(out >= 8, out - 16, out)
+
+
+def check_refs(wl, g: dict, Xk, Xv):
+    ref_pos = oracle.schedule(len(Xk), wl.stride0, wl.refs_per_phase)
+    assert np.array_equal(g["pos"], ref_pos)
+    assert np.array_equal(g["refK"], oracle.build_refs(Xk, ref_pos))
+    assert np.array_equal(g["refV"], oracle.build_refs(Xv, ref_pos))
+    rv = oracle.bf16_value(g["refK"]).astype(np.float64)
+    np.testing.assert_allclose(g["hn"], 0.5 * (rv * rv).sum(axis=1), rtol=2e-6, atol=1e-30)
+    return ref_pos
+
+
+def check_compress(wl, g: dict, Xk, Xv, positions=None, stats=None):
+    """Selection (tie-band aware) and codes of compressed positions against the oracle."""
+    n = len(Xk)
+    ref_pos = oracle.schedule(n, wl.stride0, wl.refs_per_phase)
+    cpos, _ = oracle.positions_split(n, ref_pos)
+    if positions is None:
+        positions = cpos
+    positions = np.asarray(positions, dtype=np.int32)
+    if len(positions) == 0:
+        return
+    slots = slots_of(positions, ref_pos)
+    refK = g["refK"]
+    refV = g["refV"]
+    gidx = g["idx"][slots]
+    oidx, okeff, odist = oracle.select(Xk[positions], positions, refK, ref_pos, wl.k)
+    k = wl.k
+    mism = 0
+    for t in np.nonzero(np.any(gidx != oidx, axis=1))[0]:
+        mism += 1
+        ke = okeff[t]
+        dk, dk1 = odist[t, ke - 1], odist[t, ke]
+        assert ke < k + 1 and not math.isnan(dk1), f"selection differs at position {positions[t]} with no tie"
+        assert dk1 - dk <= IDX_TIE_BAND * dk, (
+            f"selection differs outside the tie band at position {positions[t]}: "
+            f"gpu {gidx[t]} oracle {oidx[t]} d_k={dk} d_k+1={dk1}")
+        sel = gidx[t][gidx[t] != oracle.SENTINEL]
+        assert len(sel) == ke and np.all(np.diff(sel.astype(int)) > 0) and np.all(ref_pos[sel] < positions[t])
+        rv = oracle.bf16_value(refK)
+        worst = max(oracle.l2(Xk[positions[t]], rv[j]) for j in sel)
+        assert worst <= dk1 * (1 + IDX_TIE_BAND)
+    # codes: the oracle's encoder fed the GPU's index sets
+    ek = oracle.encode(Xk[positions], refK, gidx, wl.bits, wl.group)
+    ev = oracle.encode(Xv[positions], refV, gidx, wl.bits, wl.group)
+    assert ek["overflow"] == 0 and ev["overflow"] == 0
+    D = wl.head_dim
+    for name, e in (("K", ek), ("V", ev)):
+        assert np.array_equal(g["scales" + name][slots], e["scales"]), f"{name} scales differ"
+        gc = _unpack(g["codes" + name][slots], D, wl.bits)
+        oc = _unpack(e["codes"], D, wl.bits)
+        diff = np.abs(gc - oc)
+        assert diff.max(initial=0) <= 1, f"{name} codes differ by more than one step"
+        assert diff.astype(bool).mean() <= CODE_LSB_FRACTION
+    if stats is not None:
+        stats["tokens"] = stats.get("tokens", 0) + len(positions)
+        stats["idx_tie_mismatch"] = stats.get("idx_tie_mismatch", 0) + mism
+
+
+def oracle_decode_on_gpu_cache(wl, g: dict, q_group: np.ndarray):
+    """The oracle's reconstruction and attention over the cache the GPU produced."""
+    n = g["n"]
+    if n == 0:
+        return np.zeros((q_group.shape[0], wl.head_dim))
+    Kh, Vh = oracle.unit_cache_rows(n, g["pos"], g["refK"], g["refV"], g["idx"], g["codesK"], g["scalesK"],
+                                    g["codesV"], g["scalesV"], wl.bits, wl.group)
+    return oracle.attention(q_group.astype(np.float64), Kh, Vh)
+
+
+def check_decode(run: GpuRun, q: np.ndarray, units=None, threads=8):
+    """Decode output of every (or the listed) unit against the oracle on the GPU's cache."""
+    wl = run.wl
+    out = run.decode(q)
+    qf = synth.as_f32(wl, q)
+    G = wl.n_q_heads // wl.n_kv_heads
+    units = [(b, h) for b in range(len(run.lengths)) for h in range(wl.n_kv_heads)] if units is None else units
+    gus = {u: run.unit(*u) for u in units}
+
+    def one(u):
+        b, h = u
+        return u, oracle_decode_on_gpu_cache(wl, gus[u], qf[b, h * G:(h + 1) * G])
+
+    with ThreadPoolExecutor(threads) as ex:
+        refs = dict(ex.map(one, units))
+    worst = 0.0
+    for (b, h), ref in refs.items():
+        got = out[b, h * G:(h + 1) * G].astype(np.float64)
+        if run.cfg.out_dtype == rkv.RKV_DTYPE_F32:
+            tol = ATTN_ABS
+        else:
+            tol = ATTN_ABS + np.abs(ref) * 2.0 ** -8          # half an ulp of bf16 on top
+        err = np.abs(got - ref)
+        assert np.all(err <= tol), f"decode unit {(b, h)}: max err {err.max()}"
+        worst = max(worst, float(err.max(initial=0)))
+    return worst
+
+
+def check_reconstruct(run: GpuRun, g: dict, b: int, h: int, positions=None):
+    wl = run.wl
+    n = g["n"]
+    Kh, Vh = oracle.unit_cache_rows(n, g["pos"], g["refK"], g["refV"], g["idx"], g["codesK"], g["scalesK"],
+                                    g["codesV"], g["scalesV"], wl.bits, wl.group)
+    Kg, Vg = run.reconstruct(b, h, positions)
+    sel = np.arange(n) if positions is None else np.asarray(positions)
+    np.testing.assert_allclose(Kg, Kh[sel], atol=RECON_ABS, rtol=0)
+    np.testing.assert_allclose(Vg, Vh[sel], atol=RECON_ABS, rtol=0)
+    return float(max(np.abs(Kg - Kh[sel]).max(initial=0), np.abs(Vg - Vh[sel]).max(initial=0)))
+
+
+def sample_positions(wl, n: int, n_uniform=2048, seed=0):
+    """Deterministic row sample: the first k*s positions, phase boundaries +-2, uniform rows."""
+    ref_pos = oracle.schedule(n, wl.stride0, wl.refs_per_phase)
+    cpos, is_ref = oracle.positions_split(n, ref_pos)
+    pick = set(range(min(n, wl.k * wl.stride0)))
+    if wl.refs_per_phase:
+        for j in range(0, len(ref_pos), wl.refs_per_phase):
+            for d in (-2, -1, 1, 2):
+                pick.add(int(ref_pos[j]) + d)
+    rng = np.random.default_rng(seed)
+    if len(cpos):
+        pick.update(int(p) for p in rng.choice(cpos, min(n_uniform, len(cpos)), replace=False))
+    pick.add(n - 1)
+    return np.array(sorted(p for p in pick if 0 <= p < n and not is_ref[p]), dtype=np.int32)

@@ -1,0 +1,178 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle, element by element.
+
+Small cases run every stage on every token (several tiles, ragged tails, short
+and empty sequences, dynamic stride); the named workloads run at full size in
+the bench's launch configuration, checking sampled compressed rows exactly and
+decode over every unit.
+"""
+import numpy as np
+import pytest
+import torch
+
+import long_context_attention_rkv_b200 as rkv
+import oracle
+import synth
+from gpu_harness import (GpuRun, check_compress, check_decode, check_reconstruct, check_refs, sample_positions,
+                         to_dev, unit_rows)
+
+pytestmark = pytest.mark.gpu
+
+
+def _small(name, **kw):
+    return synth.WORKLOADS[name].with_(**kw)
+
+
+def _full_unit_checks(run, wl, K, V, lengths, recon=True):
+    stats = {}
+    for b, n in enumerate(lengths):
+        for h in range(wl.n_kv_heads):
+            g = run.unit(b, h)
+            Xk, Xv = unit_rows(wl, K, V, b, h, n)
+            if n:
+                check_refs(wl, g, Xk, Xv)
+                check_compress(wl, g, Xk, Xv, stats=stats)
+                if recon:
+                    check_reconstruct(run, g, b, h)
+    return stats
+
+
+def test_tiny_workload_every_stage():
+    wl = synth.WORKLOADS["tiny"]
+    lengths = wl.lengths()
+    K, V = synth.gen_layer(wl, 0, lengths)
+    run = GpuRun(wl, K, V, lengths)
+    stats = _full_unit_checks(run, wl, K, V, lengths)
+    assert stats["tokens"] == 1920
+    check_decode(run, synth.gen_query(wl, 0, 0))
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_bf16_ragged_batch_every_stage(bits):
+    wl = _small("llama3_8b_layer", n_kv_heads=2, n_q_heads=8, bits=bits, batch=4, seq_len=5000)
+    lengths = [5000, 777, 1, 0]
+    K, V = synth.gen_layer(wl, 0, lengths, max_len=5003)
+    run = GpuRun(wl, K, V, lengths)
+    _full_unit_checks(run, wl, K, V, lengths)
+    check_decode(run, synth.gen_query(wl, 0, 0))
+
+
+def test_dynamic_stride_every_stage():
+    wl = _small("ultra_long_1m", n_kv_heads=1, n_q_heads=4, head_dim=64, stride0=4, refs_per_phase=64, k=3,
+                bits=8, seq_len=6000, n_proto=64)
+    lengths = [6000]
+    K, V = synth.gen_layer(wl, 0, lengths)
+    run = GpuRun(wl, K, V, lengths)
+    stats = _full_unit_checks(run, wl, K, V, lengths)
+    assert stats["tokens"] == 6000 - len(oracle.schedule(6000, 4, 64))
+    check_decode(run, synth.gen_query(wl, 0, 0))
+
+
+def test_k8_stride32_group7_every_stage():
+    wl = _small("qwen2_5_7b_batch", n_kv_heads=2, n_q_heads=14, batch=2, seq_len=3000, ragged=None)
+    lengths = [3000, 2500]
+    K, V = synth.gen_layer(wl, 0, lengths)
+    run = GpuRun(wl, K, V, lengths)
+    _full_unit_checks(run, wl, K, V, lengths)
+    check_decode(run, synth.gen_query(wl, 0, 0))
+
+
+def test_simt_search_matches_default_search():
+    wl = _small("llama3_8b_layer", n_kv_heads=2, n_q_heads=8, seq_len=4100)
+    lengths = [4100]
+    K, V = synth.gen_layer(wl, 0, lengths)
+    a = GpuRun(wl, K, V, lengths)
+    b = GpuRun(wl, K, V, lengths, flags=rkv.RKV_FLAG_SELECT_SIMT)
+    for h in range(2):
+        ga, gb = a.unit(0, h), b.unit(0, h)
+        Xk, Xv = unit_rows(wl, K, V, 0, h, 4100)
+        check_compress(wl, gb, Xk, Xv)
+        same = np.all(ga["idx"] == gb["idx"], axis=1).mean()
+        assert same > 0.995
+
+
+def test_decode_sharp_query_and_bf16_output():
+    wl = _small("llama3_8b_layer", n_kv_heads=2, n_q_heads=8, seq_len=3000)
+    lengths = [3000]
+    K, V = synth.gen_layer(wl, 0, lengths)
+    Kf = synth.as_f32(wl, K)
+    q = np.zeros((1, 8, 128), dtype=np.float32)
+    for h in range(2):
+        q[0, h * 4:(h + 1) * 4] = synth.sharp_query(wl, Kf[0, h], 1234 + 77 * h, 4)
+    qb = oracle.bf16_round(q)                                  # the query is a bf16 input
+    run = GpuRun(wl, K, V, lengths)
+    check_decode(run, qb)
+    run16 = GpuRun(wl, K, V, lengths, out_dtype=rkv.RKV_DTYPE_BF16)
+    check_decode(run16, qb)
+
+
+def test_reconstruct_position_list():
+    wl = _small("llama3_8b_layer", n_kv_heads=1, n_q_heads=4, seq_len=2500)
+    lengths = [2500]
+    K, V = synth.gen_layer(wl, 0, lengths)
+    run = GpuRun(wl, K, V, lengths)
+    g = run.unit(0, 0)
+    pos = np.array([0, 1, 15, 16, 17, 2499, 1024, 3, 3], dtype=np.int32)
+    check_reconstruct(run, g, 0, 0, pos)
+
+
+def test_corrupted_cache_is_reported_not_faulted():
+    wl = _small("llama3_8b_layer", n_kv_heads=1, n_q_heads=4, seq_len=1000)
+    lengths = [1000]
+    K, V = synth.gen_layer(wl, 0, lengths)
+    run = GpuRun(wl, K, V, lengths)
+    v = run.layer.unit(0, 0)
+    off = v.idx - run.layer.cache.data_ptr()
+    saved = run.layer.cache[off:off + 2].clone()
+    run.layer.cache[off:off + 2] = torch.tensor([0xF0, 0x7F], dtype=torch.uint8, device="cuda")  # ordinal 0x7FF0
+    q = to_dev(synth.gen_query(wl, 0, 0))
+    out = torch.empty((1, 4, 128), dtype=torch.float32, device="cuda")
+    run.layer.decode(q, out)
+    assert run.layer.device_error() == rkv.STATUS_CODE["RKV_ERR_CORRUPT"]
+    assert run.layer.device_error() == 0                       # read clears it
+    Kout = torch.empty((4, 128), dtype=torch.float32, device="cuda")
+    run.layer.reconstruct(0, 0, to_dev(np.array([1, 2, 3, 5000], dtype=np.int32)), 4, Kout, None,
+                          rkv.RKV_DTYPE_F32)
+    st = run.layer.device_error()
+    assert st in (rkv.STATUS_CODE["RKV_ERR_CORRUPT"], rkv.STATUS_CODE["RKV_ERR_INVALID_ARG"])
+    run.layer.cache[off:off + 2] = saved
+    run.layer.decode(q, out)
+    assert run.layer.device_error() == 0
+
+
+# --- named workloads at full size (sampled rows for the search, full decode) ----------------
+
+def _named(name, layers, steps, n_uniform=2048):
+    wl = synth.WORKLOADS[name]
+    lengths = wl.lengths()
+    worst = 0.0
+    for layer in layers:
+        K, V = synth.gen_layer(wl, layer, lengths)
+        run = GpuRun(wl, K, V, lengths, out_dtype=rkv.RKV_DTYPE_BF16)
+        stats = {}
+        for b, n in enumerate(lengths):
+            for h in range(wl.n_kv_heads):
+                g = run.unit(b, h)
+                Xk, Xv = unit_rows(wl, K, V, b, h, n)
+                check_refs(wl, g, Xk, Xv)
+                check_compress(wl, g, Xk, Xv, sample_positions(wl, n, n_uniform, seed=b * 97 + h), stats)
+        for step in steps:
+            worst = max(worst, check_decode(run, synth.gen_query(wl, layer, step)))
+        del run
+        torch.cuda.empty_cache()
+    return worst
+
+
+def test_llama3_8b_layer_full_size():
+    _named("llama3_8b_layer", layers=[0], steps=[0])
+
+
+def test_llama3_8b_stack_full_size_two_layers():
+    _named("llama3_8b_stack", layers=[0, 31], steps=[0, 63], n_uniform=512)
+
+
+def test_qwen2_5_7b_batch_full_size_two_layers():
+    _named("qwen2_5_7b_batch", layers=[0, 27], steps=[0], n_uniform=512)
+
+
+def test_ultra_long_full_size():
+    _named("ultra_long_1m", layers=[0], steps=[0, 15], n_uniform=512)
