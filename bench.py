@@ -1,0 +1,474 @@
+#!/usr/bin/env python
+"""Benchmark of the residual KV-cache compression hot path (librkv) on B200.
+
+One step = the whole path over one layer of the Llama-3-8B-shaped workload
+(32 q / 8 kv heads, D=128, bf16, 32768 tokens, stride 16, k=4, int4 residuals):
+reference store, reference search, residual encoding, one decode-attention
+step, and a 256-row reconstruction.  Inputs are resident in HBM when the timed
+region starts; L2 is flushed (256 MiB write) before every timed step, outside
+the timed spans.  With N GPUs (torchrun) every rank runs its own replica on an
+independent layer; value is the whole-job throughput over the max-over-ranks
+step time.  `--impl reference` times the CPU oracle on a bounded sample of the
+same workload on the host cores.  Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+from concurrent.futures import ThreadPoolExecutor
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "decode-attn µs/step & HBM GB/s vs roofline; compress Mtok/s; 1 B200"
+WORKLOAD = "llama3_8b_layer"
+# kernels launched per step, by stage
+LAUNCHES = {"build_refs": 1, "search": 1, "encode": 1, "decode": 2, "reconstruct": 1}
+RECON_ROWS = 256
+
+
+def _load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm=float(p["hbm_gbs"]), bf16=float(p["bf16_tflops"]),
+                    bf16_sustained=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+# fp32 FMA issue peak of the CUDA cores: 148 SMs x 128 lanes x 2 flop x 1.965 GHz
+ALU_FP32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def workload_quantities(wl, lengths):
+    """Algorithmic work of one step over one layer (per-unit sums); the reference positions
+    come from the library's host-side schedule."""
+    import long_context_attention_rkv_b200 as rkv
+
+    D = wl.head_dim
+    per_tok = 2 * D * wl.bits // 8 + 2 * (D // 32) * 2 + 2 * wl.k
+    flops = 0
+    dec_bytes = 0
+    enc_bytes = 0
+    refs_bytes = 0
+    for n in lengths:
+        cfg = rkv.make_config(head_dim=D, n_kv_heads=wl.n_kv_heads, n_q_heads=wl.n_q_heads, k=wl.k, bits=wl.bits,
+                              stride0=wl.stride0, batch=1, max_len=max(n, 1), refs_per_phase=wl.refs_per_phase)
+        ref_pos = rkv.rkv_schedule(cfg, n)
+        R = len(ref_pos)
+        C = n - R
+        # search: every compressed token against its earlier references, 2*D flops each
+        is_ref = np.zeros(n, dtype=bool)
+        is_ref[ref_pos] = True
+        cpos = np.nonzero(~is_ref)[0]
+        ncand = np.searchsorted(ref_pos, cpos, side="right").astype(np.int64)
+        flops += wl.n_kv_heads * int(ncand.sum()) * 2 * D
+        dec_bytes += wl.n_kv_heads * (C * per_tok + R * 4 * D)
+        enc_bytes += wl.n_kv_heads * C * (2 * D * wl.elem_bytes + per_tok)
+        refs_bytes += wl.n_kv_heads * R * (2 * D * wl.elem_bytes + 4 * D + 8)
+    return dict(tokens=sum(lengths), search_flops=flops,
+                decode_bytes=dec_bytes, encode_bytes=enc_bytes, refs_bytes=refs_bytes, bytes_per_token=per_tok)
+
+
+class ClockSampler:
+    """Samples SM clock, power and clock-event reasons with NVML in a thread."""
+
+    def __init__(self, index: int, period_s: float = 0.02):
+        self.index = index
+        self.period = period_s
+        self.samples = []
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+
+    def start(self):
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            return self
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                self.samples.append((mhz, reasons))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def stop(self):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+        if not self.ok:
+            return None
+        names = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+                 0x80: "hw_power_brake_slowdown"}
+        seen = set()
+        for _, r in self.samples:
+            for bit, nm in names.items():
+                if r & bit:
+                    seen.add(nm)
+        mhz = [m for m, _ in self.samples]
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(seen), "samples": len(mhz)}
+
+
+def _src_sha(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic(kernel: str, src: list[str]):
+    """Per-launch DRAM bytes of a kernel from a committed ncu summary, if its source is unchanged."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        t = json.load(f)
+    e = t.get(kernel)
+    if not e or e.get("src_sha") != _src_sha(src):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class OracleSample:
+    """Times the CPU oracle on a bounded sample of one step: S uniformly drawn compressed positions
+    of every kv head are searched, encoded, reconstructed and attended over."""
+
+    def __init__(self, wl, lengths, layer: int, threads: int):
+        self.wl, self.lengths, self.layer, self.threads = wl, lengths, layer, threads
+        self.S = 64
+        self._prep()
+
+    def _prep(self):
+        import oracle
+        import synth
+
+        wl, lengths, layer = self.wl, self.lengths, self.layer
+        self._setup(oracle, synth, wl, lengths, layer)
+
+    def _setup(self, oracle, synth, wl, lengths, layer):
+        self.oracle = oracle
+        n = lengths[0]
+        K, V = synth.gen_layer(wl, layer, [n])
+        self.G = wl.n_q_heads // wl.n_kv_heads
+        self.qf = synth.as_f32(wl, synth.gen_query(wl, layer, 0))
+        self.ref_pos = oracle.schedule(n, wl.stride0, wl.refs_per_phase)
+        self.cpos, _ = oracle.positions_split(n, self.ref_pos)
+        self.units = [(0, h) for h in range(wl.n_kv_heads)]
+        self.Xs = {u: (synth.as_f32(wl, K[u[0], u[1], :n]), synth.as_f32(wl, V[u[0], u[1], :n])) for u in self.units}
+
+    def _work(self, u, pos):
+        oracle, wl, ref_pos, G = self.oracle, self.wl, self.ref_pos, self.G
+        Xk, Xv = self.Xs[u]
+        refK = oracle.build_refs(Xk, ref_pos)
+        refV = oracle.build_refs(Xv, ref_pos)
+        idx, _, _ = oracle.select(Xk[pos], pos, refK, ref_pos, wl.k)
+        ek = oracle.encode(Xk[pos], refK, idx, wl.bits)
+        ev = oracle.encode(Xv[pos], refV, idx, wl.bits)
+        Kh = oracle.reconstruct(refK, idx, ek["codes"], ek["scales"], wl.bits)
+        Vh = oracle.reconstruct(refV, idx, ev["codes"], ev["scales"], wl.bits)
+        h = u[1]
+        oracle.attention(self.qf[0, h * G:(h + 1) * G], Kh, Vh)
+
+    def timed(self, S, seed):
+        rng = np.random.default_rng(seed)
+        pos = np.sort(rng.choice(self.cpos, S, replace=False)).astype(np.int32)
+        t0 = time.perf_counter()
+        with ThreadPoolExecutor(self.threads) as ex:
+            list(ex.map(lambda u: self._work(u, pos), self.units))
+        return time.perf_counter() - t0
+
+    def calibrate(self, target_s: float):
+        t = self.timed(self.S, 1)
+        self.S = int(min(len(self.cpos), max(64, self.S * target_s / max(t, 1e-3))))
+        return self
+
+    def run(self, seed=2):
+        """(positions per second, sample description, seconds)."""
+        t = self.timed(self.S, seed)
+        desc = (f"{self.S} uniformly drawn compressed positions x {len(self.units)} kv heads of one layer: "
+                f"oracle reference store, top-{self.wl.k} search, encode, reconstruct and {self.G}-head "
+                f"attention over the sampled rows; {self.threads} threads across kv heads")
+        return self.S / t, desc, t
+
+
+def run_reference(args, rank, world):
+    import synth
+
+    if rank != 0:
+        return
+    wl = synth.WORKLOADS[args.workload]
+    lengths = wl.lengths()
+    threads = min(os.cpu_count() or 1, wl.n_kv_heads)
+    per_step = max(0.5, min(4.0, 150.0 / max(1, args.steps + args.warmup)))
+    sampler = OracleSample(wl, lengths, 0, threads).calibrate(per_step)
+    rates = []
+    for i in range(args.warmup + args.steps):
+        rate, desc, t = sampler.run(seed=10 + i)
+        if i >= args.warmup:
+            rates.append(rate)
+    v = statistics.mean(rates) / 1e6
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "Mtok/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * wl.seq_len / (v * 1e6),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": _config(wl, lengths),
+            "cpu_baseline": {"value": v, "unit": "Mtok/s", "cores": threads, "kind": "oracle", "sample": desc},
+            "e2e": {"value": v, "unit": "Mtok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def _config(wl, lengths):
+    return {"workload": wl.name, "layers": 1, "batch": wl.batch, "seq_len": wl.seq_len,
+            "n_kv_heads": wl.n_kv_heads, "n_q_heads": wl.n_q_heads, "head_dim": wl.head_dim,
+            "stride": wl.stride0, "k": wl.k, "bits": wl.bits, "group": wl.group, "global_batch": wl.batch,
+            "l2": "flushed before every timed step (256 MiB write, outside the timed spans)",
+            "parallelism": "replicas (one independent layer per GPU)"}
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+
+    import long_context_attention_rkv_b200 as rkv
+    import synth
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = synth.WORKLOADS[args.workload]
+    lengths = wl.lengths()
+    layer_id = rank                                   # every replica compresses its own independent layer
+    Kh, Vh = synth.gen_layer(wl, layer_id, lengths)
+    q_h = synth.gen_query(wl, layer_id, 0)
+    tdt = torch.int16 if wl.dtype == "bf16" else torch.float32
+
+    def pinned(a):
+        t = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).pin_memory()
+        return t
+
+    Kp, Vp, qp = pinned(Kh), pinned(Vh), pinned(q_h)
+    K = Kp.to(dev)
+    V = Vp.to(dev)
+    q = qp.to(dev)
+    cfg = rkv.make_config(head_dim=wl.head_dim, n_kv_heads=wl.n_kv_heads, n_q_heads=wl.n_q_heads, k=wl.k,
+                          bits=wl.bits, stride0=wl.stride0, batch=wl.batch, max_len=K.shape[2],
+                          refs_per_phase=wl.refs_per_phase, in_dtype=wl.dtype_code, out_dtype=wl.dtype_code)
+    L = rkv.Layer(cfg, lengths, device=dev)
+    out = torch.empty((wl.batch, wl.n_q_heads, wl.head_dim), dtype=tdt, device=dev)
+    out_h = torch.empty_like(out, device="cpu").pin_memory()
+    rpos = torch.arange(0, lengths[0], max(1, lengths[0] // RECON_ROWS), dtype=torch.int32,
+                        device=dev)[:RECON_ROWS].contiguous()
+    Kr = torch.empty((RECON_ROWS, wl.head_dim), dtype=torch.float32, device=dev)
+    Vr = torch.empty_like(Kr)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    stages = {
+        "build_refs": lambda: L.build_refs(K, V),
+        "search": lambda: L.search(K),
+        "encode": lambda: L.encode(K, V),
+        "decode": lambda: L.decode(q, out),
+        "reconstruct": lambda: L.reconstruct(0, 0, rpos, RECON_ROWS, Kr, Vr, rkv.RKV_DTYPE_F32),
+    }
+    names = list(stages)
+    # one CUDA graph per stage (launch gaps removed; each stage timed by events around its replay)
+    graphs = {}
+    with torch.cuda.stream(stream):
+        for nm in names:                               # eager run first (also a warm-up)
+            stages[nm]()
+        torch.cuda.synchronize(dev)
+        for nm in names:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                stages[nm]()
+            graphs[nm] = g
+    torch.cuda.synchronize(dev)
+    assert L.device_error() == 0
+
+    def step(evs=None):
+        if evs is not None:
+            evs[0].record(stream)
+        for i, nm in enumerate(names):
+            graphs[nm].replay()
+            if evs is not None:
+                evs[i + 1].record(stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            flush.zero_()
+            step()
+    torch.cuda.synchronize(dev)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            flush.zero_()
+            step(evs[i])
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    stage_ms = {nm: [] for nm in names}
+    step_ms = []
+    for e in evs:
+        for i, nm in enumerate(names):
+            stage_ms[nm].append(e[i].elapsed_time(e[i + 1]))
+        step_ms.append(e[0].elapsed_time(e[-1]))
+    mean_step = statistics.mean(step_ms)
+    if world > 1:
+        t = torch.tensor([mean_step], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        mean_step = float(t.item())
+    assert L.device_error() == 0
+
+    # end to end through the public API: host inputs copied in, output copied out, every step
+    e2e_ms = []
+    h2d = Kp.numel() * Kp.element_size() + Vp.numel() * Vp.element_size() + qp.numel() * qp.element_size()
+    d2h = out.numel() * out.element_size()
+    with torch.cuda.stream(stream):
+        for i in range(max(3, min(args.steps, 50)) + 2):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            K.copy_(Kp, non_blocking=True)
+            V.copy_(Vp, non_blocking=True)
+            q.copy_(qp, non_blocking=True)
+            for nm in names:
+                stages[nm]()
+            out_h.copy_(out, non_blocking=True)
+            e1.record(stream)
+            e1.synchronize()
+            if i >= 2:
+                e2e_ms.append(e0.elapsed_time(e1))
+    e2e_step = statistics.mean(e2e_ms)
+    if world > 1:
+        t = torch.tensor([e2e_step], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_step = float(t.item())
+
+    Q = workload_quantities(wl, lengths)
+    tokens = Q["tokens"]
+    value = world * tokens / (mean_step * 1e-3) / 1e6
+    avg = {nm: statistics.mean(v) for nm, v in stage_ms.items()}
+    peaks = _load_peaks()
+    decode_gbs = Q["decode_bytes"] / (avg["decode"] * 1e-3) / 1e9
+    encode_gbs = Q["encode_bytes"] / (avg["encode"] * 1e-3) / 1e9
+    search_tflops = Q["search_flops"] / (avg["search"] * 1e-3) / 1e12
+    search_src = ["long_context_attention_rkv_b200/csrc/kernels_select_simt.cu"]
+    search_tensor = False
+    dominant = max(("search", "encode", "decode"), key=lambda s: avg[s])
+    if dominant == "search":
+        if search_tensor:
+            peak, bound, ach, unit = peaks["bf16"], "tensor", search_tflops, "TFLOP/s"
+        else:
+            peak, bound, ach, unit = ALU_FP32_TFLOPS, "alu", search_tflops, "TFLOP/s"
+        traffic = _traffic("select_simt", search_src)
+    elif dominant == "encode":
+        peak, bound, ach, unit = peaks["hbm"], "hbm", encode_gbs, "GB/s"
+        traffic = _traffic("encode", ["long_context_attention_rkv_b200/csrc/kernels_encode.cu"])
+    else:
+        peak, bound, ach, unit = peaks["hbm"], "hbm", decode_gbs, "GB/s"
+        traffic = _traffic("decode", ["long_context_attention_rkv_b200/csrc/kernels_decode_direct.cu"])
+    roofline = {"kernel": dominant, "bound": bound, "achieved": ach, "peak": peak, "unit": unit,
+                "frac": ach / peak, "traffic": traffic, "peak_source": peaks["source"]}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        threads = min(os.cpu_count() or 1, wl.n_kv_heads)
+        rate, desc, t = OracleSample(wl, lengths, 0, threads).calibrate(args.cpu_seconds).run()
+        cpu = {"value": rate / 1e6, "unit": "Mtok/s", "cores": threads, "kind": "oracle", "sample": desc,
+               "seconds": t}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "Mtok/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": mean_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded prototype-cluster caches)",
+            "config": _config(wl, lengths),
+            "parts": {
+                "build_refs_us": 1e3 * avg["build_refs"], "search_us": 1e3 * avg["search"],
+                "encode_us": 1e3 * avg["encode"], "decode_us_per_step": 1e3 * avg["decode"],
+                "reconstruct_us": 1e3 * avg["reconstruct"],
+                "decode_hbm_gbs": decode_gbs, "decode_roofline_frac": decode_gbs / peaks["hbm"],
+                "decode_bytes_per_step": Q["decode_bytes"],
+                "search_tflops": search_tflops, "search_flops": Q["search_flops"],
+                "encode_gbs": encode_gbs, "compress_mtok_s": tokens / ((avg["search"] + avg["encode"] +
+                                                                        avg["build_refs"]) * 1e-3) / 1e6,
+            },
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": {"value": world * tokens / (e2e_step * 1e-3) / 1e6, "unit": "Mtok/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": sum(LAUNCHES.values()) * args.steps,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    for g in graphs.values():
+        g.reset()
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch
+
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -219,6 +219,20 @@ RKV_API rkv_status rkv_compress(const rkv_cache_desc* desc, const void* K, const
                         uint64_t workspace_bytes, void* stream);
 
 /*
+ * The two stages of rkv_compress, for callers that schedule or time them
+ * separately; rkv_compress is rkv_search followed by rkv_encode on the same
+ * workspace.  rkv_search (paper summary page, "Practical Deployment via
+ * Sparse-vLLM": the batched L2 distance kernel of the reference search) writes
+ * per compressed token its leading candidate references into the workspace;
+ * rkv_encode reads them, fixes the final top-k by exact distance and writes
+ * idx, codes and scales.  The workspace must not change in between.
+ */
+RKV_API rkv_status rkv_search(const rkv_cache_desc* desc, const void* K, void* workspace, uint64_t workspace_bytes,
+                              void* stream);
+RKV_API rkv_status rkv_encode(const rkv_cache_desc* desc, const void* K, const void* V, void* workspace,
+                              uint64_t workspace_bytes, void* stream);
+
+/*
  * One decode step of attention over the compressed cache (paper summary
  * page, "Training and Inference Integration" and "Practical Deployment via
  * Sparse-vLLM": reconstruction fused into attention; news page, "How

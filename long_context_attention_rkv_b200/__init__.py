@@ -28,7 +28,7 @@ STATUS = {0: "RKV_OK", 1: "RKV_ERR_INVALID_ARG", 2: "RKV_ERR_UNSUPPORTED", 3: "R
 STATUS_CODE = {v: k for k, v in STATUS.items()}
 
 EXPORTED = ["rkv_abi_version", "rkv_status_string", "rkv_schedule", "rkv_cache_size", "rkv_cache_bind",
-            "rkv_unit_view_get", "rkv_build_refs", "rkv_compress", "rkv_decode_attn", "rkv_reconstruct",
+            "rkv_unit_view_get", "rkv_build_refs", "rkv_search", "rkv_encode", "rkv_compress", "rkv_decode_attn", "rkv_reconstruct",
             "rkv_read_device_error"]
 
 
@@ -72,6 +72,8 @@ def lib() -> ctypes.CDLL:
         L.rkv_cache_bind.argtypes = [cfgp, vp, vp, u64, vp]
         L.rkv_unit_view_get.argtypes = [vp, i32, i32, ctypes.POINTER(rkv_unit_view)]
         L.rkv_build_refs.argtypes = [vp, vp, vp, vp]
+        L.rkv_search.argtypes = [vp, vp, vp, u64, vp]
+        L.rkv_encode.argtypes = [vp, vp, vp, vp, u64, vp]
         L.rkv_compress.argtypes = [vp, vp, vp, vp, u64, vp]
         L.rkv_decode_attn.argtypes = [vp, vp, vp, vp, u64, vp]
         L.rkv_reconstruct.argtypes = [vp, i32, i32, vp, i64, vp, vp, i32, vp]
@@ -169,6 +171,15 @@ def rkv_build_refs(desc: CacheDesc, K, V, stream=None):
     _check(lib().rkv_build_refs(desc.ptr, _ptr(K), _ptr(V), _stream(stream)), "rkv_build_refs")
 
 
+def rkv_search(desc: CacheDesc, K, workspace, workspace_bytes: int, stream=None):
+    _check(lib().rkv_search(desc.ptr, _ptr(K), _ptr(workspace), workspace_bytes, _stream(stream)), "rkv_search")
+
+
+def rkv_encode(desc: CacheDesc, K, V, workspace, workspace_bytes: int, stream=None):
+    _check(lib().rkv_encode(desc.ptr, _ptr(K), _ptr(V), _ptr(workspace), workspace_bytes, _stream(stream)),
+           "rkv_encode")
+
+
 def rkv_compress(desc: CacheDesc, K, V, workspace, workspace_bytes: int, stream=None):
     _check(lib().rkv_compress(desc.ptr, _ptr(K), _ptr(V), _ptr(workspace), workspace_bytes, _stream(stream)),
            "rkv_compress")
@@ -211,6 +222,12 @@ class Layer:
 
     def build_refs(self, K, V, stream=None):
         rkv_build_refs(self.desc, K, V, stream)
+
+    def search(self, K, stream=None):
+        rkv_search(self.desc, K, self.workspace, self.workspace.numel(), stream)
+
+    def encode(self, K, V, stream=None):
+        rkv_encode(self.desc, K, V, self.workspace, self.workspace.numel(), stream)
 
     def compress(self, K, V, stream=None):
         rkv_compress(self.desc, K, V, self.workspace, self.workspace.numel(), stream)

@@ -381,25 +381,58 @@ rkv_status rkv_build_refs(const rkv_cache_desc* desc, const void* K, const void*
     return cuda_status(launch_refs_copy(a, d->max_R, K, V, static_cast<cudaStream_t>(stream)));
 }
 
-rkv_status rkv_compress(const rkv_cache_desc* desc, const void* K, const void* V, void* workspace,
-                        uint64_t workspace_bytes, void* stream)
+static rkv_status check_stage_args(const Desc* d, const void* K, const void* V, const void* workspace,
+                                   uint64_t workspace_bytes)
 {
-    const Desc* d = get_desc(desc);
-    if (!d || !K || !V || !aligned(K, 16) || !aligned(V, 16) || (!workspace && d->ws_select > 0) ||
+    if (!d || !K || !aligned(K, 16) || (V && !aligned(V, 16)) || (!workspace && d->ws_select > 0) ||
         !aligned(workspace, 256))
         return RKV_ERR_INVALID_ARG;
     if (workspace_bytes < d->ws_select)
         return RKV_ERR_WORKSPACE;
+    return RKV_OK;
+}
+
+static uint16_t* cand_idx_of(const Desc* d, void* ws) { return static_cast<uint16_t*>(ws); }
+
+static float* cand_t_of(const Desc* d, void* ws)
+{
+    return reinterpret_cast<float*>(static_cast<char*>(ws) + align_up(2ull * d->total_cmp_rows * d->kc, 256));
+}
+
+rkv_status rkv_search(const rkv_cache_desc* desc, const void* K, void* workspace, uint64_t workspace_bytes,
+                      void* stream)
+{
+    const Desc* d = get_desc(desc);
+    const rkv_status s = check_stage_args(d, K, nullptr, workspace, workspace_bytes);
+    if (s != RKV_OK)
+        return s;
     const CacheArgs a = make_args(*d);
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    uint16_t* cand_idx = static_cast<uint16_t*>(workspace);
-    float* cand_t = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                             align_up(2ull * d->total_cmp_rows * d->kc, 256));
     const Tile* tiles = reinterpret_cast<const Tile*>(static_cast<char*>(d->base) + d->sec.tiles);
-    cudaError_t e = launch_select_simt(a, tiles, d->n_tiles, K, cand_idx, cand_t, st);
-    if (e == cudaSuccess)
-        e = launch_encode(a, d->max_C, K, V, cand_idx, cand_t, st);
-    return cuda_status(e);
+    return cuda_status(launch_select_simt(a, tiles, d->n_tiles, K, cand_idx_of(d, workspace),
+                                          cand_t_of(d, workspace), static_cast<cudaStream_t>(stream)));
+}
+
+rkv_status rkv_encode(const rkv_cache_desc* desc, const void* K, const void* V, void* workspace,
+                      uint64_t workspace_bytes, void* stream)
+{
+    const Desc* d = get_desc(desc);
+    if (!V)
+        return RKV_ERR_INVALID_ARG;
+    const rkv_status s = check_stage_args(d, K, V, workspace, workspace_bytes);
+    if (s != RKV_OK)
+        return s;
+    const CacheArgs a = make_args(*d);
+    return cuda_status(launch_encode(a, d->max_C, K, V, cand_idx_of(d, workspace), cand_t_of(d, workspace),
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+rkv_status rkv_compress(const rkv_cache_desc* desc, const void* K, const void* V, void* workspace,
+                        uint64_t workspace_bytes, void* stream)
+{
+    if (!V)
+        return RKV_ERR_INVALID_ARG;
+    const rkv_status s = rkv_search(desc, K, workspace, workspace_bytes, stream);
+    return s != RKV_OK ? s : rkv_encode(desc, K, V, workspace, workspace_bytes, stream);
 }
 
 rkv_status rkv_decode_attn(const rkv_cache_desc* desc, const void* q, void* out, void* workspace,
