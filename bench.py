@@ -382,15 +382,16 @@ def run_ours(args, rank, world, local_rank):
     decode_gbs = Q["decode_bytes"] / (avg["decode"] * 1e-3) / 1e9
     encode_gbs = Q["encode_bytes"] / (avg["encode"] * 1e-3) / 1e9
     search_tflops = Q["search_flops"] / (avg["search"] * 1e-3) / 1e12
-    search_src = ["long_context_attention_rkv_b200/csrc/kernels_select_simt.cu"]
-    search_tensor = False
+    search_tensor = wl.dtype == "bf16"
+    search_kernel = "select_tc" if search_tensor else "select_simt"
+    search_src = ["long_context_attention_rkv_b200/csrc/kernels_%s.cu" % search_kernel]
     dominant = max(("search", "encode", "decode"), key=lambda s: avg[s])
     if dominant == "search":
         if search_tensor:
             peak, bound, ach, unit = peaks["bf16"], "tensor", search_tflops, "TFLOP/s"
         else:
             peak, bound, ach, unit = ALU_FP32_TFLOPS, "alu", search_tflops, "TFLOP/s"
-        traffic = _traffic("select_simt", search_src)
+        traffic = _traffic(search_kernel, search_src)
     elif dominant == "encode":
         peak, bound, ach, unit = peaks["hbm"], "hbm", encode_gbs, "GB/s"
         traffic = _traffic("encode", ["long_context_attention_rkv_b200/csrc/kernels_encode.cu"])

@@ -119,7 +119,7 @@ rkv_status compute_layout(const rkv_config* c, const int32_t* lengths, Desc& d)
     d.n_groups = D / c->group;
     d.n_units = c->batch * Hkv;
     d.max_n = max_n;
-    int64_t ref_rows = 0, cmp_rows = 0, tiles = 0;
+    int64_t ref_rows = 0, cmp_rows = 0, tiles = 0, pairs = 0;
     for (int b = 0; b < c->batch; ++b) {
         const int64_t n = lengths[b];
         const int64_t R = host_ref_count(d.ph, n);
@@ -135,6 +135,7 @@ rkv_status compute_layout(const rkv_config* c, const int32_t* lengths, Desc& d)
         ref_rows += static_cast<int64_t>(Hkv) * d.Rpad[b];
         cmp_rows += static_cast<int64_t>(Hkv) * d.Cpad[b];
         tiles += static_cast<int64_t>(Hkv) * ceil_div(n, kPosTile);
+        pairs += static_cast<int64_t>(Hkv) * ceil_div(n, 2 * kPosTile);
         d.max_R = std::max<int32_t>(d.max_R, d.R[b]);
         d.max_C = std::max<int32_t>(d.max_C, d.C[b]);
     }
@@ -143,6 +144,7 @@ rkv_status compute_layout(const rkv_config* c, const int32_t* lengths, Desc& d)
     d.total_ref_rows = ref_rows;
     d.total_cmp_rows = cmp_rows;
     d.n_tiles = static_cast<int32_t>(tiles);
+    d.n_pairs = static_cast<int32_t>(pairs);
     uint64_t off = 0;
     auto take = [&](uint64_t bytes) {
         const uint64_t o = off;
@@ -153,9 +155,11 @@ rkv_status compute_layout(const rkv_config* c, const int32_t* lengths, Desc& d)
     s.err = take(256);
     s.units = take(sizeof(UnitMeta) * d.n_units);
     s.tiles = take(sizeof(Tile) * std::max<int64_t>(1, tiles));
+    s.pairs = take(sizeof(Tile) * std::max<int64_t>(1, pairs));
     s.ref_K = take(2ull * ref_rows * D);
     s.ref_V = take(2ull * ref_rows * D);
-    s.ref_hn = take(4ull * ref_rows);
+    s.ref_hn = take(4ull * (ref_rows + 256));  // tail slack: tile scans read up to 32 entries past a unit
+    s.ref_aug = take(32ull * ref_rows);
     s.ref_pos = take(4ull * ref_rows);
     s.codes_K = take(static_cast<uint64_t>(cmp_rows) * d.code_bytes);
     s.codes_V = take(static_cast<uint64_t>(cmp_rows) * d.code_bytes);
@@ -203,6 +207,7 @@ CacheArgs make_args(const Desc& d)
     a.ref_K = reinterpret_cast<uint16_t*>(base + d.sec.ref_K);
     a.ref_V = reinterpret_cast<uint16_t*>(base + d.sec.ref_V);
     a.ref_hn = reinterpret_cast<float*>(base + d.sec.ref_hn);
+    a.ref_aug = reinterpret_cast<uint16_t*>(base + d.sec.ref_aug);
     a.ref_pos = reinterpret_cast<int32_t*>(base + d.sec.ref_pos);
     a.codes_K = reinterpret_cast<uint8_t*>(base + d.sec.codes_K);
     a.codes_V = reinterpret_cast<uint8_t*>(base + d.sec.codes_V);
@@ -327,17 +332,32 @@ rkv_status rkv_cache_bind(const rkv_config* cfg, const int32_t* lengths, void* d
                 work.push_back({host_refs_upto(d->ph, last), Tile{u, t}});
             }
         }
-    std::stable_sort(work.begin(), work.end(),
-                     [](const std::pair<int64_t, Tile>& x, const std::pair<int64_t, Tile>& y) { return x.first > y.first; });
+    auto heavier = [](const std::pair<int64_t, Tile>& x, const std::pair<int64_t, Tile>& y) { return x.first > y.first; };
+    std::stable_sort(work.begin(), work.end(), heavier);
     std::vector<Tile> tiles(work.size());
     for (size_t i = 0; i < work.size(); ++i)
         tiles[i] = work[i].second;
+    std::vector<std::pair<int64_t, Tile>> pwork;
+    pwork.reserve(d->n_pairs);
+    for (int u = 0; u < d->n_units; ++u) {
+        const int np = static_cast<int>(ceil_div(units[u].n, 2 * kPosTile));
+        for (int t = 0; t < np; ++t) {
+            const int64_t last = std::min<int64_t>(static_cast<int64_t>(t + 1) * 2 * kPosTile, units[u].n) - 1;
+            pwork.push_back({host_refs_upto(d->ph, last), Tile{u, t}});
+        }
+    }
+    std::stable_sort(pwork.begin(), pwork.end(), heavier);
+    std::vector<Tile> pairs(pwork.size());
+    for (size_t i = 0; i < pwork.size(); ++i)
+        pairs[i] = pwork[i].second;
     char* base = static_cast<char*>(dev_buf);
     cudaError_t e = cudaMemset(base + d->sec.err, 0, 256);
     if (e == cudaSuccess)
         e = cudaMemcpy(base + d->sec.units, units.data(), sizeof(UnitMeta) * units.size(), cudaMemcpyHostToDevice);
     if (e == cudaSuccess && !tiles.empty())
         e = cudaMemcpy(base + d->sec.tiles, tiles.data(), sizeof(Tile) * tiles.size(), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && !pairs.empty())
+        e = cudaMemcpy(base + d->sec.pairs, pairs.data(), sizeof(Tile) * pairs.size(), cudaMemcpyHostToDevice);
     if (e != cudaSuccess) {
         std::memset(desc, 0, sizeof(*desc));
         return RKV_ERR_CUDA;
@@ -408,8 +428,15 @@ rkv_status rkv_search(const rkv_cache_desc* desc, const void* K, void* workspace
         return s;
     const CacheArgs a = make_args(*d);
     const Tile* tiles = reinterpret_cast<const Tile*>(static_cast<char*>(d->base) + d->sec.tiles);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (select_tc_supported(a) && !(d->cfg.flags & RKV_FLAG_SELECT_SIMT)) {
+        const int64_t in_rows = static_cast<int64_t>(d->n_units) * d->cfg.max_len;
+        const Tile* pairs = reinterpret_cast<const Tile*>(static_cast<char*>(d->base) + d->sec.pairs);
+        return cuda_status(launch_select_tc(a, pairs, d->n_pairs, K, in_rows, d->total_ref_rows,
+                                            cand_idx_of(d, workspace), cand_t_of(d, workspace), st));
+    }
     return cuda_status(launch_select_simt(a, tiles, d->n_tiles, K, cand_idx_of(d, workspace),
-                                          cand_t_of(d, workspace), static_cast<cudaStream_t>(stream)));
+                                          cand_t_of(d, workspace), st));
 }
 
 rkv_status rkv_encode(const rkv_cache_desc* desc, const void* K, const void* V, void* workspace,

@@ -1,7 +1,8 @@
 // Reference store: copies the key/value rows at the reference positions of every
 // unit into the cache as bf16 and records 0.5*|r|^2 of each key reference
 // (ResidualKV paper summary page, "DeltaKV Framework Architecture": the
-// reference set T is kept uncompressed).
+// reference set T is kept uncompressed), plus -|r|^2/2 as three bf16 terms for
+// the augmented column of the tensor-core search.
 //
 // One warp per reference row; each lane moves D/32 consecutive channels, so a
 // warp reads and writes one contiguous row (256 B for bf16, D = 128).
@@ -45,8 +46,18 @@ __global__ void __launch_bounds__(256) refs_copy_kernel(CacheArgs a, const void*
     }
     ss = warp_sum(ss);
     if (lane == 0) {
-        a.ref_hn[um.ref_row + j] = 0.5f * ss;
+        const float hn = 0.5f * ss;
+        a.ref_hn[um.ref_row + j] = hn;
         a.ref_pos[um.ref_row + j] = p;
+        // -hn split into three bf16 terms (hi + mid + lo = hn to ~2^-24 relative): a 16-wide
+        // extra K block of the search GEMM adds them to every dot product
+        const uint16_t hi = f32_to_bf16_bits(hn);
+        const float r1 = hn - bf16_bits_to_f32(hi);
+        const uint16_t mid = f32_to_bf16_bits(r1);
+        const uint16_t lo = f32_to_bf16_bits(r1 - bf16_bits_to_f32(mid));
+        uint4* aug = reinterpret_cast<uint4*>(a.ref_aug + (um.ref_row + j) * 16);
+        aug[0] = make_uint4((hi ^ 0x8000u) | ((mid ^ 0x8000u) << 16), lo ^ 0x8000u, 0u, 0u);
+        aug[1] = make_uint4(0u, 0u, 0u, 0u);
     }
 }
 

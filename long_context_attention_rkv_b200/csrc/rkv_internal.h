@@ -40,7 +40,8 @@ struct UnitMeta {
 
 // Byte offsets of the cache sections inside the caller's buffer.
 struct Sections {
-    uint64_t err, units, tiles, ref_K, ref_V, ref_hn, ref_pos, codes_K, codes_V, scale_K, scale_V, idx, end;
+    uint64_t err, units, tiles, pairs, ref_K, ref_V, ref_hn, ref_aug, ref_pos, codes_K, codes_V, scale_K, scale_V, idx,
+        end;
 };
 
 // Host-side descriptor stored in rkv_cache_desc::opaque.
@@ -51,6 +52,8 @@ struct Desc {
     uint64_t bytes;
     int32_t n_units;
     int32_t n_tiles;
+    int32_t n_pairs;
+    int32_t pad0;
     int32_t kc;
     int32_t code_bytes;
     int32_t n_groups;
@@ -83,6 +86,7 @@ struct CacheArgs {
     uint16_t* ref_K;
     uint16_t* ref_V;
     float* ref_hn;
+    uint16_t* ref_aug;   // [rows][16] bf16: -hi, -mid, -lo of 0.5|r|^2, then zeros (augmented GEMM column)
     int32_t* ref_pos;
     uint8_t* codes_K;
     uint8_t* codes_V;
@@ -91,7 +95,8 @@ struct CacheArgs {
     uint16_t* idx;
 };
 
-// Selection work item: one tile of kPosTile positions of one unit.
+// Selection work item: one tile of kPosTile positions of one unit (CUDA-core search), or a pair
+// of consecutive tiles (tensor-core search; `tile` is then the pair index).
 struct Tile {
     int32_t unit;
     int32_t tile;
