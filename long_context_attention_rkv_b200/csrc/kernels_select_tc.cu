@@ -58,7 +58,7 @@ constexpr int kAcc = 2;           // accumulator sets (each kTiles x kN columns)
 constexpr int kEpiWarps = 4 * kTiles;
 constexpr int kEpiThreads = 32 * kEpiWarps;
 constexpr int kThreads = 64 + kEpiThreads;
-constexpr int kQC = 16;           // queue entries per epilogue thread
+constexpr int kQC = 24;           // queue entries per epilogue thread
 constexpr uint32_t kTmemCols = kAcc * kTiles * kN;  // 512
 
 template <int D>
@@ -89,6 +89,9 @@ struct Bars {
 };
 static_assert(sizeof(Bars) <= 256, "barrier block");
 
+// Inserts t into the list kept in descending t.  Exact ties of t are not ordered here: the
+// encoder re-ranks every candidate within its error bound of the k-th by exact distance
+// and ordinal, and rescans all candidates when the kept list could be incomplete.
 template <int KC>
 __device__ __forceinline__ void topk_insert(float (&tv)[KC], int (&ti)[KC], float t, int j)
 {
@@ -96,7 +99,7 @@ __device__ __forceinline__ void topk_insert(float (&tv)[KC], int (&ti)[KC], floa
     int ci = j;
 #pragma unroll
     for (int s = 0; s < KC; ++s) {
-        const bool before = (cv > tv[s]) || (cv == tv[s] && ci < ti[s]);
+        const bool before = cv > tv[s];
         const float ft = tv[s];
         const int it = ti[s];
         tv[s] = before ? cv : ft;
@@ -104,6 +107,31 @@ __device__ __forceinline__ void topk_insert(float (&tv)[KC], int (&ti)[KC], floa
         cv = before ? ft : cv;
         ci = before ? it : ci;
     }
+}
+
+// Orders entries of equal t by ascending ordinal (odd-even transposition passes).
+template <int KC>
+__device__ __forceinline__ void order_ties(float (&tv)[KC], int (&ti)[KC])
+{
+#pragma unroll
+    for (int pass = 0; pass < KC; ++pass) {
+#pragma unroll
+        for (int s = pass & 1; s + 1 < KC; s += 2) {
+            const bool sw = tv[s] == tv[s + 1] && ti[s] > ti[s + 1];
+            const int x = ti[s];
+            ti[s] = sw ? ti[s + 1] : x;
+            ti[s + 1] = sw ? x : ti[s + 1];
+        }
+    }
+}
+
+// Item taken by this CTA in round r: rounds alternate direction over the
+// heaviest-first list, so every CTA gets a balanced share of the work.
+__device__ __forceinline__ int item_of(int r)
+{
+    const int g = static_cast<int>(gridDim.x);
+    const int b = static_cast<int>(blockIdx.x);
+    return r * g + ((r & 1) ? (g - 1 - b) : b);
 }
 
 // Candidates of the last position of an item (its causal limit).
@@ -192,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int last_a = -1;
             int last_b[kStagesB] = {-1, -1, -1};
             bool ok = true;
-            for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
+            for (int rnd = 0, w = item_of(0); w < n_items && ok; w = item_of(++rnd)) {
                 const Tile it = items[w];
                 const UnitMeta um = a.units[it.unit];
                 const int p0 = it.tile * kTiles * kM;
@@ -209,8 +237,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     &bars->full_a);
                 last_a = static_cast<int>(ni);
                 ++ni;
-                if (w + static_cast<int>(gridDim.x) < n_items) {
-                    const Tile nx = items[w + gridDim.x];
+                if (item_of(rnd + 1) < n_items) {
+                    const Tile nx = items[item_of(rnd + 1)];
                     const int nrow = nx.unit * a.max_len + nx.tile * kTiles * kM;
 #pragma unroll
                     for (int t = 0; t < kTiles; ++t)
@@ -253,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t it_b = 0, it_c = 0, ni = 0;
             bool ok = true;
             bool issued = false;
-            for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
+            for (int rnd = 0, w = item_of(0); w < n_items && ok; w = item_of(++rnd)) {
                 const Tile it = items[w];
                 const UnitMeta um = a.units[it.unit];
                 const int nrt = (item_candidates(a, um, it.tile * kTiles * kM) + kN - 1) / kN;
@@ -317,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
         uint32_t it_c = 0;
         bool ok = true;
-        for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
+        for (int rnd = 0, w = item_of(0); w < n_items && ok; w = item_of(++rnd)) {
             const Tile it = items[w];
             const UnitMeta um = a.units[it.unit];
             const int p0 = it.tile * kTiles * kM;
@@ -334,6 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ti[s] = 0x7fffffff;
             }
             int cnt = 0;
+            float seed = -FLT_MAX;   // lower bound of the kc-th best t (from sub-block maxima)
             for (int r = 0; r < nrt; ++r) {
                 const int acc = it_c % kAcc;
                 // one lane waits, the warp follows: the TMEM loads below are warp-collective
@@ -346,6 +375,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const int j0 = r * kN;
                 const uint32_t col0 = lane_base + (acc * kTiles + t) * kN;
+                if (r == 0 && nc_max >= kN && KC <= kN / 16) {
+                    // the kc largest of kN/16 sub-block maxima are distinct elements, so the
+                    // smallest of them bounds the kc-th best t from below
+                    float mxs[kN / 16];
+#pragma unroll
+                    for (int c0 = 0; c0 < kN; c0 += 32) {
+                        float v[32];
+                        tmem_ld32(col0 + c0, v);
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            float m = -FLT_MAX;
+#pragma unroll
+                            for (int i = 0; i < 16; ++i)
+                                m = fmaxf(m, (c0 + h * 16 + i < ncand) ? v[h * 16 + i] : -FLT_MAX);
+                            mxs[c0 / 16 + h] = m;
+                        }
+                    }
+                    // kc-th largest of the maxima (kc <= 8 = kN/16: the minimum when kc == 8)
+                    float lo = FLT_MAX;
+#pragma unroll
+                    for (int i = 0; i < kN / 16; ++i)
+                        lo = fminf(lo, mxs[i]);
+                    seed = (KC == kN / 16) ? lo : -FLT_MAX;
+                }
                 for (int c0 = 0; c0 < kN && j0 + c0 < nc_max; c0 += 32) {
                     float v[32];
                     tmem_ld32(col0 + c0, v);
@@ -357,27 +410,32 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         if (__any_sync(0xffffffffu, cnt > kQC - 16)) {
-                            __syncwarp();
                             drain<KC>(myq, cnt, tv, ti);
                             cnt = 0;
                         }
-                        const float thr = tv[KC - 1];
+                        // appends at >= seed keep the element that defines the seed
+                        const float thr = fmaxf(tv[KC - 1], seed);
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
                             const int k = h * 16 + i;
                             myq[cnt * kEpiThreads] = make_float2(v[k], __int_as_float(j0 + c0 + k));
-                            cnt += (v[k] > thr) ? 1 : 0;
+                            cnt += (v[k] > thr || (v[k] == seed && v[k] > tv[KC - 1])) ? 1 : 0;
                         }
                     }
                 }
                 tc_fence_before();
                 mbar_arrive(&bars->acc_empty[acc]);
                 ++it_c;
+                // drain at reference-tile boundaries so the threshold keeps up
+                if (__any_sync(0xffffffffu, cnt > 0)) {
+                    drain<KC>(myq, cnt, tv, ti);
+                    cnt = 0;
+                }
             }
             if (!ok)
                 break;
-            __syncwarp();
             drain<KC>(myq, cnt, tv, ti);
+            order_ties<KC>(tv, ti);
             if (valid) {
                 const int64_t orow = um.cmp_row + (p - ncand);
                 const int nv = min(KC, ncand);
