@@ -200,6 +200,7 @@ CacheArgs make_args(const Desc& d)
     a.n_groups = d.n_groups;
     a.kc = d.kc;
     a.max_len = c.max_len;
+    a.max_refs = d.max_R;
     a.ph = d.ph;
     char* base = static_cast<char*>(d.base);
     a.err = reinterpret_cast<int32_t*>(base + d.sec.err);
@@ -472,6 +473,15 @@ rkv_status rkv_decode_attn(const rkv_cache_desc* desc, const void* q, void* out,
         return RKV_ERR_WORKSPACE;
     const CacheArgs a = make_args(*d);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (decode_fact_supported(a) && !(d->cfg.flags & RKV_FLAG_DECODE_DIRECT)) {
+        int dev = 0, sms = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e == cudaSuccess)
+            e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e == cudaSuccess)
+            e = launch_decode_fact(a, decode_fact_cluster(a, sms), q, out, st);
+        return cuda_status(e);
+    }
     const int splits = decode_splits(d->n_units, d->max_n);
     float* part = static_cast<float*>(workspace);
     cudaError_t e = launch_decode_direct(a, splits, q, part, st);

@@ -3,19 +3,22 @@
 // KV - KV_R; news page "New KV Cache Compression Method Cuts Long-Context
 // Inference Costs by 85%", "How ResidualKV Works": quantized residual codes).
 //
-// One warp per compressed token; each lane owns D/32 consecutive channels.
+// Eight lanes per compressed token (four tokens per warp); a lane owns D/8
+// consecutive channels (16 for D = 128), i.e. half of a 32-channel group.
 //  1. Final top-k.  The search handed over its kc best candidates by
-//     t = k.r - |r|^2/2 computed with fp32 accumulation.  Every candidate
-//     whose t is within 2*delta of the k-th (delta = 2^-13 (|k|^2 + max|r|^2),
-//     far above the accumulation error of a 128-term dot product) is re-ranked
-//     by its exact-order fp32 distance sum_c (k_c - r_c)^2, ties to the lower
-//     ordinal.  If even the last kept candidate is that close, the list may be
-//     incomplete and the warp rescans every candidate exactly.
-//  2. Mean of the chosen rows in ascending ordinal order (fp32, left to right)
-//     and one IEEE division by k_eff; residual = x - mean (fp32).
+//     t = k.r - |r|^2/2 from fp32 accumulation.  With
+//     delta = 2^-16 (|k|^2 + max|r|^2) (four times the worst-case error of a
+//     128-term fp32 dot product, 2^-18 (|k|^2 + |r|^2), and about 25 times the
+//     largest tensor-core vs. CUDA-core difference measured on these inputs): if the (k+1)-th t is more than 2*delta below the k-th, the
+//     first k candidates are the top-k.  Otherwise every candidate within 2*delta
+//     of the k-th is re-ranked by its exact-order fp32 distance sum_c (k_c - r_c)^2
+//     (ties to the lower ordinal); if even the last kept candidate is that close,
+//     the list may be incomplete and all candidates are rescanned exactly.
+//  2. Mean of the chosen rows in ascending ordinal order (fp32, left to right),
+//     one IEEE division by k_eff; residual = x - mean (fp32).
 //  3. Per 32-channel group: a = max|residual|, scale = binary16 rounded up from
-//     a / qmax, code = round-half-even(residual / scale).  All of step 2-3 use
-//     correctly rounded fp32 operations with no contraction, so codes match an
+//     a / qmax, code = round-half-even(residual / scale).  Steps 2-3 use
+//     correctly rounded fp32 operations without contraction, so the codes equal an
 //     IEEE fp32 evaluation of the same steps bit for bit.
 #include <cfloat>
 
@@ -27,102 +30,89 @@ namespace rkv {
 namespace {
 
 constexpr int kWarps = 8;
+constexpr int kLPT = 8;                  // lanes per token
+constexpr int kTPW = 32 / kLPT;          // tokens per warp
 
-template <int NPL>
-__device__ __forceinline__ float partial_dist(const float (&x)[NPL], const uint16_t* r)
+__device__ __forceinline__ unsigned group_mask(int lane) { return 0xffu << (lane & ~(kLPT - 1)); }
+
+// Sum over the 8 lanes of a token group.
+__device__ __forceinline__ float tsum(float v)
 {
-    float rv[NPL];
-    load_bf16<NPL>(r, rv);
+    v += __shfl_xor_sync(0xffffffffu, v, 1);
+    v += __shfl_xor_sync(0xffffffffu, v, 2);
+    v += __shfl_xor_sync(0xffffffffu, v, 4);
+    return v;
+}
+
+__device__ __forceinline__ float tmax(float v)
+{
+    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+    return v;
+}
+
+// CPL consecutive bf16 values (CPL = 8 or 16) as floats.
+template <int CPL>
+__device__ __forceinline__ void load_bf16_row(const uint16_t* p, float (&out)[CPL])
+{
+#pragma unroll
+    for (int h = 0; h < CPL / 8; ++h) {
+        const uint4 v = *reinterpret_cast<const uint4*>(p + h * 8);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            out[h * 8 + 2 * i] = bf16_bits_to_f32(w[i] & 0xffffu);
+            out[h * 8 + 2 * i + 1] = bf16_bits_to_f32(w[i] >> 16);
+        }
+    }
+}
+
+template <int CPL>
+__device__ __forceinline__ void load_input_row(const void* base, int64_t elem, int in_dtype, float (&out)[CPL])
+{
+    if (in_dtype == RKV_DTYPE_F32) {
+        const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(base) + elem);
+#pragma unroll
+        for (int h = 0; h < CPL / 4; ++h) {
+            const float4 v = p[h];
+            out[4 * h] = v.x;
+            out[4 * h + 1] = v.y;
+            out[4 * h + 2] = v.z;
+            out[4 * h + 3] = v.w;
+        }
+    } else {
+        load_bf16_row<CPL>(static_cast<const uint16_t*>(base) + elem, out);
+    }
+}
+
+// Exact-order fp32 squared distance between this token's key and a reference row (this
+// lane's part; sum over the token group with tsum).
+template <int CPL>
+__device__ __forceinline__ float part_dist(const float (&x)[CPL], const uint16_t* r)
+{
+    float rv[CPL];
+    load_bf16_row<CPL>(r, rv);
     float s = 0.0f;
 #pragma unroll
-    for (int i = 0; i < NPL; ++i) {
+    for (int i = 0; i < CPL; ++i) {
         const float d = __fsub_rn(x[i], rv[i]);
         s = __fmaf_rn(d, d, s);
     }
     return s;
 }
 
-// Exhaustive exact top-k over candidates [0, ncand) for one warp.  The key row is
-// staged in xs (shared, D floats).  Afterwards lanes 0..keff-1 hold the chosen ordinals.
-template <int NPL>
-__device__ void exhaustive_topk(const CacheArgs& a, const UnitMeta& um, const float* xs, int ncand, int k, int lane,
-                                int& my_ord)
+template <int CPL>
+__device__ __forceinline__ void quantise_store(const float (&x)[CPL], const float (&m)[CPL], int bits, int sub,
+                                               bool store, uint8_t* codes_row, uint16_t* scale_row, int32_t* err)
 {
-    constexpr int D = NPL * 32;
-    float bd[RKV_MAX_K];
-    int bo[RKV_MAX_K];
-#pragma unroll
-    for (int s = 0; s < RKV_MAX_K; ++s) {
-        bd[s] = FLT_MAX;
-        bo[s] = 0x7fffffff;
-    }
-    for (int j = lane; j < ncand; j += 32) {
-        const uint16_t* r = a.ref_K + (um.ref_row + j) * D;
-        float d = 0.0f;
-        for (int c = 0; c < D; c += 2) {
-            float rv[2];
-            load_bf16<2>(r + c, rv);
-            const float e0 = __fsub_rn(xs[c], rv[0]);
-            const float e1 = __fsub_rn(xs[c + 1], rv[1]);
-            d = __fmaf_rn(e0, e0, d);
-            d = __fmaf_rn(e1, e1, d);
-        }
-        // insert by (d ascending, ordinal ascending) into the first k slots
-        float cv = d;
-        int ci = j;
-#pragma unroll
-        for (int s = 0; s < RKV_MAX_K; ++s) {
-            if (s < k) {
-                const bool before = (cv < bd[s]) || (cv == bd[s] && ci < bo[s]);
-                const float fd = bd[s];
-                const int fo = bo[s];
-                bd[s] = before ? cv : fd;
-                bo[s] = before ? ci : fo;
-                cv = before ? fd : cv;
-                ci = before ? fo : ci;
-            }
-        }
-    }
-    // merge the 32 per-lane lists: k rounds of a warp-wide (d, ordinal) minimum
-    int head = 0;
-    my_ord = RKV_IDX_UNUSED;
-    for (int r = 0; r < k && r < ncand; ++r) {
-        float hd = FLT_MAX;
-        int ho = 0x7fffffff;
-#pragma unroll
-        for (int s = 0; s < RKV_MAX_K; ++s)
-            if (s == head) {
-                hd = bd[s];
-                ho = bo[s];
-            }
-        float wd = hd;
-        int wo = ho;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            const float od = __shfl_xor_sync(0xffffffffu, wd, off);
-            const int oo = __shfl_xor_sync(0xffffffffu, wo, off);
-            if (od < wd || (od == wd && oo < wo)) {
-                wd = od;
-                wo = oo;
-            }
-        }
-        if (ho == wo && hd == wd)
-            ++head;
-        if (lane == r)
-            my_ord = wo;
-    }
-}
-
-template <int NPL>
-__device__ __forceinline__ void quantise_store(const float (&x)[NPL], const float (&m)[NPL], int bits, int lane,
-                                               uint8_t* codes_row, uint16_t* scale_row, int32_t* err)
-{
-    constexpr int LPG = 32 / NPL;  // lanes per 32-channel group
+    // lanes per 32-channel group: 2 when CPL = 16, 4 when CPL = 8
+    constexpr int LPG = 32 / CPL;
     const int qmax = (bits == 8) ? 127 : 7;
-    float d[NPL];
+    float d[CPL];
     float amax = 0.0f;
 #pragma unroll
-    for (int i = 0; i < NPL; ++i) {
+    for (int i = 0; i < CPL; ++i) {
         d[i] = __fsub_rn(x[i], m[i]);
         amax = fmaxf(amax, fabsf(d[i]));
     }
@@ -130,181 +120,337 @@ __device__ __forceinline__ void quantise_store(const float (&x)[NPL], const floa
     for (int off = 1; off < LPG; off <<= 1)
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
     uint16_t sbits = 0;
-    float s = 0.0f;
+    float s = 1.0f;
     if (amax > 0.0f) {
         const __half h = __float2half_ru(__fdiv_rn(amax, static_cast<float>(qmax)));
         sbits = __half_as_ushort(h);
         s = __half2float(h);
-        if ((sbits & 0x7c00u) == 0x7c00u)
+        if (store && (sbits & 0x7c00u) == 0x7c00u)
             report(err, RKV_ERR_UNSUPPORTED);
     }
-    int q[NPL];
+    int q[CPL];
 #pragma unroll
-    for (int i = 0; i < NPL; ++i) {
-        int c = 0;
-        if (amax > 0.0f) {
-            c = static_cast<int>(rintf(__fdiv_rn(d[i], s)));
-            c = max(-qmax, min(qmax, c));
-        }
-        q[i] = c;
+    for (int i = 0; i < CPL; ++i) {
+        int c = static_cast<int>(rintf(__fdiv_rn(d[i], s)));
+        q[i] = (amax > 0.0f) ? max(-qmax, min(qmax, c)) : 0;
     }
+    if (!store)
+        return;
     if (bits == 8) {
-        if constexpr (NPL == 4) {
-            const uint32_t w = (q[0] & 0xff) | ((q[1] & 0xff) << 8) | ((q[2] & 0xff) << 16) | (uint32_t(q[3] & 0xff) << 24);
-            reinterpret_cast<uint32_t*>(codes_row)[lane] = w;
-        } else {
-            const uint16_t w = static_cast<uint16_t>((q[0] & 0xff) | ((q[1] & 0xff) << 8));
-            reinterpret_cast<uint16_t*>(codes_row)[lane] = w;
-        }
+        uint32_t w[CPL / 4];
+#pragma unroll
+        for (int i = 0; i < CPL / 4; ++i)
+            w[i] = (q[4 * i] & 0xff) | ((q[4 * i + 1] & 0xff) << 8) | ((q[4 * i + 2] & 0xff) << 16) |
+                   (uint32_t(q[4 * i + 3] & 0xff) << 24);
+        if constexpr (CPL == 16)
+            *reinterpret_cast<uint4*>(codes_row + sub * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+        else
+            *reinterpret_cast<uint2*>(codes_row + sub * 8) = make_uint2(w[0], w[1]);
     } else {
-        if constexpr (NPL == 4) {
-            const uint16_t w = static_cast<uint16_t>((q[0] & 0xf) | ((q[1] & 0xf) << 4) | ((q[2] & 0xf) << 8) | ((q[3] & 0xf) << 12));
-            reinterpret_cast<uint16_t*>(codes_row)[lane] = w;
-        } else {
-            codes_row[lane] = static_cast<uint8_t>((q[0] & 0xf) | ((q[1] & 0xf) << 4));
+        uint32_t w[CPL / 8];
+#pragma unroll
+        for (int i = 0; i < CPL / 8; ++i) {
+            uint32_t x8 = 0;
+#pragma unroll
+            for (int b = 0; b < 8; ++b)
+                x8 |= static_cast<uint32_t>(q[8 * i + b] & 0xf) << (4 * b);
+            w[i] = x8;
         }
+        if constexpr (CPL == 16)
+            *reinterpret_cast<uint2*>(codes_row + sub * 8) = make_uint2(w[0], w[1]);
+        else
+            *reinterpret_cast<uint32_t*>(codes_row + sub * 4) = w[0];
     }
-    if ((lane % LPG) == 0)
-        scale_row[lane / LPG] = sbits;
+    if ((sub % LPG) == 0)
+        scale_row[sub / LPG] = sbits;
 }
 
-template <int NPL, int KC>
-__global__ void __launch_bounds__(kWarps * 32) encode_kernel(CacheArgs a, const void* __restrict__ K,
+template <int CPL, int KC>
+__global__ void __launch_bounds__(kWarps * 32, 2) encode_kernel(CacheArgs a, const void* __restrict__ K,
                                                              const void* __restrict__ V,
                                                              const uint16_t* __restrict__ cand_idx,
                                                              const float* __restrict__ cand_t)
 {
-    constexpr int D = NPL * 32;
-    __shared__ float xs[kWarps][D];
-    __shared__ int sorted[kWarps][RKV_MAX_K];
+    constexpr int D = CPL * kLPT;
+    constexpr int KM = KC - 4;               // largest k served by this candidate width
+    __shared__ float xs[kWarps][kTPW][D];
+    __shared__ int sorted[kWarps][kTPW][KM];
 
     const int u = blockIdx.y;
     const UnitMeta um = a.units[u];
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int c = blockIdx.x * kWarps + warp;
-    if (c >= um.C)
+    const int tg = lane / kLPT;              // token slot within the warp
+    const int sub = lane % kLPT;             // lane within the token group
+    const int c = (blockIdx.x * kWarps + warp) * kTPW + tg;
+    const bool active = c < um.C;
+    if (__all_sync(0xffffffffu, !active))
         return;
     const int k = a.k;
-    const int p = slot_pos(a.ph, c);
+    const int cc = active ? c : 0;           // inactive slots shadow token 0 and store nothing
+    const int p = slot_pos(a.ph, cc);
     const int ncand = min(refs_upto(a.ph, p), um.R);
-    const int64_t row = um.cmp_row + c;
-    const int64_t e = (static_cast<int64_t>(u) * a.max_len + p) * D + lane * NPL;
-    float xk[NPL], xv[NPL];
-    load_row_part<NPL>(K, e, a.in_dtype, xk);
-    load_row_part<NPL>(V, e, a.in_dtype, xv);
+    const int64_t row = um.cmp_row + cc;
+    const int64_t e = (static_cast<int64_t>(u) * a.max_len + p) * D + sub * CPL;
+    float xk[CPL];
+    load_input_row<CPL>(K, e, a.in_dtype, xk);
 
     // ---- 1. final top-k -------------------------------------------------------------
     const int nvalid = min(KC, ncand);
-    int my_ord = RKV_IDX_UNUSED;
-    float my_t = -FLT_MAX;
-    if (lane < nvalid) {
-        my_ord = cand_idx[row * KC + lane];
-        my_t = cand_t[row * KC + lane];
+    // candidate slot i of this token lives on lane sub == i % 8, register i / 8
+    constexpr int PER = (KC + kLPT - 1) / kLPT;
+    int co[PER];
+    float ct[PER];
+    bool bad = false;
+#pragma unroll
+    for (int r = 0; r < PER; ++r) {
+        const int i = r * kLPT + sub;
+        co[r] = RKV_IDX_UNUSED;
+        ct[r] = -FLT_MAX;
+        if (i < nvalid) {
+            co[r] = cand_idx[row * KC + i];
+            ct[r] = cand_t[row * KC + i];
+            bad |= co[r] >= ncand;
+        }
     }
-    const bool bad = (lane < nvalid) && (my_ord >= ncand);
-    if (__any_sync(0xffffffffu, bad)) {
+    if (__any_sync(0xffffffffu, bad && active)) {
         if (lane == 0)
             report(a.err, RKV_ERR_CORRUPT);
         return;
     }
-    bool chosen = false;
+    auto slot_ord = [&](int i) {   // ordinal of candidate slot i (warp-collective)
+        int v = co[0];
+#pragma unroll
+        for (int r = 1; r < PER; ++r)
+            v = (i / kLPT == r) ? co[r] : v;
+        return __shfl_sync(0xffffffffu, v, (lane & ~(kLPT - 1)) + i % kLPT);
+    };
+    auto slot_t = [&](int i) {
+        float v = ct[0];
+#pragma unroll
+        for (int r = 1; r < PER; ++r)
+            v = (i / kLPT == r) ? ct[r] : v;
+        return __shfl_sync(0xffffffffu, v, (lane & ~(kLPT - 1)) + i % kLPT);
+    };
     int keff = min(k, nvalid);
-    if (nvalid <= k) {
-        chosen = lane < nvalid;
+    int chosen[KM];   // chosen ordinals (the same in all 8 lanes of the token)
+    // mode: 0 first k by t, 1 exact re-rank of the near set, 2 exhaustive rescan
+    int mode = 0;
+    // all shuffles below run in every lane (the four tokens of a warp may differ in nvalid)
+    float xx = 0.0f;
+#pragma unroll
+    for (int i = 0; i < CPL; ++i)
+        xx = fmaf(xk[i], xk[i], xx);
+    xx = tsum(xx);
+    float hm = 0.0f;
+#pragma unroll
+    for (int r = 0; r < PER; ++r)
+        if (r * kLPT + sub < nvalid)
+            hm = fmaxf(hm, a.ref_hn[um.ref_row + co[r]]);
+    hm = tmax(hm);
+    const float delta = ldexpf(xx + 2.0f * hm, -16);
+    const float tk = slot_t(k - 1);
+    const float tk1 = slot_t(k);
+    const float tlast = slot_t(KC - 1);
+    if (nvalid > k && tk1 >= tk - 2.0f * delta)
+        mode = ((nvalid == KC) && (ncand > KC) && (tlast >= tk - 2.0f * delta)) ? 2 : 1;
+    const int any_mode = __reduce_max_sync(0xffffffffu, mode);
+    if (any_mode == 0) {
+#pragma unroll
+        for (int i = 0; i < KM; ++i)
+            if (i < k)
+                chosen[i] = slot_ord(i);
     } else {
-        float xx = 0.0f;
+        // warp-collective slow paths, taken by the whole warp; tokens in mode 0 keep the
+        // first k candidates
 #pragma unroll
-        for (int i = 0; i < NPL; ++i)
-            xx = fmaf(xk[i], xk[i], xx);
-        xx = warp_sum(xx);
-        const float hmax = warp_max(lane < nvalid ? a.ref_hn[um.ref_row + my_ord] : 0.0f);
-        const float delta = ldexpf(xx + 2.0f * hmax, -13);
-        const float tk = __shfl_sync(0xffffffffu, my_t, k - 1);
-        const float tlast = __shfl_sync(0xffffffffu, my_t, KC - 1);
-        const bool incomplete = (nvalid == KC) && (ncand > KC) && (tlast >= tk - 2.0f * delta);
-        if (incomplete) {
+        for (int i = 0; i < KM; ++i)
+            if (i < k)
+                chosen[i] = slot_ord(i);
+        if (any_mode >= 1) {
+            // exact distances of the near set: candidates i < k, plus those within 2*delta
+            float dist[KC];
+            int ords[KC];
+            bool in[KC];
 #pragma unroll
-            for (int i = 0; i < NPL; ++i)
-                xs[warp][lane * NPL + i] = xk[i];
+            for (int i = 0; i < KC; ++i) {
+                ords[i] = slot_ord(i);
+                const float ti = slot_t(i);
+                in[i] = (mode == 1) && i < nvalid && (i < k || ti >= tk - 2.0f * delta);
+                const bool need = __any_sync(0xffffffffu, in[i]);
+                float d = 0.0f;
+                if (need) {
+                    const int o = in[i] ? ords[i] : 0;
+                    d = tsum(part_dist<CPL>(xk, a.ref_K + (um.ref_row + o) * D + sub * CPL));
+                }
+                dist[i] = d;
+            }
+            if (mode == 1) {
+                // rank by (distance, ordinal) within the near set
+                int nch = 0;
+#pragma unroll
+                for (int i = 0; i < KC; ++i) {
+                    int rank = 0;
+#pragma unroll
+                    for (int j2 = 0; j2 < KC; ++j2)
+                        rank += (in[j2] && (dist[j2] < dist[i] || (dist[j2] == dist[i] && ords[j2] < ords[i]))) ? 1 : 0;
+                    if (in[i] && rank < k) {
+#pragma unroll
+                        for (int s2 = 0; s2 < KM; ++s2)
+                            if (s2 == rank)
+                                chosen[s2] = ords[i];
+                        ++nch;
+                    }
+                }
+            }
+        }
+        if (any_mode == 2) {
+            // exhaustive exact scan for tokens whose candidate list may be incomplete:
+            // the lanes of such a token split the candidates; each keeps its own best k
+            const bool ex = (mode == 2);
+#pragma unroll
+            for (int i = 0; i < CPL; ++i)
+                xs[warp][tg][sub * CPL + i] = xk[i];
             __syncwarp();
-            exhaustive_topk<NPL>(a, um, xs[warp], ncand, k, lane, my_ord);
-            chosen = lane < keff;
-        } else {
-            const bool inset = (lane < nvalid) && (lane < k || my_t >= tk - 2.0f * delta);
-            const unsigned set = __ballot_sync(0xffffffffu, inset);
-            float my_d = FLT_MAX;
-            for (unsigned m = set; m; m &= m - 1) {
-                const int l = __ffs(m) - 1;
-                const int o = __shfl_sync(0xffffffffu, my_ord, l);
-                const float d = warp_sum(partial_dist<NPL>(xk, a.ref_K + (um.ref_row + o) * D + lane * NPL));
-                if (lane == l)
-                    my_d = d;
+            float bd[KM];
+            int bo[KM];
+#pragma unroll
+            for (int s2 = 0; s2 < KM; ++s2) {
+                bd[s2] = FLT_MAX;
+                bo[s2] = 0x7fffffff;
             }
-            int rank = 0;
-            for (unsigned m = set; m; m &= m - 1) {
-                const int l = __ffs(m) - 1;
-                const float d = __shfl_sync(0xffffffffu, my_d, l);
-                const int o = __shfl_sync(0xffffffffu, my_ord, l);
-                rank += (d < my_d || (d == my_d && o < my_ord)) ? 1 : 0;
+            const int nscan = ex ? ncand : 0;
+            for (int j = sub; j < nscan; j += kLPT) {
+                const uint16_t* r = a.ref_K + (um.ref_row + j) * D;
+                float d = 0.0f;
+                for (int c2 = 0; c2 < D; c2 += 2) {
+                    const uint32_t w = *reinterpret_cast<const uint32_t*>(r + c2);
+                    const float e0 = __fsub_rn(xs[warp][tg][c2], bf16_bits_to_f32(w & 0xffffu));
+                    const float e1 = __fsub_rn(xs[warp][tg][c2 + 1], bf16_bits_to_f32(w >> 16));
+                    d = __fmaf_rn(e0, e0, d);
+                    d = __fmaf_rn(e1, e1, d);
+                }
+                float cv = d;
+                int ci = j;
+#pragma unroll
+                for (int s2 = 0; s2 < KM; ++s2) {
+                    if (s2 < k) {
+                        const bool before = (cv < bd[s2]) || (cv == bd[s2] && ci < bo[s2]);
+                        const float fd = bd[s2];
+                        const int fo = bo[s2];
+                        bd[s2] = before ? cv : fd;
+                        bo[s2] = before ? ci : fo;
+                        cv = before ? fd : cv;
+                        ci = before ? fo : ci;
+                    }
+                }
             }
-            chosen = inset && rank < k;
+            // merge the 8 lane lists of each token: k rounds of a group-wide minimum
+            int head = 0;
+            for (int r = 0; r < k; ++r) {
+                float hd = FLT_MAX;
+                int ho = 0x7fffffff;
+#pragma unroll
+                for (int s2 = 0; s2 < KM; ++s2)
+                    if (s2 == head) {
+                        hd = bd[s2];
+                        ho = bo[s2];
+                    }
+                float wd = hd;
+                int wo = ho;
+#pragma unroll
+                for (int off = 1; off < kLPT; off <<= 1) {
+                    const float od = __shfl_xor_sync(0xffffffffu, wd, off);
+                    const int oo = __shfl_xor_sync(0xffffffffu, wo, off);
+                    if (od < wd || (od == wd && oo < wo)) {
+                        wd = od;
+                        wo = oo;
+                    }
+                }
+                if (ho == wo && hd == wd)
+                    ++head;
+                if (ex) {
+#pragma unroll
+                    for (int s2 = 0; s2 < KM; ++s2)
+                        if (s2 == r)
+                            chosen[s2] = wo;
+                }
+            }
         }
     }
-    // ascending ordinal order of the chosen set
-    const unsigned cm = __ballot_sync(0xffffffffu, chosen);
-    int pos = 0;
-    for (unsigned m = cm; m; m &= m - 1) {
-        const int l = __ffs(m) - 1;
-        const int o = __shfl_sync(0xffffffffu, my_ord, l);
-        pos += (o < my_ord) ? 1 : 0;
+    // ascending ordinal order of the chosen set (identical in the 8 lanes of a token)
+    if (sub == 0) {
+#pragma unroll
+        for (int i = 0; i < KM; ++i)
+            if (i < keff) {
+                int pos = 0;
+#pragma unroll
+                for (int j2 = 0; j2 < KM; ++j2)
+                    pos += (j2 < keff && chosen[j2] < chosen[i]) ? 1 : 0;
+                sorted[warp][tg][pos] = chosen[i];
+            }
     }
-    if (chosen)
-        sorted[warp][pos] = my_ord;
     __syncwarp();
-    if (lane < k)
-        a.idx[row * k + lane] = (lane < keff) ? static_cast<uint16_t>(sorted[warp][lane])
-                                              : static_cast<uint16_t>(RKV_IDX_UNUSED);
+    if (active && sub == 0) {
+        for (int i = 0; i < k; ++i)
+            a.idx[row * k + i] = (i < keff) ? static_cast<uint16_t>(sorted[warp][tg][i])
+                                            : static_cast<uint16_t>(RKV_IDX_UNUSED);
+    }
 
     // ---- 2. mean reference (fp32, ascending ordinals, one division) -------------------
-    float mk[NPL], mv[NPL];
+    float mk[CPL], mv[CPL];
     {
-        const int o = sorted[warp][0];
-        load_bf16<NPL>(a.ref_K + (um.ref_row + o) * D + lane * NPL, mk);
-        load_bf16<NPL>(a.ref_V + (um.ref_row + o) * D + lane * NPL, mv);
+        const int o = sorted[warp][tg][0];
+        load_bf16_row<CPL>(a.ref_K + (um.ref_row + o) * D + sub * CPL, mk);
+        load_bf16_row<CPL>(a.ref_V + (um.ref_row + o) * D + sub * CPL, mv);
     }
     for (int i = 1; i < keff; ++i) {
-        const int o = sorted[warp][i];
-        float rk[NPL], rv[NPL];
-        load_bf16<NPL>(a.ref_K + (um.ref_row + o) * D + lane * NPL, rk);
-        load_bf16<NPL>(a.ref_V + (um.ref_row + o) * D + lane * NPL, rv);
+        const int o = sorted[warp][tg][i];
+        float rk[CPL], rv[CPL];
+        load_bf16_row<CPL>(a.ref_K + (um.ref_row + o) * D + sub * CPL, rk);
+        load_bf16_row<CPL>(a.ref_V + (um.ref_row + o) * D + sub * CPL, rv);
 #pragma unroll
-        for (int j = 0; j < NPL; ++j) {
-            mk[j] = __fadd_rn(mk[j], rk[j]);
-            mv[j] = __fadd_rn(mv[j], rv[j]);
+        for (int j2 = 0; j2 < CPL; ++j2) {
+            mk[j2] = __fadd_rn(mk[j2], rk[j2]);
+            mv[j2] = __fadd_rn(mv[j2], rv[j2]);
         }
     }
-    const float fk = static_cast<float>(keff);
+    if (keff & (keff - 1)) {
+        const float fk = static_cast<float>(keff);
 #pragma unroll
-    for (int j = 0; j < NPL; ++j) {
-        mk[j] = __fdiv_rn(mk[j], fk);
-        mv[j] = __fdiv_rn(mv[j], fk);
+        for (int j2 = 0; j2 < CPL; ++j2) {
+            mk[j2] = __fdiv_rn(mk[j2], fk);
+            mv[j2] = __fdiv_rn(mv[j2], fk);
+        }
+    } else {
+        // keff a power of two: the division is an exact scaling
+        const float inv = 1.0f / static_cast<float>(keff);
+#pragma unroll
+        for (int j2 = 0; j2 < CPL; ++j2) {
+            mk[j2] = __fmul_rn(mk[j2], inv);
+            mv[j2] = __fmul_rn(mv[j2], inv);
+        }
     }
 
     // ---- 3. residual and group quantiser ---------------------------------------------
-    quantise_store<NPL>(xk, mk, a.bits, lane, a.codes_K + row * a.code_bytes, a.scale_K + row * a.n_groups, a.err);
-    quantise_store<NPL>(xv, mv, a.bits, lane, a.codes_V + row * a.code_bytes, a.scale_V + row * a.n_groups, a.err);
+    float xv[CPL];
+    load_input_row<CPL>(V, e, a.in_dtype, xv);
+    quantise_store<CPL>(xk, mk, a.bits, sub, active, a.codes_K + row * a.code_bytes, a.scale_K + row * a.n_groups,
+                        a.err);
+    quantise_store<CPL>(xv, mv, a.bits, sub, active, a.codes_V + row * a.code_bytes, a.scale_V + row * a.n_groups,
+                        a.err);
 }
 
-template <int NPL>
-cudaError_t launch_npl(const CacheArgs& a, int max_C, const void* K, const void* V, const uint16_t* ci,
+template <int CPL>
+cudaError_t launch_cpl(const CacheArgs& a, int max_C, const void* K, const void* V, const uint16_t* ci,
                        const float* ct, cudaStream_t st)
 {
-    const dim3 grid((max_C + kWarps - 1) / kWarps, a.n_units);
+    const int per_block = kWarps * kTPW;
+    const dim3 grid((max_C + per_block - 1) / per_block, a.n_units);
     switch (a.kc) {
-    case 8: encode_kernel<NPL, 8><<<grid, kWarps * 32, 0, st>>>(a, K, V, ci, ct); break;
-    case 12: encode_kernel<NPL, 12><<<grid, kWarps * 32, 0, st>>>(a, K, V, ci, ct); break;
-    default: encode_kernel<NPL, 20><<<grid, kWarps * 32, 0, st>>>(a, K, V, ci, ct); break;
+    case 8: encode_kernel<CPL, 8><<<grid, kWarps * 32, 0, st>>>(a, K, V, ci, ct); break;
+    case 12: encode_kernel<CPL, 12><<<grid, kWarps * 32, 0, st>>>(a, K, V, ci, ct); break;
+    default: encode_kernel<CPL, 20><<<grid, kWarps * 32, 0, st>>>(a, K, V, ci, ct); break;
     }
     return cudaGetLastError();
 }
@@ -316,8 +462,8 @@ cudaError_t launch_encode(const CacheArgs& a, int max_C, const void* K, const vo
 {
     if (max_C <= 0)
         return cudaSuccess;
-    return (a.D == 128) ? launch_npl<4>(a, max_C, K, V, cand_idx, cand_t, st)
-                        : launch_npl<2>(a, max_C, K, V, cand_idx, cand_t, st);
+    return (a.D == 128) ? launch_cpl<16>(a, max_C, K, V, cand_idx, cand_t, st)
+                        : launch_cpl<8>(a, max_C, K, V, cand_idx, cand_t, st);
 }
 
 }  // namespace rkv

@@ -26,6 +26,11 @@ cudaError_t launch_reconstruct(const CacheArgs& a, int unit, const int32_t* posi
 // Literal decode: per token gather + mean of the reference rows, dequantise, add, attend.
 cudaError_t launch_decode_direct(const CacheArgs& a, int splits, const void* q, float* partials, cudaStream_t st);
 
+// Factorised decode (reference scores + scattered reference weights), one cluster per unit.
+bool decode_fact_supported(const CacheArgs& a);
+int decode_fact_cluster(const CacheArgs& a, int sms);
+cudaError_t launch_decode_fact(const CacheArgs& a, int cluster, const void* q, void* out, cudaStream_t st);
+
 // Merge of per-split partial softmax states into the output.
 cudaError_t launch_decode_combine(const CacheArgs& a, int batch, int splits, const float* partials, void* out,
                                   cudaStream_t st);

@@ -79,7 +79,7 @@ static_assert(sizeof(Desc) <= RKV_CACHE_DESC_BYTES, "descriptor too large");
 // Everything a kernel needs about one bound cache, passed by value.
 struct CacheArgs {
     int32_t D, Hkv, Hq, G, k, bits, group, in_dtype, out_dtype;
-    int32_t n_units, code_bytes, n_groups, kc, max_len;
+    int32_t n_units, code_bytes, n_groups, kc, max_len, max_refs;
     Phases ph;
     const UnitMeta* units;
     int32_t* err;

@@ -176,3 +176,11 @@ def test_qwen2_5_7b_batch_full_size_two_layers():
 
 def test_ultra_long_full_size():
     _named("ultra_long_1m", layers=[0], steps=[0, 15], n_uniform=512)
+
+
+def test_direct_decode_flag_matches_oracle():
+    wl = _small("qwen2_5_7b_batch", n_kv_heads=2, n_q_heads=14, batch=2, seq_len=2100, ragged=None)
+    lengths = [2100, 900]
+    K, V = synth.gen_layer(wl, 0, lengths)
+    run = GpuRun(wl, K, V, lengths, flags=rkv.RKV_FLAG_DECODE_DIRECT)
+    check_decode(run, synth.gen_query(wl, 0, 0))
