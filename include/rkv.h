@@ -260,6 +260,31 @@ RKV_API rkv_status rkv_reconstruct(const rkv_cache_desc* desc, int32_t seq, int3
                            int64_t n_pos, void* K_out, void* V_out, int32_t out_dtype, void* stream);
 
 /*
+ * rkv_compress without a caller-provided workspace (no counterpart on the
+ * pages; this is an interface convenience of this library).
+ *
+ * Some callers cannot call cudaMalloc or lend a workspace: code that runs
+ * while a stream is being captured into a CUDA graph (allocation calls are not
+ * allowed there), or an engine that has handed all device memory to its own
+ * fixed pool.  This entry point does the same work as rkv_compress, with the
+ * search -> encoder candidate lists kept in a file-scope device array of
+ * RKV_NOALLOC_SCRATCH_BYTES inside the library instead of in a workspace.  It
+ * allocates nothing; every GPU that loads the library holds the array until
+ * the process exits.
+ *   - Limit: the candidate lists of one layer (6 bytes per compressed row per
+ *     kept candidate, rounded to 256-byte sections) must fit the array;
+ *     larger caches get RKV_ERR_WORKSPACE before anything is enqueued.
+ *   - Set-up: the first call on a device (with that device current) looks up the
+ *     array's device address; make that first call before any stream capture.
+ *   - Sharing: all calls on a device use the same array and it keeps the last
+ *     call's contents; nothing in it needs to start at zero (the search writes
+ *     every entry the encoder reads).  Calls that overlap on the GPU race on it:
+ *     serialise them (one stream, or events).
+ */
+#define RKV_NOALLOC_SCRATCH_BYTES (16u << 20)
+RKV_API rkv_status rkv_compress_noalloc(const rkv_cache_desc* desc, const void* K, const void* V, void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the cache's device error word.
  * *device_status gets RKV_OK or the first RKV_ERR_* a kernel recorded since
  * the last read.  Returns RKV_ERR_CUDA if the synchronisation failed.

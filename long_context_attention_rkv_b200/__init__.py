@@ -29,7 +29,7 @@ STATUS_CODE = {v: k for k, v in STATUS.items()}
 
 EXPORTED = ["rkv_abi_version", "rkv_status_string", "rkv_schedule", "rkv_cache_size", "rkv_cache_bind",
             "rkv_unit_view_get", "rkv_build_refs", "rkv_search", "rkv_encode", "rkv_compress", "rkv_decode_attn", "rkv_reconstruct",
-            "rkv_read_device_error"]
+            "rkv_read_device_error", "rkv_compress_noalloc"]
 
 
 class RkvError(RuntimeError):
@@ -78,6 +78,7 @@ def lib() -> ctypes.CDLL:
         L.rkv_decode_attn.argtypes = [vp, vp, vp, vp, u64, vp]
         L.rkv_reconstruct.argtypes = [vp, i32, i32, vp, i64, vp, vp, i32, vp]
         L.rkv_read_device_error.argtypes = [vp, vp, ctypes.POINTER(i32)]
+        L.rkv_compress_noalloc.argtypes = [vp, vp, vp, vp]
         for name in EXPORTED[2:]:
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -185,6 +186,12 @@ def rkv_compress(desc: CacheDesc, K, V, workspace, workspace_bytes: int, stream=
            "rkv_compress")
 
 
+def rkv_compress_noalloc(desc: CacheDesc, K, V, stream=None):
+    """rkv_compress with the library's own fixed scratch array instead of a workspace (for callers
+    that cannot allocate); see include/rkv.h for its limit and sharing rules."""
+    _check(lib().rkv_compress_noalloc(desc.ptr, _ptr(K), _ptr(V), _stream(stream)), "rkv_compress_noalloc")
+
+
 def rkv_decode_attn(desc: CacheDesc, q, out, workspace, workspace_bytes: int, stream=None):
     _check(lib().rkv_decode_attn(desc.ptr, _ptr(q), _ptr(out), _ptr(workspace), workspace_bytes, _stream(stream)),
            "rkv_decode_attn")
@@ -216,8 +223,9 @@ class Layer:
         self.cache = torch.empty(self.cache_bytes, dtype=torch.uint8, device=device)
         if workspace is None:
             workspace = torch.empty(max(256, self.ws_bytes), dtype=torch.uint8, device=device)
-        assert workspace.numel() >= self.ws_bytes
-        self.workspace = workspace
+        if workspace is not False:           # False: no workspace (calls that need none)
+            assert workspace.numel() >= self.ws_bytes
+        self.workspace = workspace if workspace is not False else None
         self.desc = rkv_cache_bind(cfg, self.lengths, self.cache, self.cache_bytes)
 
     def build_refs(self, K, V, stream=None):

@@ -3,8 +3,10 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <climits>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -529,6 +531,61 @@ rkv_status rkv_read_device_error(const rkv_cache_desc* desc, void* stream, int32
         return RKV_ERR_CUDA;
     *device_status = v;
     return RKV_OK;
+}
+
+// ---- compress without a workspace ------------------------------------------------------
+// For callers that cannot allocate (see rkv_compress_noalloc in rkv.h): the candidate lists
+// live in this file-scope device array.  Host code only ever uses its device address, looked
+// up once per device with cudaGetSymbolAddress while that device is current.
+
+}  // extern "C"
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[RKV_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::atomic<void*> g_noalloc_addr[kMaxDevices];
+std::mutex g_noalloc_mutex;
+
+// Device address of the scratch array on the current device (looked up on first use).
+rkv_status noalloc_scratch(void** out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return RKV_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices)
+        return RKV_ERR_UNSUPPORTED;
+    void* p = g_noalloc_addr[dev].load(std::memory_order_acquire);
+    if (!p) {
+        std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+        p = g_noalloc_addr[dev].load(std::memory_order_relaxed);
+        if (!p) {
+            if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p)
+                return RKV_ERR_CUDA;
+            g_noalloc_addr[dev].store(p, std::memory_order_release);
+        }
+    }
+    *out = p;
+    return RKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+rkv_status rkv_compress_noalloc(const rkv_cache_desc* desc, const void* K, const void* V, void* stream)
+{
+    const Desc* d = get_desc(desc);
+    if (!d || !V)
+        return RKV_ERR_INVALID_ARG;
+    if (d->ws_select > RKV_NOALLOC_SCRATCH_BYTES)
+        return RKV_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    const rkv_status st = noalloc_scratch(&scratch);
+    if (st != RKV_OK)
+        return st;
+    return rkv_compress(desc, K, V, scratch, RKV_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 }  // extern "C"
