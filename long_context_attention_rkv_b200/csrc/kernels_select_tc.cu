@@ -363,6 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             int cnt = 0;
             float seed = -FLT_MAX;   // lower bound of the kc-th best t (from sub-block maxima)
+            float seed_lo = -FLT_MAX;
             for (int r = 0; r < nrt; ++r) {
                 const int acc = it_c % kAcc;
                 // one lane waits, the warp follows: the TMEM loads below are warp-collective
@@ -398,6 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int i = 0; i < kN / 16; ++i)
                         lo = fminf(lo, mxs[i]);
                     seed = (KC == kN / 16) ? lo : -FLT_MAX;
+                    seed_lo = (seed > -FLT_MAX) ? nextafterf(seed, -FLT_MAX) : -FLT_MAX;
                 }
                 for (int c0 = 0; c0 < kN && j0 + c0 < nc_max; c0 += 32) {
                     float v[32];
@@ -413,14 +415,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                             drain<KC>(myq, cnt, tv, ti);
                             cnt = 0;
                         }
-                        // appends at >= seed keep the element that defines the seed
-                        const float thr = fmaxf(tv[KC - 1], seed);
+                        // one compare per element: seed_lo is just below the seed, so the element
+                        // that defines the seed is still appended
+                        const float thr = fmaxf(tv[KC - 1], seed_lo);
+                        int o = cnt * kEpiThreads;
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
                             const int k = h * 16 + i;
-                            myq[cnt * kEpiThreads] = make_float2(v[k], __int_as_float(j0 + c0 + k));
-                            cnt += (v[k] > thr || (v[k] == seed && v[k] > tv[KC - 1])) ? 1 : 0;
+                            myq[o] = make_float2(v[k], __int_as_float(j0 + c0 + k));
+                            o += (v[k] > thr) ? kEpiThreads : 0;
                         }
+                        cnt = o / kEpiThreads;
                     }
                 }
                 tc_fence_before();
