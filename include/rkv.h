@@ -72,6 +72,7 @@ extern "C" {
  * library's tolerances whichever is chosen; the defaults are the fast paths. */
 #define RKV_FLAG_SELECT_SIMT 0x1u    /* reference search on CUDA cores even for bf16 inputs */
 #define RKV_FLAG_DECODE_DIRECT 0x2u  /* decode by gathering and averaging reference rows per token */
+#define RKV_FLAG_DECODE_SIMT 0x4u    /* factorised decode on CUDA cores even where the tensor-core form applies */
 
 typedef enum rkv_status {
     RKV_OK = 0,
@@ -242,7 +243,11 @@ RKV_API rkv_status rkv_encode(const rkv_cache_desc* desc, const void* K, const v
  * over all lengths[b] cached positions, where reference rows are the stored
  * bf16 rows and compressed rows are mean(references) + code * scale.  The
  * reconstructed cache is never written to memory.  A sequence of length 0
- * gives zeros.  workspace: device, scratch, >= rkv_cache_size's size.
+ * gives zeros.  workspace: device, scratch, >= rkv_cache_size's size; it holds
+ * state between the kernels of one call, so concurrent calls on different
+ * streams need different workspaces.  With bf16 inputs, head_dim 128, int4
+ * codes, k <= 8 and at most 8 query heads per kv-head the per-token dot
+ * products run on the tensor cores (flag RKV_FLAG_DECODE_SIMT turns that off).
  */
 RKV_API rkv_status rkv_decode_attn(const rkv_cache_desc* desc, const void* q, void* out, void* workspace,
                            uint64_t workspace_bytes, void* stream);

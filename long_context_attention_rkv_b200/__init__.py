@@ -20,6 +20,7 @@ RKV_DTYPE_BF16 = 0
 RKV_DTYPE_F32 = 1
 RKV_FLAG_SELECT_SIMT = 0x1
 RKV_FLAG_DECODE_DIRECT = 0x2
+RKV_FLAG_DECODE_SIMT = 0x4
 RKV_IDX_UNUSED = 0xFFFF
 RKV_CACHE_DESC_BYTES = 32768
 

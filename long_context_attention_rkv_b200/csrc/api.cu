@@ -96,6 +96,8 @@ int decode_splits(int n_units, int max_tokens)
     return s;
 }
 
+CacheArgs make_args(const Desc& d);
+
 rkv_status compute_layout(const rkv_config* c, const int32_t* lengths, Desc& d)
 {
     rkv_status st = validate_config(c);
@@ -172,6 +174,9 @@ rkv_status compute_layout(const rkv_config* c, const int32_t* lengths, Desc& d)
     d.ws_select = align_up(2ull * cmp_rows * d.kc, 256) + align_up(4ull * cmp_rows * d.kc, 256);
     const int splits = decode_splits(d.n_units, max_n);
     d.ws_decode = align_up(4ull * d.n_units * splits * G * (D + 2), 256);
+    const CacheArgs a = make_args(d);
+    if (decode_mma_supported(a))
+        d.ws_decode = std::max<uint64_t>(d.ws_decode, decode_mma_ws_bytes(a, d.total_ref_rows));
     return RKV_OK;
 }
 
@@ -475,6 +480,9 @@ rkv_status rkv_decode_attn(const rkv_cache_desc* desc, const void* q, void* out,
         return RKV_ERR_WORKSPACE;
     const CacheArgs a = make_args(*d);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (!(d->cfg.flags & (RKV_FLAG_DECODE_DIRECT | RKV_FLAG_DECODE_SIMT)) && decode_mma_supported(a) &&
+        workspace_bytes >= decode_mma_ws_bytes(a, d->total_ref_rows))
+        return cuda_status(launch_decode_mma(a, d->total_ref_rows, d->total_cmp_rows, q, out, workspace, st));
     if (decode_fact_supported(a) && !(d->cfg.flags & RKV_FLAG_DECODE_DIRECT)) {
         int dev = 0, sms = 0;
         cudaError_t e = cudaGetDevice(&dev);

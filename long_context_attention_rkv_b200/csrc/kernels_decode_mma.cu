@@ -1,0 +1,923 @@
+// Decode attention over the compressed cache with the two per-token contractions on
+// the tensor cores (ResidualKV paper summary page, "Practical Deployment via
+// Sparse-vLLM": reconstruction fused into attention; news page, "How ResidualKV
+// Works": tokens rebuilt on the fly when attention needs them).
+//
+// The algebra is the factorised one (reference scores s_j = q.refK_j, reference
+// weights w_j = sum of p_i / k_eff over the tokens that chose j):
+//   logit_i = mean_{j in S(i)} s_j + sum_g sK_ig * (q . codeK_i)_g
+//   out     = (sum_i p_i sum_g sV_ig codeV_i|g + sum_j (p_j + w_j) refV_j) / (sum_i p_i + sum_j p_j)
+// with every p taken against one common offset m = max_j s_j per (unit, q-head), so
+// partial sums from any number of CTAs add without rescaling.
+//
+// Per query step a G-head group does 2 * G * D multiply-adds per token against 152
+// bytes of codes, scales and ordinals (int4, D = 128, k = 4): at G >= 4 that is more
+// arithmetic per byte than the CUDA cores deliver per byte of HBM bandwidth, so the
+// per-token dot products run as bf16 MMAs and the CUDA cores only unpack codes and
+// run the softmax.  Three kernels, chained with programmatic dependent launch:
+//   1. scores:  s_j for every reference (fp32, log2 units) and per-64-reference maxima;
+//               zeroes the accumulators of step 3;
+//   2. tokens:  persistent, one CTA per SM over a contiguous range of 128-token tiles.
+//               A producer warp streams each tile into a shared-memory ring (codes by
+//               TMA with the 64-byte swizzle, scales and ordinals by bulk copies);
+//               consumer warps take 16 tokens each:
+//                 K side  D[tok][(head, group)] = codes (int4 -> bf16, exact) x q, one
+//                         m16n8k16 MMA per 16 channels, the group scale applied after;
+//                 softmax p = 2^(logit - m), reference weights by shared atomics;
+//                 V side  D[channel][(head, group)] = codes^T x (p * sV), the group
+//                         scale folded into the B operand (a hi + lo pair of bf16);
+//               partial outputs, sums and weights go to global accumulators;
+//   3. refs:    sum_j (p_j + w_j) refV_j per 64-reference chunk; the last chunk of a
+//               unit to finish normalises and writes the output.
+// Codes enter the MMAs as 136 + v (v the signed code; the bf16 bit pattern of 128 + n
+// for a nibble n): the constant 136 is taken off afterwards with exact row/column sums.
+#include <cudaTypedefs.h>
+
+#include <cfloat>
+#include <cmath>
+
+#include "device_common.cuh"
+#include "launchers.h"
+#include "sm100_ptx.cuh"
+
+namespace rkv {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kTok = 128;            // tokens per pipeline stage (= compressed-row padding)
+constexpr int kRefChunk = 64;        // references per CTA of the scores and refs kernels
+constexpr int kWarpTok = 16;         // tokens per consumer warp and stage
+constexpr int kConsWarps = kTok / kWarpTok;
+constexpr int kCodeRow = 64;         // bytes of one int4 code row at D = 128
+constexpr uint32_t kNibMask = 0x000F000Fu;
+constexpr uint32_t kNibMagic = 0x43084308u;   // bf16 128.0 in each half, sign bit of the nibble flipped
+constexpr float kCodeOffset = 136.0f;         // (128 + (v + 8)) - v
+
+// Stage layout (bytes): codes K | codes V (64-byte swizzle, 1024-aligned) | scales K | scales V | ordinals
+constexpr int kStCodes = kTok * kCodeRow;                 // 8192
+constexpr int kStScale = kTok * 4 * 2;                    // 4 groups x fp16
+constexpr int kStIdxMax = kTok * 8 * 2;                   // k <= 8 ordinals x u16
+constexpr int kStageBytes = 2 * kStCodes + 2 * kStScale + kStIdxMax;   // 20480
+
+// ---- small PTX wrappers ------------------------------------------------------------------
+
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// One-dimensional bulk copy global -> shared, completion counted on bar (16-byte aligned, size % 16 == 0).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_addr(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_addr(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4])
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4])
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+// D += A * B, m16n8k16, bf16 inputs, fp32 accumulators.
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Two nibbles (bits 0-3 and 16-19 of w) to a bf16 pair {136 + v_lo, 136 + v_hi}.
+__device__ __forceinline__ uint32_t nib2(uint32_t w) { return (w & kNibMask) ^ kNibMagic; }
+
+// A pair of fp32 values as two bf16 pairs, hi = bf16(x) and lo = bf16(x - hi), so that
+// hi + lo carries about 16 significant bits; sum accumulates the four values exactly as
+// the MMAs will see them.
+__device__ __forceinline__ void split_bf16(float x0, float x1, uint32_t& hi, uint32_t& lo, float& sum)
+{
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    const float h0 = __uint_as_float(hi << 16), h1 = __uint_as_float(hi & 0xffff0000u);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - h0, x1 - h1);
+    lo = *reinterpret_cast<const uint32_t*>(&l);
+    sum += (h0 + __uint_as_float(lo << 16)) + (h1 + __uint_as_float(lo & 0xffff0000u));
+}
+
+__device__ __forceinline__ float half_bits_to_f32(uint32_t b) { return __half2float(__ushort_as_half(static_cast<unsigned short>(b))); }
+
+// Bytes offset of (row, 16-byte chunk) in a 64-byte-row tile written by TMA with the 64-byte swizzle.
+__device__ __forceinline__ uint32_t sw64(int row, int chunk)
+{
+    return static_cast<uint32_t>(row * kCodeRow + ((chunk ^ ((row >> 1) & 3)) << 4));
+}
+
+}  // namespace
+
+// Workspace carve-up of this decode (device pointers); see decode_mma_ws_bytes.
+struct MmaWs {
+    float* s_tab;     // [ref rows][Gp]  reference scores, log2 units
+    float* W;         // [ref rows][Gp]  reference weights sum_i p_i / k_eff
+    float* mpart;     // [units][n_chunk][Gp]  maxima of 64-reference chunks
+    float* O;         // [units][Gp][D]  output numerators
+    float* L;         // [units][Gp]     softmax denominators
+    uint32_t* cnt;    // [units]         finished chunks of the refs kernel
+    int n_chunk;
+    int n_tiles;
+    float cK;         // log2(e) / sqrt(D)
+};
+
+namespace {
+
+// ==== 1. reference scores ==================================================================
+
+template <int Gp>
+__global__ void __launch_bounds__(256) mma_scores_kernel(const CacheArgs a, const void* __restrict__ q, const MmaWs w)
+{
+    grid_dep_launch();
+    constexpr int D = 128;
+    __shared__ float qs[Gp][D];
+    __shared__ float wmax[8][Gp];
+    const int u = blockIdx.y, ch = blockIdx.x;
+    const UnitMeta um = a.units[u];
+    const int kvh = u - um.seq * a.Hkv;
+    const int tid = threadIdx.x;
+    const int R = um.R;
+    const int r0 = ch * kRefChunk;
+    const int r1 = min(R, r0 + kRefChunk);
+    if (ch == 0) {
+        for (int i = tid; i < Gp * D; i += 256)
+            w.O[static_cast<int64_t>(u) * Gp * D + i] = 0.0f;
+        if (tid < Gp)
+            w.L[u * Gp + tid] = 0.0f;
+        if (tid == 0)
+            w.cnt[u] = 0u;
+    }
+    for (int i = tid; i < (r1 - r0) * Gp; i += 256)
+        w.W[(um.ref_row + r0) * Gp + i] = 0.0f;
+    for (int i = tid; i < Gp * D; i += 256) {
+        const int h = i / D, c = i % D;
+        qs[h][c] = (h < a.G) ? bf16_bits_to_f32(static_cast<const uint16_t*>(
+                                   q)[(static_cast<int64_t>(um.seq) * a.Hq + kvh * a.G + h) * D + c]) * w.cK
+                             : 0.0f;
+    }
+    __syncthreads();
+    // eight lanes per reference row, sixteen channels each
+    const int grp = tid >> 3, sub = tid & 7;
+    float mloc[Gp];
+#pragma unroll
+    for (int h = 0; h < Gp; ++h)
+        mloc[h] = -FLT_MAX;
+    for (int r = r0 + grp; r - grp < r1; r += 32) {
+        const bool ok = r < r1;
+        float x[16];
+        if (ok) {
+            const uint16_t* rp = a.ref_K + (um.ref_row + r) * D + sub * 16;
+            const uint4 v0 = *reinterpret_cast<const uint4*>(rp);
+            const uint4 v1 = *reinterpret_cast<const uint4*>(rp + 8);
+            const uint32_t ww[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                x[2 * i] = bf16_bits_to_f32(ww[i] & 0xffffu);
+                x[2 * i + 1] = bf16_bits_to_f32(ww[i] >> 16);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                x[i] = 0.0f;
+        }
+        float sv[Gp];
+#pragma unroll
+        for (int h = 0; h < Gp; ++h) {
+            float d = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                d = fmaf(qs[h][sub * 16 + i], x[i], d);
+            d += __shfl_xor_sync(0xffffffffu, d, 1);
+            d += __shfl_xor_sync(0xffffffffu, d, 2);
+            d += __shfl_xor_sync(0xffffffffu, d, 4);
+            sv[h] = d;
+            if (ok && h < a.G)
+                mloc[h] = fmaxf(mloc[h], d);
+        }
+        if (ok && sub == 0) {
+            float* dst = w.s_tab + (um.ref_row + r) * Gp;
+#pragma unroll
+            for (int h = 0; h < Gp; h += 4)
+                *reinterpret_cast<float4*>(dst + h) = make_float4(sv[h], sv[h + 1], sv[h + 2], sv[h + 3]);
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < Gp; ++h) {
+        const float v = warp_max(mloc[h]);
+        if ((tid & 31) == 0)
+            wmax[tid >> 5][h] = v;
+    }
+    __syncthreads();
+    if (tid < Gp) {
+        float v = -FLT_MAX;
+        for (int i = 0; i < 8; ++i)
+            v = fmaxf(v, wmax[i][tid]);
+        w.mpart[(static_cast<int64_t>(u) * w.n_chunk + ch) * Gp + tid] = v;
+    }
+}
+
+// Common offset m of a unit's q-head: the maximum reference score (0 for a unit without references).
+template <int Gp>
+__device__ __forceinline__ float unit_max(const MmaWs& w, int u, int R, int h)
+{
+    const int nch = (R + kRefChunk - 1) / kRefChunk;
+    float v = -FLT_MAX;
+    for (int c = 0; c < nch; ++c)
+        v = fmaxf(v, w.mpart[(static_cast<int64_t>(u) * w.n_chunk + c) * Gp + h]);
+    return (v == -FLT_MAX) ? 0.0f : v;
+}
+
+// ==== 2. compressed tokens ================================================================
+
+// Dynamic shared memory of the tokens kernel (byte offsets from a 1024-aligned base).
+struct TokLayout {
+    int stages, s_sm, w_sm, o_sm, p_sm, q_sm, bar, misc, total;
+    __host__ __device__ TokLayout(int Gp, int ncons, int R_max, int nst)
+    {
+        auto up = [](int x) { return (x + 127) & ~127; };
+        int off = 0;
+        stages = off; off += nst * kStageBytes;
+        s_sm = off;   off += up(R_max * Gp * 4);
+        w_sm = off;   off += up(R_max * Gp * 4);
+        o_sm = off;   off += up(Gp * 128 * 4);
+        p_sm = off;   off += up(ncons * kWarpTok * Gp * 4);
+        q_sm = off;   off += up(Gp * 128 * 2);
+        bar = off;    off += 2 * 8 * 8;
+        misc = off;   off += up((6 * Gp + 4) * 4);
+        total = off;
+    }
+};
+
+__device__ __forceinline__ void consumer_sync(int n_threads)
+{
+    asm volatile("bar.sync 1, %0;" ::"r"(n_threads) : "memory");
+}
+
+template <int Gp, int NTEAM>
+__global__ void __launch_bounds__(32 * (1 + kConsWarps * NTEAM), 1)
+    mma_tokens_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                      const CacheArgs a, const void* __restrict__ q, const MmaWs w, const int nst)
+{
+    constexpr int D = 128;
+    constexpr int GPS = 8 / Gp;           // scale groups sharing one set of eight MMA columns
+    constexpr int NS = 4 / GPS;           // column sets
+    constexpr int NH = Gp / 4;            // q-heads per thread in the softmax step
+    constexpr int NCONS = kConsWarps * NTEAM;
+    constexpr int NCT = NCONS * 32;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* sm = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const TokLayout L(Gp, NCONS, a.max_refs, nst);
+    unsigned char* stages = sm + L.stages;
+    float* s_sm = reinterpret_cast<float*>(sm + L.s_sm);
+    float* w_sm = reinterpret_cast<float*>(sm + L.w_sm);
+    float* o_sm = reinterpret_cast<float*>(sm + L.o_sm);
+    float* p_sm = reinterpret_cast<float*>(sm + L.p_sm);
+    uint16_t* q_sm = reinterpret_cast<uint16_t*>(sm + L.q_sm);
+    uint64_t* full = reinterpret_cast<uint64_t*>(sm + L.bar);
+    uint64_t* empty = full + 8;
+    float* m_sm = reinterpret_cast<float*>(sm + L.misc);
+    float* qc_sm = m_sm + Gp;             // [4 groups][Gp]
+    float* l_sm = qc_sm + 4 * Gp;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(l_sm + Gp);
+    volatile int* zero_flag = abort_flag + 1;
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int nb = gridDim.x, b = blockIdx.x;
+    const int t_lo = static_cast<int>(static_cast<int64_t>(w.n_tiles) * b / nb);
+    const int t_hi = static_cast<int>(static_cast<int64_t>(w.n_tiles) * (b + 1) / nb);
+
+    if (tid == 0) {
+        for (int s = 0; s < nst; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsWarps);
+        }
+        *abort_flag = 0;
+        *zero_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    // ---- producer warp ------------------------------------------------------------------
+    if (warp == NCONS) {
+        if (lane == 0) {
+            prefetch_tensormap(&tmK);
+            prefetch_tensormap(&tmV);
+            const uint32_t idx_bytes = static_cast<uint32_t>(kTok * a.k * 2);
+            const uint32_t tx = 2 * kStCodes + 2 * kStScale + idx_bytes;
+            int i = 0;
+            for (int t = t_lo; t < t_hi; ++t, ++i) {
+                const int s = i % nst;
+                if (i >= nst && !mbar_wait(&empty[s], ((i / nst) & 1) ^ 1, abort_flag)) {
+                    if (!*abort_flag)
+                        report(a.err, RKV_ERR_TIMEOUT);
+                    *abort_flag = 1;
+                    break;
+                }
+                unsigned char* st = stages + s * kStageBytes;
+                const int64_t row0 = static_cast<int64_t>(t) * kTok;
+                mbar_arrive_expect_tx(&full[s], tx);
+                tma_load_2d(st, &tmK, 0, static_cast<int>(row0), &full[s]);
+                tma_load_2d(st + kStCodes, &tmV, 0, static_cast<int>(row0), &full[s]);
+                bulk_load(st + 2 * kStCodes, a.scale_K + row0 * 4, kStScale, &full[s]);
+                bulk_load(st + 2 * kStCodes + kStScale, a.scale_V + row0 * 4, kStScale, &full[s]);
+                bulk_load(st + 2 * kStCodes + 2 * kStScale, a.idx + row0 * a.k, idx_bytes, &full[s]);
+            }
+            // the copies of the last stages land before the CTA may exit
+            for (int j = (i > nst ? i - nst : 0); j < i; ++j)
+                mbar_wait(&full[j % nst], (j / nst) & 1, zero_flag);
+        }
+        return;
+    }
+
+    // ---- consumer warps -----------------------------------------------------------------
+    const int team = warp / kConsWarps, wi = warp % kConsWarps;
+    const int gid = lane >> 2, tq = lane & 3;
+    const int G = a.G;
+    grid_dep_wait();   // reference scores, maxima and zeroed accumulators of the scores kernel
+
+    // unit of the first tile: the last unit whose rows start at or before it
+    int u = 0;
+    {
+        int lo = 0, hi = a.n_units - 1;
+        const int64_t row = static_cast<int64_t>(t_lo) * kTok;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (a.units[mid].cmp_row <= row)
+                lo = mid;
+            else
+                hi = mid - 1;
+        }
+        u = lo;
+    }
+    bool overflow = false, corrupt = false;
+    int t = t_lo, i = 0;
+    while (t < t_hi && u < a.n_units) {
+        const UnitMeta um = a.units[u];
+        const int t_end = static_cast<int>((um.cmp_row + ((um.C + kTok - 1) / kTok) * kTok) / kTok);
+        if (t >= t_end) {
+            ++u;
+            continue;
+        }
+        const int seg_end = min(t_hi, t_end);
+        const int R = um.R;
+        const int kvh = u - um.seq * a.Hkv;
+
+        // ---- unit setup: q, reference scores, cleared weights ----------------------------
+        consumer_sync(NCT);
+        for (int x = tid; x < Gp * D; x += NCT) {
+            const int h = x / D, c = x % D;
+            q_sm[x] = (h < G) ? static_cast<const uint16_t*>(q)[(static_cast<int64_t>(um.seq) * a.Hq + kvh * G + h) * D + c]
+                              : static_cast<uint16_t>(0);
+            o_sm[x] = 0.0f;
+        }
+        {
+            const float4* src = reinterpret_cast<const float4*>(w.s_tab + um.ref_row * Gp);
+            float4* dst = reinterpret_cast<float4*>(s_sm);
+            float4* wz = reinterpret_cast<float4*>(w_sm);
+            for (int x = tid; x < R * Gp / 4; x += NCT) {
+                dst[x] = src[x];
+                wz[x] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            }
+        }
+        if (tid < Gp) {
+            m_sm[tid] = unit_max<Gp>(w, u, R, tid);
+            l_sm[tid] = 0.0f;
+        }
+        consumer_sync(NCT);
+        if (tid < 4 * Gp) {
+            const int g = tid / Gp, h = tid % Gp;
+            float sum = 0.0f;
+            for (int c = 0; c < 32; ++c)
+                sum += bf16_bits_to_f32(q_sm[h * D + 32 * g + c]);
+            qc_sm[g * Gp + h] = kCodeOffset * sum;
+        }
+        consumer_sync(NCT);
+        // K-side B operand: column gid is (head gid / GPS, group residue gid % GPS); k-slot
+        // order within a group follows the nibble order of the A fragments
+        uint32_t bk[8][2];
+        {
+            const int hcol = gid / GPS, gcol = gid % GPS;
+#pragma unroll
+            for (int kb = 0; kb < 8; ++kb) {
+                const int g = kb >> 1, sub = kb & 1;
+                const bool on = (g % GPS) == gcol && hcol < G;
+                const uint16_t* qr = q_sm + hcol * D + 32 * g + 8 * tq + 2 * sub;
+                bk[kb][0] = on ? (static_cast<uint32_t>(qr[0]) | (static_cast<uint32_t>(qr[4]) << 16)) : 0u;
+                bk[kb][1] = on ? (static_cast<uint32_t>(qr[1]) | (static_cast<uint32_t>(qr[5]) << 16)) : 0u;
+            }
+        }
+        float m_h[NH], qc_h[4][NH], l_acc[NH];
+#pragma unroll
+        for (int e = 0; e < NH; ++e) {
+            const int h = (Gp == 4) ? tq : 2 * tq + e;
+            m_h[e] = m_sm[h];
+            l_acc[e] = 0.0f;
+#pragma unroll
+            for (int g = 0; g < 4; ++g)
+                qc_h[g][e] = qc_sm[g * Gp + h];
+        }
+        float dv[8][4];
+        float colsum[NS];
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+                dv[mt][x] = 0.0f;
+#pragma unroll
+        for (int s = 0; s < NS; ++s)
+            colsum[s] = 0.0f;
+
+        // ---- the unit's tiles: this team takes every NTEAM-th stage ----------------------
+        for (; t < seg_end; ++t, ++i) {
+            if (i % NTEAM != team)
+                continue;
+            const int s = i % nst;
+            if (!*abort_flag && !mbar_wait(&full[s], (i / nst) & 1, abort_flag)) {
+                if (!*abort_flag)
+                    report(a.err, RKV_ERR_TIMEOUT);
+                *abort_flag = 1;
+            }
+            if (!*abort_flag) {
+                unsigned char* st = stages + s * kStageBytes;
+                const uint32_t stK = smem_addr(st), stV = stK + kStCodes;
+                const uint16_t* sK = reinterpret_cast<const uint16_t*>(st + 2 * kStCodes);
+                const uint16_t* sV = sK + kTok * 4;
+                const uint16_t* ix = reinterpret_cast<const uint16_t*>(st + 2 * kStCodes + 2 * kStScale);
+                const int rb = wi * kWarpTok;                                   // first row of this warp
+                const int tok0 = static_cast<int>(static_cast<int64_t>(t) * kTok - um.cmp_row) + rb;
+                float* pw = p_sm + warp * kWarpTok * Gp;
+
+                // K side: D[token][column set] over the 128 channels, one MMA per 16 channels
+                uint32_t wk0[4], wk1[4];
+                ldsm_x4(stK + sw64(rb + (lane & 7), lane >> 3), wk0);
+                ldsm_x4(stK + sw64(rb + 8 + (lane & 7), lane >> 3), wk1);
+                float dk[NS][4];
+#pragma unroll
+                for (int x = 0; x < NS; ++x)
+                    dk[x][0] = dk[x][1] = dk[x][2] = dk[x][3] = 0.0f;
+#pragma unroll
+                for (int g = 0; g < 4; ++g)
+#pragma unroll
+                    for (int sub = 0; sub < 2; ++sub) {
+                        const int sh = 8 * sub;
+                        mma_bf16(dk[g / GPS], nib2(wk0[g] >> sh), nib2(wk1[g] >> sh), nib2(wk0[g] >> (sh + 4)),
+                                 nib2(wk1[g] >> (sh + 4)), bk[2 * g + sub][0], bk[2 * g + sub][1]);
+                    }
+
+                // softmax of this thread's two tokens (rows gid, gid + 8) and NH heads
+#pragma unroll
+                for (int rr = 0; rr < 2; ++rr) {
+                    const int row = rb + gid + 8 * rr;
+                    const bool valid = tok0 + gid + 8 * rr < um.C;
+                    const uint2 skw = *reinterpret_cast<const uint2*>(sK + row * 4);
+                    const float sk[4] = {half_bits_to_f32(skw.x & 0xffffu), half_bits_to_f32(skw.x >> 16),
+                                         half_bits_to_f32(skw.y & 0xffffu), half_bits_to_f32(skw.y >> 16)};
+                    int oi[8];
+                    if (a.k == 4) {
+                        const uint2 v = *reinterpret_cast<const uint2*>(ix + row * 4);
+                        oi[0] = v.x & 0xffff; oi[1] = v.x >> 16; oi[2] = v.y & 0xffff; oi[3] = v.y >> 16;
+                        oi[4] = oi[5] = oi[6] = oi[7] = RKV_IDX_UNUSED;
+                    } else if (a.k == 8) {
+                        const uint4 v = *reinterpret_cast<const uint4*>(ix + row * 8);
+                        oi[0] = v.x & 0xffff; oi[1] = v.x >> 16; oi[2] = v.y & 0xffff; oi[3] = v.y >> 16;
+                        oi[4] = v.z & 0xffff; oi[5] = v.z >> 16; oi[6] = v.w & 0xffff; oi[7] = v.w >> 16;
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            oi[j] = (j < a.k) ? ix[row * a.k + j] : RKV_IDX_UNUSED;
+                    }
+                    int keff = 0;
+                    float sref[NH];
+#pragma unroll
+                    for (int e = 0; e < NH; ++e)
+                        sref[e] = 0.0f;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const bool has = valid && oi[j] != RKV_IDX_UNUSED;
+                        corrupt |= has && oi[j] >= R;
+                        const bool use = has && oi[j] < R;
+                        oi[j] = use ? oi[j] : -1;
+                        keff += use ? 1 : 0;
+                        if (use) {
+                            if constexpr (NH == 1) {
+                                sref[0] += s_sm[oi[j] * Gp + tq];
+                            } else {
+                                const float2 v = *reinterpret_cast<const float2*>(s_sm + oi[j] * Gp + 2 * tq);
+                                sref[0] += v.x;
+                                sref[1] += v.y;
+                            }
+                        }
+                    }
+                    const float rk = 1.0f / static_cast<float>(max(keff, 1));
+#pragma unroll
+                    for (int e = 0; e < NH; ++e) {
+                        const int h = (Gp == 4) ? tq : 2 * tq + e;
+                        float acc = 0.0f;
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) {
+                            const float raw = (Gp == 4) ? dk[g >> 1][(g & 1) + 2 * rr] : dk[g][e + 2 * rr];
+                            acc = fmaf(sk[g], raw - qc_h[g][e], acc);
+                        }
+                        const float logit = fmaf(w.cK, acc, sref[e] * rk);
+                        const float ex = logit - m_h[e];
+                        const bool live = valid && keff > 0 && h < G;
+                        overflow |= live && ex > 100.0f;
+                        const float p = live ? exp2f(fminf(ex, 100.0f)) : 0.0f;
+                        l_acc[e] += p;
+                        pw[(gid + 8 * rr) * Gp + h] = p;
+                        const float pr = p * rk;
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            if (oi[j] >= 0 && live)
+                                atomicAdd(&w_sm[oi[j] * Gp + h], pr);
+                    }
+                }
+                __syncwarp();
+
+                // V-side B operand: column gid is (head gid / GPS, group residue gid % GPS),
+                // k-slots are the tokens 2tq, 2tq+1, 2tq+8, 2tq+9 of the warp's block; p * sV
+                // enters as a hi + lo pair of bf16 operands (two MMAs into one accumulator)
+                uint32_t bv[NS][2], bl[NS][2];
+                {
+                    const int hv = gid / GPS, gv = gid % GPS;
+                    const int tv[4] = {2 * tq, 2 * tq + 1, 2 * tq + 8, 2 * tq + 9};
+                    float pv[4];
+                    uint2 svw[4];
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        pv[x] = pw[tv[x] * Gp + hv];
+                        svw[x] = *reinterpret_cast<const uint2*>(sV + (rb + tv[x]) * 4);
+                    }
+#pragma unroll
+                    for (int s2 = 0; s2 < NS; ++s2) {
+                        const int g = s2 * GPS + gv;
+                        float v[4];
+#pragma unroll
+                        for (int x = 0; x < 4; ++x) {
+                            const uint32_t word = (g < 2) ? svw[x].x : svw[x].y;
+                            const float sc = half_bits_to_f32((g & 1) ? (word >> 16) : (word & 0xffffu));
+                            v[x] = (pv[x] != 0.0f) ? pv[x] * sc : 0.0f;
+                        }
+                        split_bf16(v[0], v[1], bv[s2][0], bl[s2][0], colsum[s2]);
+                        split_bf16(v[2], v[3], bv[s2][1], bl[s2][1], colsum[s2]);
+                    }
+                }
+                __syncwarp();
+
+                // V side: D[channel][column] += codes^T x B, two MMAs (32 channels) per group
+                uint32_t xv[2][4];
+#pragma unroll
+                for (int c = 0; c < 2; ++c)
+                    ldsm_x4_t(stV + sw64(rb + 8 * ((lane >> 3) & 1) + (lane & 7), 2 * c + (lane >> 4)), xv[c]);
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    const uint32_t xl = xv[g >> 1][(g & 1) * 2], xh = xv[g >> 1][(g & 1) * 2 + 1];
+                    const int s2 = g / GPS;
+                    const uint32_t a0 = nib2(xl), a1 = nib2(xl >> 4), a2 = nib2(xh), a3 = nib2(xh >> 4);
+                    const uint32_t c0 = nib2(xl >> 8), c1 = nib2(xl >> 12), c2 = nib2(xh >> 8), c3 = nib2(xh >> 12);
+                    mma_bf16(dv[2 * g], a0, a1, a2, a3, bv[s2][0], bv[s2][1]);
+                    mma_bf16(dv[2 * g + 1], c0, c1, c2, c3, bv[s2][0], bv[s2][1]);
+                    mma_bf16(dv[2 * g], a0, a1, a2, a3, bl[s2][0], bl[s2][1]);
+                    mma_bf16(dv[2 * g + 1], c0, c1, c2, c3, bl[s2][0], bl[s2][1]);
+                }
+            }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&empty[s]);
+        }
+
+        // ---- flush the unit's partial sums -----------------------------------------------
+        consumer_sync(NCT);
+        {
+            // column sums of the V-side B operand (sum over the four lanes of a column), then
+            // the sums of the two columns this thread's accumulators hold
+            float cs[NS][2];
+#pragma unroll
+            for (int s2 = 0; s2 < NS; ++s2) {
+                float tot = colsum[s2];
+                tot += __shfl_xor_sync(0xffffffffu, tot, 1);
+                tot += __shfl_xor_sync(0xffffffffu, tot, 2);
+                cs[s2][0] = __shfl_sync(0xffffffffu, tot, (2 * tq) * 4);
+                cs[s2][1] = __shfl_sync(0xffffffffu, tot, (2 * tq + 1) * 4);
+            }
+#pragma unroll
+            for (int g = 0; g < 4; ++g)
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+                    for (int rr = 0; rr < 2; ++rr) {
+                        const int ch = 32 * g + 4 * gid + 2 * hf + rr;
+                        const float* d = dv[2 * g + hf];
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            // Gp 4: column 2tq + e is (head tq, group residue e); Gp 8: head 2tq + e
+                            const int h = (Gp == 4) ? tq : 2 * tq + e;
+                            const bool mine = (Gp == 4) ? (e == (g & 1)) : true;
+                            if (mine && h < G && !*abort_flag)
+                                atomicAdd(&o_sm[h * D + ch], d[e + 2 * rr] - kCodeOffset * cs[g / GPS][e]);
+                        }
+                    }
+#pragma unroll
+            for (int e = 0; e < NH; ++e) {
+                float v = l_acc[e];
+                v += __shfl_xor_sync(0xffffffffu, v, 4);
+                v += __shfl_xor_sync(0xffffffffu, v, 8);
+                v += __shfl_xor_sync(0xffffffffu, v, 16);
+                const int h = (Gp == 4) ? tq : 2 * tq + e;
+                if (gid == 0 && h < G)
+                    atomicAdd(&l_sm[h], v);
+            }
+        }
+        consumer_sync(NCT);
+        if (!*abort_flag) {
+            const float4* ws4 = reinterpret_cast<const float4*>(w_sm);
+            float* Wg = w.W + um.ref_row * Gp;
+            for (int x = tid; x < R * Gp / 4; x += NCT) {
+                const float4 v = ws4[x];
+                if (v.x != 0.0f) atomicAdd(Wg + 4 * x, v.x);
+                if (v.y != 0.0f) atomicAdd(Wg + 4 * x + 1, v.y);
+                if (v.z != 0.0f) atomicAdd(Wg + 4 * x + 2, v.z);
+                if (v.w != 0.0f) atomicAdd(Wg + 4 * x + 3, v.w);
+            }
+            for (int x = tid; x < G * D; x += NCT)
+                atomicAdd(&w.O[static_cast<int64_t>(u) * Gp * D + x], o_sm[x]);
+            if (tid < G)
+                atomicAdd(&w.L[u * Gp + tid], l_sm[tid]);
+        }
+        t = seg_end;
+        ++u;
+    }
+    if (__any_sync(0xffffffffu, overflow) && lane == 0)
+        report(a.err, RKV_ERR_UNSUPPORTED);
+    if (__any_sync(0xffffffffu, corrupt) && lane == 0)
+        report(a.err, RKV_ERR_CORRUPT);
+}
+
+// ==== 3. reference tokens, reference weights, output =========================================
+
+template <int Gp>
+__global__ void __launch_bounds__(256) mma_refs_kernel(const CacheArgs a, void* __restrict__ out, const MmaWs w)
+{
+    constexpr int D = 128;
+    __shared__ float wt[kRefChunk][Gp];
+    __shared__ float red[4][Gp][D];
+    __shared__ float lred[Gp];
+    __shared__ float msm[Gp];
+    __shared__ int last;
+    const int u = blockIdx.y, ch = blockIdx.x, tid = threadIdx.x;
+    grid_dep_wait();   // weights and partial sums of the tokens kernel
+    const UnitMeta um = a.units[u];
+    const int R = um.R;
+    const int nch = max(1, (R + kRefChunk - 1) / kRefChunk);
+    if (ch >= nch)
+        return;
+    const int G = a.G;
+    const int kvh = u - um.seq * a.Hkv;
+    const int r0 = ch * kRefChunk, r1 = min(R, r0 + kRefChunk);
+    if (tid < Gp) {
+        lred[tid] = 0.0f;
+        msm[tid] = unit_max<Gp>(w, u, R, tid);
+    }
+    __syncthreads();
+    // weight of reference r: its own softmax term p_r plus w_r from the tokens that chose it
+    for (int x = tid; x < kRefChunk * Gp; x += 256) {
+        const int r = r0 + x / Gp, h = x % Gp;
+        float v = 0.0f;
+        if (r < r1 && h < G) {
+            const int64_t e = (um.ref_row + r) * Gp + h;
+            const float pj = exp2f(w.s_tab[e] - msm[h]);
+            v = w.W[e] + pj;
+            atomicAdd(&lred[h], pj);
+        }
+        wt[x / Gp][h] = v;
+    }
+    __syncthreads();
+    // sum_r wt[r][h] refV[r][c]: thread (channel pair, quarter of the chunk)
+    {
+        const int cp = tid & 63, qq = tid >> 6;
+        float acc[Gp][2];
+#pragma unroll
+        for (int h = 0; h < Gp; ++h)
+            acc[h][0] = acc[h][1] = 0.0f;
+#pragma unroll 4
+        for (int rr = 0; rr < kRefChunk / 4; ++rr) {
+            const int r = r0 + qq * (kRefChunk / 4) + rr;
+            if (r < r1) {
+                const uint32_t v = *reinterpret_cast<const uint32_t*>(a.ref_V + (um.ref_row + r) * D + 2 * cp);
+                const float x0 = bf16_bits_to_f32(v & 0xffffu), x1 = bf16_bits_to_f32(v >> 16);
+#pragma unroll
+                for (int h = 0; h < Gp; ++h) {
+                    acc[h][0] = fmaf(wt[r - r0][h], x0, acc[h][0]);
+                    acc[h][1] = fmaf(wt[r - r0][h], x1, acc[h][1]);
+                }
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < Gp; ++h) {
+            red[qq][h][2 * cp] = acc[h][0];
+            red[qq][h][2 * cp + 1] = acc[h][1];
+        }
+    }
+    __syncthreads();
+    for (int x = tid; x < G * D; x += 256) {
+        const int h = x / D, c = x % D;
+        atomicAdd(&w.O[static_cast<int64_t>(u) * Gp * D + x], red[0][h][c] + red[1][h][c] + red[2][h][c] + red[3][h][c]);
+    }
+    if (tid < G)
+        atomicAdd(&w.L[u * Gp + tid], lred[tid]);
+    __threadfence();
+    __syncthreads();
+    if (tid == 0)
+        last = (atomicAdd(&w.cnt[u], 1u) == static_cast<uint32_t>(nch - 1)) ? 1 : 0;
+    __syncthreads();
+    if (!last)
+        return;
+    __threadfence();
+    for (int x = tid; x < G * D; x += 256) {
+        const int h = x / D, c = x % D;
+        const float o = __ldcg(&w.O[static_cast<int64_t>(u) * Gp * D + x]);
+        const float l = __ldcg(&w.L[u * Gp + h]);
+        const float res = (l > 0.0f) ? o / l : 0.0f;
+        const int64_t e = (static_cast<int64_t>(um.seq) * a.Hq + kvh * G + h) * D + c;
+        if (a.out_dtype == RKV_DTYPE_F32)
+            static_cast<float*>(out)[e] = res;
+        else
+            static_cast<uint16_t*>(out)[e] = f32_to_bf16_bits(res);
+    }
+}
+
+// ==== host side ==============================================================================
+
+constexpr int kTeams = 1;
+
+int heads_padded(int G) { return G <= 4 ? 4 : 8; }
+
+// Opt-in shared memory per block on sm_100 (227 KB); a constant so that workspace sizes do
+// not depend on the device present when they are computed.
+constexpr int kSmemOptin = 232448;
+
+// Pipeline depth that fits next to the unit tables (0 if fewer than two stages fit).
+int tok_stages(const CacheArgs& a)
+{
+    const int Gp = heads_padded(a.G);
+    const int fixed = TokLayout(Gp, kConsWarps * kTeams, a.max_refs, 0).total + 1024;
+    const int avail = kSmemOptin - fixed;
+    const int n = avail / kStageBytes;
+    return n < 2 ? 0 : (n > 8 ? 8 : n);
+}
+
+struct WsOffsets {
+    uint64_t s_tab, W, mpart, O, L, cnt, end;
+};
+
+WsOffsets ws_offsets(const CacheArgs& a, int64_t ref_rows)
+{
+    const int Gp = heads_padded(a.G);
+    const int n_chunk = (a.max_refs + kRefChunk - 1) / kRefChunk > 0 ? (a.max_refs + kRefChunk - 1) / kRefChunk : 1;
+    uint64_t off = 0;
+    auto take = [&](uint64_t bytes) {
+        const uint64_t o = off;
+        off = (off + bytes + 255) / 256 * 256;
+        return o;
+    };
+    WsOffsets o;
+    o.s_tab = take(4ull * ref_rows * Gp);
+    o.W = take(4ull * ref_rows * Gp);
+    o.mpart = take(4ull * a.n_units * n_chunk * Gp);
+    o.O = take(4ull * a.n_units * Gp * 128);
+    o.L = take(4ull * a.n_units * Gp);
+    o.cnt = take(4ull * a.n_units);
+    o.end = off;
+    return o;
+}
+
+using EncodeFn = PFN_cuTensorMapEncodeTiled_v12000;
+
+EncodeFn encoder()
+{
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qr) != cudaSuccess ||
+        qr != cudaDriverEntryPointSuccess)
+        return nullptr;
+    return reinterpret_cast<EncodeFn>(fn);
+}
+
+// Byte-typed 2D map over the int4 code rows (64 bytes each), 128-row boxes, 64-byte swizzle.
+bool code_map(EncodeFn enc, CUtensorMap* m, const void* base, int64_t rows)
+{
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(kCodeRow), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(kCodeRow)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(kCodeRow), static_cast<cuuint32_t>(kTok)};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename Kern, typename... Args>
+cudaError_t launch_pdl(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+template <int Gp>
+cudaError_t launch_gp(const CacheArgs& a, int64_t cmp_rows, const void* q, void* out, const MmaWs& w, int nst,
+                      cudaStream_t st)
+{
+    EncodeFn enc = encoder();
+    if (!enc)
+        return cudaErrorNotSupported;
+    alignas(64) CUtensorMap mK;
+    alignas(64) CUtensorMap mV;
+    if (!code_map(enc, &mK, a.codes_K, cmp_rows) || !code_map(enc, &mV, a.codes_V, cmp_rows))
+        return cudaErrorInvalidValue;
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess)
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess)
+        return e;
+    const dim3 rgrid(w.n_chunk, a.n_units);
+    mma_scores_kernel<Gp><<<rgrid, 256, 0, st>>>(a, q, w);
+    e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return e;
+    if (w.n_tiles > 0) {
+        auto kern = mma_tokens_kernel<Gp, kTeams>;
+        const size_t smem = TokLayout(Gp, kConsWarps * kTeams, a.max_refs, nst).total + 1024;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e != cudaSuccess)
+            return e;
+        const int grid = w.n_tiles < sms ? w.n_tiles : sms;
+        e = launch_pdl(kern, dim3(grid), dim3(32 * (1 + kConsWarps * kTeams)), smem, st, mK, mV, a, q, w, nst);
+        if (e != cudaSuccess)
+            return e;
+    }
+    return launch_pdl(mma_refs_kernel<Gp>, rgrid, dim3(256), 0, st, a, out, w);
+}
+
+}  // namespace
+
+bool decode_mma_supported(const CacheArgs& a)
+{
+    return a.D == 128 && a.bits == 4 && a.group == 32 && a.in_dtype == RKV_DTYPE_BF16 && a.G >= 1 && a.G <= 8 &&
+           a.k >= 1 && a.k <= 8 && tok_stages(a) >= 2;
+}
+
+uint64_t decode_mma_ws_bytes(const CacheArgs& a, int64_t ref_rows) { return ws_offsets(a, ref_rows).end; }
+
+cudaError_t launch_decode_mma(const CacheArgs& a, int64_t ref_rows, int64_t cmp_rows, const void* q, void* out,
+                              void* workspace, cudaStream_t st)
+{
+    const WsOffsets o = ws_offsets(a, ref_rows);
+    char* base = static_cast<char*>(workspace);
+    MmaWs w;
+    w.s_tab = reinterpret_cast<float*>(base + o.s_tab);
+    w.W = reinterpret_cast<float*>(base + o.W);
+    w.mpart = reinterpret_cast<float*>(base + o.mpart);
+    w.O = reinterpret_cast<float*>(base + o.O);
+    w.L = reinterpret_cast<float*>(base + o.L);
+    w.cnt = reinterpret_cast<uint32_t*>(base + o.cnt);
+    w.n_chunk = (a.max_refs + kRefChunk - 1) / kRefChunk > 0 ? (a.max_refs + kRefChunk - 1) / kRefChunk : 1;
+    w.n_tiles = static_cast<int>(cmp_rows / kTok);
+    w.cK = static_cast<float>(1.4426950408889634 / std::sqrt(128.0));
+    const int nst = tok_stages(a);
+    if (nst < 2)
+        return cudaErrorNotSupported;
+    return heads_padded(a.G) == 4 ? launch_gp<4>(a, cmp_rows, q, out, w, nst, st)
+                                  : launch_gp<8>(a, cmp_rows, q, out, w, nst, st);
+}
+
+}  // namespace rkv

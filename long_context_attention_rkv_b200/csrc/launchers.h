@@ -31,6 +31,13 @@ bool decode_fact_supported(const CacheArgs& a);
 int decode_fact_cluster(const CacheArgs& a, int sms);
 cudaError_t launch_decode_fact(const CacheArgs& a, int cluster, const void* q, void* out, cudaStream_t st);
 
+// Factorised decode with the per-token contractions on the tensor cores (bf16 inputs,
+// head_dim 128, int4 codes): scores, tokens and references kernels.
+bool decode_mma_supported(const CacheArgs& a);
+uint64_t decode_mma_ws_bytes(const CacheArgs& a, int64_t ref_rows);
+cudaError_t launch_decode_mma(const CacheArgs& a, int64_t ref_rows, int64_t cmp_rows, const void* q, void* out,
+                              void* workspace, cudaStream_t st);
+
 // Merge of per-split partial softmax states into the output.
 cudaError_t launch_decode_combine(const CacheArgs& a, int batch, int splits, const float* partials, void* out,
                                   cudaStream_t st);

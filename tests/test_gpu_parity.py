@@ -184,3 +184,26 @@ def test_direct_decode_flag_matches_oracle():
     K, V = synth.gen_layer(wl, 0, lengths)
     run = GpuRun(wl, K, V, lengths, flags=rkv.RKV_FLAG_DECODE_DIRECT)
     check_decode(run, synth.gen_query(wl, 0, 0))
+
+
+def test_simt_decode_flag_matches_oracle():
+    wl = _small("llama3_8b_layer", n_kv_heads=2, n_q_heads=8, batch=2, seq_len=3100, ragged=None)
+    lengths = [3100, 1500]
+    K, V = synth.gen_layer(wl, 0, lengths)
+    run = GpuRun(wl, K, V, lengths, flags=rkv.RKV_FLAG_DECODE_SIMT)
+    check_decode(run, synth.gen_query(wl, 0, 0))
+
+
+@pytest.mark.parametrize("n_q_heads", [6, 16])
+def test_decode_many_short_units(n_q_heads):
+    """More 128-token tiles than SMs, so one CTA of the tensor-core decode crosses unit
+    boundaries; group sizes 3 (heads padded to 4) and 8."""
+    wl = _small("llama3_8b_layer", n_kv_heads=2, n_q_heads=n_q_heads, batch=16, seq_len=1700, ragged=None)
+    lengths = [1700 - 97 * i for i in range(16)]
+    K, V = synth.gen_layer(wl, 0, lengths)
+    run = GpuRun(wl, K, V, lengths)
+    check_decode(run, synth.gen_query(wl, 0, 0))
+    simt = GpuRun(wl, K, V, lengths, flags=rkv.RKV_FLAG_DECODE_SIMT)
+    q = synth.gen_query(wl, 0, 0)
+    a, b = run.decode(q), simt.decode(q)
+    assert np.abs(a - b).max() <= 2e-3
