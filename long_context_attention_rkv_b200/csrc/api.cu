@@ -5,6 +5,8 @@
 #include <algorithm>
 #include <atomic>
 #include <climits>
+#include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <new>
@@ -225,7 +227,17 @@ CacheArgs make_args(const Desc& d)
     return a;
 }
 
-rkv_status cuda_status(cudaError_t e) { return e == cudaSuccess ? RKV_OK : RKV_ERR_CUDA; }
+// A failed CUDA call becomes RKV_ERR_CUDA; with RKV_DEBUG set in the environment its
+// CUDA error string is also printed to stderr.
+rkv_status cuda_status(cudaError_t e)
+{
+    if (e == cudaSuccess)
+        return RKV_OK;
+    static const bool verbose = std::getenv("RKV_DEBUG") != nullptr;
+    if (verbose)
+        std::fprintf(stderr, "librkv: CUDA error %d: %s\n", static_cast<int>(e), cudaGetErrorString(e));
+    return RKV_ERR_CUDA;
+}
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 

@@ -16,23 +16,27 @@
 // per-token dot products run as bf16 MMAs and the CUDA cores only unpack codes and
 // run the softmax.  Three kernels, chained with programmatic dependent launch:
 //   1. scores:  s_j for every reference (fp32, log2 units) and per-64-reference maxima;
-//               zeroes the accumulators of step 3;
+//               zeroes the weight and output accumulators;
 //   2. tokens:  persistent, one CTA per SM over a contiguous range of 128-token tiles.
-//               A producer warp streams each tile into a shared-memory ring (codes by
-//               TMA with the 64-byte swizzle, scales and ordinals by bulk copies);
-//               consumer warps take 16 tokens each:
+//               Each tile is streamed into a shared-memory ring (codes by TMA with the
+//               64-byte swizzle, scales and ordinals by bulk copies); the last of the
+//               eight warps to finish a stage refills it, so no warp is spent on loads
+//               (two warps per scheduler keep the register file at up to 255 a thread);
+//               each warp takes 16 tokens of a tile:
 //                 K side  D[tok][(head, group)] = codes (int4 -> bf16, exact) x q, one
 //                         m16n8k16 MMA per 16 channels, the group scale applied after;
 //                 softmax p = 2^(logit - m), reference weights by shared atomics;
 //                 V side  D[channel][(head, group)] = codes^T x (p * sV), the group
 //                         scale folded into the B operand (a hi + lo pair of bf16);
-//               partial outputs, sums and weights go to global accumulators;
+//               reference weights go to global memory with vector reductions as they
+//               are produced, partial outputs and sums at the end of each unit;
 //   3. refs:    sum_j (p_j + w_j) refV_j per 64-reference chunk; the last chunk of a
 //               unit to finish normalises and writes the output.
 // Codes enter the MMAs as 136 + v (v the signed code; the bf16 bit pattern of 128 + n
 // for a nibble n): the constant 136 is taken off afterwards with exact row/column sums.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cfloat>
 #include <cmath>
 
@@ -119,6 +123,28 @@ __device__ __forceinline__ void split_bf16(float x0, float x1, uint32_t& hi, uin
 
 __device__ __forceinline__ float half_bits_to_f32(uint32_t b) { return __half2float(__ushort_as_half(static_cast<unsigned short>(b))); }
 
+__device__ __forceinline__ void red_shared(float* p, float v)
+{
+    asm volatile("red.shared.add.f32 [%0], %1;" ::"r"(smem_addr(p)), "f"(v) : "memory");
+}
+
+__device__ __forceinline__ void red_global_v4(float* p, float a, float b, float c, float d)
+{
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
+
+// Order-preserving map of floats to unsigned keys (0 is below every float) and back.
+__device__ __forceinline__ uint32_t fkey(float f)
+{
+    const uint32_t b = __float_as_uint(f);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+__device__ __forceinline__ float fkey_inv(uint32_t k)
+{
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
 // Bytes offset of (row, 16-byte chunk) in a 64-byte-row tile written by TMA with the 64-byte swizzle.
 __device__ __forceinline__ uint32_t sw64(int row, int chunk)
 {
@@ -137,6 +163,7 @@ struct MmaWs {
     uint32_t* cnt;    // [units]         finished chunks of the refs kernel
     int n_chunk;
     int n_tiles;
+    int n_cta;        // CTAs of the tokens kernel
     float cK;         // log2(e) / sqrt(D)
 };
 
@@ -166,6 +193,22 @@ __global__ void __launch_bounds__(256) mma_scores_kernel(const CacheArgs a, cons
         if (tid == 0)
             w.cnt[u] = 0u;
     }
+    // eight lanes per reference row, sixteen channels each, two rows per lane group; the
+    // reference rows are fetched before the query is staged
+    const int grp = tid >> 3, sub = tid & 7;
+    static_assert(kRefChunk == 64, "two passes of 32 rows");
+    uint4 rk[2][2];
+#pragma unroll
+    for (int ps = 0; ps < 2; ++ps) {
+        const int r = r0 + grp + 32 * ps;
+        if (r < r1) {
+            const uint16_t* rp = a.ref_K + (um.ref_row + r) * D + sub * 16;
+            rk[ps][0] = *reinterpret_cast<const uint4*>(rp);
+            rk[ps][1] = *reinterpret_cast<const uint4*>(rp + 8);
+        } else {
+            rk[ps][0] = rk[ps][1] = make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
     for (int i = tid; i < (r1 - r0) * Gp; i += 256)
         w.W[(um.ref_row + r0) * Gp + i] = 0.0f;
     for (int i = tid; i < Gp * D; i += 256) {
@@ -175,29 +218,21 @@ __global__ void __launch_bounds__(256) mma_scores_kernel(const CacheArgs a, cons
                              : 0.0f;
     }
     __syncthreads();
-    // eight lanes per reference row, sixteen channels each
-    const int grp = tid >> 3, sub = tid & 7;
     float mloc[Gp];
 #pragma unroll
     for (int h = 0; h < Gp; ++h)
         mloc[h] = -FLT_MAX;
-    for (int r = r0 + grp; r - grp < r1; r += 32) {
+#pragma unroll
+    for (int ps = 0; ps < 2; ++ps) {
+        const int r = r0 + grp + 32 * ps;
         const bool ok = r < r1;
         float x[16];
-        if (ok) {
-            const uint16_t* rp = a.ref_K + (um.ref_row + r) * D + sub * 16;
-            const uint4 v0 = *reinterpret_cast<const uint4*>(rp);
-            const uint4 v1 = *reinterpret_cast<const uint4*>(rp + 8);
-            const uint32_t ww[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        const uint32_t ww[8] = {rk[ps][0].x, rk[ps][0].y, rk[ps][0].z, rk[ps][0].w,
+                                rk[ps][1].x, rk[ps][1].y, rk[ps][1].z, rk[ps][1].w};
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                x[2 * i] = bf16_bits_to_f32(ww[i] & 0xffffu);
-                x[2 * i + 1] = bf16_bits_to_f32(ww[i] >> 16);
-            }
-        } else {
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-                x[i] = 0.0f;
+        for (int i = 0; i < 8; ++i) {
+            x[2 * i] = bf16_bits_to_f32(ww[i] & 0xffffu);
+            x[2 * i + 1] = bf16_bits_to_f32(ww[i] >> 16);
         }
         float sv[Gp];
 #pragma unroll
@@ -235,29 +270,36 @@ __global__ void __launch_bounds__(256) mma_scores_kernel(const CacheArgs a, cons
     }
 }
 
-// Common offset m of a unit's q-head: the maximum reference score (0 for a unit without references).
+// Common offset m of a unit's q-heads: the maximum reference score (0 for a unit without
+// references).  All threads of the group load the chunk maxima in parallel and fold them
+// into key[Gp] (shared, zeroed beforehand) with atomic maxima; read back with unit_m.
 template <int Gp>
-__device__ __forceinline__ float unit_max(const MmaWs& w, int u, int R, int h)
+__device__ __forceinline__ void unit_max_fold(const MmaWs& w, int u, int R, int tid, int nthreads, uint32_t* key)
 {
-    const int nch = (R + kRefChunk - 1) / kRefChunk;
-    float v = -FLT_MAX;
-    for (int c = 0; c < nch; ++c)
-        v = fmaxf(v, w.mpart[(static_cast<int64_t>(u) * w.n_chunk + c) * Gp + h]);
-    return (v == -FLT_MAX) ? 0.0f : v;
+    const int n = ((R + kRefChunk - 1) / kRefChunk) * Gp;
+    const float* src = w.mpart + static_cast<int64_t>(u) * w.n_chunk * Gp;
+    for (int x = tid; x < n; x += nthreads)
+        atomicMax(&key[x % Gp], fkey(src[x]));
+}
+
+__device__ __forceinline__ float unit_m(const uint32_t* key, int h)
+{
+    const uint32_t k = key[h];
+    const float v = fkey_inv(k);
+    return (k == 0u || v == -FLT_MAX) ? 0.0f : v;
 }
 
 // ==== 2. compressed tokens ================================================================
 
 // Dynamic shared memory of the tokens kernel (byte offsets from a 1024-aligned base).
 struct TokLayout {
-    int stages, s_sm, w_sm, o_sm, p_sm, q_sm, bar, misc, total;
+    int stages, s_sm, o_sm, p_sm, q_sm, bar, misc, total;
     __host__ __device__ TokLayout(int Gp, int ncons, int R_max, int nst)
     {
         auto up = [](int x) { return (x + 127) & ~127; };
         int off = 0;
         stages = off; off += nst * kStageBytes;
         s_sm = off;   off += up(R_max * Gp * 4);
-        w_sm = off;   off += up(R_max * Gp * 4);
         o_sm = off;   off += up(Gp * 128 * 4);
         p_sm = off;   off += up(ncons * kWarpTok * Gp * 4);
         q_sm = off;   off += up(Gp * 128 * 2);
@@ -272,8 +314,8 @@ __device__ __forceinline__ void consumer_sync(int n_threads)
     asm volatile("bar.sync 1, %0;" ::"r"(n_threads) : "memory");
 }
 
-template <int Gp, int NTEAM>
-__global__ void __launch_bounds__(32 * (1 + kConsWarps * NTEAM), 1)
+template <int Gp, int KK>
+__global__ void __launch_bounds__(32 * kConsWarps, 1)
     mma_tokens_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       const CacheArgs a, const void* __restrict__ q, const MmaWs w, const int nst)
 {
@@ -281,77 +323,67 @@ __global__ void __launch_bounds__(32 * (1 + kConsWarps * NTEAM), 1)
     constexpr int GPS = 8 / Gp;           // scale groups sharing one set of eight MMA columns
     constexpr int NS = 4 / GPS;           // column sets
     constexpr int NH = Gp / 4;            // q-heads per thread in the softmax step
-    constexpr int NCONS = kConsWarps * NTEAM;
-    constexpr int NCT = NCONS * 32;
+    constexpr int NCT = kConsWarps * 32;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    const TokLayout L(Gp, NCONS, a.max_refs, nst);
+    const TokLayout L(Gp, kConsWarps, a.max_refs, nst);
     unsigned char* stages = sm + L.stages;
     float* s_sm = reinterpret_cast<float*>(sm + L.s_sm);
-    float* w_sm = reinterpret_cast<float*>(sm + L.w_sm);
     float* o_sm = reinterpret_cast<float*>(sm + L.o_sm);
     float* p_sm = reinterpret_cast<float*>(sm + L.p_sm);
     uint16_t* q_sm = reinterpret_cast<uint16_t*>(sm + L.q_sm);
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + L.bar);
-    uint64_t* empty = full + 8;
-    float* m_sm = reinterpret_cast<float*>(sm + L.misc);
-    float* qc_sm = m_sm + Gp;             // [4 groups][Gp]
+    int* done_cnt = reinterpret_cast<int*>(full + 8);        // warps finished with a stage
+    float* qc_sm = reinterpret_cast<float*>(sm + L.misc);    // [4 groups][Gp]
     float* l_sm = qc_sm + 4 * Gp;
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(l_sm + Gp);
+    uint32_t* key_sm = reinterpret_cast<uint32_t*>(l_sm + Gp);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(key_sm + Gp);
     volatile int* zero_flag = abort_flag + 1;
+    int* issued = const_cast<int*>(zero_flag + 1);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
     const int nb = gridDim.x, b = blockIdx.x;
     const int t_lo = static_cast<int>(static_cast<int64_t>(w.n_tiles) * b / nb);
     const int t_hi = static_cast<int>(static_cast<int64_t>(w.n_tiles) * (b + 1) / nb);
+    const int n_local = t_hi - t_lo;
+    const uint32_t idx_bytes = static_cast<uint32_t>(kTok * a.k * 2);
+    const uint32_t tx = 2 * kStCodes + 2 * kStScale + idx_bytes;
+    // loads local tile j into stage j % nst (one thread)
+    auto issue = [&](int j) {
+        const int s = j % nst;
+        unsigned char* st = stages + s * kStageBytes;
+        const int64_t row0 = static_cast<int64_t>(t_lo + j) * kTok;
+        mbar_arrive_expect_tx(&full[s], tx);
+        tma_load_2d(st, &tmK, 0, static_cast<int>(row0), &full[s]);
+        tma_load_2d(st + kStCodes, &tmV, 0, static_cast<int>(row0), &full[s]);
+        bulk_load(st + 2 * kStCodes, a.scale_K + row0 * 4, kStScale, &full[s]);
+        bulk_load(st + 2 * kStCodes + kStScale, a.scale_V + row0 * 4, kStScale, &full[s]);
+        bulk_load(st + 2 * kStCodes + 2 * kStScale, a.idx + row0 * a.k, idx_bytes, &full[s]);
+    };
 
     if (tid == 0) {
         for (int s = 0; s < nst; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kConsWarps);
+            done_cnt[s] = 0;
         }
         *abort_flag = 0;
         *zero_flag = 0;
         fence_mbar_init();
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+        // the ring fills while the scores kernel may still run: codes do not depend on it
+        const int n0 = n_local < nst ? n_local : nst;
+        for (int j = 0; j < n0; ++j)
+            issue(j);
+        *issued = n0;
     }
     __syncthreads();
-
-    // ---- producer warp ------------------------------------------------------------------
-    if (warp == NCONS) {
-        if (lane == 0) {
-            prefetch_tensormap(&tmK);
-            prefetch_tensormap(&tmV);
-            const uint32_t idx_bytes = static_cast<uint32_t>(kTok * a.k * 2);
-            const uint32_t tx = 2 * kStCodes + 2 * kStScale + idx_bytes;
-            int i = 0;
-            for (int t = t_lo; t < t_hi; ++t, ++i) {
-                const int s = i % nst;
-                if (i >= nst && !mbar_wait(&empty[s], ((i / nst) & 1) ^ 1, abort_flag)) {
-                    if (!*abort_flag)
-                        report(a.err, RKV_ERR_TIMEOUT);
-                    *abort_flag = 1;
-                    break;
-                }
-                unsigned char* st = stages + s * kStageBytes;
-                const int64_t row0 = static_cast<int64_t>(t) * kTok;
-                mbar_arrive_expect_tx(&full[s], tx);
-                tma_load_2d(st, &tmK, 0, static_cast<int>(row0), &full[s]);
-                tma_load_2d(st + kStCodes, &tmV, 0, static_cast<int>(row0), &full[s]);
-                bulk_load(st + 2 * kStCodes, a.scale_K + row0 * 4, kStScale, &full[s]);
-                bulk_load(st + 2 * kStCodes + kStScale, a.scale_V + row0 * 4, kStScale, &full[s]);
-                bulk_load(st + 2 * kStCodes + 2 * kStScale, a.idx + row0 * a.k, idx_bytes, &full[s]);
-            }
-            // the copies of the last stages land before the CTA may exit
-            for (int j = (i > nst ? i - nst : 0); j < i; ++j)
-                mbar_wait(&full[j % nst], (j / nst) & 1, zero_flag);
-        }
-        return;
-    }
+    grid_dep_launch();   // the references kernel may be scheduled once every CTA runs
 
     // ---- consumer warps -----------------------------------------------------------------
-    const int team = warp / kConsWarps, wi = warp % kConsWarps;
+    const int wi = warp;
     const int gid = lane >> 2, tq = lane & 3;
     const int G = a.G;
     grid_dep_wait();   // reference scores, maxima and zeroed accumulators of the scores kernel
@@ -383,8 +415,12 @@ __global__ void __launch_bounds__(32 * (1 + kConsWarps * NTEAM), 1)
         const int R = um.R;
         const int kvh = u - um.seq * a.Hkv;
 
-        // ---- unit setup: q, reference scores, cleared weights ----------------------------
+        // ---- unit setup: q, reference scores, common offsets ------------------------------
         consumer_sync(NCT);
+        if (tid < Gp) {
+            key_sm[tid] = 0u;
+            l_sm[tid] = 0.0f;
+        }
         for (int x = tid; x < Gp * D; x += NCT) {
             const int h = x / D, c = x % D;
             q_sm[x] = (h < G) ? static_cast<const uint16_t*>(q)[(static_cast<int64_t>(um.seq) * a.Hq + kvh * G + h) * D + c]
@@ -392,22 +428,32 @@ __global__ void __launch_bounds__(32 * (1 + kConsWarps * NTEAM), 1)
             o_sm[x] = 0.0f;
         }
         {
+            // eight float4 loads in flight per thread
             const float4* src = reinterpret_cast<const float4*>(w.s_tab + um.ref_row * Gp);
             float4* dst = reinterpret_cast<float4*>(s_sm);
-            float4* wz = reinterpret_cast<float4*>(w_sm);
-            for (int x = tid; x < R * Gp / 4; x += NCT) {
-                dst[x] = src[x];
-                wz[x] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            const int n4 = R * Gp / 4;
+            for (int base = 0; base < n4; base += 8 * NCT) {
+                float4 tmp[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int x = base + j * NCT + tid;
+                    if (x < n4)
+                        tmp[j] = src[x];
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int x = base + j * NCT + tid;
+                    if (x < n4)
+                        dst[x] = tmp[j];
+                }
             }
         }
-        if (tid < Gp) {
-            m_sm[tid] = unit_max<Gp>(w, u, R, tid);
-            l_sm[tid] = 0.0f;
-        }
         consumer_sync(NCT);
+        unit_max_fold<Gp>(w, u, R, tid, NCT, key_sm);
         if (tid < 4 * Gp) {
             const int g = tid / Gp, h = tid % Gp;
             float sum = 0.0f;
+#pragma unroll 8
             for (int c = 0; c < 32; ++c)
                 sum += bf16_bits_to_f32(q_sm[h * D + 32 * g + c]);
             qc_sm[g * Gp + h] = kCodeOffset * sum;
@@ -431,7 +477,7 @@ __global__ void __launch_bounds__(32 * (1 + kConsWarps * NTEAM), 1)
 #pragma unroll
         for (int e = 0; e < NH; ++e) {
             const int h = (Gp == 4) ? tq : 2 * tq + e;
-            m_h[e] = m_sm[h];
+            m_h[e] = unit_m(key_sm, h);
             l_acc[e] = 0.0f;
 #pragma unroll
             for (int g = 0; g < 4; ++g)
@@ -448,12 +494,10 @@ __global__ void __launch_bounds__(32 * (1 + kConsWarps * NTEAM), 1)
         for (int s = 0; s < NS; ++s)
             colsum[s] = 0.0f;
 
-        // ---- the unit's tiles: this team takes every NTEAM-th stage ----------------------
+        // ---- the unit's tiles, 16 tokens per warp ---------------------------------------
         for (; t < seg_end; ++t, ++i) {
-            if (i % NTEAM != team)
-                continue;
             const int s = i % nst;
-            if (!*abort_flag && !mbar_wait(&full[s], (i / nst) & 1, abort_flag)) {
+            if (!*abort_flag && !mbar_wait_sleep(&full[s], (i / nst) & 1, abort_flag)) {
                 if (!*abort_flag)
                     report(a.err, RKV_ERR_TIMEOUT);
                 *abort_flag = 1;
@@ -493,18 +537,18 @@ __global__ void __launch_bounds__(32 * (1 + kConsWarps * NTEAM), 1)
                     const uint2 skw = *reinterpret_cast<const uint2*>(sK + row * 4);
                     const float sk[4] = {half_bits_to_f32(skw.x & 0xffffu), half_bits_to_f32(skw.x >> 16),
                                          half_bits_to_f32(skw.y & 0xffffu), half_bits_to_f32(skw.y >> 16)};
-                    int oi[8];
-                    if (a.k == 4) {
+                    int oi[KK];
+                    if (KK == 4 && a.k == 4) {
                         const uint2 v = *reinterpret_cast<const uint2*>(ix + row * 4);
                         oi[0] = v.x & 0xffff; oi[1] = v.x >> 16; oi[2] = v.y & 0xffff; oi[3] = v.y >> 16;
-                        oi[4] = oi[5] = oi[6] = oi[7] = RKV_IDX_UNUSED;
-                    } else if (a.k == 8) {
+                    } else if (KK == 8 && a.k == 8) {
                         const uint4 v = *reinterpret_cast<const uint4*>(ix + row * 8);
                         oi[0] = v.x & 0xffff; oi[1] = v.x >> 16; oi[2] = v.y & 0xffff; oi[3] = v.y >> 16;
-                        oi[4] = v.z & 0xffff; oi[5] = v.z >> 16; oi[6] = v.w & 0xffff; oi[7] = v.w >> 16;
+                        oi[KK > 4 ? 4 : 0] = v.z & 0xffff; oi[KK > 5 ? 5 : 0] = v.z >> 16;
+                        oi[KK > 6 ? 6 : 0] = v.w & 0xffff; oi[KK > 7 ? 7 : 0] = v.w >> 16;
                     } else {
 #pragma unroll
-                        for (int j = 0; j < 8; ++j)
+                        for (int j = 0; j < KK; ++j)
                             oi[j] = (j < a.k) ? ix[row * a.k + j] : RKV_IDX_UNUSED;
                     }
                     int keff = 0;
@@ -513,23 +557,24 @@ __global__ void __launch_bounds__(32 * (1 + kConsWarps * NTEAM), 1)
                     for (int e = 0; e < NH; ++e)
                         sref[e] = 0.0f;
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
+                    for (int j = 0; j < KK; ++j) {
                         const bool has = valid && oi[j] != RKV_IDX_UNUSED;
                         corrupt |= has && oi[j] >= R;
                         const bool use = has && oi[j] < R;
                         oi[j] = use ? oi[j] : -1;
                         keff += use ? 1 : 0;
-                        if (use) {
-                            if constexpr (NH == 1) {
-                                sref[0] += s_sm[oi[j] * Gp + tq];
-                            } else {
-                                const float2 v = *reinterpret_cast<const float2*>(s_sm + oi[j] * Gp + 2 * tq);
-                                sref[0] += v.x;
-                                sref[1] += v.y;
-                            }
+                        const int oc = use ? oi[j] : 0;     // unconditional load, selected sum
+                        if constexpr (NH == 1) {
+                            const float v = s_sm[oc * Gp + tq];
+                            sref[0] += use ? v : 0.0f;
+                        } else {
+                            const float2 v = *reinterpret_cast<const float2*>(s_sm + oc * Gp + 2 * tq);
+                            sref[0] += use ? v.x : 0.0f;
+                            sref[1] += use ? v.y : 0.0f;
                         }
                     }
-                    const float rk = 1.0f / static_cast<float>(max(keff, 1));
+                    const float rk = __frcp_rn(static_cast<float>(max(keff, 1)));
+                    float pe[NH];
 #pragma unroll
                     for (int e = 0; e < NH; ++e) {
                         const int h = (Gp == 4) ? tq : 2 * tq + e;
@@ -546,11 +591,26 @@ __global__ void __launch_bounds__(32 * (1 + kConsWarps * NTEAM), 1)
                         const float p = live ? exp2f(fminf(ex, 100.0f)) : 0.0f;
                         l_acc[e] += p;
                         pw[(gid + 8 * rr) * Gp + h] = p;
-                        const float pr = p * rk;
+                        pe[e] = p * rk;
+                    }
+                    // reference weights: the four lanes of the row share all q-heads' p / k_eff,
+                    // then lane tq adds them to references tq and tq + 4 with vector reductions
+                    float pall[Gp];
 #pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            if (oi[j] >= 0 && live)
-                                atomicAdd(&w_sm[oi[j] * Gp + h], pr);
+                    for (int t2 = 0; t2 < 4; ++t2)
+#pragma unroll
+                        for (int e = 0; e < NH; ++e)
+                            pall[NH * t2 + e] = __shfl_sync(0xffffffffu, pe[e], (lane & ~3) | t2);
+#pragma unroll
+                    for (int jj = 0; jj < KK / 4; ++jj) {
+                        const int o = (tq == 0) ? oi[4 * jj] : (tq == 1) ? oi[4 * jj + 1]
+                                    : (tq == 2) ? oi[4 * jj + 2] : oi[4 * jj + 3];
+                        if (o >= 0) {
+                            float* dst = w.W + (um.ref_row + o) * Gp;
+#pragma unroll
+                            for (int h4 = 0; h4 < Gp; h4 += 4)
+                                red_global_v4(dst + h4, pall[h4], pall[h4 + 1], pall[h4 + 2], pall[h4 + 3]);
+                        }
                     }
                 }
                 __syncwarp();
@@ -602,9 +662,20 @@ __global__ void __launch_bounds__(32 * (1 + kConsWarps * NTEAM), 1)
                     mma_bf16(dv[2 * g + 1], c0, c1, c2, c3, bl[s2][0], bl[s2][1]);
                 }
             }
+            // the last warp done with the stage refills it with local tile i + nst
             __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&empty[s]);
+            if (lane == 0) {
+                __threadfence_block();
+                if (atomicAdd(&done_cnt[s], 1) == kConsWarps - 1) {
+                    done_cnt[s] = 0;
+                    const int j = i + nst;
+                    if (j < n_local && !*abort_flag) {
+                        fence_proxy_async_smem();
+                        issue(j);
+                        atomicMax(issued, j + 1);
+                    }
+                }
+            }
         }
 
         // ---- flush the unit's partial sums -----------------------------------------------
@@ -635,7 +706,7 @@ __global__ void __launch_bounds__(32 * (1 + kConsWarps * NTEAM), 1)
                             const int h = (Gp == 4) ? tq : 2 * tq + e;
                             const bool mine = (Gp == 4) ? (e == (g & 1)) : true;
                             if (mine && h < G && !*abort_flag)
-                                atomicAdd(&o_sm[h * D + ch], d[e + 2 * rr] - kCodeOffset * cs[g / GPS][e]);
+                                red_shared(&o_sm[h * D + ch], d[e + 2 * rr] - kCodeOffset * cs[g / GPS][e]);
                         }
                     }
 #pragma unroll
@@ -646,20 +717,11 @@ __global__ void __launch_bounds__(32 * (1 + kConsWarps * NTEAM), 1)
                 v += __shfl_xor_sync(0xffffffffu, v, 16);
                 const int h = (Gp == 4) ? tq : 2 * tq + e;
                 if (gid == 0 && h < G)
-                    atomicAdd(&l_sm[h], v);
+                    red_shared(&l_sm[h], v);
             }
         }
         consumer_sync(NCT);
         if (!*abort_flag) {
-            const float4* ws4 = reinterpret_cast<const float4*>(w_sm);
-            float* Wg = w.W + um.ref_row * Gp;
-            for (int x = tid; x < R * Gp / 4; x += NCT) {
-                const float4 v = ws4[x];
-                if (v.x != 0.0f) atomicAdd(Wg + 4 * x, v.x);
-                if (v.y != 0.0f) atomicAdd(Wg + 4 * x + 1, v.y);
-                if (v.z != 0.0f) atomicAdd(Wg + 4 * x + 2, v.z);
-                if (v.w != 0.0f) atomicAdd(Wg + 4 * x + 3, v.w);
-            }
             for (int x = tid; x < G * D; x += NCT)
                 atomicAdd(&w.O[static_cast<int64_t>(u) * Gp * D + x], o_sm[x]);
             if (tid < G)
@@ -672,6 +734,14 @@ __global__ void __launch_bounds__(32 * (1 + kConsWarps * NTEAM), 1)
         report(a.err, RKV_ERR_UNSUPPORTED);
     if (__any_sync(0xffffffffu, corrupt) && lane == 0)
         report(a.err, RKV_ERR_CORRUPT);
+    // the copies of the last stages land before the CTA may exit (only after an abort can
+    // one still be in flight here)
+    consumer_sync(NCT);
+    if (tid == 0) {
+        const int n = *issued;
+        for (int j = (n > nst ? n - nst : 0); j < n; ++j)
+            mbar_wait_sleep(&full[j % nst], (j / nst) & 1, zero_flag);
+    }
 }
 
 // ==== 3. reference tokens, reference weights, output =========================================
@@ -680,13 +750,13 @@ template <int Gp>
 __global__ void __launch_bounds__(256) mma_refs_kernel(const CacheArgs a, void* __restrict__ out, const MmaWs w)
 {
     constexpr int D = 128;
+    constexpr int RQ = kRefChunk / 4;      // references per thread quarter
     __shared__ float wt[kRefChunk][Gp];
     __shared__ float red[4][Gp][D];
     __shared__ float lred[Gp];
-    __shared__ float msm[Gp];
+    __shared__ uint32_t key[Gp];
     __shared__ int last;
     const int u = blockIdx.y, ch = blockIdx.x, tid = threadIdx.x;
-    grid_dep_wait();   // weights and partial sums of the tokens kernel
     const UnitMeta um = a.units[u];
     const int R = um.R;
     const int nch = max(1, (R + kRefChunk - 1) / kRefChunk);
@@ -695,10 +765,21 @@ __global__ void __launch_bounds__(256) mma_refs_kernel(const CacheArgs a, void* 
     const int G = a.G;
     const int kvh = u - um.seq * a.Hkv;
     const int r0 = ch * kRefChunk, r1 = min(R, r0 + kRefChunk);
+    const int cp = tid & 63, qq = tid >> 6;
+    // the reference V rows do not depend on the earlier kernels: fetch them first
+    uint32_t rv[RQ];
+#pragma unroll
+    for (int rr = 0; rr < RQ; ++rr) {
+        const int r = r0 + qq * RQ + rr;
+        rv[rr] = (r < r1) ? *reinterpret_cast<const uint32_t*>(a.ref_V + (um.ref_row + r) * D + 2 * cp) : 0u;
+    }
     if (tid < Gp) {
         lred[tid] = 0.0f;
-        msm[tid] = unit_max<Gp>(w, u, R, tid);
+        key[tid] = 0u;
     }
+    grid_dep_wait();   // weights and partial sums of the tokens kernel
+    __syncthreads();
+    unit_max_fold<Gp>(w, u, R, tid, 256, key);
     __syncthreads();
     // weight of reference r: its own softmax term p_r plus w_r from the tokens that chose it
     for (int x = tid; x < kRefChunk * Gp; x += 256) {
@@ -706,31 +787,27 @@ __global__ void __launch_bounds__(256) mma_refs_kernel(const CacheArgs a, void* 
         float v = 0.0f;
         if (r < r1 && h < G) {
             const int64_t e = (um.ref_row + r) * Gp + h;
-            const float pj = exp2f(w.s_tab[e] - msm[h]);
+            const float pj = exp2f(w.s_tab[e] - unit_m(key, h));
             v = w.W[e] + pj;
-            atomicAdd(&lred[h], pj);
+            red_shared(&lred[h], pj);
         }
         wt[x / Gp][h] = v;
     }
     __syncthreads();
     // sum_r wt[r][h] refV[r][c]: thread (channel pair, quarter of the chunk)
     {
-        const int cp = tid & 63, qq = tid >> 6;
         float acc[Gp][2];
 #pragma unroll
         for (int h = 0; h < Gp; ++h)
             acc[h][0] = acc[h][1] = 0.0f;
-#pragma unroll 4
-        for (int rr = 0; rr < kRefChunk / 4; ++rr) {
-            const int r = r0 + qq * (kRefChunk / 4) + rr;
-            if (r < r1) {
-                const uint32_t v = *reinterpret_cast<const uint32_t*>(a.ref_V + (um.ref_row + r) * D + 2 * cp);
-                const float x0 = bf16_bits_to_f32(v & 0xffffu), x1 = bf16_bits_to_f32(v >> 16);
 #pragma unroll
-                for (int h = 0; h < Gp; ++h) {
-                    acc[h][0] = fmaf(wt[r - r0][h], x0, acc[h][0]);
-                    acc[h][1] = fmaf(wt[r - r0][h], x1, acc[h][1]);
-                }
+        for (int rr = 0; rr < RQ; ++rr) {
+            const float x0 = bf16_bits_to_f32(rv[rr] & 0xffffu), x1 = bf16_bits_to_f32(rv[rr] >> 16);
+            const float* wr = wt[qq * RQ + rr];
+#pragma unroll
+            for (int h = 0; h < Gp; ++h) {
+                acc[h][0] = fmaf(wr[h], x0, acc[h][0]);
+                acc[h][1] = fmaf(wr[h], x1, acc[h][1]);
             }
         }
 #pragma unroll
@@ -769,8 +846,6 @@ __global__ void __launch_bounds__(256) mma_refs_kernel(const CacheArgs a, void* 
 
 // ==== host side ==============================================================================
 
-constexpr int kTeams = 1;
-
 int heads_padded(int G) { return G <= 4 ? 4 : 8; }
 
 // Opt-in shared memory per block on sm_100 (227 KB); a constant so that workspace sizes do
@@ -781,11 +856,13 @@ constexpr int kSmemOptin = 232448;
 int tok_stages(const CacheArgs& a)
 {
     const int Gp = heads_padded(a.G);
-    const int fixed = TokLayout(Gp, kConsWarps * kTeams, a.max_refs, 0).total + 1024;
+    const int fixed = TokLayout(Gp, kConsWarps, a.max_refs, 0).total + 1024;
     const int avail = kSmemOptin - fixed;
     const int n = avail / kStageBytes;
     return n < 2 ? 0 : (n > 8 ? 8 : n);
 }
+
+constexpr int kMaxCta = 160;   // grid cap of the tokens kernel
 
 struct WsOffsets {
     uint64_t s_tab, W, mpart, O, L, cnt, end;
@@ -863,25 +940,19 @@ cudaError_t launch_gp(const CacheArgs& a, int64_t cmp_rows, const void* q, void*
     alignas(64) CUtensorMap mV;
     if (!code_map(enc, &mK, a.codes_K, cmp_rows) || !code_map(enc, &mV, a.codes_V, cmp_rows))
         return cudaErrorInvalidValue;
-    int dev = 0, sms = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e == cudaSuccess)
-        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess)
-        return e;
     const dim3 rgrid(w.n_chunk, a.n_units);
     mma_scores_kernel<Gp><<<rgrid, 256, 0, st>>>(a, q, w);
-    e = cudaGetLastError();
+    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;
     if (w.n_tiles > 0) {
-        auto kern = mma_tokens_kernel<Gp, kTeams>;
-        const size_t smem = TokLayout(Gp, kConsWarps * kTeams, a.max_refs, nst).total + 1024;
+        auto kern = (a.k <= 4) ? mma_tokens_kernel<Gp, 4> : mma_tokens_kernel<Gp, 8>;
+        const size_t smem = TokLayout(Gp, kConsWarps, a.max_refs, nst).total + 1024;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
         if (e != cudaSuccess)
             return e;
-        const int grid = w.n_tiles < sms ? w.n_tiles : sms;
-        e = launch_pdl(kern, dim3(grid), dim3(32 * (1 + kConsWarps * kTeams)), smem, st, mK, mV, a, q, w, nst);
+        const int grid = w.n_cta;
+        e = launch_pdl(kern, dim3(grid), dim3(32 * kConsWarps), smem, st, mK, mV, a, q, w, nst);
         if (e != cudaSuccess)
             return e;
     }
@@ -912,6 +983,15 @@ cudaError_t launch_decode_mma(const CacheArgs& a, int64_t ref_rows, int64_t cmp_
     w.cnt = reinterpret_cast<uint32_t*>(base + o.cnt);
     w.n_chunk = (a.max_refs + kRefChunk - 1) / kRefChunk > 0 ? (a.max_refs + kRefChunk - 1) / kRefChunk : 1;
     w.n_tiles = static_cast<int>(cmp_rows / kTok);
+    {
+        int dev = 0, sms = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e == cudaSuccess)
+            e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess)
+            return e;
+        w.n_cta = std::min(std::min(sms, kMaxCta), std::max(w.n_tiles, 1));
+    }
     w.cK = static_cast<float>(1.4426950408889634 / std::sqrt(128.0));
     const int nst = tok_stages(a);
     if (nst < 2)

@@ -85,6 +85,32 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     return true;
 }
 
+// mbar_wait with a suspend-time hint: a waiting thread sleeps in the barrier instead of
+// polling (same time limit and abort flag).
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, volatile int* abort)
+{
+    uint64_t t0 = 0;
+    for (;;) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(smem_addr(bar)), "r"(parity), "r"(1000000u)
+            : "memory");
+        if (ok)
+            return true;
+        if (*abort)
+            return false;
+        const uint64_t now = global_ns();
+        if (t0 == 0)
+            t0 = now;
+        else if (now - t0 > kWaitNs)
+            return false;
+    }
+}
+
 // 2D tiled TMA load (no multicast) into shared memory, completion counted on bar.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar)
 {
