@@ -172,99 +172,89 @@ namespace {
 // ==== 1. reference scores ==================================================================
 
 template <int Gp>
-__global__ void __launch_bounds__(256) mma_scores_kernel(const CacheArgs a, const void* __restrict__ q, const MmaWs w)
+__global__ void __launch_bounds__(128) mma_scores_kernel(const CacheArgs a, const void* __restrict__ q, const MmaWs w)
 {
+    // s[r][h] = cK * (refK_r . q_h) as m16n8k16 MMAs: one warp per 16 references, columns are
+    // the (up to 8) q-heads.  The k-slot -> channel map gives lane tq the 32 channels
+    // 32 tq .. 32 tq + 31 in every k-block (k-block kb, slots 2tq, 2tq+1 -> channels
+    // 32 tq + 4 kb + {0, 1}; slots 2tq+8, 2tq+9 -> + {2, 3}), so A and B fragments are
+    // four 16-byte loads of a row each.
     grid_dep_launch();
     constexpr int D = 128;
-    __shared__ float qs[Gp][D];
-    __shared__ float wmax[8][Gp];
+    __shared__ float wmax[4][Gp];
     const int u = blockIdx.y, ch = blockIdx.x;
     const UnitMeta um = a.units[u];
     const int kvh = u - um.seq * a.Hkv;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int gid = lane >> 2, tq = lane & 3;
     const int R = um.R;
     const int r0 = ch * kRefChunk;
     const int r1 = min(R, r0 + kRefChunk);
+    const int rw = r0 + warp * 16;               // first reference of this warp
+    // A rows gid and gid + 8 (zero past the unit), B column gid (zero past the group)
+    uint4 ar[2][4], bq[4];
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+        const int r = rw + gid + 8 * rr;
+        const uint4* src = reinterpret_cast<const uint4*>(a.ref_K + (um.ref_row + r) * D + 32 * tq);
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+            ar[rr][x] = (r < r1) ? src[x] : make_uint4(0u, 0u, 0u, 0u);
+    }
+    {
+        const uint4* src = reinterpret_cast<const uint4*>(
+            static_cast<const uint16_t*>(q) + (static_cast<int64_t>(um.seq) * a.Hq + kvh * a.G + gid) * D + 32 * tq);
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+            bq[x] = (gid < a.G) ? src[x] : make_uint4(0u, 0u, 0u, 0u);
+    }
     if (ch == 0) {
-        for (int i = tid; i < Gp * D; i += 256)
+        for (int i = tid; i < Gp * D; i += 128)
             w.O[static_cast<int64_t>(u) * Gp * D + i] = 0.0f;
         if (tid < Gp)
             w.L[u * Gp + tid] = 0.0f;
         if (tid == 0)
             w.cnt[u] = 0u;
     }
-    // eight lanes per reference row, sixteen channels each, two rows per lane group; the
-    // reference rows are fetched before the query is staged
-    const int grp = tid >> 3, sub = tid & 7;
-    static_assert(kRefChunk == 64, "two passes of 32 rows");
-    uint4 rk[2][2];
-#pragma unroll
-    for (int ps = 0; ps < 2; ++ps) {
-        const int r = r0 + grp + 32 * ps;
-        if (r < r1) {
-            const uint16_t* rp = a.ref_K + (um.ref_row + r) * D + sub * 16;
-            rk[ps][0] = *reinterpret_cast<const uint4*>(rp);
-            rk[ps][1] = *reinterpret_cast<const uint4*>(rp + 8);
-        } else {
-            rk[ps][0] = rk[ps][1] = make_uint4(0u, 0u, 0u, 0u);
-        }
-    }
-    for (int i = tid; i < (r1 - r0) * Gp; i += 256)
+    for (int i = tid; i < (r1 - r0) * Gp; i += 128)
         w.W[(um.ref_row + r0) * Gp + i] = 0.0f;
-    for (int i = tid; i < Gp * D; i += 256) {
-        const int h = i / D, c = i % D;
-        qs[h][c] = (h < a.G) ? bf16_bits_to_f32(static_cast<const uint16_t*>(
-                                   q)[(static_cast<int64_t>(um.seq) * a.Hq + kvh * a.G + h) * D + c]) * w.cK
-                             : 0.0f;
-    }
-    __syncthreads();
-    float mloc[Gp];
+    float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    auto word = [](const uint4 (&v)[4], int i) {
+        const uint4 x = v[i >> 2];
+        return (i & 3) == 0 ? x.x : (i & 3) == 1 ? x.y : (i & 3) == 2 ? x.z : x.w;
+    };
 #pragma unroll
-    for (int h = 0; h < Gp; ++h)
-        mloc[h] = -FLT_MAX;
+    for (int kb = 0; kb < 8; ++kb)
+        mma_bf16(d, word(ar[0], 2 * kb), word(ar[1], 2 * kb), word(ar[0], 2 * kb + 1), word(ar[1], 2 * kb + 1),
+                 word(bq, 2 * kb), word(bq, 2 * kb + 1));
+    // d: rows gid / gid + 8, heads 2tq / 2tq + 1
+    float mloc[2] = {-FLT_MAX, -FLT_MAX};
 #pragma unroll
-    for (int ps = 0; ps < 2; ++ps) {
-        const int r = r0 + grp + 32 * ps;
-        const bool ok = r < r1;
-        float x[16];
-        const uint32_t ww[8] = {rk[ps][0].x, rk[ps][0].y, rk[ps][0].z, rk[ps][0].w,
-                                rk[ps][1].x, rk[ps][1].y, rk[ps][1].z, rk[ps][1].w};
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            x[2 * i] = bf16_bits_to_f32(ww[i] & 0xffffu);
-            x[2 * i + 1] = bf16_bits_to_f32(ww[i] >> 16);
-        }
-        float sv[Gp];
-#pragma unroll
-        for (int h = 0; h < Gp; ++h) {
-            float d = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-                d = fmaf(qs[h][sub * 16 + i], x[i], d);
-            d += __shfl_xor_sync(0xffffffffu, d, 1);
-            d += __shfl_xor_sync(0xffffffffu, d, 2);
-            d += __shfl_xor_sync(0xffffffffu, d, 4);
-            sv[h] = d;
-            if (ok && h < a.G)
-                mloc[h] = fmaxf(mloc[h], d);
-        }
-        if (ok && sub == 0) {
-            float* dst = w.s_tab + (um.ref_row + r) * Gp;
-#pragma unroll
-            for (int h = 0; h < Gp; h += 4)
-                *reinterpret_cast<float4*>(dst + h) = make_float4(sv[h], sv[h + 1], sv[h + 2], sv[h + 3]);
+    for (int rr = 0; rr < 2; ++rr) {
+        const int r = rw + gid + 8 * rr;
+        const float s0 = d[2 * rr] * w.cK, s1 = d[2 * rr + 1] * w.cK;
+        if (r < r1) {
+            if (2 * tq < Gp)
+                *reinterpret_cast<float2*>(w.s_tab + (um.ref_row + r) * Gp + 2 * tq) = make_float2(s0, s1);
+            if (2 * tq < a.G)
+                mloc[0] = fmaxf(mloc[0], s0);
+            if (2 * tq + 1 < a.G)
+                mloc[1] = fmaxf(mloc[1], s1);
         }
     }
 #pragma unroll
-    for (int h = 0; h < Gp; ++h) {
-        const float v = warp_max(mloc[h]);
-        if ((tid & 31) == 0)
-            wmax[tid >> 5][h] = v;
+    for (int e = 0; e < 2; ++e) {
+        float v = mloc[e];
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+        if (gid == 0 && 2 * tq + e < Gp)
+            wmax[warp][2 * tq + e] = v;
     }
     __syncthreads();
     if (tid < Gp) {
         float v = -FLT_MAX;
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < 4; ++i)
             v = fmaxf(v, wmax[i][tid]);
         w.mpart[(static_cast<int64_t>(u) * w.n_chunk + ch) * Gp + tid] = v;
     }
@@ -293,16 +283,17 @@ __device__ __forceinline__ float unit_m(const uint32_t* key, int h)
 
 // Dynamic shared memory of the tokens kernel (byte offsets from a 1024-aligned base).
 struct TokLayout {
-    int stages, s_sm, o_sm, p_sm, q_sm, bar, misc, total;
+    int stages, s_sm, o_sm, p_sm, q_sm, bk_sm, bar, misc, total;
     __host__ __device__ TokLayout(int Gp, int ncons, int R_max, int nst)
     {
         auto up = [](int x) { return (x + 127) & ~127; };
         int off = 0;
         stages = off; off += nst * kStageBytes;
-        s_sm = off;   off += up(R_max * Gp * 4);
-        o_sm = off;   off += up(Gp * 128 * 4);
+        s_sm = off;   off += 2 * up(R_max * Gp * 4);      // two table buffers
+        o_sm = off;   off += up(ncons * Gp * 128 * 4);    // per-warp output partials
         p_sm = off;   off += up(ncons * kWarpTok * Gp * 4);
         q_sm = off;   off += up(Gp * 128 * 2);
+        bk_sm = off;  off += 8 * 2 * 8 * 16;     // K-side B operand, ldmatrix layout
         bar = off;    off += 2 * 8 * 8;
         misc = off;   off += up((6 * Gp + 4) * 4);
         total = off;
@@ -314,8 +305,8 @@ __device__ __forceinline__ void consumer_sync(int n_threads)
     asm volatile("bar.sync 1, %0;" ::"r"(n_threads) : "memory");
 }
 
-template <int Gp, int KK>
-__global__ void __launch_bounds__(32 * kConsWarps, 1)
+template <int Gp, int KK, int NTEAM>
+__global__ void __launch_bounds__(32 * kConsWarps * NTEAM, 1)
     mma_tokens_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       const CacheArgs a, const void* __restrict__ q, const MmaWs w, const int nst)
 {
@@ -323,18 +314,21 @@ __global__ void __launch_bounds__(32 * kConsWarps, 1)
     constexpr int GPS = 8 / Gp;           // scale groups sharing one set of eight MMA columns
     constexpr int NS = 4 / GPS;           // column sets
     constexpr int NH = Gp / 4;            // q-heads per thread in the softmax step
-    constexpr int NCT = kConsWarps * 32;
+    constexpr int NCT = kConsWarps * NTEAM * 32;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    const TokLayout L(Gp, kConsWarps, a.max_refs, nst);
+    const TokLayout L(Gp, kConsWarps * NTEAM, a.max_refs, nst);
     unsigned char* stages = sm + L.stages;
-    float* s_sm = reinterpret_cast<float*>(sm + L.s_sm);
+    float* s_buf = reinterpret_cast<float*>(sm + L.s_sm);
+    const int s_stride = ((a.max_refs * Gp * 4 + 127) & ~127) / 4;
     float* o_sm = reinterpret_cast<float*>(sm + L.o_sm);
     float* p_sm = reinterpret_cast<float*>(sm + L.p_sm);
     uint16_t* q_sm = reinterpret_cast<uint16_t*>(sm + L.q_sm);
+    uint16_t* bk_sm = reinterpret_cast<uint16_t*>(sm + L.bk_sm);
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + L.bar);
     int* done_cnt = reinterpret_cast<int*>(full + 8);        // warps finished with a stage
+    uint64_t* tbar = reinterpret_cast<uint64_t*>(done_cnt + 8);   // table buffer loaded
     float* qc_sm = reinterpret_cast<float*>(sm + L.misc);    // [4 groups][Gp]
     float* l_sm = qc_sm + 4 * Gp;
     uint32_t* key_sm = reinterpret_cast<uint32_t*>(l_sm + Gp);
@@ -368,6 +362,8 @@ __global__ void __launch_bounds__(32 * kConsWarps, 1)
             mbar_init(&full[s], 1);
             done_cnt[s] = 0;
         }
+        mbar_init(&tbar[0], 1);
+        mbar_init(&tbar[1], 1);
         *abort_flag = 0;
         *zero_flag = 0;
         fence_mbar_init();
@@ -383,7 +379,7 @@ __global__ void __launch_bounds__(32 * kConsWarps, 1)
     grid_dep_launch();   // the references kernel may be scheduled once every CTA runs
 
     // ---- consumer warps -----------------------------------------------------------------
-    const int wi = warp;
+    const int team = warp / kConsWarps, wi = warp % kConsWarps;
     const int gid = lane >> 2, tq = lane & 3;
     const int G = a.G;
     grid_dep_wait();   // reference scores, maxima and zeroed accumulators of the scores kernel
@@ -402,16 +398,39 @@ __global__ void __launch_bounds__(32 * kConsWarps, 1)
         }
         u = lo;
     }
+    // segments: the runs of this CTA's tiles that belong to one unit.  Their score tables
+    // are bulk-copied into two alternating buffers, the next one while the current is used.
+    auto unit_end = [&](int uu) {
+        const UnitMeta m = a.units[uu];
+        return static_cast<int>((m.cmp_row + ((m.C + kTok - 1) / kTok) * kTok) / kTok);
+    };
+    auto unit_at = [&](int uu, int T) {   // first unit from uu whose tiles reach past tile T
+        while (uu < a.n_units && T >= unit_end(uu))
+            ++uu;
+        return uu;
+    };
+    int tables_issued[2] = {0, 0};             // (thread 0)
+    auto load_table = [&](int buf, int uu) {   // one thread
+        ++tables_issued[buf];
+        const UnitMeta m = a.units[uu];
+        const uint32_t bytes = static_cast<uint32_t>(m.R * Gp * 4);
+        mbar_arrive_expect_tx(&tbar[buf], bytes);
+        if (bytes)
+            bulk_load(s_buf + buf * s_stride, w.s_tab + m.ref_row * Gp, bytes, &tbar[buf]);
+    };
+    u = unit_at(u, t_lo);
+    if (tid == 0 && t_lo < t_hi) {
+        load_table(0, u);
+        const int t1 = min(t_hi, unit_end(u));
+        if (t1 < t_hi)
+            load_table(1, unit_at(u, t1));
+    }
     bool overflow = false, corrupt = false;
-    int t = t_lo, i = 0;
+    int t = t_lo, i = 0, seg = 0;
     while (t < t_hi && u < a.n_units) {
         const UnitMeta um = a.units[u];
-        const int t_end = static_cast<int>((um.cmp_row + ((um.C + kTok - 1) / kTok) * kTok) / kTok);
-        if (t >= t_end) {
-            ++u;
-            continue;
-        }
-        const int seg_end = min(t_hi, t_end);
+        const int seg_end = min(t_hi, unit_end(u));
+        const float* s_sm = s_buf + (seg & 1) * s_stride;
         const int R = um.R;
         const int kvh = u - um.seq * a.Hkv;
 
@@ -425,28 +444,11 @@ __global__ void __launch_bounds__(32 * kConsWarps, 1)
             const int h = x / D, c = x % D;
             q_sm[x] = (h < G) ? static_cast<const uint16_t*>(q)[(static_cast<int64_t>(um.seq) * a.Hq + kvh * G + h) * D + c]
                               : static_cast<uint16_t>(0);
-            o_sm[x] = 0.0f;
         }
-        {
-            // eight float4 loads in flight per thread
-            const float4* src = reinterpret_cast<const float4*>(w.s_tab + um.ref_row * Gp);
-            float4* dst = reinterpret_cast<float4*>(s_sm);
-            const int n4 = R * Gp / 4;
-            for (int base = 0; base < n4; base += 8 * NCT) {
-                float4 tmp[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int x = base + j * NCT + tid;
-                    if (x < n4)
-                        tmp[j] = src[x];
-                }
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int x = base + j * NCT + tid;
-                    if (x < n4)
-                        dst[x] = tmp[j];
-                }
-            }
+        if (!*abort_flag && !mbar_wait_sleep(&tbar[seg & 1], (seg >> 1) & 1, abort_flag)) {
+            if (!*abort_flag)
+                report(a.err, RKV_ERR_TIMEOUT);
+            *abort_flag = 1;
         }
         consumer_sync(NCT);
         unit_max_fold<Gp>(w, u, R, tid, NCT, key_sm);
@@ -458,21 +460,20 @@ __global__ void __launch_bounds__(32 * kConsWarps, 1)
                 sum += bf16_bits_to_f32(q_sm[h * D + 32 * g + c]);
             qc_sm[g * Gp + h] = kCodeOffset * sum;
         }
-        consumer_sync(NCT);
-        // K-side B operand: column gid is (head gid / GPS, group residue gid % GPS); k-slot
+        // K-side B operand in the ldmatrix layout: matrix (k-block, half) holds rows n (the
+        // eight columns: head n / GPS, group residue n % GPS) of eight k-slots; the k-slot
         // order within a group follows the nibble order of the A fragments
-        uint32_t bk[8][2];
-        {
-            const int hcol = gid / GPS, gcol = gid % GPS;
-#pragma unroll
-            for (int kb = 0; kb < 8; ++kb) {
-                const int g = kb >> 1, sub = kb & 1;
-                const bool on = (g % GPS) == gcol && hcol < G;
-                const uint16_t* qr = q_sm + hcol * D + 32 * g + 8 * tq + 2 * sub;
-                bk[kb][0] = on ? (static_cast<uint32_t>(qr[0]) | (static_cast<uint32_t>(qr[4]) << 16)) : 0u;
-                bk[kb][1] = on ? (static_cast<uint32_t>(qr[1]) | (static_cast<uint32_t>(qr[5]) << 16)) : 0u;
-            }
+        for (int x = tid; x < 8 * 2 * 8 * 8; x += NCT) {
+            const int kb = x >> 7, half = (x >> 6) & 1, n = (x >> 3) & 7, slot = x & 7;
+            const int g = kb >> 1, sub = kb & 1, tq2 = slot >> 1, e = slot & 1;
+            const int nib = 2 * sub + half + 4 * e;
+            const int h = n / GPS;
+            const bool on = (g % GPS) == (n % GPS) && h < G;
+            bk_sm[x] = on ? q_sm[h * D + 32 * g + 8 * tq2 + nib] : static_cast<uint16_t>(0);
         }
+        consumer_sync(NCT);
+        // ldmatrix row address of this lane for the K-side B operand of group 0 (+512 B per group)
+        const uint32_t bk_base = smem_addr(bk_sm) + static_cast<uint32_t>(((lane >> 3) * 8 + (lane & 7)) * 16);
         float m_h[NH], qc_h[4][NH], l_acc[NH];
 #pragma unroll
         for (int e = 0; e < NH; ++e) {
@@ -496,6 +497,8 @@ __global__ void __launch_bounds__(32 * kConsWarps, 1)
 
         // ---- the unit's tiles, 16 tokens per warp ---------------------------------------
         for (; t < seg_end; ++t, ++i) {
+            if (NTEAM > 1 && (i % NTEAM) != team)
+                continue;
             const int s = i % nst;
             if (!*abort_flag && !mbar_wait_sleep(&full[s], (i / nst) & 1, abort_flag)) {
                 if (!*abort_flag)
@@ -512,22 +515,23 @@ __global__ void __launch_bounds__(32 * kConsWarps, 1)
                 const int tok0 = static_cast<int>(static_cast<int64_t>(t) * kTok - um.cmp_row) + rb;
                 float* pw = p_sm + warp * kWarpTok * Gp;
 
-                // K side: D[token][column set] over the 128 channels, one MMA per 16 channels
+                // K side: D[token][column] per scale group, one MMA per 16 channels
                 uint32_t wk0[4], wk1[4];
                 ldsm_x4(stK + sw64(rb + (lane & 7), lane >> 3), wk0);
                 ldsm_x4(stK + sw64(rb + 8 + (lane & 7), lane >> 3), wk1);
-                float dk[NS][4];
+                float dk[4][4];
 #pragma unroll
-                for (int x = 0; x < NS; ++x)
-                    dk[x][0] = dk[x][1] = dk[x][2] = dk[x][3] = 0.0f;
-#pragma unroll
-                for (int g = 0; g < 4; ++g)
+                for (int g = 0; g < 4; ++g) {
+                    uint32_t bq[4];
+                    ldsm_x4(bk_base + g * 512, bq);
+                    dk[g][0] = dk[g][1] = dk[g][2] = dk[g][3] = 0.0f;
 #pragma unroll
                     for (int sub = 0; sub < 2; ++sub) {
                         const int sh = 8 * sub;
-                        mma_bf16(dk[g / GPS], nib2(wk0[g] >> sh), nib2(wk1[g] >> sh), nib2(wk0[g] >> (sh + 4)),
-                                 nib2(wk1[g] >> (sh + 4)), bk[2 * g + sub][0], bk[2 * g + sub][1]);
+                        mma_bf16(dk[g], nib2(wk0[g] >> sh), nib2(wk1[g] >> sh), nib2(wk0[g] >> (sh + 4)),
+                                 nib2(wk1[g] >> (sh + 4)), bq[2 * sub], bq[2 * sub + 1]);
                     }
+                }
 
                 // softmax of this thread's two tokens (rows gid, gid + 8) and NH heads
 #pragma unroll
@@ -581,7 +585,7 @@ __global__ void __launch_bounds__(32 * kConsWarps, 1)
                         float acc = 0.0f;
 #pragma unroll
                         for (int g = 0; g < 4; ++g) {
-                            const float raw = (Gp == 4) ? dk[g >> 1][(g & 1) + 2 * rr] : dk[g][e + 2 * rr];
+                            const float raw = (Gp == 4) ? dk[g][(g & 1) + 2 * rr] : dk[g][e + 2 * rr];
                             acc = fmaf(sk[g], raw - qc_h[g][e], acc);
                         }
                         const float logit = fmaf(w.cK, acc, sref[e] * rk);
@@ -705,8 +709,8 @@ __global__ void __launch_bounds__(32 * kConsWarps, 1)
                             // Gp 4: column 2tq + e is (head tq, group residue e); Gp 8: head 2tq + e
                             const int h = (Gp == 4) ? tq : 2 * tq + e;
                             const bool mine = (Gp == 4) ? (e == (g & 1)) : true;
-                            if (mine && h < G && !*abort_flag)
-                                red_shared(&o_sm[h * D + ch], d[e + 2 * rr] - kCodeOffset * cs[g / GPS][e]);
+                            if (mine)
+                                o_sm[(warp * Gp + h) * D + ch] = d[e + 2 * rr] - kCodeOffset * cs[g / GPS][e];
                         }
                     }
 #pragma unroll
@@ -721,14 +725,29 @@ __global__ void __launch_bounds__(32 * kConsWarps, 1)
             }
         }
         consumer_sync(NCT);
+        // the table buffer of this segment is free: the segment after next loads into it
+        if (tid == 0 && seg_end < t_hi) {
+            const int u1 = unit_at(u, seg_end);
+            const int t2 = min(t_hi, unit_end(u1));
+            if (t2 < t_hi && !*abort_flag) {
+                fence_proxy_async_smem();
+                load_table(seg & 1, unit_at(u1, t2));
+            }
+        }
         if (!*abort_flag) {
-            for (int x = tid; x < G * D; x += NCT)
-                atomicAdd(&w.O[static_cast<int64_t>(u) * Gp * D + x], o_sm[x]);
+            for (int x = tid; x < G * D; x += NCT) {
+                float v = 0.0f;
+#pragma unroll 4
+                for (int wv = 0; wv < kConsWarps * NTEAM; ++wv)
+                    v += o_sm[wv * Gp * D + x];
+                atomicAdd(&w.O[static_cast<int64_t>(u) * Gp * D + x], v);
+            }
             if (tid < G)
                 atomicAdd(&w.L[u * Gp + tid], l_sm[tid]);
         }
         t = seg_end;
-        ++u;
+        u = unit_at(u, t);
+        ++seg;
     }
     if (__any_sync(0xffffffffu, overflow) && lane == 0)
         report(a.err, RKV_ERR_UNSUPPORTED);
@@ -741,6 +760,9 @@ __global__ void __launch_bounds__(32 * kConsWarps, 1)
         const int n = *issued;
         for (int j = (n > nst ? n - nst : 0); j < n; ++j)
             mbar_wait_sleep(&full[j % nst], (j / nst) & 1, zero_flag);
+        for (int bf = 0; bf < 2; ++bf)
+            if (tables_issued[bf] > 0)
+                mbar_wait_sleep(&tbar[bf], (tables_issued[bf] - 1) & 1, zero_flag);
     }
 }
 
@@ -846,6 +868,8 @@ __global__ void __launch_bounds__(256) mma_refs_kernel(const CacheArgs a, void* 
 
 // ==== host side ==============================================================================
 
+constexpr int kTeams = 2;      // warp teams of the tokens kernel (each takes every other stage)
+
 int heads_padded(int G) { return G <= 4 ? 4 : 8; }
 
 // Opt-in shared memory per block on sm_100 (227 KB); a constant so that workspace sizes do
@@ -856,7 +880,7 @@ constexpr int kSmemOptin = 232448;
 int tok_stages(const CacheArgs& a)
 {
     const int Gp = heads_padded(a.G);
-    const int fixed = TokLayout(Gp, kConsWarps, a.max_refs, 0).total + 1024;
+    const int fixed = TokLayout(Gp, kConsWarps * kTeams, a.max_refs, 0).total + 1024;
     const int avail = kSmemOptin - fixed;
     const int n = avail / kStageBytes;
     return n < 2 ? 0 : (n > 8 ? 8 : n);
@@ -941,18 +965,18 @@ cudaError_t launch_gp(const CacheArgs& a, int64_t cmp_rows, const void* q, void*
     if (!code_map(enc, &mK, a.codes_K, cmp_rows) || !code_map(enc, &mV, a.codes_V, cmp_rows))
         return cudaErrorInvalidValue;
     const dim3 rgrid(w.n_chunk, a.n_units);
-    mma_scores_kernel<Gp><<<rgrid, 256, 0, st>>>(a, q, w);
+    mma_scores_kernel<Gp><<<rgrid, 128, 0, st>>>(a, q, w);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;
     if (w.n_tiles > 0) {
-        auto kern = (a.k <= 4) ? mma_tokens_kernel<Gp, 4> : mma_tokens_kernel<Gp, 8>;
-        const size_t smem = TokLayout(Gp, kConsWarps, a.max_refs, nst).total + 1024;
+        auto kern = (a.k <= 4) ? mma_tokens_kernel<Gp, 4, kTeams> : mma_tokens_kernel<Gp, 8, kTeams>;
+        const size_t smem = TokLayout(Gp, kConsWarps * kTeams, a.max_refs, nst).total + 1024;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
         if (e != cudaSuccess)
             return e;
         const int grid = w.n_cta;
-        e = launch_pdl(kern, dim3(grid), dim3(32 * kConsWarps), smem, st, mK, mV, a, q, w, nst);
+        e = launch_pdl(kern, dim3(grid), dim3(32 * kConsWarps * kTeams), smem, st, mK, mV, a, q, w, nst);
         if (e != cudaSuccess)
             return e;
     }
