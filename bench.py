@@ -32,7 +32,7 @@ import numpy as np  # noqa: E402
 METRIC = "decode-attn µs/step & HBM GB/s vs roofline; compress Mtok/s; 1 B200"
 WORKLOAD = "llama3_8b_layer"
 # kernels launched per step, by stage
-LAUNCHES = {"build_refs": 1, "search": 1, "encode": 1, "decode": 2, "reconstruct": 1}
+LAUNCHES = {"build_refs": 1, "search": 1, "encode": 1, "decode": 3, "reconstruct": 1}
 RECON_ROWS = 256
 
 
@@ -415,7 +415,7 @@ def run_ours(args, rank, world, local_rank):
         traffic = _traffic("encode", ["long_context_attention_rkv_b200/csrc/kernels_encode.cu"])
     else:
         peak, bound, ach, unit = peaks["hbm"], "hbm", decode_gbs, "GB/s"
-        traffic = _traffic("decode", ["long_context_attention_rkv_b200/csrc/kernels_decode_direct.cu"])
+        traffic = _traffic("decode", ["long_context_attention_rkv_b200/csrc/kernels_decode_mma.cu"])
     roofline = {"kernel": dominant, "bound": bound, "achieved": ach, "peak": peak, "unit": unit,
                 "frac": ach / peak, "traffic": traffic, "peak_source": peaks["source"]}
 
