@@ -3,8 +3,10 @@
 // KV - KV_R; news page "New KV Cache Compression Method Cuts Long-Context
 // Inference Costs by 85%", "How ResidualKV Works": quantized residual codes).
 //
-// Eight lanes per compressed token (four tokens per warp); a lane owns D/8
-// consecutive channels (16 for D = 128), i.e. half of a 32-channel group.
+// Sixteen lanes per compressed token at D = 128 (eight at D = 64; two or four tokens
+// per warp); a lane owns 8 consecutive channels, a quarter of a 32-channel group.
+// Short per-lane state keeps four 256-thread blocks resident per SM: the kernel is
+// bound by the latency of its gathers of reference rows, so resident warps matter.
 //  1. Final top-k.  The search handed over its kc best candidates by
 //     t = k.r - |r|^2/2 from fp32 accumulation.  With
 //     delta = 2^-16 (|k|^2 + max|r|^2) (four times the worst-case error of a
@@ -30,25 +32,24 @@ namespace rkv {
 namespace {
 
 constexpr int kWarps = 8;
-constexpr int kLPT = 8;                  // lanes per token
-constexpr int kTPW = 32 / kLPT;          // tokens per warp
+constexpr int kCpl128 = 8;   // channels per lane at D = 128 (16 lanes per token)
 
-__device__ __forceinline__ unsigned group_mask(int lane) { return 0xffu << (lane & ~(kLPT - 1)); }
-
-// Sum over the 8 lanes of a token group.
+// Sum over the LPT lanes of a token group.
+template <int LPT>
 __device__ __forceinline__ float tsum(float v)
 {
-    v += __shfl_xor_sync(0xffffffffu, v, 1);
-    v += __shfl_xor_sync(0xffffffffu, v, 2);
-    v += __shfl_xor_sync(0xffffffffu, v, 4);
+#pragma unroll
+    for (int o = 1; o < LPT; o <<= 1)
+        v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
 }
 
+template <int LPT>
 __device__ __forceinline__ float tmax(float v)
 {
-    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
-    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
-    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+#pragma unroll
+    for (int o = 1; o < LPT; o <<= 1)
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
     return v;
 }
 
@@ -165,13 +166,20 @@ __device__ __forceinline__ void quantise_store(const float (&x)[CPL], const floa
         scale_row[sub / LPG] = sbits;
 }
 
-template <int CPL, int KC>
-__global__ void __launch_bounds__(kWarps * 32, 2) encode_kernel(CacheArgs a, const void* __restrict__ K,
+// Resident blocks per SM the register budget is set for: four (64 registers) where the code
+// fits without spills, two otherwise.
+template <int KC, int LPT>
+constexpr int encode_min_blocks() { return (LPT == 16 && KC <= 12) ? 4 : 2; }
+
+template <int CPL, int KC, int LPT>
+__global__ void __launch_bounds__(kWarps * 32, encode_min_blocks<KC, LPT>()) encode_kernel(CacheArgs a, const void* __restrict__ K,
                                                              const void* __restrict__ V,
                                                              const uint16_t* __restrict__ cand_idx,
                                                              const float* __restrict__ cand_t)
 {
-    constexpr int D = CPL * kLPT;
+    constexpr int D = CPL * LPT;
+    constexpr int kLPT = LPT;                // lanes per token
+    constexpr int kTPW = 32 / kLPT;          // tokens per warp
     constexpr int KM = KC - 4;               // largest k served by this candidate width
     __shared__ float xs[kWarps][kTPW][D];
     __shared__ int sorted[kWarps][kTPW][KM];
@@ -241,13 +249,13 @@ __global__ void __launch_bounds__(kWarps * 32, 2) encode_kernel(CacheArgs a, con
 #pragma unroll
     for (int i = 0; i < CPL; ++i)
         xx = fmaf(xk[i], xk[i], xx);
-    xx = tsum(xx);
+    xx = tsum<kLPT>(xx);
     float hm = 0.0f;
 #pragma unroll
     for (int r = 0; r < PER; ++r)
         if (r * kLPT + sub < nvalid)
             hm = fmaxf(hm, a.ref_hn[um.ref_row + co[r]]);
-    hm = tmax(hm);
+    hm = tmax<kLPT>(hm);
     const float delta = ldexpf(xx + 2.0f * hm, -16);
     const float tk = slot_t(k - 1);
     const float tk1 = slot_t(k);
@@ -281,7 +289,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) encode_kernel(CacheArgs a, con
                 float d = 0.0f;
                 if (need) {
                     const int o = in[i] ? ords[i] : 0;
-                    d = tsum(part_dist<CPL>(xk, a.ref_K + (um.ref_row + o) * D + sub * CPL));
+                    d = tsum<kLPT>(part_dist<CPL>(xk, a.ref_K + (um.ref_row + o) * D + sub * CPL));
                 }
                 dist[i] = d;
             }
@@ -441,16 +449,16 @@ __global__ void __launch_bounds__(kWarps * 32, 2) encode_kernel(CacheArgs a, con
                         a.err);
 }
 
-template <int CPL>
+template <int CPL, int LPT>
 cudaError_t launch_cpl(const CacheArgs& a, int max_C, const void* K, const void* V, const uint16_t* ci,
                        const float* ct, cudaStream_t st)
 {
-    const int per_block = kWarps * kTPW;
+    const int per_block = kWarps * (32 / LPT);
     const dim3 grid((max_C + per_block - 1) / per_block, a.n_units);
     switch (a.kc) {
-    case 8: encode_kernel<CPL, 8><<<grid, kWarps * 32, 0, st>>>(a, K, V, ci, ct); break;
-    case 12: encode_kernel<CPL, 12><<<grid, kWarps * 32, 0, st>>>(a, K, V, ci, ct); break;
-    default: encode_kernel<CPL, 20><<<grid, kWarps * 32, 0, st>>>(a, K, V, ci, ct); break;
+    case 8: encode_kernel<CPL, 8, LPT><<<grid, kWarps * 32, 0, st>>>(a, K, V, ci, ct); break;
+    case 12: encode_kernel<CPL, 12, LPT><<<grid, kWarps * 32, 0, st>>>(a, K, V, ci, ct); break;
+    default: encode_kernel<CPL, 20, LPT><<<grid, kWarps * 32, 0, st>>>(a, K, V, ci, ct); break;
     }
     return cudaGetLastError();
 }
@@ -462,8 +470,8 @@ cudaError_t launch_encode(const CacheArgs& a, int max_C, const void* K, const vo
 {
     if (max_C <= 0)
         return cudaSuccess;
-    return (a.D == 128) ? launch_cpl<16>(a, max_C, K, V, cand_idx, cand_t, st)
-                        : launch_cpl<8>(a, max_C, K, V, cand_idx, cand_t, st);
+    return (a.D == 128) ? launch_cpl<kCpl128, 128 / kCpl128>(a, max_C, K, V, cand_idx, cand_t, st)
+                        : launch_cpl<8, 8>(a, max_C, K, V, cand_idx, cand_t, st);
 }
 
 }  // namespace rkv
