@@ -266,10 +266,18 @@ __global__ void __launch_bounds__(128) mma_scores_kernel(const CacheArgs a, cons
 template <int Gp>
 __device__ __forceinline__ void unit_max_fold(const MmaWs& w, int u, int R, int tid, int nthreads, uint32_t* key)
 {
+    // entry x holds head x % Gp: lanes 0 .. Gp-1 of each warp fold their lane classes
     const int n = ((R + kRefChunk - 1) / kRefChunk) * Gp;
     const float* src = w.mpart + static_cast<int64_t>(u) * w.n_chunk * Gp;
-    for (int x = tid; x < n; x += nthreads)
-        atomicMax(&key[x % Gp], fkey(src[x]));
+    for (int base = 0; base < n; base += nthreads) {
+        const int x = base + tid;
+        uint32_t k = (x < n) ? fkey(__ldcg(src + x)) : 0u;
+#pragma unroll
+        for (int o = Gp; o < 32; o <<= 1)
+            k = max(k, __shfl_xor_sync(0xffffffffu, k, o));
+        if ((tid & 31) < Gp && k != 0u)
+            atomicMax(&key[tid % Gp], k);
+    }
 }
 
 __device__ __forceinline__ float unit_m(const uint32_t* key, int h)
@@ -376,13 +384,16 @@ __global__ void __launch_bounds__(32 * kConsWarps * NTEAM, 1)
         *issued = n0;
     }
     __syncthreads();
-    grid_dep_launch();   // the references kernel may be scheduled once every CTA runs
 
     // ---- consumer warps -----------------------------------------------------------------
     const int team = warp / kConsWarps, wi = warp % kConsWarps;
     const int gid = lane >> 2, tq = lane & 3;
     const int G = a.G;
     grid_dep_wait();   // reference scores, maxima and zeroed accumulators of the scores kernel
+    // The references kernel may be scheduled once every CTA has passed this wait: the scores
+    // kernel has then completed, so the references kernel may read its outputs (through L2)
+    // before waiting for this one.
+    grid_dep_launch();
 
     // unit of the first tile: the last unit whose rows start at or before it
     int u = 0;
@@ -788,32 +799,53 @@ __global__ void __launch_bounds__(256) mma_refs_kernel(const CacheArgs a, void* 
     const int kvh = u - um.seq * a.Hkv;
     const int r0 = ch * kRefChunk, r1 = min(R, r0 + kRefChunk);
     const int cp = tid & 63, qq = tid >> 6;
-    // the reference V rows do not depend on the earlier kernels: fetch them first
+    // Before the wait on the tokens kernel: the reference V rows, and what depends only on the
+    // scores kernel (complete once this kernel runs; read through L2): the common offsets,
+    // the reference tokens' own terms p_r and their sum.
     uint32_t rv[RQ];
 #pragma unroll
     for (int rr = 0; rr < RQ; ++rr) {
         const int r = r0 + qq * RQ + rr;
         rv[rr] = (r < r1) ? *reinterpret_cast<const uint32_t*>(a.ref_V + (um.ref_row + r) * D + 2 * cp) : 0u;
     }
-    if (tid < Gp) {
-        lred[tid] = 0.0f;
+    if (tid < Gp)
         key[tid] = 0u;
-    }
-    grid_dep_wait();   // weights and partial sums of the tokens kernel
     __syncthreads();
     unit_max_fold<Gp>(w, u, R, tid, 256, key);
     __syncthreads();
-    // weight of reference r: its own softmax term p_r plus w_r from the tokens that chose it
-    for (int x = tid; x < kRefChunk * Gp; x += 256) {
+    float pj[kRefChunk * Gp / 256 > 0 ? kRefChunk * Gp / 256 : 1];
+    constexpr int PJ = kRefChunk * Gp / 256;
+    float lsum = 0.0f;
+#pragma unroll
+    for (int z = 0; z < PJ; ++z) {
+        const int x = tid + 256 * z;
         const int r = r0 + x / Gp, h = x % Gp;
         float v = 0.0f;
-        if (r < r1 && h < G) {
-            const int64_t e = (um.ref_row + r) * Gp + h;
-            const float pj = exp2f(w.s_tab[e] - unit_m(key, h));
-            v = w.W[e] + pj;
-            red_shared(&lred[h], pj);
-        }
-        wt[x / Gp][h] = v;
+        if (r < r1 && h < G)
+            v = exp2f(__ldcg(w.s_tab + (um.ref_row + r) * Gp + h) - unit_m(key, h));
+        pj[z] = v;
+        lsum += v;
+    }
+    // per-head sums: entry x holds head x % Gp (256 % Gp == 0)
+#pragma unroll
+    for (int o = Gp; o < 32; o <<= 1)
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+    grid_dep_wait();   // weights and partial sums of the tokens kernel
+    if ((tid & 31) < Gp)
+        (&red[0][0][0])[(tid >> 5) * Gp + (tid & 31)] = lsum;   // scratch: 8 warps x Gp
+    // weight of reference r: its own softmax term p_r plus w_r from the tokens that chose it
+#pragma unroll
+    for (int z = 0; z < PJ; ++z) {
+        const int x = tid + 256 * z;
+        const int r = r0 + x / Gp, h = x % Gp;
+        wt[x / Gp][h] = (r < r1 && h < G) ? w.W[(um.ref_row + r) * Gp + h] + pj[z] : 0.0f;
+    }
+    __syncthreads();
+    if (tid < Gp) {
+        float v = 0.0f;
+        for (int i = 0; i < 8; ++i)
+            v += red[0][0][i * Gp + tid];
+        lred[tid] = v;
     }
     __syncthreads();
     // sum_r wt[r][h] refV[r][c]: thread (channel pair, quarter of the chunk)
