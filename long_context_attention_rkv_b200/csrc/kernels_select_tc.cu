@@ -28,8 +28,9 @@
 //
 // Top-kc per position (ties to the lower ordinal): each thread appends, without
 // branching, every t above its current threshold to a private queue in shared
-// memory; when any lane's queue could overflow, the warp drains all queues in
-// lockstep into the sorted per-thread lists and raises the thresholds.  This
+// memory; when any lane's queue could overflow, and at the end of an item, the warp
+// drains all queues in lockstep into the sorted per-thread lists, which raises the
+// thresholds.  This
 // keeps the per-element cost at a compare and a store, and the sorted
 // insertions coherent across the warp.
 //
@@ -431,11 +432,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_before();
                 mbar_arrive(&bars->acc_empty[acc]);
                 ++it_c;
-                // drain at reference-tile boundaries so the threshold keeps up
-                if (__any_sync(0xffffffffu, cnt > 0)) {
-                    drain<KC>(myq, cnt, tv, ti);
-                    cnt = 0;
-                }
+                // (queues drain only when one could overflow, and at the end of the item:
+                // draining at every reference-tile boundary as well measured slower)
             }
             if (!ok)
                 break;
