@@ -313,7 +313,9 @@ __device__ __forceinline__ void consumer_sync(int n_threads)
     asm volatile("bar.sync 1, %0;" ::"r"(n_threads) : "memory");
 }
 
-template <int Gp, int KK, int NTEAM>
+// GT: the units' reference-score tables are read from global memory (L2) instead of being
+// copied into shared memory (units with more references than shared memory holds).
+template <int Gp, int KK, int NTEAM, bool GT>
 __global__ void __launch_bounds__(32 * kConsWarps * NTEAM, 1)
     mma_tokens_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       const CacheArgs a, const void* __restrict__ q, const MmaWs w, const int nst)
@@ -326,7 +328,7 @@ __global__ void __launch_bounds__(32 * kConsWarps * NTEAM, 1)
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    const TokLayout L(Gp, kConsWarps * NTEAM, a.max_refs, nst);
+    const TokLayout L(Gp, kConsWarps * NTEAM, GT ? 0 : a.max_refs, nst);
     unsigned char* stages = sm + L.stages;
     float* s_buf = reinterpret_cast<float*>(sm + L.s_sm);
     const int s_stride = ((a.max_refs * Gp * 4 + 127) & ~127) / 4;
@@ -430,7 +432,7 @@ __global__ void __launch_bounds__(32 * kConsWarps * NTEAM, 1)
             bulk_load(s_buf + buf * s_stride, w.s_tab + m.ref_row * Gp, bytes, &tbar[buf]);
     };
     u = unit_at(u, t_lo);
-    if (tid == 0 && t_lo < t_hi) {
+    if (!GT && tid == 0 && t_lo < t_hi) {
         load_table(0, u);
         const int t1 = min(t_hi, unit_end(u));
         if (t1 < t_hi)
@@ -441,7 +443,7 @@ __global__ void __launch_bounds__(32 * kConsWarps * NTEAM, 1)
     while (t < t_hi && u < a.n_units) {
         const UnitMeta um = a.units[u];
         const int seg_end = min(t_hi, unit_end(u));
-        const float* s_sm = s_buf + (seg & 1) * s_stride;
+        const float* s_sm = GT ? w.s_tab + um.ref_row * Gp : s_buf + (seg & 1) * s_stride;
         const int R = um.R;
         const int kvh = u - um.seq * a.Hkv;
 
@@ -456,7 +458,7 @@ __global__ void __launch_bounds__(32 * kConsWarps * NTEAM, 1)
             q_sm[x] = (h < G) ? static_cast<const uint16_t*>(q)[(static_cast<int64_t>(um.seq) * a.Hq + kvh * G + h) * D + c]
                               : static_cast<uint16_t>(0);
         }
-        if (!*abort_flag && !mbar_wait_sleep(&tbar[seg & 1], (seg >> 1) & 1, abort_flag)) {
+        if (!GT && !*abort_flag && !mbar_wait_sleep(&tbar[seg & 1], (seg >> 1) & 1, abort_flag)) {
             if (!*abort_flag)
                 report(a.err, RKV_ERR_TIMEOUT);
             *abort_flag = 1;
@@ -580,10 +582,11 @@ __global__ void __launch_bounds__(32 * kConsWarps * NTEAM, 1)
                         keff += use ? 1 : 0;
                         const int oc = use ? oi[j] : 0;     // unconditional load, selected sum
                         if constexpr (NH == 1) {
-                            const float v = s_sm[oc * Gp + tq];
+                            const float v = GT ? __ldg(s_sm + oc * Gp + tq) : s_sm[oc * Gp + tq];
                             sref[0] += use ? v : 0.0f;
                         } else {
-                            const float2 v = *reinterpret_cast<const float2*>(s_sm + oc * Gp + 2 * tq);
+                            const float2 v = GT ? __ldg(reinterpret_cast<const float2*>(s_sm + oc * Gp + 2 * tq))
+                                                : *reinterpret_cast<const float2*>(s_sm + oc * Gp + 2 * tq);
                             sref[0] += use ? v.x : 0.0f;
                             sref[1] += use ? v.y : 0.0f;
                         }
@@ -737,7 +740,7 @@ __global__ void __launch_bounds__(32 * kConsWarps * NTEAM, 1)
         }
         consumer_sync(NCT);
         // the table buffer of this segment is free: the segment after next loads into it
-        if (tid == 0 && seg_end < t_hi) {
+        if (!GT && tid == 0 && seg_end < t_hi) {
             const int u1 = unit_at(u, seg_end);
             const int t2 = min(t_hi, unit_end(u1));
             if (t2 < t_hi && !*abort_flag) {
@@ -908,15 +911,19 @@ int heads_padded(int G) { return G <= 4 ? 4 : 8; }
 // not depend on the device present when they are computed.
 constexpr int kSmemOptin = 232448;
 
-// Pipeline depth that fits next to the unit tables (0 if fewer than two stages fit).
-int tok_stages(const CacheArgs& a)
+// Pipeline depth that fits next to the unit tables (0 if fewer than four stages fit);
+// table_refs = 0 when the tables stay in global memory.
+int tok_stages(const CacheArgs& a, int table_refs)
 {
     const int Gp = heads_padded(a.G);
-    const int fixed = TokLayout(Gp, kConsWarps * kTeams, a.max_refs, 0).total + 1024;
+    const int fixed = TokLayout(Gp, kConsWarps * kTeams, table_refs, 0).total + 1024;
     const int avail = kSmemOptin - fixed;
     const int n = avail / kStageBytes;
-    return n < 2 ? 0 : (n > 8 ? 8 : n);
+    return n < 4 ? 0 : (n > 8 ? 8 : n);
 }
+
+// Score tables in shared memory when they fit next to four or more stages, else in L2.
+bool tables_global(const CacheArgs& a) { return tok_stages(a, a.max_refs) == 0; }
 
 constexpr int kMaxCta = 160;   // grid cap of the tokens kernel
 
@@ -1002,8 +1009,10 @@ cudaError_t launch_gp(const CacheArgs& a, int64_t cmp_rows, const void* q, void*
     if (e != cudaSuccess)
         return e;
     if (w.n_tiles > 0) {
-        auto kern = (a.k <= 4) ? mma_tokens_kernel<Gp, 4, kTeams> : mma_tokens_kernel<Gp, 8, kTeams>;
-        const size_t smem = TokLayout(Gp, kConsWarps * kTeams, a.max_refs, nst).total + 1024;
+        const bool gt = tables_global(a);
+        auto kern = gt ? ((a.k <= 4) ? mma_tokens_kernel<Gp, 4, kTeams, true> : mma_tokens_kernel<Gp, 8, kTeams, true>)
+                       : ((a.k <= 4) ? mma_tokens_kernel<Gp, 4, kTeams, false> : mma_tokens_kernel<Gp, 8, kTeams, false>);
+        const size_t smem = TokLayout(Gp, kConsWarps * kTeams, gt ? 0 : a.max_refs, nst).total + 1024;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
         if (e != cudaSuccess)
             return e;
@@ -1020,7 +1029,7 @@ cudaError_t launch_gp(const CacheArgs& a, int64_t cmp_rows, const void* q, void*
 bool decode_mma_supported(const CacheArgs& a)
 {
     return a.D == 128 && a.bits == 4 && a.group == 32 && a.in_dtype == RKV_DTYPE_BF16 && a.G >= 1 && a.G <= 8 &&
-           a.k >= 1 && a.k <= 8 && tok_stages(a) >= 2;
+           a.k >= 1 && a.k <= 8 && tok_stages(a, 0) > 0;
 }
 
 uint64_t decode_mma_ws_bytes(const CacheArgs& a, int64_t ref_rows) { return ws_offsets(a, ref_rows).end; }
@@ -1049,8 +1058,8 @@ cudaError_t launch_decode_mma(const CacheArgs& a, int64_t ref_rows, int64_t cmp_
         w.n_cta = std::min(std::min(sms, kMaxCta), std::max(w.n_tiles, 1));
     }
     w.cK = static_cast<float>(1.4426950408889634 / std::sqrt(128.0));
-    const int nst = tok_stages(a);
-    if (nst < 2)
+    const int nst = tok_stages(a, tables_global(a) ? 0 : a.max_refs);
+    if (nst < 4)
         return cudaErrorNotSupported;
     return heads_padded(a.G) == 4 ? launch_gp<4>(a, cmp_rows, q, out, w, nst, st)
                                   : launch_gp<8>(a, cmp_rows, q, out, w, nst, st);
