@@ -253,6 +253,27 @@ RKV_API rkv_status rkv_decode_attn(const rkv_cache_desc* desc, const void* q, vo
                            uint64_t workspace_bytes, void* stream);
 
 /*
+ * One decode step over a subset of the cached positions: selective decompression
+ * (paper summary page, "Training and Inference Integration": only the tokens that
+ * sparse attention selects are rebuilt, from their references and residual codes).
+ * For unit u = b * n_kv_heads + h, the G query heads of kv-head h of sequence b attend
+ * to positions[u * max_sel + i], i < counts[u]: the same softmax attention as
+ * rkv_decode_attn restricted to those rows.  Reference positions use their stored
+ * rows; compressed positions are rebuilt from their codes, scales and k reference
+ * rows; nothing else of the cache is read.
+ *   positions  device int32 [n_units][max_sel], each in [0, lengths[b]), distinct
+ *              within a unit, any order; a position outside its sequence is skipped
+ *              and reported as RKV_ERR_INVALID_ARG through the device error word
+ *   counts     device int32 [n_units], 0 <= counts[u] <= max_sel (larger is clamped);
+ *              a unit with count 0 gives zeros
+ *   max_sel    >= 1, the row stride of positions
+ * q, out, workspace and stream as for rkv_decode_attn.
+ */
+RKV_API rkv_status rkv_decode_attn_sparse(const rkv_cache_desc* desc, const void* q, const int32_t* positions,
+                                          const int32_t* counts, int32_t max_sel, void* out, void* workspace,
+                                          uint64_t workspace_bytes, void* stream);
+
+/*
  * Materialises reconstructed rows of one unit (paper summary page, "DeltaKV
  * Framework Architecture", reconstruction KV = KV_delta + KV_R; "Training and
  * Inference Integration", selective decompression of only the rows needed).

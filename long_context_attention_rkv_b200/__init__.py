@@ -30,7 +30,7 @@ STATUS_CODE = {v: k for k, v in STATUS.items()}
 
 EXPORTED = ["rkv_abi_version", "rkv_status_string", "rkv_schedule", "rkv_cache_size", "rkv_cache_bind",
             "rkv_unit_view_get", "rkv_build_refs", "rkv_search", "rkv_encode", "rkv_compress", "rkv_decode_attn", "rkv_reconstruct",
-            "rkv_read_device_error", "rkv_compress_noalloc"]
+            "rkv_read_device_error", "rkv_compress_noalloc", "rkv_decode_attn_sparse"]
 
 
 class RkvError(RuntimeError):
@@ -80,6 +80,7 @@ def lib() -> ctypes.CDLL:
         L.rkv_reconstruct.argtypes = [vp, i32, i32, vp, i64, vp, vp, i32, vp]
         L.rkv_read_device_error.argtypes = [vp, vp, ctypes.POINTER(i32)]
         L.rkv_compress_noalloc.argtypes = [vp, vp, vp, vp]
+        L.rkv_decode_attn_sparse.argtypes = [vp, vp, vp, vp, i32, vp, vp, u64, vp]
         for name in EXPORTED[2:]:
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -198,6 +199,12 @@ def rkv_decode_attn(desc: CacheDesc, q, out, workspace, workspace_bytes: int, st
            "rkv_decode_attn")
 
 
+def rkv_decode_attn_sparse(desc: CacheDesc, q, positions, counts, max_sel: int, out, workspace, workspace_bytes: int,
+                           stream=None):
+    _check(lib().rkv_decode_attn_sparse(desc.ptr, _ptr(q), _ptr(positions), _ptr(counts), max_sel, _ptr(out),
+                                        _ptr(workspace), workspace_bytes, _stream(stream)), "rkv_decode_attn_sparse")
+
+
 def rkv_reconstruct(desc: CacheDesc, seq: int, kv_head: int, positions, n_pos: int, K_out, V_out,
                     out_dtype: int, stream=None):
     _check(lib().rkv_reconstruct(desc.ptr, seq, kv_head, _ptr(positions), n_pos, _ptr(K_out), _ptr(V_out),
@@ -243,6 +250,11 @@ class Layer:
 
     def decode(self, q, out, stream=None):
         rkv_decode_attn(self.desc, q, out, self.workspace, self.workspace.numel(), stream)
+
+    def decode_sparse(self, q, positions, counts, out, stream=None):
+        """positions: int32 [n_units, max_sel] on the device, counts: int32 [n_units] on the device."""
+        rkv_decode_attn_sparse(self.desc, q, positions, counts, positions.shape[-1], out, self.workspace,
+                               self.workspace.numel(), stream)
 
     def reconstruct(self, seq, kv_head, positions, n_pos, K_out, V_out, out_dtype, stream=None):
         rkv_reconstruct(self.desc, seq, kv_head, positions, n_pos, K_out, V_out, out_dtype, stream)

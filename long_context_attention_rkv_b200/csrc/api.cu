@@ -90,6 +90,15 @@ rkv_status validate_config(const rkv_config* c)
     return RKV_OK;
 }
 
+// Splits of the gather decode over a position list: about 32 positions per CTA (8 per warp;
+// each position is a chain of dependent gathers), within the workspace reserved for them.
+int sparse_splits_max(int n_units) { return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(256, 65536 / n_units))); }
+
+int sparse_splits(int n_units, int max_sel)
+{
+    return static_cast<int>(std::min<int64_t>(sparse_splits_max(n_units), std::max<int64_t>(1, ceil_div(max_sel, 32))));
+}
+
 int decode_splits(int n_units, int max_tokens)
 {
     int s = static_cast<int>(ceil_div(4 * 148, n_units));
@@ -174,7 +183,7 @@ rkv_status compute_layout(const rkv_config* c, const int32_t* lengths, Desc& d)
     s.idx = take(2ull * cmp_rows * c->k);
     s.end = off;
     d.ws_select = align_up(2ull * cmp_rows * d.kc, 256) + align_up(4ull * cmp_rows * d.kc, 256);
-    const int splits = decode_splits(d.n_units, max_n);
+    const int splits = std::max(decode_splits(d.n_units, max_n), sparse_splits_max(d.n_units));
     d.ws_decode = align_up(4ull * d.n_units * splits * G * (D + 2), 256);
     const CacheArgs a = make_args(d);
     if (decode_mma_supported(a))
@@ -507,6 +516,26 @@ rkv_status rkv_decode_attn(const rkv_cache_desc* desc, const void* q, void* out,
     const int splits = decode_splits(d->n_units, d->max_n);
     float* part = static_cast<float*>(workspace);
     cudaError_t e = launch_decode_direct(a, splits, q, part, st);
+    if (e == cudaSuccess)
+        e = launch_decode_combine(a, d->cfg.batch, splits, part, out, st);
+    return cuda_status(e);
+}
+
+rkv_status rkv_decode_attn_sparse(const rkv_cache_desc* desc, const void* q, const int32_t* positions,
+                                  const int32_t* counts, int32_t max_sel, void* out, void* workspace,
+                                  uint64_t workspace_bytes, void* stream)
+{
+    const Desc* d = get_desc(desc);
+    if (!d || !q || !out || !positions || !counts || max_sel < 1 || !workspace || !aligned(q, 16) ||
+        !aligned(out, 16) || !aligned(workspace, 256) || !aligned(positions, 4) || !aligned(counts, 4))
+        return RKV_ERR_INVALID_ARG;
+    if (workspace_bytes < d->ws_decode)
+        return RKV_ERR_WORKSPACE;
+    const CacheArgs a = make_args(*d);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int splits = sparse_splits(d->n_units, std::min<int>(max_sel, std::max(1, d->max_n)));
+    float* part = static_cast<float*>(workspace);
+    cudaError_t e = launch_decode_direct(a, splits, q, part, st, positions, counts, max_sel);
     if (e == cudaSuccess)
         e = launch_decode_combine(a, d->cfg.batch, splits, part, out, st);
     return cuda_status(e);

@@ -11,7 +11,9 @@
 // Grid: (splits, units); each CTA takes one contiguous range of the unit's
 // tokens (references first, then compressed tokens) and writes one partial
 // softmax state (m, l, o[D]) per query head, in log2 units.  The combine
-// kernel merges the splits.
+// kernel merges the splits.  With a position list (selective decompression)
+// the CTA ranges split the unit's listed positions instead, each mapped to its
+// reference row or compressed slot.
 #include <cfloat>
 #include <cmath>
 
@@ -73,7 +75,9 @@ __device__ __forceinline__ bool rebuild_compressed(const CacheArgs& a, const Uni
 template <int NPL, int GMAX>
 __global__ void __launch_bounds__(kWarps * 32) decode_direct_kernel(CacheArgs a, const void* __restrict__ q,
                                                                     float* __restrict__ part, int splits,
-                                                                    float qscale)
+                                                                    float qscale, const int32_t* __restrict__ sel,
+                                                                    const int32_t* __restrict__ sel_cnt,
+                                                                    int sel_stride)
 {
     constexpr int D = NPL * 32;
     __shared__ float s_m[kWarps][GMAX];
@@ -87,7 +91,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_direct_kernel(CacheArgs a,
     const int lane = threadIdx.x & 31;
     const int G = a.G;
     const int h = u - um.seq * a.Hkv;
-    const int T = um.R + um.C;
+    const int T = sel ? max(0, min(sel_cnt[u], sel_stride)) : um.R + um.C;
     const int per = (T + splits - 1) / splits;
     const int v0 = split * per;
     const int v1 = min(T, v0 + per);
@@ -112,7 +116,19 @@ __global__ void __launch_bounds__(kWarps * 32) decode_direct_kernel(CacheArgs a,
         }
     }
 
-    for (int v = v0 + warp; v < v1; v += kWarps) {
+    for (int vi = v0 + warp; vi < v1; vi += kWarps) {
+        int v = vi;
+        if (sel) {
+            // listed position -> storage index: reference ordinal, or R + compressed slot
+            const int p = sel[static_cast<int64_t>(u) * sel_stride + vi];
+            if (p < 0 || p >= um.n) {
+                if (lane == 0)
+                    report(a.err, RKV_ERR_INVALID_ARG);
+                continue;
+            }
+            const int nr = refs_upto(a.ph, p);
+            v = is_ref_pos(a.ph, p) ? nr - 1 : um.R + (p - nr);
+        }
         float xk[NPL], xv[NPL];
         if (v < um.R) {
             const int64_t r = (um.ref_row + v) * D + lane * NPL;
@@ -214,20 +230,25 @@ __global__ void decode_combine_kernel(CacheArgs a, int splits, const float* __re
 
 }  // namespace
 
-cudaError_t launch_decode_direct(const CacheArgs& a, int splits, const void* q, float* partials, cudaStream_t st)
+cudaError_t launch_decode_direct(const CacheArgs& a, int splits, const void* q, float* partials, cudaStream_t st,
+                                 const int32_t* sel, const int32_t* sel_cnt, int sel_stride)
 {
     const dim3 grid(splits, a.n_units);
     const float qscale = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(a.D)));
     if (a.D == 128) {
         if (a.G <= 8)
-            decode_direct_kernel<4, 8><<<grid, kWarps * 32, 0, st>>>(a, q, partials, splits, qscale);
+            decode_direct_kernel<4, 8><<<grid, kWarps * 32, 0, st>>>(a, q, partials, splits, qscale, sel, sel_cnt,
+                                                                      sel_stride);
         else
-            decode_direct_kernel<4, 16><<<grid, kWarps * 32, 0, st>>>(a, q, partials, splits, qscale);
+            decode_direct_kernel<4, 16><<<grid, kWarps * 32, 0, st>>>(a, q, partials, splits, qscale, sel, sel_cnt,
+                                                                       sel_stride);
     } else {
         if (a.G <= 8)
-            decode_direct_kernel<2, 8><<<grid, kWarps * 32, 0, st>>>(a, q, partials, splits, qscale);
+            decode_direct_kernel<2, 8><<<grid, kWarps * 32, 0, st>>>(a, q, partials, splits, qscale, sel, sel_cnt,
+                                                                      sel_stride);
         else
-            decode_direct_kernel<2, 16><<<grid, kWarps * 32, 0, st>>>(a, q, partials, splits, qscale);
+            decode_direct_kernel<2, 16><<<grid, kWarps * 32, 0, st>>>(a, q, partials, splits, qscale, sel, sel_cnt,
+                                                                       sel_stride);
     }
     return cudaGetLastError();
 }

@@ -24,7 +24,11 @@ cudaError_t launch_reconstruct(const CacheArgs& a, int unit, const int32_t* posi
                                void* V_out, int out_dtype, cudaStream_t st);
 
 // Literal decode: per token gather + mean of the reference rows, dequantise, add, attend.
-cudaError_t launch_decode_direct(const CacheArgs& a, int splits, const void* q, float* partials, cudaStream_t st);
+// With sel (device [n_units][sel_stride] positions, sel_cnt [n_units] counts) only the listed
+// positions are attended to.
+cudaError_t launch_decode_direct(const CacheArgs& a, int splits, const void* q, float* partials, cudaStream_t st,
+                                 const int32_t* sel = nullptr, const int32_t* sel_cnt = nullptr,
+                                 int sel_stride = 0);
 
 // Factorised decode (reference scores + scattered reference weights), one cluster per unit.
 bool decode_fact_supported(const CacheArgs& a);

@@ -74,7 +74,8 @@ def test_calls_reject_unbound_handles():
     for fn, args in [(rkv.lib().rkv_build_refs, (d.ptr, 16, 16, None)),
                      (rkv.lib().rkv_compress, (d.ptr, 16, 16, 256, 0, None)),
                      (rkv.lib().rkv_decode_attn, (d.ptr, 16, 16, 256, 0, None)),
-                     (rkv.lib().rkv_reconstruct, (d.ptr, 0, 0, None, 0, 16, 16, 0, None))]:
+                     (rkv.lib().rkv_reconstruct, (d.ptr, 0, 0, None, 0, 16, 16, 0, None)),
+                     (rkv.lib().rkv_decode_attn_sparse, (d.ptr, 16, 16, 16, 1, 16, 256, 0, None))]:
         assert fn(*args) == rkv.STATUS_CODE["RKV_ERR_INVALID_ARG"]
 
 

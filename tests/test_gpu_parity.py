@@ -207,3 +207,86 @@ def test_decode_many_short_units(n_q_heads):
     q = synth.gen_query(wl, 0, 0)
     a, b = run.decode(q), simt.decode(q)
     assert np.abs(a - b).max() <= 2e-3
+
+
+def _sparse_check(run, wl, lengths, sel, q):
+    """Sparse decode on the GPU against the oracle's attention over the listed rows."""
+    n_units = len(lengths) * wl.n_kv_heads
+    max_sel = max(1, max(len(x) for x in sel))
+    pos = np.zeros((n_units, max_sel), dtype=np.int32)
+    cnt = np.zeros(n_units, dtype=np.int32)
+    for u, x in enumerate(sel):
+        pos[u, :len(x)] = x
+        cnt[u] = len(x)
+    out = torch.empty((len(lengths), wl.n_q_heads, wl.head_dim), dtype=torch.float32, device="cuda")
+    run.layer.decode_sparse(to_dev(q), torch.from_numpy(pos).cuda(), torch.from_numpy(cnt).cuda(), out)
+    torch.cuda.synchronize()
+    assert run.layer.device_error() == 0
+    got = out.cpu().numpy().astype(np.float64)
+    qf = synth.as_f32(wl, q)
+    G = wl.n_q_heads // wl.n_kv_heads
+    for b, n in enumerate(lengths):
+        for h in range(wl.n_kv_heads):
+            u = b * wl.n_kv_heads + h
+            g = run.unit(b, h)
+            if len(sel[u]) == 0:
+                assert np.all(got[b, h * G:(h + 1) * G] == 0.0)
+                continue
+            Kh, Vh = oracle.unit_cache_rows(n, g["pos"], g["refK"], g["refV"], g["idx"], g["codesK"], g["scalesK"],
+                                            g["codesV"], g["scalesV"], wl.bits, wl.group)
+            ref = oracle.attention(qf[b, h * G:(h + 1) * G].astype(np.float64), Kh[sel[u]], Vh[sel[u]])
+            err = np.abs(got[b, h * G:(h + 1) * G] - ref)
+            assert err.max() <= 2e-3, f"sparse decode unit {(b, h)}: max err {err.max()}"
+
+
+@pytest.mark.parametrize("name", ["llama3_8b_layer", "qwen2_5_7b_batch"])
+def test_sparse_decode_matches_oracle_on_listed_rows(name):
+    """Selective decompression: random position lists per unit (references and compressed
+    tokens mixed, any order), a unit with an empty list, and one that lists every position."""
+    wl = _small(name, n_kv_heads=2, n_q_heads=2 * (synth.WORKLOADS[name].n_q_heads // synth.WORKLOADS[name].n_kv_heads),
+                batch=2, seq_len=3000, ragged=None)
+    lengths = [3000, 1700]
+    K, V = synth.gen_layer(wl, 0, lengths)
+    run = GpuRun(wl, K, V, lengths)
+    rng = np.random.default_rng(7)
+    sel = []
+    for b, n in enumerate(lengths):
+        for h in range(wl.n_kv_heads):
+            u = b * wl.n_kv_heads + h
+            if u == 1:
+                sel.append(np.zeros(0, dtype=np.int64))                # nothing selected
+            elif u == 2:
+                sel.append(rng.permutation(n))                         # everything, shuffled
+            else:
+                sel.append(rng.choice(n, size=min(n, 257), replace=False))
+    _sparse_check(run, wl, lengths, sel, synth.gen_query(wl, 0, 0))
+
+
+def test_sparse_decode_full_list_equals_dense_decode():
+    wl = _small("llama3_8b_layer", n_kv_heads=2, n_q_heads=8, seq_len=2500)
+    lengths = [2500]
+    K, V = synth.gen_layer(wl, 0, lengths)
+    run = GpuRun(wl, K, V, lengths)
+    q = synth.gen_query(wl, 0, 0)
+    dense = run.decode(q)
+    sel = [np.arange(2500) for _ in range(2)]
+    _sparse_check(run, wl, lengths, sel, q)
+    pos = torch.from_numpy(np.stack(sel).astype(np.int32)).cuda()
+    cnt = torch.full((2,), 2500, dtype=torch.int32, device="cuda")
+    out = torch.empty((1, 8, 128), dtype=torch.float32, device="cuda")
+    run.layer.decode_sparse(to_dev(q), pos, cnt, out)
+    torch.cuda.synchronize()
+    assert np.abs(out.cpu().numpy() - dense).max() <= 2e-3
+
+
+def test_sparse_decode_reports_out_of_range_positions():
+    wl = _small("llama3_8b_layer", n_kv_heads=1, n_q_heads=4, seq_len=1000)
+    lengths = [1000]
+    K, V = synth.gen_layer(wl, 0, lengths)
+    run = GpuRun(wl, K, V, lengths)
+    pos = torch.tensor([[5, 999, 1000, -1]], dtype=torch.int32, device="cuda")   # two outside [0, 1000)
+    cnt = torch.tensor([4], dtype=torch.int32, device="cuda")
+    out = torch.empty((1, 4, 128), dtype=torch.float32, device="cuda")
+    run.layer.decode_sparse(to_dev(synth.gen_query(wl, 0, 0)), pos, cnt, out)
+    torch.cuda.synchronize()
+    assert run.layer.device_error() == rkv.STATUS_CODE["RKV_ERR_INVALID_ARG"]
