@@ -8,8 +8,9 @@ step, and a 256-row reconstruction.  Inputs are resident in HBM when the timed
 region starts; L2 is flushed (256 MiB write) before every timed step, outside
 the timed spans.  With N GPUs (torchrun) every rank runs its own replica on an
 independent layer; value is the whole-job throughput over the max-over-ranks
-step time.  `--impl reference` times the CPU oracle on a bounded sample of the
-same workload on the host cores.  Prints one JSON line on rank 0.
+step time.  Outside the step, a selective decode (2048 seeded positions per unit)
+is timed as well.  `--impl reference` times the CPU oracle on a bounded sample of
+the same workload on the host cores.  Prints one JSON line on rank 0.
 """
 from __future__ import annotations
 
@@ -34,6 +35,7 @@ WORKLOAD = "llama3_8b_layer"
 # kernels launched per step, by stage
 LAUNCHES = {"build_refs": 1, "search": 1, "encode": 1, "decode": 3, "reconstruct": 1}
 RECON_ROWS = 256
+SPARSE_SEL = 2048          # positions per unit of the selective-decode measurement
 
 
 def replica_layer(rank: int) -> int:
@@ -392,6 +394,32 @@ def run_ours(args, rank, world, local_rank):
                 e2e_ms.append(e0.elapsed_time(e1))
     e2e_step = max_over_ranks(statistics.mean(e2e_ms), world, dev)
 
+    # selective decode (outside the step): SPARSE_SEL seeded uniform positions per unit
+    rng = np.random.default_rng(0x5E1)
+    n_units = wl.batch * wl.n_kv_heads
+    sel = np.zeros((n_units, SPARSE_SEL), dtype=np.int32)
+    cnt = np.zeros(n_units, dtype=np.int32)
+    for u in range(n_units):
+        n = lengths[u // wl.n_kv_heads]
+        m = min(n, SPARSE_SEL)
+        sel[u, :m] = np.sort(rng.choice(n, m, replace=False))
+        cnt[u] = m
+    sel_d, cnt_d = torch.from_numpy(sel).to(dev), torch.from_numpy(cnt).to(dev)
+    sp_ms = []
+    with torch.cuda.stream(stream):
+        for i in range(max(3, min(args.steps, 20)) + 2):
+            flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            L.decode_sparse(q, sel_d, cnt_d, out)
+            e1.record(stream)
+            e1.synchronize()
+            if i >= 2:
+                sp_ms.append(e0.elapsed_time(e1))
+    assert L.device_error() == 0
+    sparse_us = 1e3 * statistics.mean(sp_ms)
+
     Q = workload_quantities(wl, lengths)
     tokens = Q["tokens"]
     value = job_throughput(world, tokens, mean_step)
@@ -441,6 +469,7 @@ def run_ours(args, rank, world, local_rank):
                 "search_tflops": search_tflops, "search_flops": Q["search_flops"],
                 "encode_gbs": encode_gbs, "compress_mtok_s": tokens / ((avg["search"] + avg["encode"] +
                                                                         avg["build_refs"]) * 1e-3) / 1e6,
+                "sparse_decode_us": sparse_us, "sparse_decode_positions_per_unit": SPARSE_SEL,
             },
             "roofline": roofline,
             "cpu_baseline": cpu,
