@@ -253,6 +253,31 @@ RKV_API rkv_status rkv_decode_attn(const rkv_cache_desc* desc, const void* q, vo
                            uint64_t workspace_bytes, void* stream);
 
 /*
+ * Current lengths of the sequences of a bound cache (host array of batch entries,
+ * 0 <= lengths[b] <= the length the cache was bound with, which is its capacity).
+ * rkv_build_refs, rkv_compress, the decodes and rkv_reconstruct then work on the
+ * first lengths[b] positions; rkv_append grows them.  Binding sets the current
+ * lengths to the bound ones.  Host arguments; queues one small copy on stream.
+ */
+RKV_API rkv_status rkv_cache_set_lengths(rkv_cache_desc* desc, const int32_t* lengths, void* stream);
+
+/*
+ * Incremental compression (paper summary page, "DeltaKV Framework Architecture";
+ * news page, "How ResidualKV Works": each new token is stored as a reference or as
+ * a residual against its nearest earlier references).  For every sequence b with
+ * active[b] != 0 (active: host array of batch flags, NULL = all) the token at
+ * position p = current length is added to each kv-head unit: a reference if p is
+ * on the schedule, otherwise compressed against the references so far exactly as
+ * rkv_compress would (nearest by exact L2 distance, ties to the lower ordinal).
+ *   K_new, V_new  device [batch][n_kv_heads][head_dim], the cache's input dtype;
+ *                 rows of inactive sequences are not read
+ * Fails with RKV_ERR_INVALID_ARG, launching nothing, if an active sequence is at
+ * capacity.  The current lengths advance on return (the work is queued on stream).
+ */
+RKV_API rkv_status rkv_append(rkv_cache_desc* desc, const void* K_new, const void* V_new, const uint8_t* active,
+                              void* stream);
+
+/*
  * One decode step over a subset of the cached positions: selective decompression
  * (paper summary page, "Training and Inference Integration": only the tokens that
  * sparse attention selects are rebuilt, from their references and residual codes).

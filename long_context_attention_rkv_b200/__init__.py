@@ -30,7 +30,8 @@ STATUS_CODE = {v: k for k, v in STATUS.items()}
 
 EXPORTED = ["rkv_abi_version", "rkv_status_string", "rkv_schedule", "rkv_cache_size", "rkv_cache_bind",
             "rkv_unit_view_get", "rkv_build_refs", "rkv_search", "rkv_encode", "rkv_compress", "rkv_decode_attn", "rkv_reconstruct",
-            "rkv_read_device_error", "rkv_compress_noalloc", "rkv_decode_attn_sparse"]
+            "rkv_read_device_error", "rkv_compress_noalloc", "rkv_decode_attn_sparse", "rkv_cache_set_lengths",
+            "rkv_append"]
 
 
 class RkvError(RuntimeError):
@@ -81,6 +82,8 @@ def lib() -> ctypes.CDLL:
         L.rkv_read_device_error.argtypes = [vp, vp, ctypes.POINTER(i32)]
         L.rkv_compress_noalloc.argtypes = [vp, vp, vp, vp]
         L.rkv_decode_attn_sparse.argtypes = [vp, vp, vp, vp, i32, vp, vp, u64, vp]
+        L.rkv_cache_set_lengths.argtypes = [vp, vp, vp]
+        L.rkv_append.argtypes = [vp, vp, vp, vp, vp]
         for name in EXPORTED[2:]:
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -199,6 +202,16 @@ def rkv_decode_attn(desc: CacheDesc, q, out, workspace, workspace_bytes: int, st
            "rkv_decode_attn")
 
 
+def rkv_cache_set_lengths(desc: CacheDesc, lengths, stream=None):
+    arr, p = _lengths(lengths)
+    _check(lib().rkv_cache_set_lengths(desc.ptr, p, _stream(stream)), "rkv_cache_set_lengths")
+
+
+def rkv_append(desc: CacheDesc, K_new, V_new, active=None, stream=None):
+    act = None if active is None else (ctypes.c_uint8 * len(active))(*[1 if x else 0 for x in active])
+    _check(lib().rkv_append(desc.ptr, _ptr(K_new), _ptr(V_new), act, _stream(stream)), "rkv_append")
+
+
 def rkv_decode_attn_sparse(desc: CacheDesc, q, positions, counts, max_sel: int, out, workspace, workspace_bytes: int,
                            stream=None):
     _check(lib().rkv_decode_attn_sparse(desc.ptr, _ptr(q), _ptr(positions), _ptr(counts), max_sel, _ptr(out),
@@ -250,6 +263,14 @@ class Layer:
 
     def decode(self, q, out, stream=None):
         rkv_decode_attn(self.desc, q, out, self.workspace, self.workspace.numel(), stream)
+
+    def set_lengths(self, lengths, stream=None):
+        """Current lengths (<= the bound ones, which are the capacity)."""
+        rkv_cache_set_lengths(self.desc, lengths, stream)
+
+    def append(self, K_new, V_new, active=None, stream=None):
+        """One new token per active sequence: K_new, V_new [batch, kv_heads, head_dim] on the device."""
+        rkv_append(self.desc, K_new, V_new, active, stream)
 
     def decode_sparse(self, q, positions, counts, out, stream=None):
         """positions: int32 [n_units, max_sel] on the device, counts: int32 [n_units] on the device."""

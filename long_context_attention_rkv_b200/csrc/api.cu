@@ -141,6 +141,7 @@ rkv_status compute_layout(const rkv_config* c, const int32_t* lengths, Desc& d)
         if (R > RKV_MAX_REFS)
             return RKV_ERR_UNSUPPORTED;
         d.len[b] = static_cast<int32_t>(n);
+        d.cur_len[b] = static_cast<int32_t>(n);
         d.R[b] = static_cast<int32_t>(R);
         d.C[b] = static_cast<int32_t>(n - R);
         d.Rpad[b] = static_cast<int32_t>(align_up(R, kRefPad));
@@ -403,9 +404,11 @@ rkv_status rkv_unit_view_get(const rkv_cache_desc* desc, int32_t seq, int32_t kv
     const int64_t ref_row = d->ref_seq_row[seq] + static_cast<int64_t>(kv_head) * d->Rpad[seq];
     const int64_t cmp_row = d->cmp_seq_row[seq] + static_cast<int64_t>(kv_head) * d->Cpad[seq];
     std::memset(out, 0, sizeof(*out));
-    out->n = d->len[seq];
-    out->n_ref = d->R[seq];
-    out->n_cmp = d->C[seq];
+    const int64_t ncur = d->cur_len[seq];
+    const int64_t rcur = host_ref_count(d->ph, ncur);
+    out->n = static_cast<int32_t>(ncur);
+    out->n_ref = static_cast<int32_t>(rcur);
+    out->n_cmp = static_cast<int32_t>(ncur - rcur);
     out->k = d->cfg.k;
     out->code_bytes = d->code_bytes;
     out->n_groups = d->n_groups;
@@ -521,6 +524,67 @@ rkv_status rkv_decode_attn(const rkv_cache_desc* desc, const void* q, void* out,
     return cuda_status(e);
 }
 
+rkv_status rkv_cache_set_lengths(rkv_cache_desc* desc, const int32_t* lengths, void* stream)
+{
+    const Desc* cd = get_desc(desc);
+    if (!cd || !lengths)
+        return RKV_ERR_INVALID_ARG;
+    Desc* d = const_cast<Desc*>(cd);
+    for (int b = 0; b < d->cfg.batch; ++b)
+        if (lengths[b] < 0 || lengths[b] > d->len[b])
+            return RKV_ERR_INVALID_ARG;
+    const int Hkv = d->cfg.n_kv_heads;
+    std::vector<UnitMeta> units(d->n_units);
+    for (int b = 0; b < d->cfg.batch; ++b)
+        for (int h = 0; h < Hkv; ++h) {
+            UnitMeta& m = units[b * Hkv + h];
+            m.n = lengths[b];
+            m.R = static_cast<int32_t>(host_ref_count(d->ph, lengths[b]));
+            m.C = m.n - m.R;
+            m.seq = b;
+            m.ref_row = d->ref_seq_row[b] + static_cast<int64_t>(h) * d->Rpad[b];
+            m.cmp_row = d->cmp_seq_row[b] + static_cast<int64_t>(h) * d->Cpad[b];
+        }
+    // pageable source: the copy has read it when the call returns
+    const cudaError_t e = cudaMemcpyAsync(static_cast<char*>(d->base) + d->sec.units, units.data(),
+                                          sizeof(UnitMeta) * units.size(), cudaMemcpyHostToDevice,
+                                          static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess)
+        return RKV_ERR_CUDA;
+    for (int b = 0; b < d->cfg.batch; ++b)
+        d->cur_len[b] = lengths[b];
+    return RKV_OK;
+}
+
+rkv_status rkv_append(rkv_cache_desc* desc, const void* K_new, const void* V_new, const uint8_t* active,
+                      void* stream)
+{
+    const Desc* cd = get_desc(desc);
+    if (!cd || !K_new || !V_new || !aligned(K_new, 16) || !aligned(V_new, 16))
+        return RKV_ERR_INVALID_ARG;
+    Desc* d = const_cast<Desc*>(cd);
+    uint32_t bits[8] = {};
+    bool any = false;
+    for (int b = 0; b < d->cfg.batch; ++b) {
+        if (active && !active[b])
+            continue;
+        if (d->cur_len[b] >= d->len[b])
+            return RKV_ERR_INVALID_ARG;            // capacity reached: nothing is launched
+        bits[b >> 5] |= 1u << (b & 31);
+        any = true;
+    }
+    if (!any)
+        return RKV_OK;
+    const CacheArgs a = make_args(*d);
+    const cudaError_t e = launch_append(a, K_new, V_new, bits, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess)
+        return RKV_ERR_CUDA;
+    for (int b = 0; b < d->cfg.batch; ++b)
+        if (bits[b >> 5] >> (b & 31) & 1u)
+            ++d->cur_len[b];
+    return RKV_OK;
+}
+
 rkv_status rkv_decode_attn_sparse(const rkv_cache_desc* desc, const void* q, const int32_t* positions,
                                   const int32_t* counts, int32_t max_sel, void* out, void* workspace,
                                   uint64_t workspace_bytes, void* stream)
@@ -549,7 +613,7 @@ rkv_status rkv_reconstruct(const rkv_cache_desc* desc, int32_t seq, int32_t kv_h
         return RKV_ERR_INVALID_ARG;
     if (out_dtype != RKV_DTYPE_BF16 && out_dtype != RKV_DTYPE_F32)
         return RKV_ERR_INVALID_ARG;
-    if (!positions && n_pos != d->len[seq])
+    if (!positions && n_pos != d->cur_len[seq])
         return RKV_ERR_INVALID_ARG;
     if ((K_out && !aligned(K_out, 16)) || (V_out && !aligned(V_out, 16)) || (positions && !aligned(positions, 4)))
         return RKV_ERR_INVALID_ARG;

@@ -449,6 +449,226 @@ __global__ void __launch_bounds__(kWarps * 32, encode_min_blocks<KC, LPT>()) enc
                         a.err);
 }
 
+// ---- incremental compression: one new token per unit ----------------------------------
+// (ResidualKV paper summary page, "DeltaKV Framework Architecture"; news page, "How
+// ResidualKV Works": tokens are compressed as they arrive during generation.)  The token at
+// position p = n of a unit becomes reference n_ref if p is on the schedule (stored exactly as
+// the reference store does), otherwise compressed slot n_cmp: its k nearest references by
+// exact distance (double, channel order, no contraction; ties to the lower ordinal: the
+// search's definition evaluated directly), the mean in ascending ordinal order and the group
+// quantiser of the encoder.  The unit's counts advance on the device.
+constexpr int kAppendThreads = 128;
+
+template <int D>
+__global__ void __launch_bounds__(kAppendThreads) append_kernel(CacheArgs a, const void* __restrict__ Kn,
+                                                                 const void* __restrict__ Vn, uint32_t act0,
+                                                                 uint32_t act1, uint32_t act2, uint32_t act3,
+                                                                 uint32_t act4, uint32_t act5, uint32_t act6,
+                                                                 uint32_t act7)
+{
+    constexpr int KM = 16;                      // largest k
+    constexpr int CPL = 8;                      // channels per lane in the encode step
+    constexpr int LPT = D / CPL;
+    __shared__ float xs[D];
+    __shared__ double bd_s[kAppendThreads / 32][KM];
+    __shared__ int bo_s[kAppendThreads / 32][KM];
+    __shared__ int chosen_s[KM];
+    const int u = blockIdx.x;
+    UnitMeta* um_ptr = const_cast<UnitMeta*>(a.units) + u;
+    const UnitMeta um = *um_ptr;
+    const uint32_t act[8] = {act0, act1, act2, act3, act4, act5, act6, act7};
+    if (!((act[um.seq >> 5] >> (um.seq & 31)) & 1u))
+        return;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int p = um.n;
+    const int64_t e_row = static_cast<int64_t>(u) * D;      // the new rows: [unit][D]
+    if (is_ref_pos(a.ph, p)) {
+        // reference ordinal um.R, written as the reference store writes it
+        if (warp == 0) {
+            constexpr int NPL = D / 32;
+            const int j = um.R;
+            float kx[NPL], vx[NPL];
+            load_row_part<NPL>(Kn, e_row + lane * NPL, a.in_dtype, kx);
+            load_row_part<NPL>(Vn, e_row + lane * NPL, a.in_dtype, vx);
+            float ss = 0.0f;
+            const int64_t o = (um.ref_row + j) * D + lane * NPL;
+#pragma unroll
+            for (int i = 0; i < NPL; ++i) {
+                const uint16_t kb = f32_to_bf16_bits(kx[i]);
+                const uint16_t vb = f32_to_bf16_bits(vx[i]);
+                a.ref_K[o + i] = kb;
+                a.ref_V[o + i] = vb;
+                const float r = bf16_bits_to_f32(kb);
+                ss = fmaf(r, r, ss);
+            }
+            ss = warp_sum(ss);
+            if (lane == 0) {
+                const float hn = 0.5f * ss;
+                a.ref_hn[um.ref_row + j] = hn;
+                a.ref_pos[um.ref_row + j] = p;
+                const uint16_t hi = f32_to_bf16_bits(hn);
+                const float r1 = hn - bf16_bits_to_f32(hi);
+                const uint16_t mid = f32_to_bf16_bits(r1);
+                const uint16_t lo = f32_to_bf16_bits(r1 - bf16_bits_to_f32(mid));
+                uint4* aug = reinterpret_cast<uint4*>(a.ref_aug + (um.ref_row + j) * 16);
+                aug[0] = make_uint4((hi ^ 0x8000u) | ((mid ^ 0x8000u) << 16), lo ^ 0x8000u, 0u, 0u);
+                aug[1] = make_uint4(0u, 0u, 0u, 0u);
+                __threadfence();
+                um_ptr->R = j + 1;
+                um_ptr->n = p + 1;
+            }
+        }
+        return;
+    }
+    // ---- compressed token: exact top-k over the references so far -------------------------
+    const int R = um.R;
+    const int k = a.k;
+    const int keff = min(k, R);
+    for (int c = tid; c < D; c += kAppendThreads)
+        xs[c] = (a.in_dtype == RKV_DTYPE_F32) ? static_cast<const float*>(Kn)[e_row + c]
+                                              : bf16_bits_to_f32(static_cast<const uint16_t*>(Kn)[e_row + c]);
+    __syncthreads();
+    double bd[KM];
+    int bo[KM];
+#pragma unroll
+    for (int s2 = 0; s2 < KM; ++s2) {
+        bd[s2] = DBL_MAX;
+        bo[s2] = 0x7fffffff;
+    }
+    for (int j = tid; j < R; j += kAppendThreads) {
+        const uint16_t* r = a.ref_K + (um.ref_row + j) * D;
+        double d = 0.0;
+        for (int c = 0; c < D; ++c) {
+            const double t = __dsub_rn(static_cast<double>(xs[c]), static_cast<double>(bf16_bits_to_f32(r[c])));
+            d = __dadd_rn(d, __dmul_rn(t, t));
+        }
+        double cv = d;
+        int ci = j;
+#pragma unroll
+        for (int s2 = 0; s2 < KM; ++s2) {
+            if (s2 < k) {
+                const bool before = (cv < bd[s2]) || (cv == bd[s2] && ci < bo[s2]);
+                const double fd = bd[s2];
+                const int fo = bo[s2];
+                bd[s2] = before ? cv : fd;
+                bo[s2] = before ? ci : fo;
+                cv = before ? fd : cv;
+                ci = before ? fo : ci;
+            }
+        }
+    }
+    // merge: k rounds of a warp-wide minimum, then the warps' lists in thread 0
+    {
+        int head = 0;
+        for (int r2 = 0; r2 < k; ++r2) {
+            double hd = DBL_MAX;
+            int ho = 0x7fffffff;
+#pragma unroll
+            for (int s2 = 0; s2 < KM; ++s2)
+                if (s2 == head) {
+                    hd = bd[s2];
+                    ho = bo[s2];
+                }
+            double wd = hd;
+            int wo = ho;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const double od = __shfl_xor_sync(0xffffffffu, wd, off);
+                const int oo = __shfl_xor_sync(0xffffffffu, wo, off);
+                if (od < wd || (od == wd && oo < wo)) {
+                    wd = od;
+                    wo = oo;
+                }
+            }
+            if (ho == wo && hd == wd)
+                ++head;
+            if (lane == 0) {
+                bd_s[warp][r2] = wd;
+                bo_s[warp][r2] = wo;
+            }
+        }
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int hp[kAppendThreads / 32] = {};
+        int ch[KM];
+        for (int r2 = 0; r2 < keff; ++r2) {
+            int bw = 0;
+            for (int w2 = 1; w2 < kAppendThreads / 32; ++w2) {
+                const double dw = bd_s[w2][hp[w2]], db = bd_s[bw][hp[bw]];
+                if (dw < db || (dw == db && bo_s[w2][hp[w2]] < bo_s[bw][hp[bw]]))
+                    bw = w2;
+            }
+            ch[r2] = bo_s[bw][hp[bw]];
+            ++hp[bw];
+        }
+        // ascending ordinal order
+        for (int i2 = 1; i2 < keff; ++i2)
+            for (int j2 = i2; j2 > 0 && ch[j2 - 1] > ch[j2]; --j2) {
+                const int t = ch[j2];
+                ch[j2] = ch[j2 - 1];
+                ch[j2 - 1] = t;
+            }
+        for (int i2 = 0; i2 < KM; ++i2)
+            chosen_s[i2] = (i2 < keff) ? ch[i2] : 0;
+        const int64_t row = um.cmp_row + um.C;
+        for (int i2 = 0; i2 < k; ++i2)
+            a.idx[row * k + i2] = (i2 < keff) ? static_cast<uint16_t>(ch[i2]) : static_cast<uint16_t>(RKV_IDX_UNUSED);
+    }
+    __syncthreads();
+    // ---- mean, residual and quantiser: warp 0, LPT lanes of CPL channels (lanes past LPT
+    // shadow lane 0 and store nothing)
+    if (warp == 0) {
+        const int sub = (lane < LPT) ? lane : 0;
+        const bool store = lane < LPT;
+        const int64_t row = um.cmp_row + um.C;
+        float xk[CPL], xv[CPL], mk[CPL], mv[CPL];
+        load_input_row<CPL>(Kn, e_row + sub * CPL, a.in_dtype, xk);
+        load_input_row<CPL>(Vn, e_row + sub * CPL, a.in_dtype, xv);
+        {
+            const int o = chosen_s[0];
+            load_bf16_row<CPL>(a.ref_K + (um.ref_row + o) * D + sub * CPL, mk);
+            load_bf16_row<CPL>(a.ref_V + (um.ref_row + o) * D + sub * CPL, mv);
+        }
+        for (int i2 = 1; i2 < keff; ++i2) {
+            const int o = chosen_s[i2];
+            float rk[CPL], rv[CPL];
+            load_bf16_row<CPL>(a.ref_K + (um.ref_row + o) * D + sub * CPL, rk);
+            load_bf16_row<CPL>(a.ref_V + (um.ref_row + o) * D + sub * CPL, rv);
+#pragma unroll
+            for (int j2 = 0; j2 < CPL; ++j2) {
+                mk[j2] = __fadd_rn(mk[j2], rk[j2]);
+                mv[j2] = __fadd_rn(mv[j2], rv[j2]);
+            }
+        }
+        if (keff & (keff - 1)) {
+            const float fk = static_cast<float>(keff);
+#pragma unroll
+            for (int j2 = 0; j2 < CPL; ++j2) {
+                mk[j2] = __fdiv_rn(mk[j2], fk);
+                mv[j2] = __fdiv_rn(mv[j2], fk);
+            }
+        } else {
+            const float inv = 1.0f / static_cast<float>(keff);
+#pragma unroll
+            for (int j2 = 0; j2 < CPL; ++j2) {
+                mk[j2] = __fmul_rn(mk[j2], inv);
+                mv[j2] = __fmul_rn(mv[j2], inv);
+            }
+        }
+        quantise_store<CPL>(xk, mk, a.bits, sub, store, a.codes_K + row * a.code_bytes,
+                            a.scale_K + row * a.n_groups, a.err);
+        quantise_store<CPL>(xv, mv, a.bits, sub, store, a.codes_V + row * a.code_bytes,
+                            a.scale_V + row * a.n_groups, a.err);
+        __syncwarp();
+        if (lane == 0) {
+            __threadfence();
+            um_ptr->C = um.C + 1;
+            um_ptr->n = p + 1;
+        }
+    }
+}
+
 template <int CPL, int LPT>
 cudaError_t launch_cpl(const CacheArgs& a, int max_C, const void* K, const void* V, const uint16_t* ci,
                        const float* ct, cudaStream_t st)
@@ -464,6 +684,18 @@ cudaError_t launch_cpl(const CacheArgs& a, int max_C, const void* K, const void*
 }
 
 }  // namespace
+
+cudaError_t launch_append(const CacheArgs& a, const void* K_new, const void* V_new, const uint32_t (&active)[8],
+                          cudaStream_t st)
+{
+    if (a.D == 128)
+        append_kernel<128><<<a.n_units, kAppendThreads, 0, st>>>(a, K_new, V_new, active[0], active[1], active[2],
+                                                               active[3], active[4], active[5], active[6], active[7]);
+    else
+        append_kernel<64><<<a.n_units, kAppendThreads, 0, st>>>(a, K_new, V_new, active[0], active[1], active[2],
+                                                              active[3], active[4], active[5], active[6], active[7]);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_encode(const CacheArgs& a, int max_C, const void* K, const void* V, const uint16_t* cand_idx,
                           const float* cand_t, cudaStream_t st)

@@ -20,6 +20,11 @@ cudaError_t launch_select_tc(const CacheArgs& a, const Tile* tiles, int n_tiles,
 cudaError_t launch_encode(const CacheArgs& a, int max_C, const void* K, const void* V, const uint16_t* cand_idx,
                           const float* cand_t, cudaStream_t st);
 
+// Incremental compression: one new token ([unit][D] rows) for every unit of the sequences whose
+// bit is set in active (256 bits).
+cudaError_t launch_append(const CacheArgs& a, const void* K_new, const void* V_new, const uint32_t (&active)[8],
+                          cudaStream_t st);
+
 cudaError_t launch_reconstruct(const CacheArgs& a, int unit, const int32_t* positions, int64_t n_pos, void* K_out,
                                void* V_out, int out_dtype, cudaStream_t st);
 

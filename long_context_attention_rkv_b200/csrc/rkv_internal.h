@@ -73,6 +73,7 @@ struct Desc {
     int32_t Cpad[RKV_MAX_BATCH];
     int64_t ref_seq_row[RKV_MAX_BATCH];
     int64_t cmp_seq_row[RKV_MAX_BATCH];
+    int32_t cur_len[RKV_MAX_BATCH];   // current lengths (len[] is the capacity the layout holds)
 };
 static_assert(sizeof(Desc) <= RKV_CACHE_DESC_BYTES, "descriptor too large");
 

@@ -39,15 +39,37 @@ class GpuRun:
     """One layer compressed on the GPU through the C ABI."""
 
     def __init__(self, wl: synth.Workload, K: np.ndarray, V: np.ndarray, lengths, out_dtype=rkv.RKV_DTYPE_F32,
-                 flags=0):
+                 flags=0, start_lengths=None):
+        """lengths: the bound (capacity) lengths; start_lengths: a shorter prefix to compress
+        first (grown later with append_until)."""
         self.wl = wl
         self.lengths = list(lengths)
         self.cfg = config(wl, lengths, max_len=K.shape[2], out_dtype=out_dtype, flags=flags)
         self.layer = rkv.Layer(self.cfg, self.lengths)
         self.Kd = to_dev(K)
         self.Vd = to_dev(V)
+        self.cur = list(self.lengths if start_lengths is None else start_lengths)
+        if start_lengths is not None:
+            self.layer.set_lengths(self.cur)
         self.layer.build_refs(self.Kd, self.Vd)
         self.layer.compress(self.Kd, self.Vd)
+        torch.cuda.synchronize()
+        err = self.layer.device_error()
+        assert err == 0, f"device error {rkv.STATUS.get(err, err)}"
+
+    def append_until(self, target):
+        """Appends each sequence's next tokens (from the same K, V) until it reaches target."""
+        B, Hkv = len(self.lengths), self.wl.n_kv_heads
+        bi = torch.arange(B, device="cuda").repeat_interleave(Hkv)
+        hi = torch.arange(Hkv, device="cuda").repeat(B)
+        while any(c < t for c, t in zip(self.cur, target)):
+            act = [1 if self.cur[b] < target[b] else 0 for b in range(B)]
+            pos = torch.tensor([min(self.cur[b], self.Kd.shape[2] - 1) for b in range(B)],
+                               device="cuda").repeat_interleave(Hkv)
+            Kn = self.Kd[bi, hi, pos].contiguous()
+            Vn = self.Vd[bi, hi, pos].contiguous()
+            self.layer.append(Kn, Vn, act)
+            self.cur = [c + a for c, a in zip(self.cur, act)]
         torch.cuda.synchronize()
         err = self.layer.device_error()
         assert err == 0, f"device error {rkv.STATUS.get(err, err)}"

@@ -290,3 +290,33 @@ def test_sparse_decode_reports_out_of_range_positions():
     run.layer.decode_sparse(to_dev(synth.gen_query(wl, 0, 0)), pos, cnt, out)
     torch.cuda.synchronize()
     assert run.layer.device_error() == rkv.STATUS_CODE["RKV_ERR_INVALID_ARG"]
+
+
+@pytest.mark.parametrize("case", ["llama_int4", "dynamic_int8_d64"])
+def test_append_equals_compressing_the_whole_sequence(case):
+    """Incremental compression: a prefix compressed, then one token appended at a time (to
+    both sequences, then to one of them), checked against the oracle's compression of the
+    full sequences and decode over the grown cache."""
+    if case == "llama_int4":
+        wl = _small("llama3_8b_layer", n_kv_heads=2, n_q_heads=8, batch=2, seq_len=2600, ragged=None)
+        cap, start = [2600, 2100], [1700, 900]
+    else:
+        wl = _small("ultra_long_1m", n_kv_heads=1, n_q_heads=4, head_dim=64, stride0=4, refs_per_phase=64, k=3,
+                    bits=8, seq_len=1500, n_proto=64)
+        cap, start = [1500], [200]
+    K, V = synth.gen_layer(wl, 0, cap)
+    run = GpuRun(wl, K, V, cap, start_lengths=start)
+    mid = [min(c, s + 300) for c, s in zip(cap, start)]
+    run.append_until(mid)                        # every sequence
+    run.append_until(cap)                        # then each up to its own capacity
+    for b, n in enumerate(cap):
+        for h in range(wl.n_kv_heads):
+            g = run.unit(b, h)
+            assert g["n"] == n
+            Xk, Xv = unit_rows(wl, K, V, b, h, n)
+            check_refs(wl, g, Xk, Xv)
+            check_compress(wl, g, Xk, Xv)
+    check_decode(run, synth.gen_query(wl, 0, 0))
+    with pytest.raises(rkv.RkvError) as ei:      # at capacity: refused, nothing launched
+        run.layer.append(run.Kd[:, :, 0].contiguous(), run.Vd[:, :, 0].contiguous())
+    assert ei.value.status == rkv.STATUS_CODE["RKV_ERR_INVALID_ARG"]
