@@ -9,7 +9,8 @@ region starts; L2 is flushed (256 MiB write) before every timed step, outside
 the timed spans.  With N GPUs (torchrun) every rank runs its own replica on an
 independent layer; value is the whole-job throughput over the max-over-ranks
 step time.  Outside the step, a selective decode (2048 seeded positions per unit)
-is timed as well.  `--impl reference` times the CPU oracle on a bounded sample of
+and incremental compression (the last 64 tokens appended one at a time) are timed as
+well.  `--impl reference` times the CPU oracle on a bounded sample of
 the same workload on the host cores.  Prints one JSON line on rank 0.
 """
 from __future__ import annotations
@@ -36,6 +37,7 @@ WORKLOAD = "llama3_8b_layer"
 LAUNCHES = {"build_refs": 1, "search": 1, "encode": 1, "decode": 3, "reconstruct": 1}
 RECON_ROWS = 256
 SPARSE_SEL = 2048          # positions per unit of the selective-decode measurement
+APPEND_TOKENS = 64         # tokens appended one at a time in the incremental-compression measurement
 
 
 def replica_layer(rank: int) -> int:
@@ -420,6 +422,36 @@ def run_ours(args, rank, world, local_rank):
     assert L.device_error() == 0
     sparse_us = 1e3 * statistics.mean(sp_ms)
 
+    # incremental compression (outside the step): the last APPEND_TOKENS positions of every
+    # sequence appended one at a time to a layer compressed up to them
+    La = rkv.Layer(cfg, lengths, device=dev)
+    start = [max(0, n - APPEND_TOKENS) for n in lengths]
+    La.set_lengths(start)
+    La.build_refs(K, V)
+    La.compress(K, V)
+    Hkv = wl.n_kv_heads
+    bi = torch.arange(wl.batch, device=dev).repeat_interleave(Hkv)
+    hi = torch.arange(Hkv, device=dev).repeat(wl.batch)
+    rows = []
+    for t in range(APPEND_TOKENS):
+        pos = torch.tensor([min(s0 + t, K.shape[2] - 1) for s0 in start], device=dev).repeat_interleave(Hkv)
+        rows.append((K[bi, hi, pos].contiguous(), V[bi, hi, pos].contiguous()))
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        # a busy-wait ahead of the timed span keeps the device behind the host while the
+        # appends are issued, so the span holds the appends' device time, not Python's
+        torch.cuda._sleep(20_000_000)
+        e0.record(stream)
+        for Kn, Vn in rows:
+            La.append(Kn, Vn, stream=stream)
+        e1.record(stream)
+        e1.synchronize()
+    assert La.device_error() == 0
+    append_us = 1e3 * e0.elapsed_time(e1) / APPEND_TOKENS
+    del La
+
     Q = workload_quantities(wl, lengths)
     tokens = Q["tokens"]
     value = job_throughput(world, tokens, mean_step)
@@ -470,6 +502,7 @@ def run_ours(args, rank, world, local_rank):
                 "encode_gbs": encode_gbs, "compress_mtok_s": tokens / ((avg["search"] + avg["encode"] +
                                                                         avg["build_refs"]) * 1e-3) / 1e6,
                 "sparse_decode_us": sparse_us, "sparse_decode_positions_per_unit": SPARSE_SEL,
+                "append_us_per_token": append_us,
             },
             "roofline": roofline,
             "cpu_baseline": cpu,

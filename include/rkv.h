@@ -271,6 +271,10 @@ RKV_API rkv_status rkv_cache_set_lengths(rkv_cache_desc* desc, const int32_t* le
  * rkv_compress would (nearest by exact L2 distance, ties to the lower ordinal).
  *   K_new, V_new  device [batch][n_kv_heads][head_dim], the cache's input dtype;
  *                 rows of inactive sequences are not read
+ * Two launches: the distances to the references, split over up to 32 CTAs per unit,
+ * each keeping its k best; then per unit the merge, the mean and the quantiser.  The
+ * candidate lists live in a small scratch section of the cache buffer (about 6 KB per
+ * unit, counted by rkv_cache_size), so appends to one cache run on one stream.
  * Fails with RKV_ERR_INVALID_ARG, launching nothing, if an active sequence is at
  * capacity.  The current lengths advance on return (the work is queued on stream).
  */

@@ -182,6 +182,7 @@ rkv_status compute_layout(const rkv_config* c, const int32_t* lengths, Desc& d)
     s.scale_K = take(2ull * cmp_rows * d.n_groups);
     s.scale_V = take(2ull * cmp_rows * d.n_groups);
     s.idx = take(2ull * cmp_rows * c->k);
+    s.append = take(append_scratch_bytes(d.n_units));   // per-unit candidate lists of rkv_append
     s.end = off;
     d.ws_select = align_up(2ull * cmp_rows * d.kc, 256) + align_up(4ull * cmp_rows * d.kc, 256);
     const int splits = std::max(decode_splits(d.n_units, max_n), sparse_splits_max(d.n_units));
@@ -576,7 +577,8 @@ rkv_status rkv_append(rkv_cache_desc* desc, const void* K_new, const void* V_new
     if (!any)
         return RKV_OK;
     const CacheArgs a = make_args(*d);
-    const cudaError_t e = launch_append(a, K_new, V_new, bits, static_cast<cudaStream_t>(stream));
+    const cudaError_t e = launch_append(a, K_new, V_new, bits, static_cast<char*>(d->base) + d->sec.append,
+                                        static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess)
         return RKV_ERR_CUDA;
     for (int b = 0; b < d->cfg.batch; ++b)

@@ -458,26 +458,149 @@ __global__ void __launch_bounds__(kWarps * 32, encode_min_blocks<KC, LPT>()) enc
 // search's definition evaluated directly), the mean in ascending ordinal order and the group
 // quantiser of the encoder.  The unit's counts advance on the device.
 constexpr int kAppendThreads = 128;
+constexpr int kAppendKM = 16;                   // largest k
 
+// Per-unit candidate lists of the append search: chunk c of unit u holds the k best (distance,
+// ordinal) of its share of the references, in ascending (distance, ordinal) order.
+__host__ __device__ inline int append_chunks(int max_refs)
+{
+    const int c = (max_refs + kAppendThreads - 1) / kAppendThreads;
+    return c < 1 ? 1 : (c > 32 ? 32 : c);
+}
+
+__device__ __forceinline__ bool seq_active(const uint32_t (&act)[8], int seq) { return (act[seq >> 5] >> (seq & 31)) & 1u; }
+
+// 1. distances of the new token's key to a chunk of the unit's references, the chunk's k best.
+template <int D>
+__global__ void __launch_bounds__(kAppendThreads) append_search_kernel(CacheArgs a, const void* __restrict__ Kn,
+                                                                        uint32_t act0, uint32_t act1, uint32_t act2,
+                                                                        uint32_t act3, uint32_t act4, uint32_t act5,
+                                                                        uint32_t act6, uint32_t act7,
+                                                                        double* __restrict__ ws_d,
+                                                                        int* __restrict__ ws_j, int n_chunks)
+{
+    constexpr int KM = kAppendKM;
+    __shared__ float xs[D];
+    __shared__ double bd_s[kAppendThreads / 32][KM];
+    __shared__ int bo_s[kAppendThreads / 32][KM];
+    const int u = blockIdx.y, ch = blockIdx.x;
+    const UnitMeta um = a.units[u];
+    const uint32_t act[8] = {act0, act1, act2, act3, act4, act5, act6, act7};
+    const int p = um.n;
+    if (!seq_active(act, um.seq) || is_ref_pos(a.ph, p))
+        return;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int R = um.R, k = a.k;
+    const int per = (R + n_chunks - 1) / n_chunks;
+    const int j_lo = ch * per, j_hi = min(R, j_lo + per);
+    const int64_t e_row = static_cast<int64_t>(u) * D;
+    for (int c = tid; c < D; c += kAppendThreads)
+        xs[c] = (a.in_dtype == RKV_DTYPE_F32) ? static_cast<const float*>(Kn)[e_row + c]
+                                              : bf16_bits_to_f32(static_cast<const uint16_t*>(Kn)[e_row + c]);
+    __syncthreads();
+    double bd[KM];
+    int bo[KM];
+#pragma unroll
+    for (int s2 = 0; s2 < KM; ++s2) {
+        bd[s2] = DBL_MAX;
+        bo[s2] = 0x7fffffff;
+    }
+    for (int j = j_lo + tid; j < j_hi; j += kAppendThreads) {
+        // distance in double, channels in order, no contraction (the search's definition)
+        const uint4* r4 = reinterpret_cast<const uint4*>(a.ref_K + (um.ref_row + j) * D);
+        double d = 0.0;
+#pragma unroll 2
+        for (int c8 = 0; c8 < D / 8; ++c8) {
+            const uint4 w = r4[c8];
+            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float rv = bf16_bits_to_f32((i & 1) ? (ww[i >> 1] >> 16) : (ww[i >> 1] & 0xffffu));
+                const double t = __dsub_rn(static_cast<double>(xs[c8 * 8 + i]), static_cast<double>(rv));
+                d = __dadd_rn(d, __dmul_rn(t, t));
+            }
+        }
+        double cv = d;
+        int ci = j;
+#pragma unroll
+        for (int s2 = 0; s2 < KM; ++s2) {
+            if (s2 < k) {
+                const bool before = (cv < bd[s2]) || (cv == bd[s2] && ci < bo[s2]);
+                const double fd = bd[s2];
+                const int fo = bo[s2];
+                bd[s2] = before ? cv : fd;
+                bo[s2] = before ? ci : fo;
+                cv = before ? fd : cv;
+                ci = before ? fo : ci;
+            }
+        }
+    }
+    // k rounds of a warp-wide minimum, then the four warps' lists in thread 0
+    int head = 0;
+    for (int r2 = 0; r2 < k; ++r2) {
+        double hd = DBL_MAX;
+        int ho = 0x7fffffff;
+#pragma unroll
+        for (int s2 = 0; s2 < KM; ++s2)
+            if (s2 == head) {
+                hd = bd[s2];
+                ho = bo[s2];
+            }
+        double wd = hd;
+        int wo = ho;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const double od = __shfl_xor_sync(0xffffffffu, wd, off);
+            const int oo = __shfl_xor_sync(0xffffffffu, wo, off);
+            if (od < wd || (od == wd && oo < wo)) {
+                wd = od;
+                wo = oo;
+            }
+        }
+        if (ho == wo && hd == wd)
+            ++head;
+        if (lane == 0) {
+            bd_s[warp][r2] = wd;
+            bo_s[warp][r2] = wo;
+        }
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int hp[kAppendThreads / 32] = {};
+        const int64_t base = (static_cast<int64_t>(u) * n_chunks + ch) * KM;
+        for (int r2 = 0; r2 < k; ++r2) {
+            int bw = 0;
+            for (int w2 = 1; w2 < kAppendThreads / 32; ++w2) {
+                const double dw = bd_s[w2][hp[w2]], db = bd_s[bw][hp[bw]];
+                if (dw < db || (dw == db && bo_s[w2][hp[w2]] < bo_s[bw][hp[bw]]))
+                    bw = w2;
+            }
+            ws_d[base + r2] = bd_s[bw][hp[bw]];
+            ws_j[base + r2] = bo_s[bw][hp[bw]];
+            ++hp[bw];
+        }
+    }
+}
+
+// 2. the new token itself: a reference row, or the merge of the chunks' lists, the mean and the
+// encoder's quantiser.  The unit's counts advance on the device.
 template <int D>
 __global__ void __launch_bounds__(kAppendThreads) append_kernel(CacheArgs a, const void* __restrict__ Kn,
                                                                  const void* __restrict__ Vn, uint32_t act0,
                                                                  uint32_t act1, uint32_t act2, uint32_t act3,
                                                                  uint32_t act4, uint32_t act5, uint32_t act6,
-                                                                 uint32_t act7)
+                                                                 uint32_t act7, const double* __restrict__ ws_d,
+                                                                 const int* __restrict__ ws_j, int n_chunks)
 {
-    constexpr int KM = 16;                      // largest k
+    constexpr int KM = kAppendKM;
     constexpr int CPL = 8;                      // channels per lane in the encode step
     constexpr int LPT = D / CPL;
-    __shared__ float xs[D];
-    __shared__ double bd_s[kAppendThreads / 32][KM];
-    __shared__ int bo_s[kAppendThreads / 32][KM];
     __shared__ int chosen_s[KM];
     const int u = blockIdx.x;
     UnitMeta* um_ptr = const_cast<UnitMeta*>(a.units) + u;
     const UnitMeta um = *um_ptr;
     const uint32_t act[8] = {act0, act1, act2, act3, act4, act5, act6, act7};
-    if (!((act[um.seq >> 5] >> (um.seq & 31)) & 1u))
+    if (!seq_active(act, um.seq))
         return;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int p = um.n;
@@ -520,87 +643,26 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(CacheArgs a, con
         }
         return;
     }
-    // ---- compressed token: exact top-k over the references so far -------------------------
+    // ---- compressed token: the k best of the chunks' lists -------------------------------
     const int R = um.R;
     const int k = a.k;
     const int keff = min(k, R);
-    for (int c = tid; c < D; c += kAppendThreads)
-        xs[c] = (a.in_dtype == RKV_DTYPE_F32) ? static_cast<const float*>(Kn)[e_row + c]
-                                              : bf16_bits_to_f32(static_cast<const uint16_t*>(Kn)[e_row + c]);
-    __syncthreads();
-    double bd[KM];
-    int bo[KM];
-#pragma unroll
-    for (int s2 = 0; s2 < KM; ++s2) {
-        bd[s2] = DBL_MAX;
-        bo[s2] = 0x7fffffff;
-    }
-    for (int j = tid; j < R; j += kAppendThreads) {
-        const uint16_t* r = a.ref_K + (um.ref_row + j) * D;
-        double d = 0.0;
-        for (int c = 0; c < D; ++c) {
-            const double t = __dsub_rn(static_cast<double>(xs[c]), static_cast<double>(bf16_bits_to_f32(r[c])));
-            d = __dadd_rn(d, __dmul_rn(t, t));
-        }
-        double cv = d;
-        int ci = j;
-#pragma unroll
-        for (int s2 = 0; s2 < KM; ++s2) {
-            if (s2 < k) {
-                const bool before = (cv < bd[s2]) || (cv == bd[s2] && ci < bo[s2]);
-                const double fd = bd[s2];
-                const int fo = bo[s2];
-                bd[s2] = before ? cv : fd;
-                bo[s2] = before ? ci : fo;
-                cv = before ? fd : cv;
-                ci = before ? fo : ci;
-            }
-        }
-    }
-    // merge: k rounds of a warp-wide minimum, then the warps' lists in thread 0
-    {
-        int head = 0;
-        for (int r2 = 0; r2 < k; ++r2) {
-            double hd = DBL_MAX;
-            int ho = 0x7fffffff;
-#pragma unroll
-            for (int s2 = 0; s2 < KM; ++s2)
-                if (s2 == head) {
-                    hd = bd[s2];
-                    ho = bo[s2];
-                }
-            double wd = hd;
-            int wo = ho;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const double od = __shfl_xor_sync(0xffffffffu, wd, off);
-                const int oo = __shfl_xor_sync(0xffffffffu, wo, off);
-                if (od < wd || (od == wd && oo < wo)) {
-                    wd = od;
-                    wo = oo;
-                }
-            }
-            if (ho == wo && hd == wd)
-                ++head;
-            if (lane == 0) {
-                bd_s[warp][r2] = wd;
-                bo_s[warp][r2] = wo;
-            }
-        }
-    }
-    __syncthreads();
     if (tid == 0) {
-        int hp[kAppendThreads / 32] = {};
+        int hp[32] = {};
         int ch[KM];
+        const int64_t base = static_cast<int64_t>(u) * n_chunks * KM;
         for (int r2 = 0; r2 < keff; ++r2) {
-            int bw = 0;
-            for (int w2 = 1; w2 < kAppendThreads / 32; ++w2) {
-                const double dw = bd_s[w2][hp[w2]], db = bd_s[bw][hp[bw]];
-                if (dw < db || (dw == db && bo_s[w2][hp[w2]] < bo_s[bw][hp[bw]]))
-                    bw = w2;
+            int bc = 0;
+            for (int c2 = 1; c2 < n_chunks; ++c2) {
+                const double dc = (hp[c2] < k) ? ws_d[base + c2 * KM + hp[c2]] : DBL_MAX;
+                const int jc = (hp[c2] < k) ? ws_j[base + c2 * KM + hp[c2]] : 0x7fffffff;
+                const double db = (hp[bc] < k) ? ws_d[base + bc * KM + hp[bc]] : DBL_MAX;
+                const int jb = (hp[bc] < k) ? ws_j[base + bc * KM + hp[bc]] : 0x7fffffff;
+                if (dc < db || (dc == db && jc < jb))
+                    bc = c2;
             }
-            ch[r2] = bo_s[bw][hp[bw]];
-            ++hp[bw];
+            ch[r2] = ws_j[base + bc * KM + hp[bc]];
+            ++hp[bc];
         }
         // ascending ordinal order
         for (int i2 = 1; i2 < keff; ++i2)
@@ -685,15 +747,29 @@ cudaError_t launch_cpl(const CacheArgs& a, int max_C, const void* K, const void*
 
 }  // namespace
 
-cudaError_t launch_append(const CacheArgs& a, const void* K_new, const void* V_new, const uint32_t (&active)[8],
-                          cudaStream_t st)
+uint64_t append_scratch_bytes(int n_units)
 {
-    if (a.D == 128)
-        append_kernel<128><<<a.n_units, kAppendThreads, 0, st>>>(a, K_new, V_new, active[0], active[1], active[2],
-                                                               active[3], active[4], active[5], active[6], active[7]);
-    else
-        append_kernel<64><<<a.n_units, kAppendThreads, 0, st>>>(a, K_new, V_new, active[0], active[1], active[2],
-                                                              active[3], active[4], active[5], active[6], active[7]);
+    return static_cast<uint64_t>(n_units) * 32 * kAppendKM * (sizeof(double) + sizeof(int));
+}
+
+cudaError_t launch_append(const CacheArgs& a, const void* K_new, const void* V_new, const uint32_t (&active)[8],
+                          void* scratch, cudaStream_t st)
+{
+    const int nc = append_chunks(a.max_refs);
+    double* ws_d = static_cast<double*>(scratch);
+    int* ws_j = reinterpret_cast<int*>(ws_d + static_cast<int64_t>(a.n_units) * 32 * kAppendKM);
+    const uint32_t* b = active;
+    if (a.D == 128) {
+        append_search_kernel<128><<<dim3(nc, a.n_units), kAppendThreads, 0, st>>>(
+            a, K_new, b[0], b[1], b[2], b[3], b[4], b[5], b[6], b[7], ws_d, ws_j, nc);
+        append_kernel<128><<<a.n_units, kAppendThreads, 0, st>>>(a, K_new, V_new, b[0], b[1], b[2], b[3], b[4], b[5],
+                                                               b[6], b[7], ws_d, ws_j, nc);
+    } else {
+        append_search_kernel<64><<<dim3(nc, a.n_units), kAppendThreads, 0, st>>>(
+            a, K_new, b[0], b[1], b[2], b[3], b[4], b[5], b[6], b[7], ws_d, ws_j, nc);
+        append_kernel<64><<<a.n_units, kAppendThreads, 0, st>>>(a, K_new, V_new, b[0], b[1], b[2], b[3], b[4], b[5],
+                                                              b[6], b[7], ws_d, ws_j, nc);
+    }
     return cudaGetLastError();
 }
 

@@ -22,8 +22,10 @@ cudaError_t launch_encode(const CacheArgs& a, int max_C, const void* K, const vo
 
 // Incremental compression: one new token ([unit][D] rows) for every unit of the sequences whose
 // bit is set in active (256 bits).
+// Scratch that rkv_append needs inside the cache buffer (per-unit candidate lists).
+uint64_t append_scratch_bytes(int n_units);
 cudaError_t launch_append(const CacheArgs& a, const void* K_new, const void* V_new, const uint32_t (&active)[8],
-                          cudaStream_t st);
+                          void* scratch, cudaStream_t st);
 
 cudaError_t launch_reconstruct(const CacheArgs& a, int unit, const int32_t* positions, int64_t n_pos, void* K_out,
                                void* V_out, int out_dtype, cudaStream_t st);

@@ -41,7 +41,7 @@ struct UnitMeta {
 // Byte offsets of the cache sections inside the caller's buffer.
 struct Sections {
     uint64_t err, units, tiles, pairs, ref_K, ref_V, ref_hn, ref_aug, ref_pos, codes_K, codes_V, scale_K, scale_V, idx,
-        end;
+        append, end;
 };
 
 // Host-side descriptor stored in rkv_cache_desc::opaque.

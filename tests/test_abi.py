@@ -45,8 +45,9 @@ def test_cache_size_accounts_every_array():
     cb, wb = rkv.rkv_cache_size(_cfg(), lengths)
     R, C, H, D = 2048, 30720, 8, 128
     # reference rows (K, V bf16), half norm + position, augmented search column (16 bf16),
-    # then per compressed token: codes K/V, scales K/V, 4 ordinals
-    payload = H * (2 * R * D * 2 + R * 8 + R * 32 + C * (2 * 64 + 2 * 8 + 4 * 2))
+    # then per compressed token: codes K/V, scales K/V, 4 ordinals; per unit the append
+    # search's candidate lists (32 chunks x 16 (distance f64, ordinal i32))
+    payload = H * (2 * R * D * 2 + R * 8 + R * 32 + C * (2 * 64 + 2 * 8 + 4 * 2) + 32 * 16 * 12)
     assert payload <= cb <= payload + 64 * 1024
     assert wb >= H * C * 8 * 6            # search candidates: kc = 8 ordinals + scores per token
 
