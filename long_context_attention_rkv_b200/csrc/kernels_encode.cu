@@ -53,6 +53,29 @@ __device__ __forceinline__ float tmax(float v)
     return v;
 }
 
+// Packed fp32 pairs (sm_100 f32x2): two correctly rounded operations, no contraction, the
+// same results as two __fadd_rn / __fsub_rn / __fmul_rn.
+__device__ __forceinline__ void add2_rn(float& a0, float& a1, float b0, float b1)
+{
+    asm("{\n\t.reg .b64 x, y;\n\tmov.b64 x, {%0, %1};\n\tmov.b64 y, {%2, %3};\n\t"
+        "add.rn.f32x2 x, x, y;\n\tmov.b64 {%0, %1}, x;\n\t}"
+        : "+f"(a0), "+f"(a1) : "f"(b0), "f"(b1));
+}
+
+__device__ __forceinline__ void sub2_rn(float& d0, float& d1, float a0, float a1, float b0, float b1)
+{
+    asm("{\n\t.reg .b64 x, y;\n\tmov.b64 x, {%2, %3};\n\tmov.b64 y, {%4, %5};\n\t"
+        "sub.rn.f32x2 x, x, y;\n\tmov.b64 {%0, %1}, x;\n\t}"
+        : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+__device__ __forceinline__ void mul2_rn(float& a0, float& a1, float b0, float b1)
+{
+    asm("{\n\t.reg .b64 x, y;\n\tmov.b64 x, {%0, %1};\n\tmov.b64 y, {%2, %3};\n\t"
+        "mul.rn.f32x2 x, x, y;\n\tmov.b64 {%0, %1}, x;\n\t}"
+        : "+f"(a0), "+f"(a1) : "f"(b0), "f"(b1));
+}
+
 // CPL consecutive bf16 values (CPL = 8 or 16) as floats.
 template <int CPL>
 __device__ __forceinline__ void load_bf16_row(const uint16_t* p, float (&out)[CPL])
@@ -113,10 +136,11 @@ __device__ __forceinline__ void quantise_store(const float (&x)[CPL], const floa
     float d[CPL];
     float amax = 0.0f;
 #pragma unroll
-    for (int i = 0; i < CPL; ++i) {
-        d[i] = __fsub_rn(x[i], m[i]);
+    for (int i = 0; i < CPL; i += 2)
+        sub2_rn(d[i], d[i + 1], x[i], x[i + 1], m[i], m[i + 1]);
+#pragma unroll
+    for (int i = 0; i < CPL; ++i)
         amax = fmaxf(amax, fabsf(d[i]));
-    }
 #pragma unroll
     for (int off = 1; off < LPG; off <<= 1)
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
@@ -129,10 +153,33 @@ __device__ __forceinline__ void quantise_store(const float (&x)[CPL], const floa
         if (store && (sbits & 0x7c00u) == 0x7c00u)
             report(err, RKV_ERR_UNSUPPORTED);
     }
+    // code = rint(fl(d / s)).  y = d * fl(1/s) is within 1.5 * 2^-23 |d/s| of fl(d/s), and
+    // |d/s| <= qmax < 128, so the two differ by less than 2^-15: unless y lies within 2^-14 of
+    // a half-integer, both round to the same integer.  The rare lanes that do take the
+    // correctly rounded division for their elements.
+    const float rs = __frcp_rn(s);
+    float yv[CPL], y[CPL];
+#pragma unroll
+    for (int i = 0; i < CPL; i += 2) {
+        yv[i] = d[i];
+        yv[i + 1] = d[i + 1];
+        mul2_rn(yv[i], yv[i + 1], rs, rs);
+    }
+    bool near_half = false;
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) {
+        y[i] = rintf(yv[i]);
+        near_half |= fabsf(__fsub_rn(yv[i], y[i])) >= 0.5f - 0x1p-14f;
+    }
+    if (near_half) {
+#pragma unroll
+        for (int i = 0; i < CPL; ++i)
+            y[i] = rintf(__fdiv_rn(d[i], s));
+    }
     int q[CPL];
 #pragma unroll
     for (int i = 0; i < CPL; ++i) {
-        int c = static_cast<int>(rintf(__fdiv_rn(d[i], s)));
+        const int c = static_cast<int>(y[i]);
         q[i] = (amax > 0.0f) ? max(-qmax, min(qmax, c)) : 0;
     }
     if (!store)
@@ -418,9 +465,9 @@ __global__ void __launch_bounds__(kWarps * 32, encode_min_blocks<KC, LPT>()) enc
         load_bf16_row<CPL>(a.ref_K + (um.ref_row + o) * D + sub * CPL, rk);
         load_bf16_row<CPL>(a.ref_V + (um.ref_row + o) * D + sub * CPL, rv);
 #pragma unroll
-        for (int j2 = 0; j2 < CPL; ++j2) {
-            mk[j2] = __fadd_rn(mk[j2], rk[j2]);
-            mv[j2] = __fadd_rn(mv[j2], rv[j2]);
+        for (int j2 = 0; j2 < CPL; j2 += 2) {
+            add2_rn(mk[j2], mk[j2 + 1], rk[j2], rk[j2 + 1]);
+            add2_rn(mv[j2], mv[j2 + 1], rv[j2], rv[j2 + 1]);
         }
     }
     if (keff & (keff - 1)) {
@@ -434,9 +481,9 @@ __global__ void __launch_bounds__(kWarps * 32, encode_min_blocks<KC, LPT>()) enc
         // keff a power of two: the division is an exact scaling
         const float inv = 1.0f / static_cast<float>(keff);
 #pragma unroll
-        for (int j2 = 0; j2 < CPL; ++j2) {
-            mk[j2] = __fmul_rn(mk[j2], inv);
-            mv[j2] = __fmul_rn(mv[j2], inv);
+        for (int j2 = 0; j2 < CPL; j2 += 2) {
+            mul2_rn(mk[j2], mk[j2 + 1], inv, inv);
+            mul2_rn(mv[j2], mv[j2 + 1], inv, inv);
         }
     }
 

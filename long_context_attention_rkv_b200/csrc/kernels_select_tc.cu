@@ -142,6 +142,56 @@ __device__ __forceinline__ int item_candidates(const CacheArgs& a, const UnitMet
     return min(refs_upto(a.ph, p_last), um.R);
 }
 
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// Maxima of the eight 16-column blocks of one accumulator tile (this thread's row); columns
+// j0 + c at or past ncand count as -inf.
+__device__ __forceinline__ void block_maxima(uint32_t col, int j0, int ncand, float* mx)
+{
+#pragma unroll
+    for (int c0 = 0; c0 < kN; c0 += 32) {
+        float v[32];
+        tmem_ld32(col + c0, v);
+        if (j0 + c0 + 32 > ncand) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                v[i] = (j0 + c0 + i < ncand) ? v[i] : -FLT_MAX;
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const float* b = v + 16 * h;
+            const float m0 = fmax3(b[0], b[1], b[2]), m1 = fmax3(b[3], b[4], b[5]);
+            const float m2 = fmax3(b[6], b[7], b[8]), m3 = fmax3(b[9], b[10], b[11]);
+            const float m4 = fmax3(b[12], b[13], b[14]);
+            mx[c0 / 16 + h] = fmax3(fmax3(m0, m1, m2), fmax3(m3, m4, b[15]), -FLT_MAX);
+        }
+    }
+}
+
+// Sorts 16 values in descending order (bitonic network).
+__device__ __forceinline__ void sort16_desc(float (&x)[16])
+{
+#pragma unroll
+    for (int k = 2; k <= 16; k <<= 1)
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1)
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int l = i ^ j;
+                if (l > i) {
+                    const float a = x[i], b = x[l];
+                    const bool desc = (i & k) == 0;
+                    x[i] = desc ? fmaxf(a, b) : fminf(a, b);
+                    x[l] = desc ? fminf(a, b) : fmaxf(a, b);
+                }
+            }
+}
+
 // Drains this thread's queue (entries [0, cnt)) into its sorted list, in lockstep with the warp.
 template <int KC>
 __device__ __forceinline__ void drain(const float2* q, int cnt, float (&tv)[KC], int (&ti)[KC])
@@ -377,7 +427,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const int j0 = r * kN;
                 const uint32_t col0 = lane_base + (acc * kTiles + t) * kN;
-                if (r == 0 && nc_max >= kN && KC <= kN / 16) {
+                if (r == 0 && nrt >= 2 && KC <= 16) {
+                    // the KC-th largest of the sixteen block maxima of the first two reference
+                    // tiles (distinct elements) bounds the kc-th best t from below; the first
+                    // tile stays in TMEM while the second is read, and is scanned after
+                    float mx[16];
+                    block_maxima(col0, 0, ncand, mx);
+                    const int acc1 = (it_c + 1) % kAcc;
+                    int got1 = 1;
+                    if (lane == 0)
+                        got1 = mbar_wait(&bars->acc_full[acc1], ((it_c + 1) / kAcc) & 1, abort) ? 1 : 0;
+                    ok = __shfl_sync(0xffffffffu, got1, 0) != 0;
+                    if (!ok)
+                        break;
+                    tc_fence_after();
+                    block_maxima(lane_base + (acc1 * kTiles + t) * kN, kN, ncand, mx + 8);
+                    sort16_desc(mx);
+                    seed = mx[KC - 1];
+                    seed_lo = (seed > -FLT_MAX) ? nextafterf(seed, -FLT_MAX) : -FLT_MAX;
+                } else if (r == 0 && nc_max >= kN && KC <= kN / 16) {
                     // the kc largest of kN/16 sub-block maxima are distinct elements, so the
                     // smallest of them bounds the kc-th best t from below
                     float mxs[kN / 16];
