@@ -62,14 +62,23 @@ def lib():
         L.orc_bf16_round.argtypes = [_vp, ctypes.c_int64, _vp]
         L.orc_l2.argtypes = [ctypes.c_int, _vp, _vp]
         L.orc_l2.restype = ctypes.c_double
-        L.orc_select.argtypes = [ctypes.c_int, ctypes.c_int64, _vp, _vp, ctypes.c_int64, _vp, _vp, ctypes.c_int,
-                                 _vp, _vp, _vp]
-        L.orc_encode.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64, _vp, _vp, _vp,
-                                 ctypes.c_int, _vp, _vp, _vp, _vp, _vp]
+        sel = [ctypes.c_int, ctypes.c_int64, _vp, _vp, ctypes.c_int64, _vp, _vp, ctypes.c_int, _vp, _vp, _vp]
+        L.orc_select.argtypes = sel
+        L.orc_select_f.argtypes = sel
+        L.orc_encode.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64, _vp, _vp, ctypes.c_int64,
+                                 _vp, ctypes.c_int, _vp, _vp, _vp, _vp, _vp]
         L.orc_encode.restype = ctypes.c_int
+        L.orc_encode_f.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64, _vp, _vp, _vp,
+                                   ctypes.c_int, _vp, _vp, _vp, _vp, _vp]
+        L.orc_encode_f.restype = ctypes.c_int
+        L.orc_quantize_rows.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64, _vp, _vp, _vp]
+        L.orc_quantize_rows.restype = ctypes.c_int
+        L.orc_dequantize_rows.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64, _vp, _vp, _vp]
         L.orc_unpack_codes.argtypes = [ctypes.c_int, ctypes.c_int, _vp, _vp]
-        L.orc_reconstruct.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64, _vp, _vp,
-                                      ctypes.c_int, _vp, _vp, _vp, _vp, _vp]
+        L.orc_reconstruct.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64, _vp,
+                                      ctypes.c_int64, _vp, ctypes.c_int, _vp, _vp, _vp, _vp, _vp]
+        L.orc_reconstruct_f.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64, _vp, _vp,
+                                        ctypes.c_int, _vp, _vp, _vp, _vp, _vp]
         L.orc_attention.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp, _vp]
         L.orc_fp16_round_up.argtypes = [ctypes.c_float, _vp]
         L.orc_fp16_round_up.restype = ctypes.c_uint16
@@ -123,29 +132,40 @@ def l2(a, b) -> float:
     return lib().orc_l2(a.size, a.ctypes.data, b.ctypes.data)
 
 
+def _refs(refs):
+    """(array, is_values): bf16 reference rows (uint16 bits) or stored values (float32)."""
+    if np.asarray(refs).dtype == np.float32:
+        return _c(refs, np.float32), True
+    return _c(refs, np.uint16), False
+
+
 def select(x: np.ndarray, tok_pos: np.ndarray, refK: np.ndarray, ref_pos: np.ndarray, k: int):
-    """Top-k references per token: (idx [n][k] uint16 ascending, k_eff [n], dist [n][k+1])."""
+    """Top-k references per token: (idx [n][k] uint16 ascending, k_eff [n], dist [n][k+1]).
+
+    refK: bf16 rows (uint16 bits) or stored values (float32, e.g. the int4 reference store)."""
     x = _c(x, np.float32)
     tok_pos = _c(tok_pos, np.int32)
-    refK = _c(refK, np.uint16)
+    refK, values = _refs(refK)
     ref_pos = _c(ref_pos, np.int32)
     n, D = x.shape
     idx = np.empty((n, k), dtype=np.uint16)
     keff = np.empty(n, dtype=np.int32)
     dist = np.empty((n, k + 1), dtype=np.float64)
-    lib().orc_select(D, n, x.ctypes.data, tok_pos.ctypes.data, len(ref_pos), refK.ctypes.data, ref_pos.ctypes.data,
-                     k, idx.ctypes.data, keff.ctypes.data, dist.ctypes.data)
+    fn = lib().orc_select_f if values else lib().orc_select
+    fn(D, n, x.ctypes.data, tok_pos.ctypes.data, len(ref_pos), refK.ctypes.data, ref_pos.ctypes.data,
+       k, idx.ctypes.data, keff.ctypes.data, dist.ctypes.data)
     return idx, keff, dist
 
 
 def encode(x: np.ndarray, refs: np.ndarray, idx: np.ndarray, bits: int, group: int = 32, want_detail=False):
-    """Residual codes for rows x[n][D] against refs[R][D] (bf16 bits) and idx[n][k].
+    """Residual codes for rows x[n][D] against refs[R][D] (bf16 bits, or float32 stored values)
+    and idx[n][k].
 
     Returns dict(codes [n][D*bits/8] uint8, scales [n][D/group] uint16 fp16 bits, overflow,
     and with want_detail: mean, delta (fp32), delta_exact (bits=0, double)).
     """
     x = _c(x, np.float32)
-    refs = _c(refs, np.uint16)
+    refs, values = _refs(refs)
     idx = _c(idx, np.uint16)
     n, D = x.shape
     k = idx.shape[1]
@@ -154,8 +174,12 @@ def encode(x: np.ndarray, refs: np.ndarray, idx: np.ndarray, bits: int, group: i
     mean = np.empty((n, D), dtype=np.float32) if (want_detail or bits == 0) else None
     delta = np.empty((n, D), dtype=np.float32) if (want_detail or bits == 0) else None
     dex = np.empty((n, D), dtype=np.float64) if bits == 0 else None
-    ov = lib().orc_encode(D, bits, group, n, x.ctypes.data, refs.ctypes.data, idx.ctypes.data, k,
-                          codes.ctypes.data, scales.ctypes.data, _p(mean), _p(delta), _p(dex))
+    if values:
+        ov = lib().orc_encode_f(D, bits, group, n, x.ctypes.data, refs.ctypes.data, idx.ctypes.data, k,
+                                codes.ctypes.data, scales.ctypes.data, _p(mean), _p(delta), _p(dex))
+    else:
+        ov = lib().orc_encode(D, bits, group, n, x.ctypes.data, refs.ctypes.data, refs.shape[0], idx.ctypes.data,
+                              k, codes.ctypes.data, scales.ctypes.data, _p(mean), _p(delta), _p(dex))
     out = dict(codes=codes, scales=scales, overflow=int(ov))
     if mean is not None:
         out.update(mean=mean, delta=delta)
@@ -173,22 +197,56 @@ def unpack_codes(codes_row: np.ndarray, D: int, bits: int) -> np.ndarray:
 
 def reconstruct(refs, idx, codes, scales, bits: int, group: int = 32, D: int | None = None, delta_exact=None):
     """Reconstructed rows: float32 [n][D] (or float64 when bits == 0)."""
-    refs = _c(refs, np.uint16)
+    refs, values = _refs(refs)
     idx = _c(idx, np.uint16)
     n, k = idx.shape
     D = refs.shape[1] if D is None else D
+
+    def call(b, cp, sp, dp, op, oxp):
+        if values:
+            lib().orc_reconstruct_f(D, b, group, n, refs.ctypes.data, idx.ctypes.data, k, cp, sp, dp, op, oxp)
+        else:
+            lib().orc_reconstruct(D, b, group, n, refs.ctypes.data, refs.shape[0], idx.ctypes.data, k, cp, sp, dp,
+                                  op, oxp)
+
     if bits == 0:
         dex = _c(delta_exact, np.float64)
         out = np.empty((n, D), dtype=np.float64)
-        lib().orc_reconstruct(D, 0, group, n, refs.ctypes.data, idx.ctypes.data, k, None, None, dex.ctypes.data,
-                              None, out.ctypes.data)
+        call(0, None, None, dex.ctypes.data, None, out.ctypes.data)
         return out
     codes = _c(codes, np.uint8)
     scales = _c(scales, np.uint16)
     out = np.empty((n, D), dtype=np.float32)
-    lib().orc_reconstruct(D, bits, group, n, refs.ctypes.data, idx.ctypes.data, k, codes.ctypes.data,
-                          scales.ctypes.data, None, out.ctypes.data, None)
+    call(bits, codes.ctypes.data, scales.ctypes.data, None, out.ctypes.data, None)
     return out
+
+
+def quantize_rows(X: np.ndarray, bits: int = 4, group: int = 32):
+    """Group quantiser applied to each row of X[n][D] by itself: (codes, scales, overflow)."""
+    X = _c(X, np.float32)
+    n, D = X.shape
+    codes = np.zeros((n, D * bits // 8), dtype=np.uint8)
+    scales = np.zeros((n, D // group), dtype=np.uint16)
+    ov = lib().orc_quantize_rows(D, bits, group, n, X.ctypes.data, codes.ctypes.data, scales.ctypes.data)
+    return codes, scales, int(ov)
+
+
+def dequantize_rows(codes: np.ndarray, scales: np.ndarray, D: int, bits: int = 4, group: int = 32) -> np.ndarray:
+    """Stored values code * scale (float32 [n][D])."""
+    codes = _c(codes, np.uint8)
+    scales = _c(scales, np.uint16)
+    n = codes.shape[0]
+    out = np.empty((n, D), dtype=np.float32)
+    lib().orc_dequantize_rows(D, bits, group, n, codes.ctypes.data, scales.ctypes.data, out.ctypes.data)
+    return out
+
+
+def build_refs_quantized(X: np.ndarray, ref_pos: np.ndarray, bits: int = 4, group: int = 32):
+    """int4 reference store of float rows X at ref_pos: (codes, scales, stored values, overflow)."""
+    X = _c(X, np.float32)
+    rows = X[np.asarray(ref_pos, dtype=np.int64)]
+    codes, scales, ov = quantize_rows(rows, bits, group)
+    return codes, scales, dequantize_rows(codes, scales, X.shape[1], bits, group), ov
 
 
 def attention(q: np.ndarray, K: np.ndarray, V: np.ndarray) -> np.ndarray:
@@ -224,17 +282,25 @@ def positions_split(n: int, ref_pos: np.ndarray):
 
 
 def compress_unit(Xk: np.ndarray, Xv: np.ndarray, stride0: int, refs_per_phase: int, k: int, bits: int,
-                  group: int = 32, positions=None):
+                  group: int = 32, positions=None, ref_bits: int = 16):
     """Compress one unit given float rows Xk, Xv [n][D] (exact input values).
 
-    positions: compressed positions to encode (default: all).  Returns a dict with
-    ref_pos, refK, refV, pos (encoded positions), idx, keff, dist, codesK, scalesK,
+    positions: compressed positions to encode (default: all).  ref_bits 16: bf16 reference
+    rows (refK, refV uint16 bits); 4: the int4 reference store (refK, refV are the stored
+    values, float32, and ref_codesK/ref_scalesK/ref_codesV/ref_scalesV are added).  Returns a
+    dict with ref_pos, refK, refV, pos (encoded positions), idx, keff, dist, codesK, scalesK,
     codesV, scalesV, overflow.
     """
     n = Xk.shape[0]
     ref_pos = schedule(n, stride0, refs_per_phase)
-    refK = build_refs(Xk, ref_pos)
-    refV = build_refs(Xv, ref_pos)
+    extra = {}
+    if ref_bits == 4:
+        rcK, rsK, refK, ovk = build_refs_quantized(Xk, ref_pos, 4, group)
+        rcV, rsV, refV, ovv = build_refs_quantized(Xv, ref_pos, 4, group)
+        extra = dict(ref_codesK=rcK, ref_scalesK=rsK, ref_codesV=rcV, ref_scalesV=rsV, ref_overflow=ovk | ovv)
+    else:
+        refK = build_refs(Xk, ref_pos)
+        refV = build_refs(Xv, ref_pos)
     if positions is None:
         positions, _ = positions_split(n, ref_pos)
     positions = np.asarray(positions, dtype=np.int32)
@@ -243,18 +309,20 @@ def compress_unit(Xk: np.ndarray, Xv: np.ndarray, stride0: int, refs_per_phase: 
     ev = encode(Xv[positions], refV, idx, bits, group)
     return dict(ref_pos=ref_pos, refK=refK, refV=refV, pos=positions, idx=idx, keff=keff, dist=dist,
                 codesK=ek["codes"], scalesK=ek["scales"], codesV=ev["codes"], scalesV=ev["scales"],
-                overflow=ek["overflow"] | ev["overflow"])
+                overflow=ek["overflow"] | ev["overflow"], **extra)
 
 
 def unit_cache_rows(n: int, ref_pos, refK, refV, idx, codesK, scalesK, codesV, scalesV, bits: int,
                     group: int = 32):
-    """Reconstructed K, V [n][D] float32 of a whole unit (reference rows are the stored bf16)."""
+    """Reconstructed K, V [n][D] float32 of a whole unit (reference rows are the stored values:
+    bf16 rows given as uint16 bits, or float32 values of the int4 reference store)."""
     D = refK.shape[1]
     cpos, is_ref = positions_split(n, np.asarray(ref_pos))
     Kh = np.empty((n, D), dtype=np.float32)
     Vh = np.empty((n, D), dtype=np.float32)
-    Kh[ref_pos] = bf16_value(refK)
-    Vh[ref_pos] = bf16_value(refV)
+    stored = (lambda r: r) if np.asarray(refK).dtype == np.float32 else bf16_value
+    Kh[ref_pos] = stored(refK)
+    Vh[ref_pos] = stored(refV)
     if len(cpos):
         Kh[cpos] = reconstruct(refK, idx, codesK, scalesK, bits, group)
         Vh[cpos] = reconstruct(refV, idx, codesV, scalesV, bits, group)

@@ -24,6 +24,10 @@
 //   * dynamic stride: the stride doubles after every refs_per_phase references;
 //   * references are stored in bf16 (fp32 inputs rounded to nearest even) and
 //     selection, mean and residual use the stored values;
+//   * int4 reference store (optional): each reference row is quantised by
+//     itself with the residuals' group quantiser; the stored value is
+//     code * scale and every step uses it (the "_f" entry points take the
+//     stored values as fp32);
 //   * candidates of position i are the references at positions <= i; the
 //     distance is on the key vector only and one index set serves K and V;
 //   * top-k ranks by (distance, ordinal), keeps k_eff = min(k, #candidates),
@@ -110,15 +114,64 @@ float fp16_value(uint16_t h)
     return static_cast<float>((h & 0x8000) ? -v : v);
 }
 
-// Mean reference of one token: acc = r_j1; acc += r_j2; ...; acc / k_eff (fp32).
-void mean_reference(int D, const uint16_t* refs, const uint16_t* idx, int keff, float* m)
+// Mean reference of one token: acc = r_j1; acc += r_j2; ...; acc / k_eff (fp32), over the
+// stored reference values (bf16 rows widened, or int4 rows dequantised).
+void mean_reference(int D, const float* refs, const uint16_t* idx, int keff, float* m)
 {
     for (int c = 0; c < D; ++c) {
-        float acc = bf16_value(refs[static_cast<int64_t>(idx[0]) * D + c]);
+        float acc = refs[static_cast<int64_t>(idx[0]) * D + c];
         for (int l = 1; l < keff; ++l)
-            acc = acc + bf16_value(refs[static_cast<int64_t>(idx[l]) * D + c]);
+            acc = acc + refs[static_cast<int64_t>(idx[l]) * D + c];
         m[c] = acc / static_cast<float>(keff);
     }
+}
+
+// Stored values of bf16 reference rows.
+std::vector<float> widen_bf16(const uint16_t* rows, int64_t count)
+{
+    std::vector<float> out(static_cast<size_t>(count));
+    for (int64_t i = 0; i < count; ++i)
+        out[i] = bf16_value(rows[i]);
+    return out;
+}
+
+// The symmetric group quantiser of one row of D values ([P3] "How ResidualKV Works":
+// quantized codes; with one fp16 scale per group).  Per group: a = max|v|; a == 0 -> scale 0
+// and codes 0; else scale = fp16_round_up(a / qmax) and code = clamp(round_half_even(v /
+// scale), -qmax, qmax).  Packing: int8 one byte per channel (two's complement); int4 two
+// channels per byte, the even channel in the low nibble.  Returns 1 when a scale overflowed
+// binary16, else 0.
+int quantize_groups(int D, int bits, int group, const float* v, uint8_t* out, uint16_t* scales)
+{
+    int overflow = 0;
+    const int qmax = (bits == 8) ? 127 : 7;
+    const int code_bytes = D * bits / 8;
+    std::memset(out, 0, code_bytes);
+    for (int g = 0; g < D / group; ++g) {
+        float a = 0.0f;
+        for (int c = g * group; c < (g + 1) * group; ++c)
+            a = std::max(a, std::fabs(v[c]));
+        uint16_t sbits = 0;
+        if (a > 0.0f)
+            sbits = fp16_round_up(a / static_cast<float>(qmax), &overflow);
+        scales[g] = sbits;
+        const float s = fp16_value(sbits);
+        for (int c = g * group; c < (g + 1) * group; ++c) {
+            int code = 0;
+            if (a > 0.0f) {
+                const float qv = v[c] / s;
+                code = static_cast<int>(std::nearbyintf(qv));  // default rounding: ties to even
+                code = std::min(qmax, std::max(-qmax, code));
+            }
+            if (bits == 8) {
+                out[c] = static_cast<uint8_t>(static_cast<int8_t>(code));
+            } else {
+                const uint8_t nib = static_cast<uint8_t>(code & 0xf);
+                out[c / 2] |= (c & 1) ? static_cast<uint8_t>(nib << 4) : nib;
+            }
+        }
+    }
+    return overflow;
 }
 
 int count_keff(const uint16_t* idx, int k)
@@ -203,17 +256,16 @@ double orc_l2(int D, const float* a, const float* b)
 // padded with 0xFFFF.  dist_out[t][0..k] gets the k+1 smallest distances in
 // rank order (NaN where there are fewer candidates).
 // ---------------------------------------------------------------------------
-void orc_select(int D, int64_t n_tok, const float* x, const int32_t* tok_pos, int64_t R, const uint16_t* refK,
-                const int32_t* ref_pos, int k, uint16_t* idx_out, int32_t* keff_out, double* dist_out)
+// refK holds the stored reference values (fp32): orc_select passes bf16 rows widened,
+// orc_select_f rows given as values (the int4 reference store, dequantised).
+void orc_select_f(int D, int64_t n_tok, const float* x, const int32_t* tok_pos, int64_t R, const float* rf,
+                  const int32_t* ref_pos, int k, uint16_t* idx_out, int32_t* keff_out, double* dist_out)
 {
-    std::vector<float> rf(static_cast<size_t>(R) * D);
-    for (int64_t i = 0; i < R * D; ++i)
-        rf[i] = bf16_value(refK[i]);
     std::vector<std::pair<double, int64_t>> cand;
     for (int64_t t = 0; t < n_tok; ++t) {
         cand.clear();
         for (int64_t j = 0; j < R && ref_pos[j] <= tok_pos[t]; ++j)
-            cand.emplace_back(orc_l2(D, x + t * D, rf.data() + j * D), j);
+            cand.emplace_back(orc_l2(D, x + t * D, rf + j * D), j);
         const int64_t take = std::min<int64_t>(static_cast<int64_t>(k) + 1, static_cast<int64_t>(cand.size()));
         std::partial_sort(cand.begin(), cand.begin() + take, cand.end());  // (distance, ordinal) order
         const int keff = static_cast<int>(std::min<int64_t>(k, static_cast<int64_t>(cand.size())));
@@ -231,6 +283,13 @@ void orc_select(int D, int64_t n_tok, const float* x, const int32_t* tok_pos, in
     }
 }
 
+void orc_select(int D, int64_t n_tok, const float* x, const int32_t* tok_pos, int64_t R, const uint16_t* refK,
+                const int32_t* ref_pos, int k, uint16_t* idx_out, int32_t* keff_out, double* dist_out)
+{
+    const std::vector<float> rf = widen_bf16(refK, R * D);
+    orc_select_f(D, n_tok, x, tok_pos, R, rf.data(), ref_pos, k, idx_out, keff_out, dist_out);
+}
+
 // ---------------------------------------------------------------------------
 // Residual encoding ([P1] "DeltaKV Framework Architecture", residual
 // computation, with the compressor taken as the identity; [P3] "How
@@ -245,12 +304,12 @@ void orc_select(int D, int64_t n_tok, const float* x, const int32_t* tok_pos, in
 // delta_exact and codes/scales are untouched.
 // Returns 0, or 1 when a scale overflowed binary16.
 // ---------------------------------------------------------------------------
-int orc_encode(int D, int bits, int group, int64_t n_tok, const float* X, const uint16_t* refs,
-               const uint16_t* idx, int k, uint8_t* codes, uint16_t* scales, float* mean_out,
-               float* delta_out, double* delta_exact)
+// refs: stored reference values (fp32), as for orc_select_f.  The number of reference rows
+// is not needed (idx addresses them).
+int orc_encode_f(int D, int bits, int group, int64_t n_tok, const float* X, const float* refs, const uint16_t* idx,
+                 int k, uint8_t* codes, uint16_t* scales, float* mean_out, float* delta_out, double* delta_exact)
 {
     int overflow = 0;
-    const int qmax = (bits == 8) ? 127 : 7;
     const int code_bytes = D * bits / 8;
     const int ngroups = D / group;
     std::vector<float> m(D), delta(D);
@@ -270,33 +329,32 @@ int orc_encode(int D, int bits, int group, int64_t n_tok, const float* X, const 
                 delta_exact[t * D + c] = static_cast<double>(x[c]) - static_cast<double>(m[c]);
             continue;
         }
-        uint8_t* out = codes + t * code_bytes;
-        std::memset(out, 0, code_bytes);
-        for (int g = 0; g < ngroups; ++g) {
-            float a = 0.0f;
-            for (int c = g * group; c < (g + 1) * group; ++c)
-                a = std::max(a, std::fabs(delta[c]));
-            uint16_t sbits = 0;
-            if (a > 0.0f)
-                sbits = fp16_round_up(a / static_cast<float>(qmax), &overflow);
-            scales[t * ngroups + g] = sbits;
-            const float s = fp16_value(sbits);
-            for (int c = g * group; c < (g + 1) * group; ++c) {
-                int code = 0;
-                if (a > 0.0f) {
-                    const float qv = delta[c] / s;
-                    code = static_cast<int>(std::nearbyintf(qv));  // default rounding: ties to even
-                    code = std::min(qmax, std::max(-qmax, code));
-                }
-                if (bits == 8) {
-                    out[c] = static_cast<uint8_t>(static_cast<int8_t>(code));
-                } else {
-                    const uint8_t nib = static_cast<uint8_t>(code & 0xf);
-                    out[c / 2] |= (c & 1) ? static_cast<uint8_t>(nib << 4) : nib;
-                }
-            }
-        }
+        overflow |= quantize_groups(D, bits, group, delta.data(), codes + t * code_bytes, scales + t * ngroups);
     }
+    return overflow;
+}
+
+int orc_encode(int D, int bits, int group, int64_t n_tok, const float* X, const uint16_t* refs, int64_t n_refs,
+               const uint16_t* idx, int k, uint8_t* codes, uint16_t* scales, float* mean_out, float* delta_out,
+               double* delta_exact)
+{
+    const std::vector<float> rf = widen_bf16(refs, n_refs * D);
+    return orc_encode_f(D, bits, group, n_tok, X, rf.data(), idx, k, codes, scales, mean_out, delta_out,
+                        delta_exact);
+}
+
+// ---------------------------------------------------------------------------
+// Quantised rows (the int4 reference store: [P1] "Improvements for AI systems" and "Impact
+// and Future Directions", full-pipeline quantisation applying 4-bit quantization uniformly
+// to the compressed residuals and to the uncompressed components).  Each row of X is
+// quantised by itself with the residuals' group quantiser; the stored value of a channel is
+// code * scale in fp32 (exact: a code of at most 7 bits times a binary16 value).
+// ---------------------------------------------------------------------------
+int orc_quantize_rows(int D, int bits, int group, int64_t n, const float* X, uint8_t* codes, uint16_t* scales)
+{
+    int overflow = 0;
+    for (int64_t i = 0; i < n; ++i)
+        overflow |= quantize_groups(D, bits, group, X + i * D, codes + i * (D * bits / 8), scales + i * (D / group));
     return overflow;
 }
 
@@ -313,14 +371,26 @@ void orc_unpack_codes(int D, int bits, const uint8_t* codes, int32_t* out)
     }
 }
 
+// Stored values of quantised rows: code * scale (fp32).
+void orc_dequantize_rows(int D, int bits, int group, int64_t n, const uint8_t* codes, const uint16_t* scales,
+                         float* out)
+{
+    std::vector<int32_t> q(D);
+    for (int64_t i = 0; i < n; ++i) {
+        orc_unpack_codes(D, bits, codes + i * (D * bits / 8), q.data());
+        for (int c = 0; c < D; ++c)
+            out[i * D + c] = static_cast<float>(q[c]) * fp16_value(scales[i * (D / group) + c / group]);
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Reconstruction ([P1] "DeltaKV Framework Architecture": the decoded residual
 // plus the mean reference).  x_hat = m + code * scale in fp32.  bits == 0
 // uses delta_exact: x_hat = m + delta (double, written to out_exact).
 // ---------------------------------------------------------------------------
-void orc_reconstruct(int D, int bits, int group, int64_t n_tok, const uint16_t* refs, const uint16_t* idx, int k,
-                     const uint8_t* codes, const uint16_t* scales, const double* delta_exact, float* out,
-                     double* out_exact)
+void orc_reconstruct_f(int D, int bits, int group, int64_t n_tok, const float* refs, const uint16_t* idx, int k,
+                       const uint8_t* codes, const uint16_t* scales, const double* delta_exact, float* out,
+                       double* out_exact)
 {
     const int code_bytes = D * bits / 8;
     const int ngroups = (group > 0) ? D / group : 0;
@@ -342,6 +412,14 @@ void orc_reconstruct(int D, int bits, int group, int64_t n_tok, const uint16_t* 
             out[t * D + c] = m[c] + d;
         }
     }
+}
+
+void orc_reconstruct(int D, int bits, int group, int64_t n_tok, const uint16_t* refs, int64_t n_refs,
+                     const uint16_t* idx, int k, const uint8_t* codes, const uint16_t* scales,
+                     const double* delta_exact, float* out, double* out_exact)
+{
+    const std::vector<float> rf = widen_bf16(refs, n_refs * D);
+    orc_reconstruct_f(D, bits, group, n_tok, rf.data(), idx, k, codes, scales, delta_exact, out, out_exact);
 }
 
 // ---------------------------------------------------------------------------

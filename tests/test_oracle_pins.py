@@ -353,3 +353,119 @@ def test_compress_unit_dynamic_stride_smoke():
     assert len(c["ref_pos"]) == len(oracle.schedule(n, 2, 64))
     assert len(c["pos"]) == n - len(c["ref_pos"])
     assert c["overflow"] == 0
+
+
+# --- int4 reference store (paper summary page, "Improvements for AI systems" and "Impact
+#     and Future Directions": full-pipeline 4-bit quantisation of the uncompressed
+#     components as well) -------------------------------------------------------------------
+
+def test_reference_quantiser_invariants():
+    """Each reference row quantised by itself: the residual quantiser's invariants on x."""
+    rng = np.random.default_rng(21)
+    n, D, qmax = 300, 128, 7
+    X = (rng.standard_normal((n, D)) * rng.uniform(0.01, 8, (n, 1))).astype(np.float32)
+    X[5, 32:64] = 0.0                                        # an all-zero group
+    X[6] = 0.0                                               # an all-zero row
+    codes, scales, ov = oracle.quantize_rows(X, 4, 32)
+    assert ov == 0 and codes.shape == (n, D // 2) and scales.shape == (n, D // 32)
+    q = _numpy_unpack(codes, D, 4)
+    s = scales.view(np.float16).astype(np.float64)
+    for i in range(n):
+        for g in range(D // 32):
+            sl = slice(32 * g, 32 * g + 32)
+            a = float(np.max(np.abs(X[i, sl])))
+            if a == 0:
+                assert s[i, g] == 0 and np.all(q[i, sl] == 0)
+                continue
+            assert s[i, g] >= np.float32(np.float32(a) / np.float32(qmax))
+            assert float(np.nextafter(np.float16(s[i, g]), np.float16(0))) < np.float32(np.float32(a) / qmax)
+            assert np.max(np.abs(q[i, sl])) == qmax
+            assert np.all(np.abs(X[i, sl] - q[i, sl] * s[i, g]) <= s[i, g] / 2 * (1 + 1e-12))
+    # stored values: code * scale, decoded independently (numpy nibbles x numpy binary16)
+    vals = oracle.dequantize_rows(codes, scales, D, 4, 32)
+    np.testing.assert_array_equal(vals, (q * np.repeat(s, 32, axis=1)).astype(np.float32))
+    assert np.array_equal(vals.astype(np.float64), q * np.repeat(s, 32, axis=1))   # exact in fp32
+
+
+def test_reference_quantiser_grid_roundtrip():
+    rng = np.random.default_rng(22)
+    D = 64
+    q = rng.integers(-7, 8, (40, D))
+    q[:, ::32] = 7
+    X = (q * np.float32(0.25)).astype(np.float32)
+    codes, scales, _ = oracle.quantize_rows(X, 4, 32)
+    assert np.all(scales.view(np.float16) == np.float16(0.25))
+    assert np.array_equal(_numpy_unpack(codes, D, 4), q)
+    assert np.array_equal(oracle.dequantize_rows(codes, scales, D), X)
+
+
+def test_value_references_match_bf16_references_on_bf16_values():
+    """The stored-value entry points equal the bf16 ones when the values are bf16 rows."""
+    rng = np.random.default_rng(23)
+    n, D, s, k = 600, 32, 8, 4
+    X = _bf16_vals(rng, (n, D))
+    ref_pos = oracle.schedule(n, s)
+    refK = oracle.build_refs(X, ref_pos)
+    vals = oracle.bf16_value(refK).astype(np.float32)
+    tok = np.arange(n, dtype=np.int32)
+    a = oracle.select(X, tok, refK, ref_pos, k)
+    b = oracle.select(X, tok, vals, ref_pos, k)
+    for u, v in zip(a, b):
+        assert np.array_equal(u, v, equal_nan=True)
+    e1 = oracle.encode(X, refK, a[0], 4, want_detail=True)
+    e2 = oracle.encode(X, vals, a[0], 4, want_detail=True)
+    for key in ("codes", "scales", "mean"):
+        assert np.array_equal(e1[key], e2[key])
+    r1 = oracle.reconstruct(refK, a[0], e1["codes"], e1["scales"], 4)
+    r2 = oracle.reconstruct(vals, a[0], e1["codes"], e1["scales"], 4)
+    assert np.array_equal(r1, r2)
+
+
+def test_int4_reference_select_is_the_minimum_k_subset():
+    """Exhaustive on tiny inputs: selection ranks the stored (dequantised) references."""
+    rng = np.random.default_rng(24)
+    n, D, s = 48, 32, 4
+    X = rng.standard_normal((n, D)).astype(np.float32)
+    ref_pos = oracle.schedule(n, s)
+    _, _, vals, _ = oracle.build_refs_quantized(X, ref_pos)
+    d = cdist(X.astype(np.float64), vals.astype(np.float64), "sqeuclidean")
+    for k in (1, 2, 3):
+        idx, keff, _ = oracle.select(X, np.arange(n, dtype=np.int32), vals, ref_pos, k)
+        for t in range(n):
+            cands = [j for j in range(len(ref_pos)) if ref_pos[j] <= t]
+            kk = min(k, len(cands))
+            best = min(itertools.combinations(cands, kk), key=lambda S: sum(d[t, j] for j in S))
+            assert list(idx[t, :kk]) == sorted(best)
+
+
+def test_int4_reference_store_unquantised_residuals_rebuild_the_input():
+    """With int4 references and exact residuals, compressed positions rebuild the input
+    exactly, reference positions give the stored value, and attention over that cache equals
+    attention over [stored references, inputs]."""
+    rng = np.random.default_rng(25)
+    n, D, G = 600, 64, 2
+    Xk = _bf16_vals(rng, (n, D))
+    Xv = _bf16_vals(rng, (n, D))
+    c = oracle.compress_unit(Xk, Xv, 16, 0, 4, 4, ref_bits=4)
+    assert c["refK"].dtype == np.float32 and c["ref_overflow"] == 0
+    # a copy of a stored reference selects that reference at distance 0
+    idx, _, dist = oracle.select(c["refK"][3:4], np.array([n - 1], np.int32), c["refK"], c["ref_pos"], 1)
+    assert idx[0, 0] == 3 and dist[0, 0] == 0
+    ek = oracle.encode(Xk[c["pos"]], c["refK"], c["idx"], 0)
+    ev = oracle.encode(Xv[c["pos"]], c["refV"], c["idx"], 0)
+    Kh = np.empty((n, D))
+    Vh = np.empty((n, D))
+    Kh[c["ref_pos"]] = c["refK"]
+    Vh[c["ref_pos"]] = c["refV"]
+    Kh[c["pos"]] = oracle.reconstruct(c["refK"], c["idx"], None, None, 0, delta_exact=ek["delta_exact"])
+    Vh[c["pos"]] = oracle.reconstruct(c["refV"], c["idx"], None, None, 0, delta_exact=ev["delta_exact"])
+    assert np.array_equal(Kh[c["pos"]], Xk[c["pos"]].astype(np.float64))
+    K2, V2 = Xk.astype(np.float64), Xv.astype(np.float64)
+    K2[c["ref_pos"]] = c["refK"]
+    V2[c["ref_pos"]] = c["refV"]
+    q = rng.standard_normal((G, D))
+    np.testing.assert_allclose(oracle.attention(q, Kh, Vh), _plain_attention(q, K2, V2), rtol=1e-12, atol=1e-13)
+    # and the quantised cache's reconstruction rows sit within scale/2 of the input
+    xh = oracle.reconstruct(c["refK"], c["idx"], c["codesK"], c["scalesK"], 4)
+    sc = np.repeat(c["scalesK"].view(np.float16).astype(np.float64), 32, axis=1)
+    assert np.all(np.abs(xh - Xk[c["pos"]]) <= sc / 2 + 4 * 2 ** -24 * np.abs(Xk[c["pos"]]) + 1e-30)
