@@ -71,7 +71,8 @@ def lib():
         L.orc_encode_f.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64, _vp, _vp, _vp,
                                    ctypes.c_int, _vp, _vp, _vp, _vp, _vp]
         L.orc_encode_f.restype = ctypes.c_int
-        L.orc_quantize_rows.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64, _vp, _vp, _vp]
+        L.orc_quantize_rows.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64, _vp,
+                                        _vp, _vp]
         L.orc_quantize_rows.restype = ctypes.c_int
         L.orc_dequantize_rows.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64, _vp, _vp, _vp]
         L.orc_unpack_codes.argtypes = [ctypes.c_int, ctypes.c_int, _vp, _vp]
@@ -221,13 +222,16 @@ def reconstruct(refs, idx, codes, scales, bits: int, group: int = 32, D: int | N
     return out
 
 
-def quantize_rows(X: np.ndarray, bits: int = 4, group: int = 32):
-    """Group quantiser applied to each row of X[n][D] by itself: (codes, scales, overflow)."""
+def quantize_rows(X: np.ndarray, bits: int = 4, group: int = 32, pow2: bool = True):
+    """Group quantiser applied to each row of X[n][D] by itself: (codes, scales, overflow).
+    pow2: scales rounded up to a power of two (the int4 reference store) instead of to the
+    next binary16 value (the residuals' quantiser)."""
     X = _c(X, np.float32)
     n, D = X.shape
     codes = np.zeros((n, D * bits // 8), dtype=np.uint8)
     scales = np.zeros((n, D // group), dtype=np.uint16)
-    ov = lib().orc_quantize_rows(D, bits, group, n, X.ctypes.data, codes.ctypes.data, scales.ctypes.data)
+    ov = lib().orc_quantize_rows(D, bits, group, int(pow2), n, X.ctypes.data, codes.ctypes.data,
+                                 scales.ctypes.data)
     return codes, scales, int(ov)
 
 

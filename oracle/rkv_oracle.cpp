@@ -25,8 +25,9 @@
 //   * references are stored in bf16 (fp32 inputs rounded to nearest even) and
 //     selection, mean and residual use the stored values;
 //   * int4 reference store (optional): each reference row is quantised by
-//     itself with the residuals' group quantiser; the stored value is
-//     code * scale and every step uses it (the "_f" entry points take the
+//     itself with the residuals' group quantiser, the scale rounded up to a
+//     power of two (so code * scale is an exact bf16 value); the stored value
+//     is code * scale and every step uses it (the "_f" entry points take the
 //     stored values as fp32);
 //   * candidates of position i are the references at positions <= i; the
 //     distance is on the key vector only and one index set serves K and V;
@@ -100,6 +101,25 @@ uint16_t fp16_round_up(float f, int* overflow)
     return static_cast<uint16_t>(((E2 + 15) << 10) | static_cast<int>(frac));
 }
 
+// Smallest power of two >= f (f >= 0) as binary16 bits, within binary16's powers of two
+// 2^-24 .. 2^15; above 2^15 sets *overflow and returns +infinity.
+uint16_t pow2_round_up(float f, int* overflow)
+{
+    const double v = static_cast<double>(f);
+    if (!(v > 0.0))
+        return 0;
+    int e = 0;
+    const double fr = std::frexp(v, &e);   // v = fr * 2^e, fr in [0.5, 1)
+    int E = (fr == 0.5) ? e - 1 : e;       // smallest E with 2^E >= v
+    if (E > 15) {
+        *overflow = 1;
+        return 0x7c00;
+    }
+    if (E < -24)
+        E = -24;
+    return (E >= -14) ? static_cast<uint16_t>((E + 15) << 10) : static_cast<uint16_t>(1u << (E + 24));
+}
+
 float fp16_value(uint16_t h)
 {
     const int exp = (h >> 10) & 0x1f;
@@ -141,7 +161,7 @@ std::vector<float> widen_bf16(const uint16_t* rows, int64_t count)
 // scale), -qmax, qmax).  Packing: int8 one byte per channel (two's complement); int4 two
 // channels per byte, the even channel in the low nibble.  Returns 1 when a scale overflowed
 // binary16, else 0.
-int quantize_groups(int D, int bits, int group, const float* v, uint8_t* out, uint16_t* scales)
+int quantize_groups(int D, int bits, int group, const float* v, uint8_t* out, uint16_t* scales, bool pow2 = false)
 {
     int overflow = 0;
     const int qmax = (bits == 8) ? 127 : 7;
@@ -153,7 +173,8 @@ int quantize_groups(int D, int bits, int group, const float* v, uint8_t* out, ui
             a = std::max(a, std::fabs(v[c]));
         uint16_t sbits = 0;
         if (a > 0.0f)
-            sbits = fp16_round_up(a / static_cast<float>(qmax), &overflow);
+            sbits = pow2 ? pow2_round_up(a / static_cast<float>(qmax), &overflow)
+                         : fp16_round_up(a / static_cast<float>(qmax), &overflow);
         scales[g] = sbits;
         const float s = fp16_value(sbits);
         for (int c = g * group; c < (g + 1) * group; ++c) {
@@ -347,14 +368,18 @@ int orc_encode(int D, int bits, int group, int64_t n_tok, const float* X, const 
 // Quantised rows (the int4 reference store: [P1] "Improvements for AI systems" and "Impact
 // and Future Directions", full-pipeline quantisation applying 4-bit quantization uniformly
 // to the compressed residuals and to the uncompressed components).  Each row of X is
-// quantised by itself with the residuals' group quantiser; the stored value of a channel is
-// code * scale in fp32 (exact: a code of at most 7 bits times a binary16 value).
+// quantised by itself with the residuals' group quantiser, except that the scale is rounded
+// up to a power of two (pow2 != 0): a 4-bit code times a power of two is then an exact bf16
+// value, so the stored reference is the same number in every stage, the bf16 tensor-core
+// search included.  The stored value of a channel is code * scale in fp32.
 // ---------------------------------------------------------------------------
-int orc_quantize_rows(int D, int bits, int group, int64_t n, const float* X, uint8_t* codes, uint16_t* scales)
+int orc_quantize_rows(int D, int bits, int group, int pow2, int64_t n, const float* X, uint8_t* codes,
+                      uint16_t* scales)
 {
     int overflow = 0;
     for (int64_t i = 0; i < n; ++i)
-        overflow |= quantize_groups(D, bits, group, X + i * D, codes + i * (D * bits / 8), scales + i * (D / group));
+        overflow |= quantize_groups(D, bits, group, X + i * D, codes + i * (D * bits / 8), scales + i * (D / group),
+                                    pow2 != 0);
     return overflow;
 }
 

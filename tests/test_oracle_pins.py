@@ -360,12 +360,15 @@ def test_compress_unit_dynamic_stride_smoke():
 #     components as well) -------------------------------------------------------------------
 
 def test_reference_quantiser_invariants():
-    """Each reference row quantised by itself: the residual quantiser's invariants on x."""
+    """Each reference row quantised by itself: scale = the smallest power of two >= a / 7
+    (so every stored value is an exact bf16 number), |x - code*scale| <= scale/2."""
     rng = np.random.default_rng(21)
     n, D, qmax = 300, 128, 7
     X = (rng.standard_normal((n, D)) * rng.uniform(0.01, 8, (n, 1))).astype(np.float32)
     X[5, 32:64] = 0.0                                        # an all-zero group
     X[6] = 0.0                                               # an all-zero row
+    X[7, :32] = 1e-9                                         # below the smallest binary16 power of two x 7
+    X[8, 32:64] = 3.5                                        # a / 7 exactly a power of two
     codes, scales, ov = oracle.quantize_rows(X, 4, 32)
     assert ov == 0 and codes.shape == (n, D // 2) and scales.shape == (n, D // 32)
     q = _numpy_unpack(codes, D, 4)
@@ -377,14 +380,22 @@ def test_reference_quantiser_invariants():
             if a == 0:
                 assert s[i, g] == 0 and np.all(q[i, sl] == 0)
                 continue
-            assert s[i, g] >= np.float32(np.float32(a) / np.float32(qmax))
-            assert float(np.nextafter(np.float16(s[i, g]), np.float16(0))) < np.float32(np.float32(a) / qmax)
-            assert np.max(np.abs(q[i, sl])) == qmax
+            v = float(np.float32(np.float32(a) / np.float32(qmax)))
+            expect = max(2.0 ** int(np.ceil(np.log2(v))), 2.0 ** -24)
+            assert s[i, g] == expect, (i, g, s[i, g], v)
+            assert 4 <= np.max(np.abs(q[i, sl])) <= qmax or s[i, g] == 2.0 ** -24
             assert np.all(np.abs(X[i, sl] - q[i, sl] * s[i, g]) <= s[i, g] / 2 * (1 + 1e-12))
-    # stored values: code * scale, decoded independently (numpy nibbles x numpy binary16)
+    assert s[8, 1] == 0.5 and np.max(np.abs(q[8, 32:64])) == 7
+    # stored values: code * scale, decoded independently (numpy nibbles x numpy binary16);
+    # every one is an exact bf16 value
     vals = oracle.dequantize_rows(codes, scales, D, 4, 32)
     np.testing.assert_array_equal(vals, (q * np.repeat(s, 32, axis=1)).astype(np.float32))
     assert np.array_equal(vals.astype(np.float64), q * np.repeat(s, 32, axis=1))   # exact in fp32
+    assert np.array_equal(oracle.bf16_value(oracle.bf16_round(vals)), vals)
+    # the residuals' rounding (next binary16 instead of the next power of two) on the same rows
+    _, s16, _ = oracle.quantize_rows(X, 4, 32, pow2=False)
+    e = oracle.encode(X, oracle.bf16_round(np.zeros((1, D))), np.zeros((n, 1), dtype=np.uint16), 4)
+    assert np.array_equal(s16, e["scales"])
 
 
 def test_reference_quantiser_grid_roundtrip():
