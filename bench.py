@@ -8,8 +8,9 @@ step, and a 256-row reconstruction.  Inputs are resident in HBM when the timed
 region starts; L2 is flushed (256 MiB write) before every timed step, outside
 the timed spans.  With N GPUs (torchrun) every rank runs its own replica on an
 independent layer; value is the whole-job throughput over the max-over-ranks
-step time.  Outside the step, a selective decode (2048 seeded positions per unit)
-and incremental compression (the last 64 tokens appended one at a time) are timed as
+step time.  Outside the step, a selective decode (2048 seeded positions per unit),
+incremental compression (the last 64 tokens appended one at a time) and the same layer
+with the int4 reference store (reference store, search, encode, decode) are timed as
 well.  `--impl reference` times the CPU oracle on a bounded sample of
 the same workload on the host cores.  Prints one JSON line on rank 0.
 """
@@ -84,6 +85,7 @@ def workload_quantities(wl, lengths):
     per_tok = 2 * D * wl.bits // 8 + 2 * (D // 32) * 2 + 2 * wl.k
     flops = 0
     dec_bytes = 0
+    dec_bytes4 = 0
     enc_bytes = 0
     refs_bytes = 0
     for n in lengths:
@@ -99,10 +101,12 @@ def workload_quantities(wl, lengths):
         ncand = np.searchsorted(ref_pos, cpos, side="right").astype(np.int64)
         flops += wl.n_kv_heads * int(ncand.sum()) * 2 * D
         dec_bytes += wl.n_kv_heads * (C * per_tok + R * 4 * D)
+        # int4 reference store: codes (D/2 bytes) and binary16 scales (D/32) per row and side
+        dec_bytes4 += wl.n_kv_heads * (C * per_tok + R * 2 * (D // 2 + 2 * (D // 32)))
         enc_bytes += wl.n_kv_heads * C * (2 * D * wl.elem_bytes + per_tok)
         refs_bytes += wl.n_kv_heads * R * (2 * D * wl.elem_bytes + 4 * D + 8)
-    return dict(tokens=sum(lengths), search_flops=flops,
-                decode_bytes=dec_bytes, encode_bytes=enc_bytes, refs_bytes=refs_bytes, bytes_per_token=per_tok)
+    return dict(tokens=sum(lengths), search_flops=flops, decode_bytes=dec_bytes, decode_bytes_int4_refs=dec_bytes4,
+                encode_bytes=enc_bytes, refs_bytes=refs_bytes, bytes_per_token=per_tok)
 
 
 class ClockSampler:
@@ -452,6 +456,43 @@ def run_ours(args, rank, world, local_rank):
     append_us = 1e3 * e0.elapsed_time(e1) / APPEND_TOKENS
     del La
 
+    # int4 reference store (outside the step): the same layer with references stored as
+    # int4 codes + binary16 scales; each stage a CUDA graph, L2 flushed before each replay
+    cfg4 = rkv.make_config(head_dim=wl.head_dim, n_kv_heads=wl.n_kv_heads, n_q_heads=wl.n_q_heads, k=wl.k,
+                           bits=wl.bits, stride0=wl.stride0, batch=wl.batch, max_len=K.shape[2],
+                           refs_per_phase=wl.refs_per_phase, in_dtype=wl.dtype_code, out_dtype=wl.dtype_code,
+                           ref_bits=4)
+    L4 = rkv.Layer(cfg4, lengths, device=dev)
+    st4 = {"build_refs": lambda: L4.build_refs(K, V), "search": lambda: L4.search(K),
+           "encode": lambda: L4.encode(K, V), "decode": lambda: L4.decode(q, out)}
+    g4 = {}
+    with torch.cuda.stream(stream):
+        for nm in st4:
+            st4[nm]()
+        torch.cuda.synchronize(dev)
+        for nm in st4:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                st4[nm]()
+            g4[nm] = g
+    torch.cuda.synchronize(dev)
+    ms4 = {nm: [] for nm in st4}
+    with torch.cuda.stream(stream):
+        for i in range(max(3, min(args.steps, 20)) + 2):
+            for nm in st4:
+                flush.zero_()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                g4[nm].replay()
+                e1.record(stream)
+                e1.synchronize()
+                if i >= 2:
+                    ms4[nm].append(e0.elapsed_time(e1))
+    assert L4.device_error() == 0
+    del g4, L4
+    avg4 = {nm: statistics.mean(v) for nm, v in ms4.items()}
+
     Q = workload_quantities(wl, lengths)
     tokens = Q["tokens"]
     value = job_throughput(world, tokens, mean_step)
@@ -503,6 +544,14 @@ def run_ours(args, rank, world, local_rank):
                                                                         avg["build_refs"]) * 1e-3) / 1e6,
                 "sparse_decode_us": sparse_us, "sparse_decode_positions_per_unit": SPARSE_SEL,
                 "append_us_per_token": append_us,
+                "int4_refs": {
+                    "build_refs_us": 1e3 * avg4["build_refs"], "search_us": 1e3 * avg4["search"],
+                    "encode_us": 1e3 * avg4["encode"], "decode_us_per_step": 1e3 * avg4["decode"],
+                    "decode_bytes_per_step": Q["decode_bytes_int4_refs"],
+                    "decode_hbm_gbs": Q["decode_bytes_int4_refs"] / (avg4["decode"] * 1e-3) / 1e9,
+                    "compress_mtok_s": tokens / ((avg4["build_refs"] + avg4["search"] + avg4["encode"]) * 1e-3)
+                    / 1e6,
+                },
             },
             "roofline": roofline,
             "cpu_baseline": cpu,

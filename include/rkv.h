@@ -102,6 +102,16 @@ typedef enum rkv_status {
  *   batch           sequences, 1..RKV_MAX_BATCH
  *   max_len         row pitch (tokens) of K and V, >= every length
  *   flags           RKV_FLAG_* bits
+ *   ref_bits        0 or 16: references stored as bf16 rows.  4: the int4 reference
+ *                   store (paper summary page, "Improvements for AI systems" and "Impact
+ *                   and Future Directions": full-pipeline 4-bit quantization, applied to
+ *                   the uncompressed components too): each reference row of K and V is
+ *                   quantised by itself with the residuals' group quantiser (int4 codes,
+ *                   one scale per 32 channels stored as binary16), except that the scale
+ *                   is rounded up to a power of two, so every stored value code * scale
+ *                   is an exact bf16 number; every stage (selection, mean, residual,
+ *                   reconstruction, attention) uses that stored value.  Decode then reads
+ *                   72 instead of 256 bytes per reference row and side at D = 128.
  */
 typedef struct rkv_config {
     int32_t head_dim;
@@ -117,7 +127,9 @@ typedef struct rkv_config {
     int32_t batch;
     int32_t max_len;
     uint32_t flags;
-    int32_t reserved[3];
+    int32_t ref_bits;    /* reference store: 0 or 16 = bf16 rows; 4 = int4 codes, one binary16
+                            scale per 32 channels (see below) */
+    int32_t reserved[2];
 } rkv_config;
 
 /* Host-side handle of a bound cache.  Caller-allocated, opaque, plain data:
@@ -130,6 +142,8 @@ typedef struct rkv_cache_desc {
 /* Device pointers and sizes of one (sequence, kv-head) unit of a bound cache.
  * Layout of each array (rows contiguous):
  *   ref_K, ref_V     [n_ref][head_dim] bf16   reference rows, reference ordinal order
+ *                    (int4 reference store: [n_ref][head_dim/2] codes packed like the
+ *                    residual codes, with ref_scale_K/V [n_ref][head_dim/32] binary16)
  *   ref_half_norm    [n_ref] float            0.5 * |ref_K row|^2 (fp32)
  *   ref_pos          [n_ref] int32            position of each reference
  *   codes_K, codes_V [n_cmp][code_bytes]      residual codes of the compressed tokens in
@@ -145,7 +159,8 @@ typedef struct rkv_unit_view {
     int32_t k;
     int32_t code_bytes;
     int32_t n_groups;
-    int32_t reserved[2];
+    int32_t ref_bits;    /* 16: ref_K/ref_V are bf16 rows; 4: int4 codes [n_ref][head_dim/2] */
+    int32_t reserved;
     void* ref_K;
     void* ref_V;
     float* ref_half_norm;
@@ -155,6 +170,8 @@ typedef struct rkv_unit_view {
     uint16_t* scale_K;
     uint16_t* scale_V;
     uint16_t* idx;
+    uint16_t* ref_scale_K;   /* ref_bits 4: binary16 scales [n_ref][head_dim/32]; else NULL */
+    uint16_t* ref_scale_V;
 } rkv_unit_view;
 
 /* ABI version of the loaded library (RKV_ABI_VERSION). */

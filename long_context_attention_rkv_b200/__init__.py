@@ -43,15 +43,15 @@ class RkvError(RuntimeError):
 class rkv_config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("head_dim", "n_kv_heads", "n_q_heads", "k", "bits", "group",
                                               "stride0", "refs_per_phase", "in_dtype", "out_dtype", "batch",
-                                              "max_len")] + [("flags", ctypes.c_uint32),
-                                                             ("reserved", ctypes.c_int32 * 3)]
+                                              "max_len")] + [("flags", ctypes.c_uint32), ("ref_bits", ctypes.c_int32),
+                                                             ("reserved", ctypes.c_int32 * 2)]
 
 
 class rkv_unit_view(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_int32) for n in ("n", "n_ref", "n_cmp", "k", "code_bytes", "n_groups")] + \
-               [("reserved", ctypes.c_int32 * 2)] + \
+    _fields_ = [(n, ctypes.c_int32) for n in ("n", "n_ref", "n_cmp", "k", "code_bytes", "n_groups", "ref_bits",
+                                              "reserved")] + \
                [(n, ctypes.c_void_p) for n in ("ref_K", "ref_V", "ref_half_norm", "ref_pos", "codes_K", "codes_V",
-                                               "scale_K", "scale_V", "idx")]
+                                               "scale_K", "scale_V", "idx", "ref_scale_K", "ref_scale_V")]
 
 
 _lib = None
@@ -130,9 +130,11 @@ class CacheDesc:
 
 
 def make_config(head_dim, n_kv_heads, n_q_heads, k, bits, stride0, batch, max_len, refs_per_phase=0,
-                in_dtype=RKV_DTYPE_BF16, out_dtype=None, group=32, flags=0) -> rkv_config:
+                in_dtype=RKV_DTYPE_BF16, out_dtype=None, group=32, flags=0, ref_bits=0) -> rkv_config:
+    """ref_bits: 0 (or 16) bf16 reference rows; 4 the int4 reference store."""
     return rkv_config(head_dim, n_kv_heads, n_q_heads, k, bits, group, stride0, refs_per_phase, in_dtype,
-                      in_dtype if out_dtype is None else out_dtype, batch, max_len, flags, (ctypes.c_int32 * 3)())
+                      in_dtype if out_dtype is None else out_dtype, batch, max_len, flags, ref_bits,
+                      (ctypes.c_int32 * 2)())
 
 
 # --- the C ABI, one function each ------------------------------------------------------

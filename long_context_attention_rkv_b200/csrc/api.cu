@@ -87,6 +87,8 @@ rkv_status validate_config(const rkv_config* c)
         return RKV_ERR_UNSUPPORTED;
     if (static_cast<int64_t>(c->batch) * c->n_kv_heads > 65535)
         return RKV_ERR_UNSUPPORTED;
+    if (c->ref_bits != 0 && c->ref_bits != 16 && c->ref_bits != 4)
+        return RKV_ERR_UNSUPPORTED;
     return RKV_OK;
 }
 
@@ -172,8 +174,11 @@ rkv_status compute_layout(const rkv_config* c, const int32_t* lengths, Desc& d)
     s.units = take(sizeof(UnitMeta) * d.n_units);
     s.tiles = take(sizeof(Tile) * std::max<int64_t>(1, tiles));
     s.pairs = take(sizeof(Tile) * std::max<int64_t>(1, pairs));
-    s.ref_K = take(2ull * ref_rows * D);
-    s.ref_V = take(2ull * ref_rows * D);
+    const bool r4 = c->ref_bits == 4;
+    s.ref_K = take(r4 ? ref_rows * D / 2 : 2ull * ref_rows * D);
+    s.ref_V = take(r4 ? ref_rows * D / 2 : 2ull * ref_rows * D);
+    s.ref_sK = take(r4 ? 2ull * ref_rows * (D / 32) : 0);
+    s.ref_sV = take(r4 ? 2ull * ref_rows * (D / 32) : 0);
     s.ref_hn = take(4ull * (ref_rows + 256));  // tail slack: tile scans read up to 32 entries past a unit
     s.ref_aug = take(32ull * ref_rows);
     s.ref_pos = take(4ull * ref_rows);
@@ -185,6 +190,8 @@ rkv_status compute_layout(const rkv_config* c, const int32_t* lengths, Desc& d)
     s.append = take(append_scratch_bytes(d.n_units));   // per-unit candidate lists of rkv_append
     s.end = off;
     d.ws_select = align_up(2ull * cmp_rows * d.kc, 256) + align_up(4ull * cmp_rows * d.kc, 256);
+    if (r4)
+        d.ws_select += align_up(2ull * ref_rows * D, 256);   // the stored keys as bf16 rows (search operand)
     const int splits = std::max(decode_splits(d.n_units, max_n), sparse_splits_max(d.n_units));
     d.ws_decode = align_up(4ull * d.n_units * splits * G * (D + 2), 256);
     const CacheArgs a = make_args(d);
@@ -227,6 +234,9 @@ CacheArgs make_args(const Desc& d)
     a.units = reinterpret_cast<const UnitMeta*>(base + d.sec.units);
     a.ref_K = reinterpret_cast<uint16_t*>(base + d.sec.ref_K);
     a.ref_V = reinterpret_cast<uint16_t*>(base + d.sec.ref_V);
+    a.ref_bits = (d.cfg.ref_bits == 4) ? 4 : 16;
+    a.ref_sK = (a.ref_bits == 4) ? reinterpret_cast<uint16_t*>(base + d.sec.ref_sK) : nullptr;
+    a.ref_sV = (a.ref_bits == 4) ? reinterpret_cast<uint16_t*>(base + d.sec.ref_sV) : nullptr;
     a.ref_hn = reinterpret_cast<float*>(base + d.sec.ref_hn);
     a.ref_aug = reinterpret_cast<uint16_t*>(base + d.sec.ref_aug);
     a.ref_pos = reinterpret_cast<int32_t*>(base + d.sec.ref_pos);
@@ -413,8 +423,16 @@ rkv_status rkv_unit_view_get(const rkv_cache_desc* desc, int32_t seq, int32_t kv
     out->k = d->cfg.k;
     out->code_bytes = d->code_bytes;
     out->n_groups = d->n_groups;
-    out->ref_K = a.ref_K + ref_row * a.D;
-    out->ref_V = a.ref_V + ref_row * a.D;
+    out->ref_bits = a.ref_bits;
+    if (a.ref_bits == 4) {
+        out->ref_K = reinterpret_cast<uint8_t*>(a.ref_K) + ref_row * (a.D / 2);
+        out->ref_V = reinterpret_cast<uint8_t*>(a.ref_V) + ref_row * (a.D / 2);
+        out->ref_scale_K = a.ref_sK + ref_row * (a.D / 32);
+        out->ref_scale_V = a.ref_sV + ref_row * (a.D / 32);
+    } else {
+        out->ref_K = a.ref_K + ref_row * a.D;
+        out->ref_V = a.ref_V + ref_row * a.D;
+    }
     out->ref_half_norm = a.ref_hn + ref_row;
     out->ref_pos = a.ref_pos + ref_row;
     out->codes_K = a.codes_K + cmp_row * d->code_bytes;
@@ -465,7 +483,18 @@ rkv_status rkv_search(const rkv_cache_desc* desc, const void* K, void* workspace
     if (select_tc_supported(a) && !(d->cfg.flags & RKV_FLAG_SELECT_SIMT)) {
         const int64_t in_rows = static_cast<int64_t>(d->n_units) * d->cfg.max_len;
         const Tile* pairs = reinterpret_cast<const Tile*>(static_cast<char*>(d->base) + d->sec.pairs);
-        return cuda_status(launch_select_tc(a, pairs, d->n_pairs, K, in_rows, d->total_ref_rows,
+        const uint16_t* refB = a.ref_K;
+        if (a.ref_bits == 4) {
+            // bf16 copy of the stored keys, after the candidate lists in the workspace
+            uint16_t* copy = reinterpret_cast<uint16_t*>(static_cast<char*>(workspace) +
+                                                         align_up(2ull * d->total_cmp_rows * d->kc, 256) +
+                                                         align_up(4ull * d->total_cmp_rows * d->kc, 256));
+            const cudaError_t e = launch_refs_bf16(a, d->total_ref_rows, copy, st);
+            if (e != cudaSuccess)
+                return cuda_status(e);
+            refB = copy;
+        }
+        return cuda_status(launch_select_tc(a, pairs, d->n_pairs, K, refB, in_rows, d->total_ref_rows,
                                             cand_idx_of(d, workspace), cand_t_of(d, workspace), st));
     }
     return cuda_status(launch_select_simt(a, tiles, d->n_tiles, K, cand_idx_of(d, workspace),

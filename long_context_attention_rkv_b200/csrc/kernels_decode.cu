@@ -156,17 +156,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             const bool ok = j < j_hi;
             float r[CPL];
             if (ok) {
-                const uint16_t* rp = a.ref_K + (um.ref_row + j) * D + sub * CPL;
-#pragma unroll
-                for (int hh = 0; hh < CPL / 8; ++hh) {
-                    const uint4 v = *reinterpret_cast<const uint4*>(rp + 8 * hh);
-                    const uint32_t ww[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        r[8 * hh + 2 * i] = bf16_bits_to_f32(ww[i] & 0xffffu);
-                        r[8 * hh + 2 * i + 1] = bf16_bits_to_f32(ww[i] >> 16);
-                    }
-                }
+                load_ref<CPL>(a, 0, um.ref_row + j, sub * CPL, r);
             } else {
 #pragma unroll
                 for (int i = 0; i < CPL; ++i)
@@ -401,15 +391,18 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int g = i / (D / 2), cp = (i % (D / 2)) * 2;
         float acc0 = 0.0f, acc1 = 0.0f;
         for (int j = j_lo; j < j_hi; j += 8) {
-            uint32_t rv[8];
+            float rv[8][2];
 #pragma unroll
-            for (int t = 0; t < 8; ++t)
-                rv[t] = (j + t < j_hi) ? *reinterpret_cast<const uint32_t*>(a.ref_V + (um.ref_row + j + t) * D + cp) : 0u;
+            for (int t = 0; t < 8; ++t) {
+                rv[t][0] = rv[t][1] = 0.0f;
+                if (j + t < j_hi)
+                    load_ref<2>(a, 1, um.ref_row + j + t, cp, rv[t]);
+            }
 #pragma unroll
             for (int t = 0; t < 8; ++t) {
                 const float wj = (j + t < j_hi) ? wt[(j + t - j_lo) * G + g] : 0.0f;
-                acc0 = fmaf(wj, bf16_bits_to_f32(rv[t] & 0xffffu), acc0);
-                acc1 = fmaf(wj, bf16_bits_to_f32(rv[t] >> 16), acc1);
+                acc0 = fmaf(wj, rv[t][0], acc0);
+                acc1 = fmaf(wj, rv[t][1], acc1);
             }
         }
         osum[g * D + cp] += acc0;

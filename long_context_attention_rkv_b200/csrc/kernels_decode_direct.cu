@@ -26,7 +26,7 @@ namespace {
 
 constexpr int kWarps = 4;
 
-template <int NPL>
+template <int NPL, int RB>
 __device__ __forceinline__ bool rebuild_compressed(const CacheArgs& a, const UnitMeta& um, int c, int lane,
                                                    float (&xk)[NPL], float (&xv)[NPL])
 {
@@ -48,8 +48,8 @@ __device__ __forceinline__ bool rebuild_compressed(const CacheArgs& a, const Uni
         if (bad)
             break;
         float rk[NPL], rv[NPL];
-        load_bf16<NPL>(a.ref_K + (um.ref_row + o) * D + lane * NPL, rk);
-        load_bf16<NPL>(a.ref_V + (um.ref_row + o) * D + lane * NPL, rv);
+        load_ref<NPL, RB>(a, 0, um.ref_row + o, lane * NPL, rk);
+        load_ref<NPL, RB>(a, 1, um.ref_row + o, lane * NPL, rv);
 #pragma unroll
         for (int j = 0; j < NPL; ++j) {
             sk[j] = (l == 0) ? rk[j] : __fadd_rn(sk[j], rk[j]);
@@ -72,7 +72,7 @@ __device__ __forceinline__ bool rebuild_compressed(const CacheArgs& a, const Uni
     return true;
 }
 
-template <int NPL, int GMAX>
+template <int NPL, int GMAX, int RB>
 __global__ void __launch_bounds__(kWarps * 32) decode_direct_kernel(CacheArgs a, const void* __restrict__ q,
                                                                     float* __restrict__ part, int splits,
                                                                     float qscale, const int32_t* __restrict__ sel,
@@ -131,10 +131,9 @@ __global__ void __launch_bounds__(kWarps * 32) decode_direct_kernel(CacheArgs a,
         }
         float xk[NPL], xv[NPL];
         if (v < um.R) {
-            const int64_t r = (um.ref_row + v) * D + lane * NPL;
-            load_bf16<NPL>(a.ref_K + r, xk);
-            load_bf16<NPL>(a.ref_V + r, xv);
-        } else if (!rebuild_compressed<NPL>(a, um, v - um.R, lane, xk, xv)) {
+            load_ref<NPL, RB>(a, 0, um.ref_row + v, lane * NPL, xk);
+            load_ref<NPL, RB>(a, 1, um.ref_row + v, lane * NPL, xv);
+        } else if (!rebuild_compressed<NPL, RB>(a, um, v - um.R, lane, xk, xv)) {
             if (lane == 0)
                 report(a.err, RKV_ERR_CORRUPT);
             continue;
@@ -230,6 +229,18 @@ __global__ void decode_combine_kernel(CacheArgs a, int splits, const float* __re
 
 }  // namespace
 
+template <int NPL, int GMAX>
+static void launch_dd(const CacheArgs& a, dim3 grid, const void* q, float* partials, int splits, float qscale,
+                      const int32_t* sel, const int32_t* sel_cnt, int sel_stride, cudaStream_t st)
+{
+    if (a.ref_bits == 4)
+        decode_direct_kernel<NPL, GMAX, 4><<<grid, kWarps * 32, 0, st>>>(a, q, partials, splits, qscale, sel, sel_cnt,
+                                                                         sel_stride);
+    else
+        decode_direct_kernel<NPL, GMAX, 16><<<grid, kWarps * 32, 0, st>>>(a, q, partials, splits, qscale, sel,
+                                                                          sel_cnt, sel_stride);
+}
+
 cudaError_t launch_decode_direct(const CacheArgs& a, int splits, const void* q, float* partials, cudaStream_t st,
                                  const int32_t* sel, const int32_t* sel_cnt, int sel_stride)
 {
@@ -237,18 +248,14 @@ cudaError_t launch_decode_direct(const CacheArgs& a, int splits, const void* q, 
     const float qscale = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(a.D)));
     if (a.D == 128) {
         if (a.G <= 8)
-            decode_direct_kernel<4, 8><<<grid, kWarps * 32, 0, st>>>(a, q, partials, splits, qscale, sel, sel_cnt,
-                                                                      sel_stride);
+            launch_dd<4, 8>(a, grid, q, partials, splits, qscale, sel, sel_cnt, sel_stride, st);
         else
-            decode_direct_kernel<4, 16><<<grid, kWarps * 32, 0, st>>>(a, q, partials, splits, qscale, sel, sel_cnt,
-                                                                       sel_stride);
+            launch_dd<4, 16>(a, grid, q, partials, splits, qscale, sel, sel_cnt, sel_stride, st);
     } else {
         if (a.G <= 8)
-            decode_direct_kernel<2, 8><<<grid, kWarps * 32, 0, st>>>(a, q, partials, splits, qscale, sel, sel_cnt,
-                                                                      sel_stride);
+            launch_dd<2, 8>(a, grid, q, partials, splits, qscale, sel, sel_cnt, sel_stride, st);
         else
-            decode_direct_kernel<2, 16><<<grid, kWarps * 32, 0, st>>>(a, q, partials, splits, qscale, sel, sel_cnt,
-                                                                       sel_stride);
+            launch_dd<2, 16>(a, grid, q, partials, splits, qscale, sel, sel_cnt, sel_stride, st);
     }
     return cudaGetLastError();
 }

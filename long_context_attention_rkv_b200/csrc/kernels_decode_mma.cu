@@ -171,7 +171,7 @@ namespace {
 
 // ==== 1. reference scores ==================================================================
 
-template <int Gp>
+template <int Gp, int RB>
 __global__ void __launch_bounds__(128) mma_scores_kernel(const CacheArgs a, const void* __restrict__ q, const MmaWs w)
 {
     // s[r][h] = cK * (refK_r . q_h) as m16n8k16 MMAs: one warp per 16 references, columns are
@@ -192,14 +192,35 @@ __global__ void __launch_bounds__(128) mma_scores_kernel(const CacheArgs a, cons
     const int r1 = min(R, r0 + kRefChunk);
     const int rw = r0 + warp * 16;               // first reference of this warp
     // A rows gid and gid + 8 (zero past the unit), B column gid (zero past the group)
+    // With the int4 reference store (RB 4) the stored values code * 2^e are exact bf16
+    // numbers: the A fragments are built from the codes and scales.
     uint4 ar[2][4], bq[4];
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
         const int r = rw + gid + 8 * rr;
-        const uint4* src = reinterpret_cast<const uint4*>(a.ref_K + (um.ref_row + r) * D + 32 * tq);
+        if constexpr (RB != 4) {
+            const uint4* src = reinterpret_cast<const uint4*>(a.ref_K + (um.ref_row + r) * D + 32 * tq);
 #pragma unroll
-        for (int x = 0; x < 4; ++x)
-            ar[rr][x] = (r < r1) ? src[x] : make_uint4(0u, 0u, 0u, 0u);
+            for (int x = 0; x < 4; ++x)
+                ar[rr][x] = (r < r1) ? src[x] : make_uint4(0u, 0u, 0u, 0u);
+        } else {
+            uint32_t hw[16];
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                float v[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    v[i] = 0.0f;
+                if (r < r1)
+                    load_ref<16, 4>(a, 0, um.ref_row + r, 32 * tq + 16 * half, v);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    hw[8 * half + i] = f32_to_bf16_bits(v[2 * i]) | (uint32_t(f32_to_bf16_bits(v[2 * i + 1])) << 16);
+            }
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+                ar[rr][x] = make_uint4(hw[4 * x], hw[4 * x + 1], hw[4 * x + 2], hw[4 * x + 3]);
+        }
     }
     {
         const uint4* src = reinterpret_cast<const uint4*>(
@@ -782,7 +803,7 @@ __global__ void __launch_bounds__(32 * kConsWarps * NTEAM, 1)
 
 // ==== 3. reference tokens, reference weights, output =========================================
 
-template <int Gp>
+template <int Gp, int RB>
 __global__ void __launch_bounds__(256) mma_refs_kernel(const CacheArgs a, void* __restrict__ out, const MmaWs w)
 {
     constexpr int D = 128;
@@ -805,15 +826,42 @@ __global__ void __launch_bounds__(256) mma_refs_kernel(const CacheArgs a, void* 
     // Before the wait on the tokens kernel: the reference V rows, and what depends only on the
     // scores kernel (complete once this kernel runs; read through L2): the common offsets,
     // the reference tokens' own terms p_r and their sum.
-    uint32_t rv[RQ];
+    float rv[RQ][2];
+    __shared__ float ssc[RB == 4 ? kRefChunk * (D / 32) : 1];   // int4 store: the chunk's V scales
+    uint32_t cb[RB == 4 ? RQ : 1];
+    if constexpr (RB == 4) {
+        // one code byte (channels 2cp, 2cp+1) per row; the rows' scales staged once per CTA
+        const uint8_t* codes = reinterpret_cast<const uint8_t*>(a.ref_V);
 #pragma unroll
-    for (int rr = 0; rr < RQ; ++rr) {
-        const int r = r0 + qq * RQ + rr;
-        rv[rr] = (r < r1) ? *reinterpret_cast<const uint32_t*>(a.ref_V + (um.ref_row + r) * D + 2 * cp) : 0u;
+        for (int rr = 0; rr < RQ; ++rr) {
+            const int r = r0 + qq * RQ + rr;
+            cb[rr] = (r < r1) ? codes[(um.ref_row + r) * (D / 2) + cp] : 0u;
+        }
+        if (tid < kRefChunk * (D / 32)) {
+            const int r = r0 + tid / (D / 32);
+            ssc[tid] = (r < r1) ? __half2float(__ushort_as_half(a.ref_sV[(um.ref_row + r) * (D / 32) + tid % (D / 32)]))
+                                : 0.0f;
+        }
+    } else {
+#pragma unroll
+        for (int rr = 0; rr < RQ; ++rr) {
+            const int r = r0 + qq * RQ + rr;
+            rv[rr][0] = rv[rr][1] = 0.0f;
+            if (r < r1)
+                load_ref<2, RB>(a, 1, um.ref_row + r, 2 * cp, rv[rr]);
+        }
     }
     if (tid < Gp)
         key[tid] = 0u;
     __syncthreads();
+    if constexpr (RB == 4) {
+#pragma unroll
+        for (int rr = 0; rr < RQ; ++rr) {
+            const float sc = ssc[(qq * RQ + rr) * (D / 32) + cp / 16];
+            rv[rr][0] = __fmul_rn(static_cast<float>(static_cast<int>((cb[rr] & 0xfu) ^ 8u) - 8), sc);
+            rv[rr][1] = __fmul_rn(static_cast<float>(static_cast<int>((cb[rr] >> 4) ^ 8u) - 8), sc);
+        }
+    }
     unit_max_fold<Gp>(w, u, R, tid, 256, key);
     __syncthreads();
     float pj[kRefChunk * Gp / 256 > 0 ? kRefChunk * Gp / 256 : 1];
@@ -859,7 +907,7 @@ __global__ void __launch_bounds__(256) mma_refs_kernel(const CacheArgs a, void* 
             acc[h][0] = acc[h][1] = 0.0f;
 #pragma unroll
         for (int rr = 0; rr < RQ; ++rr) {
-            const float x0 = bf16_bits_to_f32(rv[rr] & 0xffffu), x1 = bf16_bits_to_f32(rv[rr] >> 16);
+            const float x0 = rv[rr][0], x1 = rv[rr][1];
             const float* wr = wt[qq * RQ + rr];
 #pragma unroll
             for (int h = 0; h < Gp; ++h) {
@@ -1004,7 +1052,10 @@ cudaError_t launch_gp(const CacheArgs& a, int64_t cmp_rows, const void* q, void*
     if (!code_map(enc, &mK, a.codes_K, cmp_rows) || !code_map(enc, &mV, a.codes_V, cmp_rows))
         return cudaErrorInvalidValue;
     const dim3 rgrid(w.n_chunk, a.n_units);
-    mma_scores_kernel<Gp><<<rgrid, 128, 0, st>>>(a, q, w);
+    if (a.ref_bits == 4)
+        mma_scores_kernel<Gp, 4><<<rgrid, 128, 0, st>>>(a, q, w);
+    else
+        mma_scores_kernel<Gp, 16><<<rgrid, 128, 0, st>>>(a, q, w);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;
@@ -1021,7 +1072,9 @@ cudaError_t launch_gp(const CacheArgs& a, int64_t cmp_rows, const void* q, void*
         if (e != cudaSuccess)
             return e;
     }
-    return launch_pdl(mma_refs_kernel<Gp>, rgrid, dim3(256), 0, st, a, out, w);
+    if (a.ref_bits == 4)
+        return launch_pdl(mma_refs_kernel<Gp, 4>, rgrid, dim3(256), 0, st, a, out, w);
+    return launch_pdl(mma_refs_kernel<Gp, 16>, rgrid, dim3(256), 0, st, a, out, w);
 }
 
 }  // namespace

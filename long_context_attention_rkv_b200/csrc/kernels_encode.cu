@@ -110,13 +110,13 @@ __device__ __forceinline__ void load_input_row(const void* base, int64_t elem, i
     }
 }
 
-// Exact-order fp32 squared distance between this token's key and a reference row (this
-// lane's part; sum over the token group with tsum).
-template <int CPL>
-__device__ __forceinline__ float part_dist(const float (&x)[CPL], const uint16_t* r)
+// Exact-order fp32 squared distance between this token's key and a reference row's stored
+// values (this lane's part, channels c0 ..; sum over the token group with tsum).
+template <int CPL, int RB>
+__device__ __forceinline__ float part_dist(const CacheArgs& a, const float (&x)[CPL], int64_t row, int c0)
 {
     float rv[CPL];
-    load_bf16_row<CPL>(r, rv);
+    load_ref<CPL, RB>(a, 0, row, c0, rv);
     float s = 0.0f;
 #pragma unroll
     for (int i = 0; i < CPL; ++i) {
@@ -218,7 +218,7 @@ __device__ __forceinline__ void quantise_store(const float (&x)[CPL], const floa
 template <int KC, int LPT>
 constexpr int encode_min_blocks() { return (LPT == 16 && KC <= 12) ? 4 : 2; }
 
-template <int CPL, int KC, int LPT>
+template <int CPL, int KC, int LPT, int RB>
 __global__ void __launch_bounds__(kWarps * 32, encode_min_blocks<KC, LPT>()) encode_kernel(CacheArgs a, const void* __restrict__ K,
                                                              const void* __restrict__ V,
                                                              const uint16_t* __restrict__ cand_idx,
@@ -336,7 +336,7 @@ __global__ void __launch_bounds__(kWarps * 32, encode_min_blocks<KC, LPT>()) enc
                 float d = 0.0f;
                 if (need) {
                     const int o = in[i] ? ords[i] : 0;
-                    d = tsum<kLPT>(part_dist<CPL>(xk, a.ref_K + (um.ref_row + o) * D + sub * CPL));
+                    d = tsum<kLPT>(part_dist<CPL, RB>(a, xk, um.ref_row + o, sub * CPL));
                 }
                 dist[i] = d;
             }
@@ -376,14 +376,15 @@ __global__ void __launch_bounds__(kWarps * 32, encode_min_blocks<KC, LPT>()) enc
             }
             const int nscan = ex ? ncand : 0;
             for (int j = sub; j < nscan; j += kLPT) {
-                const uint16_t* r = a.ref_K + (um.ref_row + j) * D;
                 float d = 0.0f;
-                for (int c2 = 0; c2 < D; c2 += 2) {
-                    const uint32_t w = *reinterpret_cast<const uint32_t*>(r + c2);
-                    const float e0 = __fsub_rn(xs[warp][tg][c2], bf16_bits_to_f32(w & 0xffffu));
-                    const float e1 = __fsub_rn(xs[warp][tg][c2 + 1], bf16_bits_to_f32(w >> 16));
-                    d = __fmaf_rn(e0, e0, d);
-                    d = __fmaf_rn(e1, e1, d);
+                for (int c2 = 0; c2 < D; c2 += 8) {
+                    float rv[8];
+                    load_ref<8, RB>(a, 0, um.ref_row + j, c2, rv);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float e0 = __fsub_rn(xs[warp][tg][c2 + i], rv[i]);
+                        d = __fmaf_rn(e0, e0, d);
+                    }
                 }
                 float cv = d;
                 int ci = j;
@@ -456,14 +457,14 @@ __global__ void __launch_bounds__(kWarps * 32, encode_min_blocks<KC, LPT>()) enc
     float mk[CPL], mv[CPL];
     {
         const int o = sorted[warp][tg][0];
-        load_bf16_row<CPL>(a.ref_K + (um.ref_row + o) * D + sub * CPL, mk);
-        load_bf16_row<CPL>(a.ref_V + (um.ref_row + o) * D + sub * CPL, mv);
+        load_ref<CPL, RB>(a, 0, um.ref_row + o, sub * CPL, mk);
+        load_ref<CPL, RB>(a, 1, um.ref_row + o, sub * CPL, mv);
     }
     for (int i = 1; i < keff; ++i) {
         const int o = sorted[warp][tg][i];
         float rk[CPL], rv[CPL];
-        load_bf16_row<CPL>(a.ref_K + (um.ref_row + o) * D + sub * CPL, rk);
-        load_bf16_row<CPL>(a.ref_V + (um.ref_row + o) * D + sub * CPL, rv);
+        load_ref<CPL, RB>(a, 0, um.ref_row + o, sub * CPL, rk);
+        load_ref<CPL, RB>(a, 1, um.ref_row + o, sub * CPL, rv);
 #pragma unroll
         for (int j2 = 0; j2 < CPL; j2 += 2) {
             add2_rn(mk[j2], mk[j2 + 1], rk[j2], rk[j2 + 1]);
@@ -554,16 +555,14 @@ __global__ void __launch_bounds__(kAppendThreads) append_search_kernel(CacheArgs
     }
     for (int j = j_lo + tid; j < j_hi; j += kAppendThreads) {
         // distance in double, channels in order, no contraction (the search's definition)
-        const uint4* r4 = reinterpret_cast<const uint4*>(a.ref_K + (um.ref_row + j) * D);
         double d = 0.0;
 #pragma unroll 2
         for (int c8 = 0; c8 < D / 8; ++c8) {
-            const uint4 w = r4[c8];
-            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+            float rv[8];
+            load_ref<8>(a, 0, um.ref_row + j, c8 * 8, rv);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                const float rv = bf16_bits_to_f32((i & 1) ? (ww[i >> 1] >> 16) : (ww[i >> 1] & 0xffffu));
-                const double t = __dsub_rn(static_cast<double>(xs[c8 * 8 + i]), static_cast<double>(rv));
+                const double t = __dsub_rn(static_cast<double>(xs[c8 * 8 + i]), static_cast<double>(rv[i]));
                 d = __dadd_rn(d, __dmul_rn(t, t));
             }
         }
@@ -661,15 +660,27 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(CacheArgs a, con
             load_row_part<NPL>(Kn, e_row + lane * NPL, a.in_dtype, kx);
             load_row_part<NPL>(Vn, e_row + lane * NPL, a.in_dtype, vx);
             float ss = 0.0f;
-            const int64_t o = (um.ref_row + j) * D + lane * NPL;
+            const int64_t row = um.ref_row + j;
+            if (a.ref_bits == 4) {
+                float rk[NPL], rv[NPL];
+                ref_quantise_store<NPL>(kx, lane, reinterpret_cast<uint8_t*>(a.ref_K) + row * (D / 2),
+                                        a.ref_sK + row * (D / 32), rk, a.err);
+                ref_quantise_store<NPL>(vx, lane, reinterpret_cast<uint8_t*>(a.ref_V) + row * (D / 2),
+                                        a.ref_sV + row * (D / 32), rv, a.err);
 #pragma unroll
-            for (int i = 0; i < NPL; ++i) {
-                const uint16_t kb = f32_to_bf16_bits(kx[i]);
-                const uint16_t vb = f32_to_bf16_bits(vx[i]);
-                a.ref_K[o + i] = kb;
-                a.ref_V[o + i] = vb;
-                const float r = bf16_bits_to_f32(kb);
-                ss = fmaf(r, r, ss);
+                for (int i = 0; i < NPL; ++i)
+                    ss = fmaf(rk[i], rk[i], ss);
+            } else {
+                const int64_t o = row * D + lane * NPL;
+#pragma unroll
+                for (int i = 0; i < NPL; ++i) {
+                    const uint16_t kb = f32_to_bf16_bits(kx[i]);
+                    const uint16_t vb = f32_to_bf16_bits(vx[i]);
+                    a.ref_K[o + i] = kb;
+                    a.ref_V[o + i] = vb;
+                    const float r = bf16_bits_to_f32(kb);
+                    ss = fmaf(r, r, ss);
+                }
             }
             ss = warp_sum(ss);
             if (lane == 0) {
@@ -736,14 +747,14 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(CacheArgs a, con
         load_input_row<CPL>(Vn, e_row + sub * CPL, a.in_dtype, xv);
         {
             const int o = chosen_s[0];
-            load_bf16_row<CPL>(a.ref_K + (um.ref_row + o) * D + sub * CPL, mk);
-            load_bf16_row<CPL>(a.ref_V + (um.ref_row + o) * D + sub * CPL, mv);
+            load_ref<CPL>(a, 0, um.ref_row + o, sub * CPL, mk);
+            load_ref<CPL>(a, 1, um.ref_row + o, sub * CPL, mv);
         }
         for (int i2 = 1; i2 < keff; ++i2) {
             const int o = chosen_s[i2];
             float rk[CPL], rv[CPL];
-            load_bf16_row<CPL>(a.ref_K + (um.ref_row + o) * D + sub * CPL, rk);
-            load_bf16_row<CPL>(a.ref_V + (um.ref_row + o) * D + sub * CPL, rv);
+            load_ref<CPL>(a, 0, um.ref_row + o, sub * CPL, rk);
+            load_ref<CPL>(a, 1, um.ref_row + o, sub * CPL, rv);
 #pragma unroll
             for (int j2 = 0; j2 < CPL; ++j2) {
                 mk[j2] = __fadd_rn(mk[j2], rk[j2]);
@@ -784,10 +795,18 @@ cudaError_t launch_cpl(const CacheArgs& a, int max_C, const void* K, const void*
 {
     const int per_block = kWarps * (32 / LPT);
     const dim3 grid((max_C + per_block - 1) / per_block, a.n_units);
+    if (a.ref_bits == 4) {
+        switch (a.kc) {
+        case 8: encode_kernel<CPL, 8, LPT, 4><<<grid, kWarps * 32, 0, st>>>(a, K, V, ci, ct); break;
+        case 12: encode_kernel<CPL, 12, LPT, 4><<<grid, kWarps * 32, 0, st>>>(a, K, V, ci, ct); break;
+        default: encode_kernel<CPL, 20, LPT, 4><<<grid, kWarps * 32, 0, st>>>(a, K, V, ci, ct); break;
+        }
+        return cudaGetLastError();
+    }
     switch (a.kc) {
-    case 8: encode_kernel<CPL, 8, LPT><<<grid, kWarps * 32, 0, st>>>(a, K, V, ci, ct); break;
-    case 12: encode_kernel<CPL, 12, LPT><<<grid, kWarps * 32, 0, st>>>(a, K, V, ci, ct); break;
-    default: encode_kernel<CPL, 20, LPT><<<grid, kWarps * 32, 0, st>>>(a, K, V, ci, ct); break;
+    case 8: encode_kernel<CPL, 8, LPT, 16><<<grid, kWarps * 32, 0, st>>>(a, K, V, ci, ct); break;
+    case 12: encode_kernel<CPL, 12, LPT, 16><<<grid, kWarps * 32, 0, st>>>(a, K, V, ci, ct); break;
+    default: encode_kernel<CPL, 20, LPT, 16><<<grid, kWarps * 32, 0, st>>>(a, K, V, ci, ct); break;
     }
     return cudaGetLastError();
 }

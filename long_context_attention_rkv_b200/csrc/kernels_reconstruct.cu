@@ -67,9 +67,8 @@ __global__ void __launch_bounds__(kWarps * 32) reconstruct_kernel(CacheArgs a, i
     const int nle = refs_upto(a.ph, p);
     float xk[NPL], xv[NPL];
     if (is_ref_pos(a.ph, p)) {
-        const int64_t r = (um.ref_row + nle - 1) * D + lane * NPL;
-        load_bf16<NPL>(a.ref_K + r, xk);
-        load_bf16<NPL>(a.ref_V + r, xv);
+        load_ref<NPL>(a, 0, um.ref_row + nle - 1, lane * NPL, xk);
+        load_ref<NPL>(a, 1, um.ref_row + nle - 1, lane * NPL, xv);
     } else {
         const int64_t row = um.cmp_row + (p - nle);
         const uint16_t* id = a.idx + row * a.k;
@@ -87,12 +86,12 @@ __global__ void __launch_bounds__(kWarps * 32) reconstruct_kernel(CacheArgs a, i
                 report(a.err, RKV_ERR_CORRUPT);
             return;
         }
-        load_bf16<NPL>(a.ref_K + (um.ref_row + id[0]) * D + lane * NPL, xk);
-        load_bf16<NPL>(a.ref_V + (um.ref_row + id[0]) * D + lane * NPL, xv);
+        load_ref<NPL>(a, 0, um.ref_row + id[0], lane * NPL, xk);
+        load_ref<NPL>(a, 1, um.ref_row + id[0], lane * NPL, xv);
         for (int l = 1; l < keff; ++l) {
             float rk[NPL], rv[NPL];
-            load_bf16<NPL>(a.ref_K + (um.ref_row + id[l]) * D + lane * NPL, rk);
-            load_bf16<NPL>(a.ref_V + (um.ref_row + id[l]) * D + lane * NPL, rv);
+            load_ref<NPL>(a, 0, um.ref_row + id[l], lane * NPL, rk);
+            load_ref<NPL>(a, 1, um.ref_row + id[l], lane * NPL, rv);
 #pragma unroll
             for (int j = 0; j < NPL; ++j) {
                 xk[j] = __fadd_rn(xk[j], rk[j]);

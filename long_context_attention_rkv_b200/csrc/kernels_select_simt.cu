@@ -87,7 +87,7 @@ __global__ void __launch_bounds__(128) select_simt_kernel(CacheArgs a, const Til
             const int c = (i % (D / 4)) * 4;
             float v[4] = {0.f, 0.f, 0.f, 0.f};
             if (r < nrow)
-                load_bf16<4>(a.ref_K + (um.ref_row + j0 + r) * D + c, v);
+                load_ref<4>(a, 0, um.ref_row + j0 + r, c, v);
             *reinterpret_cast<float4*>(&sr[r][c]) = make_float4(v[0], v[1], v[2], v[3]);
         }
         if (threadIdx.x < kChunk)

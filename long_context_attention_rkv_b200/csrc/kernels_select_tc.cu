@@ -574,8 +574,8 @@ cudaError_t launch_t(const CacheArgs& a, const Tile* items, int n_items, const C
 
 bool select_tc_supported(const CacheArgs& a) { return a.in_dtype == RKV_DTYPE_BF16 && (a.D == 128 || a.D == 64); }
 
-cudaError_t launch_select_tc(const CacheArgs& a, const Tile* items, int n_items, const void* K, int64_t in_rows,
-                             int64_t ref_rows, uint16_t* cand_idx, float* cand_t, cudaStream_t st)
+cudaError_t launch_select_tc(const CacheArgs& a, const Tile* items, int n_items, const void* K, const uint16_t* refB,
+                             int64_t in_rows, int64_t ref_rows, uint16_t* cand_idx, float* cand_t, cudaStream_t st)
 {
     if (n_items <= 0)
         return cudaSuccess;
@@ -586,7 +586,7 @@ cudaError_t launch_select_tc(const CacheArgs& a, const Tile* items, int n_items,
     alignas(64) CUtensorMap mB;
     alignas(64) CUtensorMap mAug;
     if (!make_map(enc, &mA, K, in_rows, a.D, 64, kM, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(enc, &mB, a.ref_K, ref_rows, a.D, 64, kN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(enc, &mB, refB, ref_rows, a.D, 64, kN, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(enc, &mAug, a.ref_aug, ref_rows, 16, 16, kN, CU_TENSOR_MAP_SWIZZLE_32B))
         return cudaErrorInvalidValue;
     int dev = 0, sms = 0;

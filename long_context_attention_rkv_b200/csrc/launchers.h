@@ -7,6 +7,7 @@
 
 namespace rkv {
 
+cudaError_t launch_refs_bf16(const CacheArgs& a, int64_t rows, uint16_t* out, cudaStream_t st);
 cudaError_t launch_refs_copy(const CacheArgs& a, int max_R, const void* K, const void* V, cudaStream_t st);
 
 cudaError_t launch_select_simt(const CacheArgs& a, const Tile* tiles, int n_tiles, const void* K, uint16_t* cand_idx,
@@ -14,8 +15,8 @@ cudaError_t launch_select_simt(const CacheArgs& a, const Tile* tiles, int n_tile
 
 // Tensor-core search (bf16 inputs, head_dim 64 or 128).
 bool select_tc_supported(const CacheArgs& a);
-cudaError_t launch_select_tc(const CacheArgs& a, const Tile* tiles, int n_tiles, const void* K, int64_t in_rows,
-                             int64_t ref_rows, uint16_t* cand_idx, float* cand_t, cudaStream_t st);
+cudaError_t launch_select_tc(const CacheArgs& a, const Tile* items, int n_items, const void* K, const uint16_t* refB,
+                             int64_t in_rows, int64_t ref_rows, uint16_t* cand_idx, float* cand_t, cudaStream_t st);
 
 cudaError_t launch_encode(const CacheArgs& a, int max_C, const void* K, const void* V, const uint16_t* cand_idx,
                           const float* cand_t, cudaStream_t st);

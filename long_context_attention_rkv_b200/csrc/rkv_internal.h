@@ -40,8 +40,8 @@ struct UnitMeta {
 
 // Byte offsets of the cache sections inside the caller's buffer.
 struct Sections {
-    uint64_t err, units, tiles, pairs, ref_K, ref_V, ref_hn, ref_aug, ref_pos, codes_K, codes_V, scale_K, scale_V, idx,
-        append, end;
+    uint64_t err, units, tiles, pairs, ref_K, ref_V, ref_sK, ref_sV, ref_hn, ref_aug, ref_pos, codes_K, codes_V,
+        scale_K, scale_V, idx, append, end;
 };
 
 // Host-side descriptor stored in rkv_cache_desc::opaque.
@@ -81,11 +81,14 @@ static_assert(sizeof(Desc) <= RKV_CACHE_DESC_BYTES, "descriptor too large");
 struct CacheArgs {
     int32_t D, Hkv, Hq, G, k, bits, group, in_dtype, out_dtype;
     int32_t n_units, code_bytes, n_groups, kc, max_len, max_refs;
+    int32_t ref_bits, pad_r;   // 16: bf16 reference rows; 4: int4 reference store
     Phases ph;
     const UnitMeta* units;
     int32_t* err;
-    uint16_t* ref_K;
+    uint16_t* ref_K;     // bf16 rows [rows][D], or int4 codes [rows][D/2] bytes (ref_bits 4)
     uint16_t* ref_V;
+    uint16_t* ref_sK;    // ref_bits 4: binary16 scales [rows][D/32]
+    uint16_t* ref_sV;
     float* ref_hn;
     uint16_t* ref_aug;   // [rows][16] bf16: -hi, -mid, -lo of 0.5|r|^2, then zeros (augmented GEMM column)
     int32_t* ref_pos;

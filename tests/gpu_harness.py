@@ -27,24 +27,25 @@ def to_dev(arr: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(a).cuda()
 
 
-def config(wl: synth.Workload, lengths, max_len=None, out_dtype=rkv.RKV_DTYPE_F32, flags=0, batch=None):
+def config(wl: synth.Workload, lengths, max_len=None, out_dtype=rkv.RKV_DTYPE_F32, flags=0, batch=None,
+           ref_bits=0):
     return rkv.make_config(head_dim=wl.head_dim, n_kv_heads=wl.n_kv_heads, n_q_heads=wl.n_q_heads, k=wl.k,
                            bits=wl.bits, stride0=wl.stride0, batch=len(lengths) if batch is None else batch,
                            max_len=max(max(lengths), 1) if max_len is None else max_len,
                            refs_per_phase=wl.refs_per_phase, in_dtype=wl.dtype_code, out_dtype=out_dtype,
-                           flags=flags)
+                           flags=flags, ref_bits=ref_bits)
 
 
 class GpuRun:
     """One layer compressed on the GPU through the C ABI."""
 
     def __init__(self, wl: synth.Workload, K: np.ndarray, V: np.ndarray, lengths, out_dtype=rkv.RKV_DTYPE_F32,
-                 flags=0, start_lengths=None):
+                 flags=0, start_lengths=None, ref_bits=0):
         """lengths: the bound (capacity) lengths; start_lengths: a shorter prefix to compress
-        first (grown later with append_until)."""
+        first (grown later with append_until); ref_bits 4: the int4 reference store."""
         self.wl = wl
         self.lengths = list(lengths)
-        self.cfg = config(wl, lengths, max_len=K.shape[2], out_dtype=out_dtype, flags=flags)
+        self.cfg = config(wl, lengths, max_len=K.shape[2], out_dtype=out_dtype, flags=flags, ref_bits=ref_bits)
         self.layer = rkv.Layer(self.cfg, self.lengths)
         self.Kd = to_dev(K)
         self.Vd = to_dev(V)
@@ -85,10 +86,21 @@ class GpuRun:
     def unit(self, b: int, h: int) -> dict:
         v = self.layer.unit(b, h)
         D, R, C, k = self.wl.head_dim, v.n_ref, v.n_cmp, v.k
+        refs = {}
+        if v.ref_bits == 4:
+            # the int4 reference store: codes and scales as stored, and their stored values
+            for side, cp, sp in (("K", v.ref_K, v.ref_scale_K), ("V", v.ref_V, v.ref_scale_V)):
+                codes = self._read(cp, R * D // 2, np.uint8, (R, D // 2))
+                scales = self._read(sp, 2 * R * (D // 32), np.uint16, (R, D // 32))
+                refs["ref_codes" + side] = codes
+                refs["ref_scales" + side] = scales
+                refs["ref" + side] = oracle.dequantize_rows(codes, scales, D, 4, 32) if R else \
+                    np.zeros((0, D), np.float32)
+        else:
+            refs["refK"] = self._read(v.ref_K, 2 * R * D, np.uint16, (R, D))
+            refs["refV"] = self._read(v.ref_V, 2 * R * D, np.uint16, (R, D))
         return dict(
-            n=v.n, R=R, C=C,
-            refK=self._read(v.ref_K, 2 * R * D, np.uint16, (R, D)),
-            refV=self._read(v.ref_V, 2 * R * D, np.uint16, (R, D)),
+            n=v.n, R=R, C=C, ref_bits=v.ref_bits, **refs,
             hn=self._read(v.ref_half_norm, 4 * R, np.float32, (R,)),
             pos=self._read(v.ref_pos, 4 * R, np.int32, (R,)),
             codesK=self._read(v.codes_K, C * v.code_bytes, np.uint8, (C, v.code_bytes)),
@@ -142,12 +154,25 @@ def _unpack(codes: np.ndarray, D: int, bits: int) -> np.ndarray:
     return np.where(out >= 8, out - 16, out)
 
 
+def stored_values(refs: np.ndarray) -> np.ndarray:
+    """Reference values as fp32: bf16 bits widened, or already values (int4 store)."""
+    return refs if refs.dtype == np.float32 else oracle.bf16_value(refs)
+
+
 def check_refs(wl, g: dict, Xk, Xv):
     ref_pos = oracle.schedule(len(Xk), wl.stride0, wl.refs_per_phase)
     assert np.array_equal(g["pos"], ref_pos)
-    assert np.array_equal(g["refK"], oracle.build_refs(Xk, ref_pos))
-    assert np.array_equal(g["refV"], oracle.build_refs(Xv, ref_pos))
-    rv = oracle.bf16_value(g["refK"]).astype(np.float64)
+    if g["ref_bits"] == 4:
+        for side, X in (("K", Xk), ("V", Xv)):
+            codes, scales, vals, ov = oracle.build_refs_quantized(X, ref_pos)
+            assert ov == 0
+            assert np.array_equal(g["ref_codes" + side], codes), f"reference {side} codes differ"
+            assert np.array_equal(g["ref_scales" + side], scales), f"reference {side} scales differ"
+            assert np.array_equal(g["ref" + side], vals)
+    else:
+        assert np.array_equal(g["refK"], oracle.build_refs(Xk, ref_pos))
+        assert np.array_equal(g["refV"], oracle.build_refs(Xv, ref_pos))
+    rv = stored_values(g["refK"]).astype(np.float64)
     np.testing.assert_allclose(g["hn"], 0.5 * (rv * rv).sum(axis=1), rtol=2e-6, atol=1e-30)
     return ref_pos
 
@@ -179,7 +204,7 @@ def check_compress(wl, g: dict, Xk, Xv, positions=None, stats=None):
             f"gpu {gidx[t]} oracle {oidx[t]} d_k={dk} d_k+1={dk1}")
         sel = gidx[t][gidx[t] != oracle.SENTINEL]
         assert len(sel) == ke and np.all(np.diff(sel.astype(int)) > 0) and np.all(ref_pos[sel] < positions[t])
-        rv = oracle.bf16_value(refK)
+        rv = stored_values(refK)
         worst = max(oracle.l2(Xk[positions[t]], rv[j]) for j in sel)
         assert worst <= dk1 * (1 + IDX_TIE_BAND)
     # codes: the oracle's encoder fed the GPU's index sets

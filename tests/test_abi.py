@@ -52,6 +52,21 @@ def test_cache_size_accounts_every_array():
     assert wb >= H * C * 8 * 6            # search candidates: kc = 8 ordinals + scores per token
 
 
+def test_int4_reference_store_sizes():
+    """int4 reference rows: D/2 code bytes and D/32 binary16 scales per row and side, and the
+    search workspace carries a bf16 copy of the stored keys."""
+    lengths = [32768]
+    c16, w16 = rkv.rkv_cache_size(_cfg(), lengths)
+    c4, w4 = rkv.rkv_cache_size(_cfg(ref_bits=4), lengths)
+    R, H, D = 2048, 8, 128
+    assert c16 - c4 == pytest.approx(H * R * 2 * (2 * D - (D // 2 + 2 * D // 32)), abs=8 * 1024)
+    assert w4 >= w16 + H * R * D * 2                       # plus the stored keys as bf16 rows
+    for bad in (8, 2, 5):
+        with pytest.raises(rkv.RkvError) as ei:
+            rkv.rkv_cache_size(_cfg(ref_bits=bad), lengths)
+        assert rkv.STATUS[ei.value.status] == "RKV_ERR_UNSUPPORTED"
+
+
 def test_ragged_sizes_and_validation():
     cfg = _cfg(n_kv_heads=4, n_q_heads=28, k=8, stride0=32, batch=3)
     cb, _ = rkv.rkv_cache_size(cfg, [16384, 0, 20000])

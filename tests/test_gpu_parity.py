@@ -320,3 +320,71 @@ def test_append_equals_compressing_the_whole_sequence(case):
     with pytest.raises(rkv.RkvError) as ei:      # at capacity: refused, nothing launched
         run.layer.append(run.Kd[:, :, 0].contiguous(), run.Vd[:, :, 0].contiguous())
     assert ei.value.status == rkv.STATUS_CODE["RKV_ERR_INVALID_ARG"]
+
+
+# --- int4 reference store (paper summary page, "Improvements for AI systems": full-pipeline
+#     4-bit quantisation of the uncompressed components too) -------------------------------
+
+@pytest.mark.parametrize("case", ["llama", "qwen", "dynamic_d64_int8", "tiny_fp32"])
+def test_int4_reference_store_every_stage(case):
+    """Reference codes and scales bit-exact; selection over the stored values (exact outside
+    the tie band); residual codes against the GPU's index sets; reconstruction; decode through
+    the tensor-core, CUDA-core and gather forms; selective decode."""
+    if case == "llama":
+        wl = _small("llama3_8b_layer", n_kv_heads=2, n_q_heads=8, batch=2, seq_len=4100, ragged=None)
+        lengths = [4100, 1333]
+    elif case == "qwen":
+        wl = _small("qwen2_5_7b_batch", n_kv_heads=2, n_q_heads=14, batch=2, seq_len=3000, ragged=None)
+        lengths = [3000, 2100]
+    elif case == "dynamic_d64_int8":
+        wl = _small("ultra_long_1m", n_kv_heads=1, n_q_heads=4, head_dim=64, stride0=4, refs_per_phase=64, k=3,
+                    bits=8, seq_len=3000, n_proto=64)
+        lengths = [3000]
+    else:
+        wl = synth.WORKLOADS["tiny"]
+        lengths = wl.lengths()
+    K, V = synth.gen_layer(wl, 0, lengths)
+    run = GpuRun(wl, K, V, lengths, ref_bits=4)
+    assert run.unit(0, 0)["ref_bits"] == 4
+    stats = _full_unit_checks(run, wl, K, V, lengths)
+    assert stats["tokens"] > 0
+    q = synth.gen_query(wl, 0, 0)
+    check_decode(run, q)
+    # a sharp query (logits of order 4 |k|): the stored reference keys must enter exactly
+    G = wl.n_q_heads // wl.n_kv_heads
+    sharp = np.zeros((len(lengths), wl.n_q_heads, wl.head_dim), dtype=np.float32)
+    for b, n in enumerate(lengths):
+        for h in range(wl.n_kv_heads):
+            sharp[b, h * G:(h + 1) * G] = synth.sharp_query(wl, synth.as_f32(wl, K[b, h, :n]), n // 2, G)
+    check_decode(run, sharp if q.dtype == np.float32 else oracle.bf16_round(sharp))
+    rng = np.random.default_rng(3)
+    sel = [rng.choice(n, size=min(n, 300), replace=False) for n in lengths for _ in range(wl.n_kv_heads)]
+    _sparse_check(run, wl, lengths, sel, q)
+
+
+@pytest.mark.parametrize("flags", ["simt", "direct"])
+def test_int4_reference_store_decode_flags(flags):
+    wl = _small("llama3_8b_layer", n_kv_heads=2, n_q_heads=8, batch=2, seq_len=2600, ragged=None)
+    lengths = [2600, 1000]
+    K, V = synth.gen_layer(wl, 0, lengths)
+    f = rkv.RKV_FLAG_DECODE_SIMT if flags == "simt" else rkv.RKV_FLAG_DECODE_DIRECT
+    run = GpuRun(wl, K, V, lengths, ref_bits=4, flags=f)
+    assert run.unit(0, 0)["ref_bits"] == 4
+    check_decode(run, synth.gen_query(wl, 0, 0))
+
+
+def test_int4_reference_store_append():
+    wl = _small("llama3_8b_layer", n_kv_heads=2, n_q_heads=8, batch=2, seq_len=2200, ragged=None)
+    cap, start = [2200, 1900], [1500, 700]
+    K, V = synth.gen_layer(wl, 0, cap)
+    run = GpuRun(wl, K, V, cap, start_lengths=start, ref_bits=4)
+    run.append_until(cap)
+    for b, n in enumerate(cap):
+        for h in range(wl.n_kv_heads):
+            g = run.unit(b, h)
+            assert g["n"] == n
+            Xk, Xv = unit_rows(wl, K, V, b, h, n)
+            check_refs(wl, g, Xk, Xv)
+            check_compress(wl, g, Xk, Xv)
+    check_decode(run, synth.gen_query(wl, 0, 0))
+
