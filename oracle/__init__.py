@@ -76,6 +76,12 @@ def lib():
         L.orc_quantize_rows.restype = ctypes.c_int
         L.orc_dequantize_rows.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64, _vp, _vp, _vp]
         L.orc_unpack_codes.argtypes = [ctypes.c_int, ctypes.c_int, _vp, _vp]
+        L.orc_coder_fc.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64, _vp, _vp, _vp, _vp, _vp]
+        L.orc_encode_latent.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                        ctypes.c_int64, _vp, _vp, _vp, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp]
+        L.orc_encode_latent.restype = ctypes.c_int
+        L.orc_reconstruct_latent.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64,
+                                             _vp, _vp, ctypes.c_int, _vp, _vp, _vp, _vp, _vp]
         L.orc_reconstruct.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64, _vp,
                                       ctypes.c_int64, _vp, ctypes.c_int, _vp, _vp, _vp, _vp, _vp]
         L.orc_reconstruct_f.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64, _vp, _vp,
@@ -253,6 +259,61 @@ def build_refs_quantized(X: np.ndarray, ref_pos: np.ndarray, bits: int = 4, grou
     return codes, scales, dequantize_rows(codes, scales, X.shape[1], bits, group), ov
 
 
+# --- learned-coder shapes (fc SwiGLU into a latent, fd linear back) ----------------------
+
+class Coder:
+    """Weights of one side's coder (float32 holding bf16 values, row-major [out][in]):
+    fc(x) = Wo (silu(Wg x) * (Wu x)), fd(z) = Wd z."""
+
+    def __init__(self, Wg, Wu, Wo, Wd):
+        self.Wg, self.Wu, self.Wo, self.Wd = (_c(w, np.float32) for w in (Wg, Wu, Wo, Wd))
+        self.H, self.D = self.Wg.shape
+        self.L = self.Wo.shape[0]
+
+
+def coder_fc(X: np.ndarray, w: Coder) -> np.ndarray:
+    X = _c(X, np.float32)
+    n = X.shape[0]
+    out = np.empty((n, w.L), dtype=np.float64)
+    lib().orc_coder_fc(w.D, w.H, w.L, n, X.ctypes.data, w.Wg.ctypes.data, w.Wu.ctypes.data, w.Wo.ctypes.data,
+                       out.ctypes.data)
+    return out
+
+
+def encode_latent(x: np.ndarray, refs: np.ndarray, idx: np.ndarray, bits: int, w: Coder, group: int = 32):
+    """Latent residual codes z = fc(x) - fc(mean of refs): dict(codes, scales, overflow, z)."""
+    x = _c(x, np.float32)
+    refs = _c(refs if np.asarray(refs).dtype == np.float32 else bf16_value(refs), np.float32)
+    idx = _c(idx, np.uint16)
+    n = x.shape[0]
+    k = idx.shape[1]
+    codes = np.zeros((n, max(1, w.L * bits // 8)), dtype=np.uint8)
+    scales = np.zeros((n, w.L // group), dtype=np.uint16)
+    z = np.empty((n, w.L), dtype=np.float64)
+    ov = lib().orc_encode_latent(w.D, w.H, w.L, bits, group, n, x.ctypes.data, refs.ctypes.data, idx.ctypes.data, k,
+                                 w.Wg.ctypes.data, w.Wu.ctypes.data, w.Wo.ctypes.data, codes.ctypes.data,
+                                 scales.ctypes.data, z.ctypes.data)
+    return dict(codes=codes, scales=scales, overflow=int(ov), z=z)
+
+
+def reconstruct_latent(refs, idx, codes, scales, bits: int, w: Coder, group: int = 32, z_exact=None) -> np.ndarray:
+    """Rebuilt rows m + fd(z_hat) (double [n][D])."""
+    refs = _c(refs if np.asarray(refs).dtype == np.float32 else bf16_value(refs), np.float32)
+    idx = _c(idx, np.uint16)
+    n, k = idx.shape
+    out = np.empty((n, w.D), dtype=np.float64)
+    if bits == 0:
+        zx = _c(z_exact, np.float64)
+        lib().orc_reconstruct_latent(w.D, w.L, 0, group, n, refs.ctypes.data, idx.ctypes.data, k, None, None,
+                                     zx.ctypes.data, w.Wd.ctypes.data, out.ctypes.data)
+        return out
+    codes = _c(codes, np.uint8)
+    scales = _c(scales, np.uint16)
+    lib().orc_reconstruct_latent(w.D, w.L, bits, group, n, refs.ctypes.data, idx.ctypes.data, k, codes.ctypes.data,
+                                 scales.ctypes.data, None, w.Wd.ctypes.data, out.ctypes.data)
+    return out
+
+
 def attention(q: np.ndarray, K: np.ndarray, V: np.ndarray) -> np.ndarray:
     """softmax(q K^T / sqrt(D)) V for q [G][D], K, V [n][D]; double."""
     q = _c(q, np.float64)
@@ -286,14 +347,15 @@ def positions_split(n: int, ref_pos: np.ndarray):
 
 
 def compress_unit(Xk: np.ndarray, Xv: np.ndarray, stride0: int, refs_per_phase: int, k: int, bits: int,
-                  group: int = 32, positions=None, ref_bits: int = 16):
+                  group: int = 32, positions=None, ref_bits: int = 16, coder=None):
     """Compress one unit given float rows Xk, Xv [n][D] (exact input values).
 
     positions: compressed positions to encode (default: all).  ref_bits 16: bf16 reference
     rows (refK, refV uint16 bits); 4: the int4 reference store (refK, refV are the stored
     values, float32, and ref_codesK/ref_scalesK/ref_codesV/ref_scalesV are added).  Returns a
     dict with ref_pos, refK, refV, pos (encoded positions), idx, keff, dist, codesK, scalesK,
-    codesV, scalesV, overflow.
+    codesV, scalesV, overflow.  coder: (Coder K, Coder V) for latent residuals (learned-coder
+    shapes) instead of the identity coder.
     """
     n = Xk.shape[0]
     ref_pos = schedule(n, stride0, refs_per_phase)
@@ -309,25 +371,33 @@ def compress_unit(Xk: np.ndarray, Xv: np.ndarray, stride0: int, refs_per_phase: 
         positions, _ = positions_split(n, ref_pos)
     positions = np.asarray(positions, dtype=np.int32)
     idx, keff, dist = select(Xk[positions], positions, refK, ref_pos, k)
-    ek = encode(Xk[positions], refK, idx, bits, group)
-    ev = encode(Xv[positions], refV, idx, bits, group)
+    if coder is not None:                       # (Coder for K, Coder for V): latent residuals
+        ek = encode_latent(Xk[positions], refK, idx, bits, coder[0], group)
+        ev = encode_latent(Xv[positions], refV, idx, bits, coder[1], group)
+    else:
+        ek = encode(Xk[positions], refK, idx, bits, group)
+        ev = encode(Xv[positions], refV, idx, bits, group)
     return dict(ref_pos=ref_pos, refK=refK, refV=refV, pos=positions, idx=idx, keff=keff, dist=dist,
                 codesK=ek["codes"], scalesK=ek["scales"], codesV=ev["codes"], scalesV=ev["scales"],
                 overflow=ek["overflow"] | ev["overflow"], **extra)
 
 
 def unit_cache_rows(n: int, ref_pos, refK, refV, idx, codesK, scalesK, codesV, scalesV, bits: int,
-                    group: int = 32):
-    """Reconstructed K, V [n][D] float32 of a whole unit (reference rows are the stored values:
-    bf16 rows given as uint16 bits, or float32 values of the int4 reference store)."""
+                    group: int = 32, coder=None):
+    """Reconstructed K, V [n][D] (float64) of a whole unit (reference rows are the stored
+    values: bf16 rows given as uint16 bits, or float32 values of the int4 reference store;
+    coder: latent residuals rebuilt through fd)."""
     D = refK.shape[1]
     cpos, is_ref = positions_split(n, np.asarray(ref_pos))
-    Kh = np.empty((n, D), dtype=np.float32)
-    Vh = np.empty((n, D), dtype=np.float32)
+    Kh = np.empty((n, D), dtype=np.float64)
+    Vh = np.empty((n, D), dtype=np.float64)
     stored = (lambda r: r) if np.asarray(refK).dtype == np.float32 else bf16_value
     Kh[ref_pos] = stored(refK)
     Vh[ref_pos] = stored(refV)
-    if len(cpos):
+    if len(cpos) and coder is not None:
+        Kh[cpos] = reconstruct_latent(refK, idx, codesK, scalesK, bits, coder[0], group)
+        Vh[cpos] = reconstruct_latent(refV, idx, codesV, scalesV, bits, coder[1], group)
+    elif len(cpos):
         Kh[cpos] = reconstruct(refK, idx, codesK, scalesK, bits, group)
         Vh[cpos] = reconstruct(refV, idx, codesV, scalesV, bits, group)
     return Kh, Vh

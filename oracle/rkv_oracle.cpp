@@ -494,4 +494,104 @@ uint16_t orc_fp16_round_up(float f, int32_t* overflow)
 
 float orc_fp16_value(uint16_t h) { return fp16_value(h); }
 
+// ---------------------------------------------------------------------------
+// Learned-coder shapes ([P1] "DeltaKV Framework Architecture": the residual is taken after
+// a compressor, z = fc(KV) - fc(KV_R), and a token is rebuilt as fd(z) + KV_R; "Improvements
+// for AI systems": fc a SwiGLU block, fd a bias-free linear projection).  The weights are
+// inputs (random in the tests; the trained ones are not available), row-major [out][in]:
+//   fc(x) = Wo (silu(Wg x) * (Wu x)),  Wg, Wu [H][D], Wo [L][H],  silu(a) = a / (1 + e^-a)
+//   fd(z) = Wd z,                      Wd [D][L]
+// Everything in double from the exact inputs.  The latent residual is rounded to fp32 and
+// then quantised by the residuals' group quantiser, as the identity coder's residual is.
+// ---------------------------------------------------------------------------
+static void fc_apply(int D, int H, int L, const float* Wg, const float* Wu, const float* Wo, const double* x,
+                     double* out)
+{
+    std::vector<double> h(H);
+    for (int j = 0; j < H; ++j) {
+        double g = 0.0, u = 0.0;
+        for (int c = 0; c < D; ++c) {
+            g += static_cast<double>(Wg[static_cast<int64_t>(j) * D + c]) * x[c];
+            u += static_cast<double>(Wu[static_cast<int64_t>(j) * D + c]) * x[c];
+        }
+        h[j] = g / (1.0 + std::exp(-g)) * u;
+    }
+    for (int l = 0; l < L; ++l) {
+        double acc = 0.0;
+        for (int j = 0; j < H; ++j)
+            acc += static_cast<double>(Wo[static_cast<int64_t>(l) * H + j]) * h[j];
+        out[l] = acc;
+    }
+}
+
+void orc_coder_fc(int D, int H, int L, int64_t n, const float* X, const float* Wg, const float* Wu, const float* Wo,
+                  double* out)
+{
+    std::vector<double> x(D);
+    for (int64_t t = 0; t < n; ++t) {
+        for (int c = 0; c < D; ++c)
+            x[c] = X[t * D + c];
+        fc_apply(D, H, L, Wg, Wu, Wo, x.data(), out + t * L);
+    }
+}
+
+// Latent residual codes: per token m = mean reference (fp32, as the identity coder forms
+// it), z = fc(x) - fc(m) (double, rounded to fp32), then the group quantiser over the L
+// latent channels.  z_out (optional) gets z in double.  Returns 1 on a binary16 overflow.
+int orc_encode_latent(int D, int H, int L, int bits, int group, int64_t n_tok, const float* X, const float* refs,
+                      const uint16_t* idx, int k, const float* Wg, const float* Wu, const float* Wo, uint8_t* codes,
+                      uint16_t* scales, double* z_out)
+{
+    int overflow = 0;
+    std::vector<float> m(D), zf(L);
+    std::vector<double> xd(D), md(D), fx(L), fm(L);
+    for (int64_t t = 0; t < n_tok; ++t) {
+        const uint16_t* id = idx + t * k;
+        mean_reference(D, refs, id, count_keff(id, k), m.data());
+        for (int c = 0; c < D; ++c) {
+            xd[c] = X[t * D + c];
+            md[c] = m[c];
+        }
+        fc_apply(D, H, L, Wg, Wu, Wo, xd.data(), fx.data());
+        fc_apply(D, H, L, Wg, Wu, Wo, md.data(), fm.data());
+        for (int l = 0; l < L; ++l) {
+            const double z = fx[l] - fm[l];
+            if (z_out)
+                z_out[t * L + l] = z;
+            zf[l] = static_cast<float>(z);
+        }
+        if (bits > 0)
+            overflow |= quantize_groups(L, bits, group, zf.data(), codes + t * (L * bits / 8), scales + t * (L / group));
+    }
+    return overflow;
+}
+
+// Rebuilt rows x = m + fd(z_hat) in double, z_hat = code * scale (or z_exact when bits == 0).
+void orc_reconstruct_latent(int D, int L, int bits, int group, int64_t n_tok, const float* refs, const uint16_t* idx,
+                            int k, const uint8_t* codes, const uint16_t* scales, const double* z_exact,
+                            const float* Wd, double* out)
+{
+    std::vector<float> m(D);
+    std::vector<int32_t> q(L);
+    std::vector<double> zh(L);
+    for (int64_t t = 0; t < n_tok; ++t) {
+        const uint16_t* id = idx + t * k;
+        mean_reference(D, refs, id, count_keff(id, k), m.data());
+        if (bits == 0) {
+            for (int l = 0; l < L; ++l)
+                zh[l] = z_exact[t * L + l];
+        } else {
+            orc_unpack_codes(L, bits, codes + t * (L * bits / 8), q.data());
+            for (int l = 0; l < L; ++l)
+                zh[l] = static_cast<double>(q[l]) * fp16_value(scales[t * (L / group) + l / group]);
+        }
+        for (int c = 0; c < D; ++c) {
+            double acc = m[c];
+            for (int l = 0; l < L; ++l)
+                acc += static_cast<double>(Wd[static_cast<int64_t>(c) * L + l]) * zh[l];
+            out[t * D + c] = acc;
+        }
+    }
+}
+
 }  // extern "C"

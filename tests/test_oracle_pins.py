@@ -480,3 +480,90 @@ def test_int4_reference_store_unquantised_residuals_rebuild_the_input():
     xh = oracle.reconstruct(c["refK"], c["idx"], c["codesK"], c["scalesK"], 4)
     sc = np.repeat(c["scalesK"].view(np.float16).astype(np.float64), 32, axis=1)
     assert np.all(np.abs(xh - Xk[c["pos"]]) <= sc / 2 + 4 * 2 ** -24 * np.abs(Xk[c["pos"]]) + 1e-30)
+
+
+# --- learned-coder shapes (paper summary page, "DeltaKV Framework Architecture": z = fc(KV)
+#     - fc(KV_R), KV = fd(z) + KV_R; "Improvements for AI systems": SwiGLU fc, linear fd) ------
+
+def _coder(rng, D, H=None, L=None, scale=None):
+    H = D if H is None else H
+    L = D if L is None else L
+    def w(o, i):
+        return oracle.bf16_value(oracle.bf16_round(rng.standard_normal((o, i)) / np.sqrt(i)))
+    return oracle.Coder(w(H, D), w(H, D), w(L, H), w(D, L))
+
+
+def test_coder_fc_matches_torch_swiglu():
+    rng = np.random.default_rng(31)
+    D, H, L = 64, 96, 48
+    c = _coder(rng, D, H, L)
+    X = _bf16_vals(rng, (50, D), 2.0)
+    x = torch.from_numpy(X.astype(np.float64))
+    g = x @ torch.from_numpy(c.Wg.astype(np.float64)).T
+    u = x @ torch.from_numpy(c.Wu.astype(np.float64)).T
+    ref = (torch.nn.functional.silu(g) * u) @ torch.from_numpy(c.Wo.astype(np.float64)).T
+    np.testing.assert_allclose(oracle.coder_fc(X, c), ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_latent_residual_is_fc_difference_and_zero_for_the_mean():
+    rng = np.random.default_rng(32)
+    n, D, R, k = 60, 64, 20, 2
+    cK = _coder(rng, D)
+    refs = oracle.bf16_round(rng.standard_normal((R, D)))
+    idx = np.sort(np.stack([rng.choice(R, k, replace=False) for _ in range(n)]), axis=1).astype(np.uint16)
+    x = _bf16_vals(rng, (n, D))
+    rv = oracle.bf16_value(refs)
+    mean = ((rv[idx[:, 0]] + rv[idx[:, 1]]) / np.float32(2)).astype(np.float32)
+    x[:5] = mean[:5]                                          # tokens equal to their mean
+    e = oracle.encode_latent(x, refs, idx, 4, cK)
+    np.testing.assert_allclose(e["z"], oracle.coder_fc(x, cK) - oracle.coder_fc(mean, cK), rtol=1e-12, atol=1e-12)
+    assert np.all(e["codes"][:5] == 0) and np.all(e["scales"][:5] == 0)
+    # the codes are the residuals' group quantiser applied to z (rounded to fp32)
+    q = _numpy_unpack(e["codes"], D, 4)
+    s = np.repeat(e["scales"].view(np.float16).astype(np.float64), 32, axis=1)
+    z32 = e["z"].astype(np.float32).astype(np.float64)
+    assert np.all(np.abs(z32 - q * s) <= s / 2 * (1 + 1e-12))
+
+
+def test_latent_decode_factorises_through_fd():
+    """Attention over rows m + fd(z) equals the factorised form the decode uses:
+    logits q.m + (Wd^T q).z, output sum p m + Wd (sum p z), over the softmax weights p."""
+    rng = np.random.default_rng(33)
+    n, D, G, R, k = 300, 64, 3, 30, 3
+    cK, cV = _coder(rng, D), _coder(rng, D)
+    refs = oracle.bf16_round(rng.standard_normal((R, D)))
+    idx = np.sort(np.stack([rng.choice(R, k, replace=False) for _ in range(n)]), axis=1).astype(np.uint16)
+    xk, xv = _bf16_vals(rng, (n, D)), _bf16_vals(rng, (n, D))
+    ek = oracle.encode_latent(xk, refs, idx, 4, cK)
+    ev = oracle.encode_latent(xv, refs, idx, 4, cV)
+    Kh = oracle.reconstruct_latent(refs, idx, ek["codes"], ek["scales"], 4, cK)
+    Vh = oracle.reconstruct_latent(refs, idx, ev["codes"], ev["scales"], 4, cV)
+    q = rng.standard_normal((G, D))
+    got = oracle.attention(q, Kh, Vh)
+    # factorised, in numpy
+    rv = oracle.bf16_value(refs).astype(np.float64)
+    m = np.stack([rv[idx[t]].astype(np.float32).sum(axis=0, dtype=np.float32) / np.float32(k) for t in range(n)])
+    zk = _numpy_unpack(ek["codes"], D, 4) * np.repeat(ek["scales"].view(np.float16).astype(np.float64), 32, axis=1)
+    zv = _numpy_unpack(ev["codes"], D, 4) * np.repeat(ev["scales"].view(np.float16).astype(np.float64), 32, axis=1)
+    qp = q @ cK.Wd.astype(np.float64)                         # Wd^T q per head
+    logits = (q @ m.astype(np.float64).T + qp @ zk.T) / np.sqrt(D)
+    p = np.exp(logits - logits.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    want = p @ m.astype(np.float64) + (p @ zv) @ cV.Wd.astype(np.float64).T
+    np.testing.assert_allclose(got, want, rtol=1e-10, atol=1e-12)
+
+
+def test_latent_reconstruction_error_bound():
+    """m + fd(z_hat) is within |Wd| (scale/2) of m + fd(z): the quantiser's bound through fd."""
+    rng = np.random.default_rng(34)
+    n, D, R, k = 200, 64, 16, 4
+    c = _coder(rng, D)
+    refs = oracle.bf16_round(rng.standard_normal((R, D)))
+    idx = np.sort(np.stack([rng.choice(R, k, replace=False) for _ in range(n)]), axis=1).astype(np.uint16)
+    x = _bf16_vals(rng, (n, D))
+    e = oracle.encode_latent(x, refs, idx, 4, c)
+    exact = oracle.reconstruct_latent(refs, idx, None, None, 0, c, z_exact=e["z"])
+    quant = oracle.reconstruct_latent(refs, idx, e["codes"], e["scales"], 4, c)
+    s = np.repeat(e["scales"].view(np.float16).astype(np.float64), 32, axis=1)
+    bound = (s / 2 + np.abs(e["z"]) * 2 ** -23) @ np.abs(c.Wd.astype(np.float64)).T
+    assert np.all(np.abs(quant - exact) <= bound * (1 + 1e-9) + 1e-12)
