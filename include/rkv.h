@@ -112,6 +112,19 @@ typedef enum rkv_status {
  *                   is an exact bf16 number; every stage (selection, mean, residual,
  *                   reconstruction, attention) uses that stored value.  Decode then reads
  *                   72 instead of 256 bytes per reference row and side at D = 128.
+ *   coder           0: the stored residual is x - mean of the k references.  1: the
+ *                   learned-coder shapes (paper summary page, "DeltaKV Framework
+ *                   Architecture": z = fc(KV) - fc(KV_R), KV = fd(z) + KV_R;
+ *                   "Improvements for AI systems": fc a SwiGLU block, fd a bias-free
+ *                   linear projection), with weights the caller binds by rkv_set_coder:
+ *                   fc(x) = Wo (silu(Wg x) * (Wu x)), fd(z) = Wd z, hidden and latent
+ *                   widths equal to head_dim.  The latent residual z is stored with the
+ *                   same quantiser and layout as the identity coder's residual.  Decode
+ *                   applies fd by linearity: the codes meet Wd^T q, and Wd is applied once
+ *                   to the softmax-weighted latent sum.  Requires head_dim 128, bits 4,
+ *                   bf16 inputs, ref_bits 16, n_q_heads / n_kv_heads <= 8 and k <= 8; the
+ *                   RKV_FLAG_DECODE_* flags, rkv_decode_attn_sparse and rkv_append answer
+ *                   RKV_ERR_UNSUPPORTED for it.
  */
 typedef struct rkv_config {
     int32_t head_dim;
@@ -129,7 +142,8 @@ typedef struct rkv_config {
     uint32_t flags;
     int32_t ref_bits;    /* reference store: 0 or 16 = bf16 rows; 4 = int4 codes, one binary16
                             scale per 32 channels (see below) */
-    int32_t reserved[2];
+    int32_t coder;       /* 0: identity coder (residual = x - mean); 1: learned-coder shapes */
+    int32_t reserved;
 } rkv_config;
 
 /* Host-side handle of a bound cache.  Caller-allocated, opaque, plain data:
@@ -268,6 +282,17 @@ RKV_API rkv_status rkv_encode(const rkv_cache_desc* desc, const void* K, const v
  */
 RKV_API rkv_status rkv_decode_attn(const rkv_cache_desc* desc, const void* q, void* out, void* workspace,
                            uint64_t workspace_bytes, void* stream);
+
+/*
+ * Weights of the learned-coder shapes (config coder = 1), device pointers, bf16, row-major
+ * [out][in], D = head_dim: w[0..3] = Wg_K [D][D], Wu_K [D][D], Wo_K [D][D], Wd_K [D][D];
+ * w[4..7] the same for V (see rkv_config.coder).  The caller keeps them alive and unchanged
+ * while the cache is used; the handle records the pointers (host call, no launch).
+ * RKV_ERR_INVALID_ARG for a NULL or misaligned (16-byte) pointer or a cache bound with
+ * coder 0.  Compression and decode of a coder-1 cache before this call fail with
+ * RKV_ERR_INVALID_ARG.
+ */
+RKV_API rkv_status rkv_set_coder(rkv_cache_desc* desc, const void* const* w);
 
 /*
  * Current lengths of the sequences of a bound cache (host array of batch entries,

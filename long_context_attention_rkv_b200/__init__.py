@@ -31,7 +31,7 @@ STATUS_CODE = {v: k for k, v in STATUS.items()}
 EXPORTED = ["rkv_abi_version", "rkv_status_string", "rkv_schedule", "rkv_cache_size", "rkv_cache_bind",
             "rkv_unit_view_get", "rkv_build_refs", "rkv_search", "rkv_encode", "rkv_compress", "rkv_decode_attn", "rkv_reconstruct",
             "rkv_read_device_error", "rkv_compress_noalloc", "rkv_decode_attn_sparse", "rkv_cache_set_lengths",
-            "rkv_append"]
+            "rkv_append", "rkv_set_coder"]
 
 
 class RkvError(RuntimeError):
@@ -44,7 +44,7 @@ class rkv_config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("head_dim", "n_kv_heads", "n_q_heads", "k", "bits", "group",
                                               "stride0", "refs_per_phase", "in_dtype", "out_dtype", "batch",
                                               "max_len")] + [("flags", ctypes.c_uint32), ("ref_bits", ctypes.c_int32),
-                                                             ("reserved", ctypes.c_int32 * 2)]
+                                                             ("coder", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 class rkv_unit_view(ctypes.Structure):
@@ -84,6 +84,7 @@ def lib() -> ctypes.CDLL:
         L.rkv_decode_attn_sparse.argtypes = [vp, vp, vp, vp, i32, vp, vp, u64, vp]
         L.rkv_cache_set_lengths.argtypes = [vp, vp, vp]
         L.rkv_append.argtypes = [vp, vp, vp, vp, vp]
+        L.rkv_set_coder.argtypes = [vp, vp]
         for name in EXPORTED[2:]:
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -130,11 +131,11 @@ class CacheDesc:
 
 
 def make_config(head_dim, n_kv_heads, n_q_heads, k, bits, stride0, batch, max_len, refs_per_phase=0,
-                in_dtype=RKV_DTYPE_BF16, out_dtype=None, group=32, flags=0, ref_bits=0) -> rkv_config:
-    """ref_bits: 0 (or 16) bf16 reference rows; 4 the int4 reference store."""
+                in_dtype=RKV_DTYPE_BF16, out_dtype=None, group=32, flags=0, ref_bits=0, coder=0) -> rkv_config:
+    """ref_bits: 0 (or 16) bf16 reference rows; 4 the int4 reference store.  coder: 0 identity,
+    1 the learned-coder shapes (weights bound with rkv_set_coder)."""
     return rkv_config(head_dim, n_kv_heads, n_q_heads, k, bits, group, stride0, refs_per_phase, in_dtype,
-                      in_dtype if out_dtype is None else out_dtype, batch, max_len, flags, ref_bits,
-                      (ctypes.c_int32 * 2)())
+                      in_dtype if out_dtype is None else out_dtype, batch, max_len, flags, ref_bits, coder, 0)
 
 
 # --- the C ABI, one function each ------------------------------------------------------
@@ -214,6 +215,13 @@ def rkv_append(desc: CacheDesc, K_new, V_new, active=None, stream=None):
     _check(lib().rkv_append(desc.ptr, _ptr(K_new), _ptr(V_new), act, _stream(stream)), "rkv_append")
 
 
+def rkv_set_coder(desc: CacheDesc, weights):
+    """weights: eight device bf16 tensors [D][D]: Wg, Wu, Wo, Wd of K, then of V."""
+    assert len(weights) == 8
+    arr = (ctypes.c_void_p * 8)(*[_ptr(w) for w in weights])
+    _check(lib().rkv_set_coder(desc.ptr, arr), "rkv_set_coder")
+
+
 def rkv_decode_attn_sparse(desc: CacheDesc, q, positions, counts, max_sel: int, out, workspace, workspace_bytes: int,
                            stream=None):
     _check(lib().rkv_decode_attn_sparse(desc.ptr, _ptr(q), _ptr(positions), _ptr(counts), max_sel, _ptr(out),
@@ -265,6 +273,11 @@ class Layer:
 
     def decode(self, q, out, stream=None):
         rkv_decode_attn(self.desc, q, out, self.workspace, self.workspace.numel(), stream)
+
+    def set_coder(self, weights):
+        """Learned-coder weights (kept referenced here so they outlive the handle's use)."""
+        self._coder_weights = list(weights)
+        rkv_set_coder(self.desc, self._coder_weights)
 
     def set_lengths(self, lengths, stream=None):
         """Current lengths (<= the bound ones, which are the capacity)."""

@@ -89,6 +89,11 @@ rkv_status validate_config(const rkv_config* c)
         return RKV_ERR_UNSUPPORTED;
     if (c->ref_bits != 0 && c->ref_bits != 16 && c->ref_bits != 4)
         return RKV_ERR_UNSUPPORTED;
+    if (c->coder != 0 && c->coder != 1)
+        return RKV_ERR_UNSUPPORTED;
+    if (c->coder == 1 && (c->head_dim != 128 || c->bits != 4 || c->in_dtype != RKV_DTYPE_BF16 || c->ref_bits == 4 ||
+                          c->n_q_heads / c->n_kv_heads > 8 || c->k > 8))
+        return RKV_ERR_UNSUPPORTED;
     return RKV_OK;
 }
 
@@ -235,6 +240,9 @@ CacheArgs make_args(const Desc& d)
     a.ref_K = reinterpret_cast<uint16_t*>(base + d.sec.ref_K);
     a.ref_V = reinterpret_cast<uint16_t*>(base + d.sec.ref_V);
     a.ref_bits = (d.cfg.ref_bits == 4) ? 4 : 16;
+    a.coder = d.cfg.coder;
+    for (int i = 0; i < 8; ++i)
+        a.cw[i] = d.coder_w[i];
     a.ref_sK = (a.ref_bits == 4) ? reinterpret_cast<uint16_t*>(base + d.sec.ref_sK) : nullptr;
     a.ref_sV = (a.ref_bits == 4) ? reinterpret_cast<uint16_t*>(base + d.sec.ref_sV) : nullptr;
     a.ref_hn = reinterpret_cast<float*>(base + d.sec.ref_hn);
@@ -470,6 +478,9 @@ static float* cand_t_of(const Desc* d, void* ws)
     return reinterpret_cast<float*>(static_cast<char*>(ws) + align_up(2ull * d->total_cmp_rows * d->kc, 256));
 }
 
+// A learned-coder cache needs its weights bound before compression, decode or reconstruction.
+static bool coder_ready(const Desc* d) { return d->cfg.coder == 0 || d->coder_w[0] != nullptr; }
+
 rkv_status rkv_search(const rkv_cache_desc* desc, const void* K, void* workspace, uint64_t workspace_bytes,
                       void* stream)
 {
@@ -510,9 +521,21 @@ rkv_status rkv_encode(const rkv_cache_desc* desc, const void* K, const void* V, 
     const rkv_status s = check_stage_args(d, K, V, workspace, workspace_bytes);
     if (s != RKV_OK)
         return s;
+    if (!coder_ready(d))
+        return RKV_ERR_INVALID_ARG;
     const CacheArgs a = make_args(*d);
-    return cuda_status(launch_encode(a, d->max_C, K, V, cand_idx_of(d, workspace), cand_t_of(d, workspace),
-                                     static_cast<cudaStream_t>(stream)));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_encode(a, d->max_C, K, V, cand_idx_of(d, workspace), cand_t_of(d, workspace), st);
+    if (e == cudaSuccess && a.coder == 1) {
+        // the latent residuals replace the codes
+        int total = 0;
+        for (int b = 0; b < d->cfg.batch; ++b) {
+            const int n = d->cur_len[b];
+            total += d->cfg.n_kv_heads * encode_latent_tiles(n - static_cast<int>(host_ref_count(d->ph, n)));
+        }
+        e = launch_encode_latent(a, K, V, total, st);
+    }
+    return cuda_status(e);
 }
 
 rkv_status rkv_compress(const rkv_cache_desc* desc, const void* K, const void* V, void* workspace,
@@ -532,8 +555,12 @@ rkv_status rkv_decode_attn(const rkv_cache_desc* desc, const void* q, void* out,
         return RKV_ERR_INVALID_ARG;
     if (workspace_bytes < d->ws_decode)
         return RKV_ERR_WORKSPACE;
+    if (!coder_ready(d))
+        return RKV_ERR_INVALID_ARG;
     const CacheArgs a = make_args(*d);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (a.coder == 1 && ((d->cfg.flags & (RKV_FLAG_DECODE_DIRECT | RKV_FLAG_DECODE_SIMT)) || !decode_mma_supported(a)))
+        return RKV_ERR_UNSUPPORTED;   // fd is folded into the tensor-core decode only
     if (!(d->cfg.flags & (RKV_FLAG_DECODE_DIRECT | RKV_FLAG_DECODE_SIMT)) && decode_mma_supported(a) &&
         workspace_bytes >= decode_mma_ws_bytes(a, d->total_ref_rows))
         return cuda_status(launch_decode_mma(a, d->total_ref_rows, d->total_cmp_rows, q, out, workspace, st));
@@ -552,6 +579,20 @@ rkv_status rkv_decode_attn(const rkv_cache_desc* desc, const void* q, void* out,
     if (e == cudaSuccess)
         e = launch_decode_combine(a, d->cfg.batch, splits, part, out, st);
     return cuda_status(e);
+}
+
+rkv_status rkv_set_coder(rkv_cache_desc* desc, const void* const* w)
+{
+    const Desc* cd = get_desc(desc);
+    if (!cd || !w || cd->cfg.coder != 1)
+        return RKV_ERR_INVALID_ARG;
+    for (int i = 0; i < 8; ++i)
+        if (!w[i] || !aligned(w[i], 16))
+            return RKV_ERR_INVALID_ARG;
+    Desc* d = const_cast<Desc*>(cd);
+    for (int i = 0; i < 8; ++i)
+        d->coder_w[i] = static_cast<const uint16_t*>(w[i]);
+    return RKV_OK;
 }
 
 rkv_status rkv_cache_set_lengths(rkv_cache_desc* desc, const int32_t* lengths, void* stream)
@@ -593,6 +634,8 @@ rkv_status rkv_append(rkv_cache_desc* desc, const void* K_new, const void* V_new
     if (!cd || !K_new || !V_new || !aligned(K_new, 16) || !aligned(V_new, 16))
         return RKV_ERR_INVALID_ARG;
     Desc* d = const_cast<Desc*>(cd);
+    if (d->cfg.coder != 0)
+        return RKV_ERR_UNSUPPORTED;
     uint32_t bits[8] = {};
     bool any = false;
     for (int b = 0; b < d->cfg.batch; ++b) {
@@ -626,6 +669,8 @@ rkv_status rkv_decode_attn_sparse(const rkv_cache_desc* desc, const void* q, con
         return RKV_ERR_INVALID_ARG;
     if (workspace_bytes < d->ws_decode)
         return RKV_ERR_WORKSPACE;
+    if (d->cfg.coder != 0)
+        return RKV_ERR_UNSUPPORTED;
     const CacheArgs a = make_args(*d);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int splits = sparse_splits(d->n_units, std::min<int>(max_sel, std::max(1, d->max_n)));
@@ -651,6 +696,8 @@ rkv_status rkv_reconstruct(const rkv_cache_desc* desc, int32_t seq, int32_t kv_h
     if (n_pos == 0)
         return RKV_OK;
     if (!K_out && !V_out)
+        return RKV_ERR_INVALID_ARG;
+    if (!coder_ready(d))
         return RKV_ERR_INVALID_ARG;
     const CacheArgs a = make_args(*d);
     return cuda_status(launch_reconstruct(a, seq * d->cfg.n_kv_heads + kv_head, positions, n_pos, K_out, V_out,

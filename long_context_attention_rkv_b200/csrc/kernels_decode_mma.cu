@@ -161,6 +161,8 @@ struct MmaWs {
     float* O;         // [units][Gp][D]  output numerators
     float* L;         // [units][Gp]     softmax denominators
     uint32_t* cnt;    // [units]         finished chunks of the refs kernel
+    float* Olat;      // [units][Gp][D]  learned-coder shapes: latent output numerators
+    uint16_t* qlat;   // [batch][Hq][D]  learned-coder shapes: Wd_K^T q (bf16)
     int n_chunk;
     int n_tiles;
     int n_cta;        // CTAs of the tokens kernel
@@ -236,6 +238,21 @@ __global__ void __launch_bounds__(128) mma_scores_kernel(const CacheArgs a, cons
             w.L[u * Gp + tid] = 0.0f;
         if (tid == 0)
             w.cnt[u] = 0u;
+        if (a.coder == 1) {
+            // learned-coder shapes: the compressed tokens' codes are latent, so they meet
+            // q' = Wd_K^T q (fd folded into the query); the latent output sums start at zero
+            for (int i = tid; i < Gp * D; i += 128)
+                w.Olat[static_cast<int64_t>(u) * Gp * D + i] = 0.0f;
+            const uint16_t* Wd = a.cw[3];
+            const uint16_t* qb = static_cast<const uint16_t*>(q) + (static_cast<int64_t>(um.seq) * a.Hq + kvh * a.G) * D;
+            uint16_t* qo = w.qlat + (static_cast<int64_t>(um.seq) * a.Hq + kvh * a.G) * D;
+            for (int g = 0; g < a.G; ++g) {
+                float acc = 0.0f;
+                for (int c = 0; c < D; ++c)
+                    acc = fmaf(bf16_bits_to_f32(Wd[c * D + tid]), bf16_bits_to_f32(qb[g * D + c]), acc);
+                qo[g * D + tid] = f32_to_bf16_bits(acc);
+            }
+        }
     }
     for (int i = tid; i < (r1 - r0) * Gp; i += 128)
         w.W[(um.ref_row + r0) * Gp + i] = 0.0f;
@@ -938,7 +955,14 @@ __global__ void __launch_bounds__(256) mma_refs_kernel(const CacheArgs a, void* 
     __threadfence();
     for (int x = tid; x < G * D; x += 256) {
         const int h = x / D, c = x % D;
-        const float o = __ldcg(&w.O[static_cast<int64_t>(u) * Gp * D + x]);
+        float o = __ldcg(&w.O[static_cast<int64_t>(u) * Gp * D + x]);
+        if (a.coder == 1) {
+            // fd applied once to the softmax-weighted latent sum: o += Wd_V (sum_i p_i z_i)
+            const uint16_t* Wd = a.cw[7] + c * D;
+            const float* ol = w.Olat + (static_cast<int64_t>(u) * Gp + h) * D;
+            for (int l = 0; l < D; ++l)
+                o = fmaf(bf16_bits_to_f32(Wd[l]), __ldcg(ol + l), o);
+        }
         const float l = __ldcg(&w.L[u * Gp + h]);
         const float res = (l > 0.0f) ? o / l : 0.0f;
         const int64_t e = (static_cast<int64_t>(um.seq) * a.Hq + kvh * G + h) * D + c;
@@ -976,7 +1000,7 @@ bool tables_global(const CacheArgs& a) { return tok_stages(a, a.max_refs) == 0; 
 constexpr int kMaxCta = 160;   // grid cap of the tokens kernel
 
 struct WsOffsets {
-    uint64_t s_tab, W, mpart, O, L, cnt, end;
+    uint64_t s_tab, W, mpart, O, L, cnt, Olat, qlat, end;
 };
 
 WsOffsets ws_offsets(const CacheArgs& a, int64_t ref_rows)
@@ -996,6 +1020,8 @@ WsOffsets ws_offsets(const CacheArgs& a, int64_t ref_rows)
     o.O = take(4ull * a.n_units * Gp * 128);
     o.L = take(4ull * a.n_units * Gp);
     o.cnt = take(4ull * a.n_units);
+    o.Olat = take(a.coder == 1 ? 4ull * a.n_units * Gp * 128 : 0);
+    o.qlat = take(a.coder == 1 ? 2ull * a.n_units * a.G * 128 : 0);
     o.end = off;
     return o;
 }
@@ -1068,7 +1094,15 @@ cudaError_t launch_gp(const CacheArgs& a, int64_t cmp_rows, const void* q, void*
         if (e != cudaSuccess)
             return e;
         const int grid = w.n_cta;
-        e = launch_pdl(kern, dim3(grid), dim3(32 * kConsWarps * kTeams), smem, st, mK, mV, a, q, w, nst);
+        // learned-coder shapes: the tokens kernel meets the latent codes with q' and sums the
+        // latent V side into Olat (the refs kernel applies fd to it)
+        MmaWs wt = w;
+        const void* qt = q;
+        if (a.coder == 1) {
+            wt.O = w.Olat;
+            qt = w.qlat;
+        }
+        e = launch_pdl(kern, dim3(grid), dim3(32 * kConsWarps * kTeams), smem, st, mK, mV, a, qt, wt, nst);
         if (e != cudaSuccess)
             return e;
     }
@@ -1099,6 +1133,8 @@ cudaError_t launch_decode_mma(const CacheArgs& a, int64_t ref_rows, int64_t cmp_
     w.O = reinterpret_cast<float*>(base + o.O);
     w.L = reinterpret_cast<float*>(base + o.L);
     w.cnt = reinterpret_cast<uint32_t*>(base + o.cnt);
+    w.Olat = reinterpret_cast<float*>(base + o.Olat);
+    w.qlat = reinterpret_cast<uint16_t*>(base + o.qlat);
     w.n_chunk = (a.max_refs + kRefChunk - 1) / kRefChunk > 0 ? (a.max_refs + kRefChunk - 1) / kRefChunk : 1;
     w.n_tiles = static_cast<int>(cmp_rows / kTok);
     {

@@ -5,7 +5,8 @@
 // One warp per requested position; lanes own D/32 consecutive channels.
 // Reference positions return the stored bf16 row.  Compressed positions return
 // mean(references) + code * scale with the mean formed exactly as the encoder
-// formed it (fp32, ascending ordinals, one division).
+// formed it (fp32, ascending ordinals, one division); with the learned-coder
+// shapes, mean + Wd (code * scale) (the decompressor fd applied to the latent).
 #include "device_common.cuh"
 #include "launchers.h"
 
@@ -45,6 +46,36 @@ __device__ __forceinline__ void dequant_add(const uint8_t* codes_row, const uint
         const int q = code_at(codes_row, bits, lane * NPL + i);
         x[i] = __fadd_rn(x[i], __fmul_rn(static_cast<float>(q), s));
     }
+}
+
+// Learned-coder shapes: x += Wd z_hat for this lane's channels, z_hat the dequantised latent
+// codes (the lanes' parts exchanged by shuffles); Wd bf16 [D][D].
+template <int NPL>
+__device__ __forceinline__ void fd_add(const uint8_t* codes_row, const uint16_t* scale_row, int bits, int lane,
+                                       const uint16_t* Wd, float (&x)[NPL])
+{
+    constexpr int D = NPL * 32;
+    constexpr int LPG = 32 / NPL;
+    const float s = __half2float(__ushort_as_half(scale_row[lane / LPG]));
+    float z[NPL], acc[NPL];
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+        z[i] = __fmul_rn(static_cast<float>(code_at(codes_row, bits, lane * NPL + i)), s);
+        acc[i] = 0.0f;
+    }
+    for (int src = 0; src < 32; ++src) {
+#pragma unroll
+        for (int e = 0; e < NPL; ++e) {
+            const float zl = __shfl_sync(0xffffffffu, z[e], src);
+            const int l = src * NPL + e;
+#pragma unroll
+            for (int i = 0; i < NPL; ++i)
+                acc[i] = fmaf(bf16_bits_to_f32(Wd[(lane * NPL + i) * D + l]), zl, acc[i]);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < NPL; ++i)
+        x[i] = __fadd_rn(x[i], acc[i]);
 }
 
 template <int NPL>
@@ -104,8 +135,13 @@ __global__ void __launch_bounds__(kWarps * 32) reconstruct_kernel(CacheArgs a, i
             xk[j] = __fdiv_rn(xk[j], fk);
             xv[j] = __fdiv_rn(xv[j], fk);
         }
-        dequant_add<NPL>(a.codes_K + row * a.code_bytes, a.scale_K + row * a.n_groups, a.bits, lane, xk);
-        dequant_add<NPL>(a.codes_V + row * a.code_bytes, a.scale_V + row * a.n_groups, a.bits, lane, xv);
+        if (a.coder == 1) {
+            fd_add<NPL>(a.codes_K + row * a.code_bytes, a.scale_K + row * a.n_groups, a.bits, lane, a.cw[3], xk);
+            fd_add<NPL>(a.codes_V + row * a.code_bytes, a.scale_V + row * a.n_groups, a.bits, lane, a.cw[7], xv);
+        } else {
+            dequant_add<NPL>(a.codes_K + row * a.code_bytes, a.scale_K + row * a.n_groups, a.bits, lane, xk);
+            dequant_add<NPL>(a.codes_V + row * a.code_bytes, a.scale_V + row * a.n_groups, a.bits, lane, xv);
+        }
     }
     const int64_t o = i * D + lane * NPL;
     if (K_out)

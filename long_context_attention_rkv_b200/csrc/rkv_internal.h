@@ -74,6 +74,7 @@ struct Desc {
     int64_t ref_seq_row[RKV_MAX_BATCH];
     int64_t cmp_seq_row[RKV_MAX_BATCH];
     int32_t cur_len[RKV_MAX_BATCH];   // current lengths (len[] is the capacity the layout holds)
+    const uint16_t* coder_w[8];       // learned-coder weights (coder 1): Wg, Wu, Wo, Wd for K, then V
 };
 static_assert(sizeof(Desc) <= RKV_CACHE_DESC_BYTES, "descriptor too large");
 
@@ -81,7 +82,7 @@ static_assert(sizeof(Desc) <= RKV_CACHE_DESC_BYTES, "descriptor too large");
 struct CacheArgs {
     int32_t D, Hkv, Hq, G, k, bits, group, in_dtype, out_dtype;
     int32_t n_units, code_bytes, n_groups, kc, max_len, max_refs;
-    int32_t ref_bits, pad_r;   // 16: bf16 reference rows; 4: int4 reference store
+    int32_t ref_bits, coder;   // 16: bf16 reference rows, 4: int4 store; coder 0 identity, 1 learned shapes
     Phases ph;
     const UnitMeta* units;
     int32_t* err;
@@ -97,6 +98,7 @@ struct CacheArgs {
     uint16_t* scale_K;
     uint16_t* scale_V;
     uint16_t* idx;
+    const uint16_t* cw[8];   // coder 1: Wg, Wu, Wo, Wd (bf16 [D][D]) of K, then of V
 };
 
 // Selection work item: one tile of kPosTile positions of one unit (CUDA-core search), or a pair

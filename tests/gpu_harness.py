@@ -28,25 +28,31 @@ def to_dev(arr: np.ndarray) -> torch.Tensor:
 
 
 def config(wl: synth.Workload, lengths, max_len=None, out_dtype=rkv.RKV_DTYPE_F32, flags=0, batch=None,
-           ref_bits=0):
+           ref_bits=0, coder=0):
     return rkv.make_config(head_dim=wl.head_dim, n_kv_heads=wl.n_kv_heads, n_q_heads=wl.n_q_heads, k=wl.k,
                            bits=wl.bits, stride0=wl.stride0, batch=len(lengths) if batch is None else batch,
                            max_len=max(max(lengths), 1) if max_len is None else max_len,
                            refs_per_phase=wl.refs_per_phase, in_dtype=wl.dtype_code, out_dtype=out_dtype,
-                           flags=flags, ref_bits=ref_bits)
+                           flags=flags, ref_bits=ref_bits, coder=coder)
 
 
 class GpuRun:
     """One layer compressed on the GPU through the C ABI."""
 
     def __init__(self, wl: synth.Workload, K: np.ndarray, V: np.ndarray, lengths, out_dtype=rkv.RKV_DTYPE_F32,
-                 flags=0, start_lengths=None, ref_bits=0):
+                 flags=0, start_lengths=None, ref_bits=0, coder=None):
         """lengths: the bound (capacity) lengths; start_lengths: a shorter prefix to compress
-        first (grown later with append_until); ref_bits 4: the int4 reference store."""
+        first (grown later with append_until); ref_bits 4: the int4 reference store; coder:
+        (oracle.Coder K, oracle.Coder V) for the learned-coder shapes."""
         self.wl = wl
         self.lengths = list(lengths)
-        self.cfg = config(wl, lengths, max_len=K.shape[2], out_dtype=out_dtype, flags=flags, ref_bits=ref_bits)
+        self.coder = coder
+        self.cfg = config(wl, lengths, max_len=K.shape[2], out_dtype=out_dtype, flags=flags, ref_bits=ref_bits,
+                          coder=0 if coder is None else 1)
         self.layer = rkv.Layer(self.cfg, self.lengths)
+        if coder is not None:
+            ws = [w for c in coder for w in (c.Wg, c.Wu, c.Wo, c.Wd)]
+            self.layer.set_coder([to_dev(oracle.bf16_round(w)) for w in ws])
         self.Kd = to_dev(K)
         self.Vd = to_dev(V)
         self.cur = list(self.lengths if start_lengths is None else start_lengths)
@@ -177,7 +183,7 @@ def check_refs(wl, g: dict, Xk, Xv):
     return ref_pos
 
 
-def check_compress(wl, g: dict, Xk, Xv, positions=None, stats=None):
+def check_compress(wl, g: dict, Xk, Xv, positions=None, stats=None, coder=None):
     """Selection (tie-band aware) and codes of compressed positions against the oracle."""
     n = len(Xk)
     ref_pos = oracle.schedule(n, wl.stride0, wl.refs_per_phase)
@@ -208,10 +214,33 @@ def check_compress(wl, g: dict, Xk, Xv, positions=None, stats=None):
         worst = max(oracle.l2(Xk[positions[t]], rv[j]) for j in sel)
         assert worst <= dk1 * (1 + IDX_TIE_BAND)
     # codes: the oracle's encoder fed the GPU's index sets
-    ek = oracle.encode(Xk[positions], refK, gidx, wl.bits, wl.group)
-    ev = oracle.encode(Xv[positions], refV, gidx, wl.bits, wl.group)
+    if coder is not None:
+        ek = oracle.encode_latent(Xk[positions], refK, gidx, wl.bits, coder[0], wl.group)
+        ev = oracle.encode_latent(Xv[positions], refV, gidx, wl.bits, coder[1], wl.group)
+    else:
+        ek = oracle.encode(Xk[positions], refK, gidx, wl.bits, wl.group)
+        ev = oracle.encode(Xv[positions], refV, gidx, wl.bits, wl.group)
     assert ek["overflow"] == 0 and ev["overflow"] == 0
     D = wl.head_dim
+    if coder is not None:
+        # the GPU forms the latent z in fp32, the oracle in double: a group's scale may take
+        # the neighbouring binary16 value where a/7 lies within that error of a binary16
+        # boundary (rare); every code still quantises the oracle's z within half a step
+        for name, e in (("K", ek), ("V", ev)):
+            gs = g["scales" + name][slots].view(np.float16).astype(np.float64)
+            os_ = e["scales"].view(np.float16).astype(np.float64)
+            diff = gs != os_
+            assert diff.mean() <= CODE_LSB_FRACTION, f"{name} latent scales differ in {diff.mean():.2e} of groups"
+            assert np.all(np.abs(gs - os_) <= os_ * 2.0 ** -9), f"{name} latent scales differ by more than a step"
+            gc = _unpack(g["codes" + name][slots], D, wl.bits)
+            sc = np.repeat(gs, 32, axis=1)
+            amax = np.repeat(np.abs(e["z"]).reshape(len(slots), -1, 32).max(axis=2), 32, axis=1)
+            err = np.abs(e["z"] - gc * sc)
+            assert np.all(err <= sc / 2 + 1e-4 * amax), f"{name} latent codes off by {(err - sc / 2).max()}"
+        if stats is not None:
+            stats["tokens"] = stats.get("tokens", 0) + len(positions)
+            stats["idx_tie_mismatch"] = stats.get("idx_tie_mismatch", 0) + mism
+        return
     for name, e in (("K", ek), ("V", ev)):
         assert np.array_equal(g["scales" + name][slots], e["scales"]), f"{name} scales differ"
         gc = _unpack(g["codes" + name][slots], D, wl.bits)
@@ -224,13 +253,13 @@ def check_compress(wl, g: dict, Xk, Xv, positions=None, stats=None):
         stats["idx_tie_mismatch"] = stats.get("idx_tie_mismatch", 0) + mism
 
 
-def oracle_decode_on_gpu_cache(wl, g: dict, q_group: np.ndarray):
+def oracle_decode_on_gpu_cache(wl, g: dict, q_group: np.ndarray, coder=None):
     """The oracle's reconstruction and attention over the cache the GPU produced."""
     n = g["n"]
     if n == 0:
         return np.zeros((q_group.shape[0], wl.head_dim))
     Kh, Vh = oracle.unit_cache_rows(n, g["pos"], g["refK"], g["refV"], g["idx"], g["codesK"], g["scalesK"],
-                                    g["codesV"], g["scalesV"], wl.bits, wl.group)
+                                    g["codesV"], g["scalesV"], wl.bits, wl.group, coder=coder)
     return oracle.attention(q_group.astype(np.float64), Kh, Vh)
 
 
@@ -245,7 +274,7 @@ def check_decode(run: GpuRun, q: np.ndarray, units=None, threads=8):
 
     def one(u):
         b, h = u
-        return u, oracle_decode_on_gpu_cache(wl, gus[u], qf[b, h * G:(h + 1) * G])
+        return u, oracle_decode_on_gpu_cache(wl, gus[u], qf[b, h * G:(h + 1) * G], run.coder)
 
     with ThreadPoolExecutor(threads) as ex:
         refs = dict(ex.map(one, units))
@@ -266,7 +295,7 @@ def check_reconstruct(run: GpuRun, g: dict, b: int, h: int, positions=None):
     wl = run.wl
     n = g["n"]
     Kh, Vh = oracle.unit_cache_rows(n, g["pos"], g["refK"], g["refV"], g["idx"], g["codesK"], g["scalesK"],
-                                    g["codesV"], g["scalesV"], wl.bits, wl.group)
+                                    g["codesV"], g["scalesV"], wl.bits, wl.group, coder=run.coder)
     Kg, Vg = run.reconstruct(b, h, positions)
     sel = np.arange(n) if positions is None else np.asarray(positions)
     np.testing.assert_allclose(Kg, Kh[sel], atol=RECON_ABS, rtol=0)

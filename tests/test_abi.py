@@ -1,5 +1,6 @@
 """The C-ABI library: it loads, exports every declared symbol, and its host-side logic
 (schedule, sizing, validation) is right.  No device calls."""
+import ctypes
 import os
 import re
 
@@ -65,6 +66,18 @@ def test_int4_reference_store_sizes():
         with pytest.raises(rkv.RkvError) as ei:
             rkv.rkv_cache_size(_cfg(ref_bits=bad), lengths)
         assert rkv.STATUS[ei.value.status] == "RKV_ERR_UNSUPPORTED"
+
+
+def test_learned_coder_validation():
+    assert rkv.rkv_cache_size(_cfg(coder=1), [4096])[0] > 0
+    for bad in (dict(coder=2), dict(coder=1, head_dim=64), dict(coder=1, bits=8), dict(coder=1, ref_bits=4),
+                dict(coder=1, k=9), dict(coder=1, n_q_heads=8 * 9)):
+        with pytest.raises(rkv.RkvError) as ei:
+            rkv.rkv_cache_size(_cfg(**bad), [4096])
+        assert rkv.STATUS[ei.value.status] == "RKV_ERR_UNSUPPORTED", bad
+    d = rkv.CacheDesc()
+    arr = (ctypes.c_void_p * 8)(*([16] * 8))
+    assert rkv.lib().rkv_set_coder(d.ptr, arr) == rkv.STATUS_CODE["RKV_ERR_INVALID_ARG"]
 
 
 def test_ragged_sizes_and_validation():

@@ -12,7 +12,7 @@ import torch
 import long_context_attention_rkv_b200 as rkv
 import oracle
 import synth
-from gpu_harness import (GpuRun, check_compress, check_decode, check_reconstruct, check_refs, sample_positions,
+from gpu_harness import (GpuRun, check_compress, check_decode, check_reconstruct, check_refs, config, sample_positions,
                          to_dev, unit_rows)
 
 pytestmark = pytest.mark.gpu
@@ -388,3 +388,62 @@ def test_int4_reference_store_append():
             check_compress(wl, g, Xk, Xv)
     check_decode(run, synth.gen_query(wl, 0, 0))
 
+
+
+# --- learned-coder shapes (paper summary page, "DeltaKV Framework Architecture": z = fc(KV) -
+#     fc(KV_R), KV = fd(z) + KV_R; "Improvements for AI systems": SwiGLU fc, linear fd) -------
+
+def _random_coders(D, seed):
+    rng = np.random.default_rng(seed)
+
+    def w():
+        return oracle.bf16_value(oracle.bf16_round(rng.standard_normal((D, D)) / np.sqrt(D)))
+    return tuple(oracle.Coder(w(), w(), w(), w()) for _ in range(2))
+
+
+@pytest.mark.parametrize("case", ["llama", "qwen"])
+def test_learned_coder_shapes_every_stage(case):
+    """Latent residual codes against the oracle's fc on the GPU's index sets; reconstruction
+    through fd; decode with fd folded into the query and the latent output sum."""
+    if case == "llama":
+        wl = _small("llama3_8b_layer", n_kv_heads=2, n_q_heads=8, batch=2, seq_len=3000, ragged=None)
+        lengths = [3000, 1200]
+    else:
+        wl = _small("qwen2_5_7b_batch", n_kv_heads=2, n_q_heads=14, batch=2, seq_len=2600, ragged=None)
+        lengths = [2600, 2000]
+    K, V = synth.gen_layer(wl, 0, lengths)
+    coder = _random_coders(wl.head_dim, 11)
+    run = GpuRun(wl, K, V, lengths, coder=coder)
+    stats = {}
+    for b, n in enumerate(lengths):
+        for h in range(wl.n_kv_heads):
+            g = run.unit(b, h)
+            Xk, Xv = unit_rows(wl, K, V, b, h, n)
+            check_refs(wl, g, Xk, Xv)
+            pos = sample_positions(wl, n, n_uniform=400, seed=b * 7 + h)
+            check_compress(wl, g, Xk, Xv, positions=pos, stats=stats, coder=coder)
+            check_reconstruct(run, g, b, h, positions=pos)
+    assert stats["tokens"] > 0
+    check_decode(run, synth.gen_query(wl, 0, 0))
+
+
+def test_learned_coder_refuses_what_it_does_not_cover():
+    wl = _small("llama3_8b_layer", n_kv_heads=1, n_q_heads=4, seq_len=600)
+    lengths = [600]
+    K, V = synth.gen_layer(wl, 0, lengths)
+    coder = _random_coders(wl.head_dim, 12)
+    run = GpuRun(wl, K, V, lengths, coder=coder)
+    q = to_dev(synth.gen_query(wl, 0, 0))
+    out = torch.empty((1, 4, 128), dtype=torch.float32, device="cuda")
+    pos = torch.zeros((1, 4), dtype=torch.int32, device="cuda")
+    cnt = torch.ones(1, dtype=torch.int32, device="cuda")
+    for call in (lambda: run.layer.decode_sparse(q, pos, cnt, out),
+                 lambda: run.layer.append(run.Kd[:, :, 0].contiguous(), run.Vd[:, :, 0].contiguous())):
+        with pytest.raises(rkv.RkvError) as ei:
+            call()
+        assert ei.value.status == rkv.STATUS_CODE["RKV_ERR_UNSUPPORTED"]
+    # a coder-1 cache without weights refuses to compress
+    bare = rkv.Layer(config(wl, lengths, max_len=K.shape[2], coder=1), lengths)
+    with pytest.raises(rkv.RkvError) as ei:
+        bare.compress(run.Kd, run.Vd)
+    assert ei.value.status == rkv.STATUS_CODE["RKV_ERR_INVALID_ARG"]
