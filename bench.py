@@ -9,9 +9,9 @@ region starts; L2 is flushed (256 MiB write) before every timed step, outside
 the timed spans.  With N GPUs (torchrun) every rank runs its own replica on an
 independent layer; value is the whole-job throughput over the max-over-ranks
 step time.  Outside the step, a selective decode (2048 seeded positions per unit),
-incremental compression (the last 64 tokens appended one at a time) and the same layer
-with the int4 reference store (reference store, search, encode, decode) are timed as
-well.  `--impl reference` times the CPU oracle on a bounded sample of
+incremental compression (the last 64 tokens appended one at a time), the same layer
+with the int4 reference store (reference store, search, encode, decode) and with the
+learned-coder shapes (random weights) are timed as well.  `--impl reference` times the CPU oracle on a bounded sample of
 the same workload on the host cores.  Prints one JSON line on rank 0.
 """
 from __future__ import annotations
@@ -86,6 +86,7 @@ def workload_quantities(wl, lengths):
     flops = 0
     dec_bytes = 0
     dec_bytes4 = 0
+    cmp_tokens = 0
     enc_bytes = 0
     refs_bytes = 0
     for n in lengths:
@@ -100,12 +101,14 @@ def workload_quantities(wl, lengths):
         cpos = np.nonzero(~is_ref)[0]
         ncand = np.searchsorted(ref_pos, cpos, side="right").astype(np.int64)
         flops += wl.n_kv_heads * int(ncand.sum()) * 2 * D
+        cmp_tokens += wl.n_kv_heads * C
         dec_bytes += wl.n_kv_heads * (C * per_tok + R * 4 * D)
         # int4 reference store: codes (D/2 bytes) and binary16 scales (D/32) per row and side
         dec_bytes4 += wl.n_kv_heads * (C * per_tok + R * 2 * (D // 2 + 2 * (D // 32)))
         enc_bytes += wl.n_kv_heads * C * (2 * D * wl.elem_bytes + per_tok)
         refs_bytes += wl.n_kv_heads * R * (2 * D * wl.elem_bytes + 4 * D + 8)
-    return dict(tokens=sum(lengths), search_flops=flops, decode_bytes=dec_bytes, decode_bytes_int4_refs=dec_bytes4,
+    return dict(tokens=sum(lengths), tokens_cmp=cmp_tokens, search_flops=flops, decode_bytes=dec_bytes,
+                decode_bytes_int4_refs=dec_bytes4,
                 encode_bytes=enc_bytes, refs_bytes=refs_bytes, bytes_per_token=per_tok)
 
 
@@ -493,6 +496,47 @@ def run_ours(args, rank, world, local_rank):
     del g4, L4
     avg4 = {nm: statistics.mean(v) for nm, v in ms4.items()}
 
+    # learned-coder shapes (outside the step): seeded random bf16 weights (scale 1/sqrt(D));
+    # encode adds the latent pass (SwiGLU fc of every token and of its mean), decode folds fd
+    wrng = np.random.default_rng(0xC0DE)
+    cw = [torch.from_numpy((wrng.standard_normal((wl.head_dim, wl.head_dim)) / np.sqrt(wl.head_dim))
+                           .astype(np.float32)).to(torch.bfloat16).to(dev) for _ in range(8)]
+    cfgc = rkv.make_config(head_dim=wl.head_dim, n_kv_heads=wl.n_kv_heads, n_q_heads=wl.n_q_heads, k=wl.k,
+                           bits=wl.bits, stride0=wl.stride0, batch=wl.batch, max_len=K.shape[2],
+                           refs_per_phase=wl.refs_per_phase, in_dtype=wl.dtype_code, out_dtype=wl.dtype_code,
+                           coder=1)
+    Lc = rkv.Layer(cfgc, lengths, device=dev)
+    Lc.set_coder(cw)
+    stc = {"build_refs": lambda: Lc.build_refs(K, V), "search": lambda: Lc.search(K),
+           "encode": lambda: Lc.encode(K, V), "decode": lambda: Lc.decode(q, out)}
+    gc = {}
+    with torch.cuda.stream(stream):
+        for nm in stc:
+            stc[nm]()
+        torch.cuda.synchronize(dev)
+        for nm in stc:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                stc[nm]()
+            gc[nm] = g
+    torch.cuda.synchronize(dev)
+    msc = {nm: [] for nm in stc}
+    with torch.cuda.stream(stream):
+        for i in range(max(3, min(args.steps, 10)) + 2):
+            for nm in stc:
+                flush.zero_()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                gc[nm].replay()
+                e1.record(stream)
+                e1.synchronize()
+                if i >= 2:
+                    msc[nm].append(e0.elapsed_time(e1))
+    assert Lc.device_error() == 0
+    del gc, Lc
+    avgc = {nm: statistics.mean(v) for nm, v in msc.items()}
+
     Q = workload_quantities(wl, lengths)
     tokens = Q["tokens"]
     value = job_throughput(world, tokens, mean_step)
@@ -550,6 +594,12 @@ def run_ours(args, rank, world, local_rank):
                     "decode_bytes_per_step": Q["decode_bytes_int4_refs"],
                     "decode_hbm_gbs": Q["decode_bytes_int4_refs"] / (avg4["decode"] * 1e-3) / 1e9,
                     "compress_mtok_s": tokens / ((avg4["build_refs"] + avg4["search"] + avg4["encode"]) * 1e-3)
+                    / 1e6,
+                },
+                "learned_coder": {
+                    "encode_us": 1e3 * avgc["encode"], "decode_us_per_step": 1e3 * avgc["decode"],
+                    "encode_latent_gflop": 2 * 2 * Q["tokens_cmp"] * 5 * wl.head_dim * wl.head_dim / 1e9,
+                    "compress_mtok_s": tokens / ((avgc["build_refs"] + avgc["search"] + avgc["encode"]) * 1e-3)
                     / 1e6,
                 },
             },

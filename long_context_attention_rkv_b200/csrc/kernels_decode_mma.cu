@@ -173,7 +173,7 @@ namespace {
 
 // ==== 1. reference scores ==================================================================
 
-template <int Gp, int RB>
+template <int Gp, int RB, bool LC>
 __global__ void __launch_bounds__(128) mma_scores_kernel(const CacheArgs a, const void* __restrict__ q, const MmaWs w)
 {
     // s[r][h] = cK * (refK_r . q_h) as m16n8k16 MMAs: one warp per 16 references, columns are
@@ -238,20 +238,39 @@ __global__ void __launch_bounds__(128) mma_scores_kernel(const CacheArgs a, cons
             w.L[u * Gp + tid] = 0.0f;
         if (tid == 0)
             w.cnt[u] = 0u;
-        if (a.coder == 1) {
+        if (LC) {
             // learned-coder shapes: the compressed tokens' codes are latent, so they meet
             // q' = Wd_K^T q (fd folded into the query); the latent output sums start at zero
             for (int i = tid; i < Gp * D; i += 128)
                 w.Olat[static_cast<int64_t>(u) * Gp * D + i] = 0.0f;
+            // thread l: q'[g][l] = sum_c Wd_K[c][l] q[g][c]; Wd_K (32 KB) staged in shared
+            // memory with 16-byte loads first
+            __shared__ float qs[8][D];
+            __shared__ __align__(16) uint16_t wds[LC ? D * D : 8];
             const uint16_t* Wd = a.cw[3];
             const uint16_t* qb = static_cast<const uint16_t*>(q) + (static_cast<int64_t>(um.seq) * a.Hq + kvh * a.G) * D;
             uint16_t* qo = w.qlat + (static_cast<int64_t>(um.seq) * a.Hq + kvh * a.G) * D;
-            for (int g = 0; g < a.G; ++g) {
-                float acc = 0.0f;
-                for (int c = 0; c < D; ++c)
-                    acc = fmaf(bf16_bits_to_f32(Wd[c * D + tid]), bf16_bits_to_f32(qb[g * D + c]), acc);
-                qo[g * D + tid] = f32_to_bf16_bits(acc);
+            if constexpr (LC) {
+#pragma unroll 4
+                for (int i = tid; i < D * D / 8; i += 128)
+                    reinterpret_cast<uint4*>(wds)[i] = reinterpret_cast<const uint4*>(Wd)[i];
             }
+            for (int i = tid; i < 8 * D; i += 128)
+                qs[i / D][i % D] = (i < a.G * D) ? bf16_bits_to_f32(qb[i]) : 0.0f;
+            __syncthreads();
+            float acc[8];
+#pragma unroll
+            for (int g = 0; g < 8; ++g)
+                acc[g] = 0.0f;
+#pragma unroll 8
+            for (int c = 0; c < D; ++c) {
+                const float wv = bf16_bits_to_f32(wds[LC ? c * D + tid : 0]);
+#pragma unroll
+                for (int g = 0; g < 8; ++g)
+                    acc[g] = fmaf(wv, qs[g][c], acc[g]);
+            }
+            for (int g = 0; g < a.G; ++g)
+                qo[g * D + tid] = f32_to_bf16_bits(acc[g]);
         }
     }
     for (int i = tid; i < (r1 - r0) * Gp; i += 128)
@@ -820,7 +839,7 @@ __global__ void __launch_bounds__(32 * kConsWarps * NTEAM, 1)
 
 // ==== 3. reference tokens, reference weights, output =========================================
 
-template <int Gp, int RB>
+template <int Gp, int RB, bool LC>
 __global__ void __launch_bounds__(256) mma_refs_kernel(const CacheArgs a, void* __restrict__ out, const MmaWs w)
 {
     constexpr int D = 128;
@@ -953,16 +972,44 @@ __global__ void __launch_bounds__(256) mma_refs_kernel(const CacheArgs a, void* 
     if (!last)
         return;
     __threadfence();
+    if constexpr (LC) {
+        // learned-coder shapes: fd applied once to the softmax-weighted latent sum, o += Wd_V
+        // (sum_i p_i z_i); the latent sums staged in shared memory, one warp per output row c
+        for (int x = tid; x < G * D; x += 256)
+            red[0][x / D][x % D] = __ldcg(&w.Olat[static_cast<int64_t>(u) * Gp * D + x]);
+        __syncthreads();
+        // thread: output row c = tid % D for the heads h = tid / D, tid / D + 2, ... (the row of
+        // Wd_V read once, sixteen 16-byte loads in flight)
+        const int c = tid % D;
+        const uint4* wrow = reinterpret_cast<const uint4*>(a.cw[7] + c * D);
+        for (int h = tid / D; h < G; h += 256 / D) {
+            const float* ol = red[0][h];
+            float acc = 0.0f;
+#pragma unroll
+            for (int i0 = 0; i0 < D / 8; i0 += 8) {
+                uint4 wr[8];                       // eight 16-byte loads in flight
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    wr[i] = wrow[i0 + i];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const uint32_t ww[4] = {wr[i].x, wr[i].y, wr[i].z, wr[i].w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        acc = fmaf(bf16_bits_to_f32(ww[e] & 0xffffu), ol[8 * (i0 + i) + 2 * e], acc);
+                        acc = fmaf(bf16_bits_to_f32(ww[e] >> 16), ol[8 * (i0 + i) + 2 * e + 1], acc);
+                    }
+                }
+            }
+            red[1][h][c] = acc;
+        }
+        __syncthreads();
+    }
     for (int x = tid; x < G * D; x += 256) {
         const int h = x / D, c = x % D;
         float o = __ldcg(&w.O[static_cast<int64_t>(u) * Gp * D + x]);
-        if (a.coder == 1) {
-            // fd applied once to the softmax-weighted latent sum: o += Wd_V (sum_i p_i z_i)
-            const uint16_t* Wd = a.cw[7] + c * D;
-            const float* ol = w.Olat + (static_cast<int64_t>(u) * Gp + h) * D;
-            for (int l = 0; l < D; ++l)
-                o = fmaf(bf16_bits_to_f32(Wd[l]), __ldcg(ol + l), o);
-        }
+        if constexpr (LC)
+            o += red[1][h][c];
         const float l = __ldcg(&w.L[u * Gp + h]);
         const float res = (l > 0.0f) ? o / l : 0.0f;
         const int64_t e = (static_cast<int64_t>(um.seq) * a.Hq + kvh * G + h) * D + c;
@@ -1078,10 +1125,12 @@ cudaError_t launch_gp(const CacheArgs& a, int64_t cmp_rows, const void* q, void*
     if (!code_map(enc, &mK, a.codes_K, cmp_rows) || !code_map(enc, &mV, a.codes_V, cmp_rows))
         return cudaErrorInvalidValue;
     const dim3 rgrid(w.n_chunk, a.n_units);
-    if (a.ref_bits == 4)
-        mma_scores_kernel<Gp, 4><<<rgrid, 128, 0, st>>>(a, q, w);
+    if (a.coder == 1)
+        mma_scores_kernel<Gp, 16, true><<<rgrid, 128, 0, st>>>(a, q, w);
+    else if (a.ref_bits == 4)
+        mma_scores_kernel<Gp, 4, false><<<rgrid, 128, 0, st>>>(a, q, w);
     else
-        mma_scores_kernel<Gp, 16><<<rgrid, 128, 0, st>>>(a, q, w);
+        mma_scores_kernel<Gp, 16, false><<<rgrid, 128, 0, st>>>(a, q, w);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;
@@ -1106,9 +1155,11 @@ cudaError_t launch_gp(const CacheArgs& a, int64_t cmp_rows, const void* q, void*
         if (e != cudaSuccess)
             return e;
     }
+    if (a.coder == 1)
+        return launch_pdl(mma_refs_kernel<Gp, 16, true>, rgrid, dim3(256), 0, st, a, out, w);
     if (a.ref_bits == 4)
-        return launch_pdl(mma_refs_kernel<Gp, 4>, rgrid, dim3(256), 0, st, a, out, w);
-    return launch_pdl(mma_refs_kernel<Gp, 16>, rgrid, dim3(256), 0, st, a, out, w);
+        return launch_pdl(mma_refs_kernel<Gp, 4, false>, rgrid, dim3(256), 0, st, a, out, w);
+    return launch_pdl(mma_refs_kernel<Gp, 16, false>, rgrid, dim3(256), 0, st, a, out, w);
 }
 
 }  // namespace
