@@ -115,7 +115,7 @@ def workload_quantities(wl, lengths):
 class ClockSampler:
     """Samples SM clock, power and clock-event reasons with NVML in a thread."""
 
-    def __init__(self, index: int, period_s: float = 0.02):
+    def __init__(self, index: int, period_s: float = 0.002):
         self.index = index
         self.period = period_s
         self.samples = []
