@@ -17,6 +17,7 @@ import synth
 IDX_TIE_BAND = 1e-4         # relative gap between the k-th and (k+1)-th oracle distance
 CODE_LSB_FRACTION = 1e-3    # codes may differ by one step on at most this fraction of elements
 RECON_ABS = 1e-2            # reconstructed K/V
+LATENT_SCALE_FRACTION = 1e-2  # learned-coder shapes: groups whose scale is one binary16 step off
 ATTN_ABS = 2e-3             # decode output (fp32 output; bf16 output adds half a bf16 ulp)
 
 
@@ -223,14 +224,16 @@ def check_compress(wl, g: dict, Xk, Xv, positions=None, stats=None, coder=None):
     assert ek["overflow"] == 0 and ev["overflow"] == 0
     D = wl.head_dim
     if coder is not None:
-        # the GPU forms the latent z in fp32, the oracle in double: a group's scale may take
-        # the neighbouring binary16 value where a/7 lies within that error of a binary16
-        # boundary (rare); every code still quantises the oracle's z within half a step
+        # the GPU forms the latent z on the tensor cores (bf16 operands split to the 24 bits of
+        # fp32, fp32 accumulation), the oracle in double: with a relative error eps of z a
+        # group's scale takes the neighbouring binary16 value where a/7 lies within eps of a
+        # binary16 boundary, about eps * 2^10 of the groups (measured 0.3 %, eps ~ 3e-6); every
+        # code still quantises the oracle's z within half a step
         for name, e in (("K", ek), ("V", ev)):
             gs = g["scales" + name][slots].view(np.float16).astype(np.float64)
             os_ = e["scales"].view(np.float16).astype(np.float64)
             diff = gs != os_
-            assert diff.mean() <= CODE_LSB_FRACTION, f"{name} latent scales differ in {diff.mean():.2e} of groups"
+            assert diff.mean() <= LATENT_SCALE_FRACTION, f"{name} latent scales differ in {diff.mean():.2e} of groups"
             assert np.all(np.abs(gs - os_) <= os_ * 2.0 ** -9), f"{name} latent scales differ by more than a step"
             gc = _unpack(g["codes" + name][slots], D, wl.bits)
             sc = np.repeat(gs, 32, axis=1)
