@@ -796,169 +796,13 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(CacheArgs a, con
 // linear, z = Wo (h(x) - h(m)).  m is the encoder's mean reference, formed again here from the
 // stored ordinals with the same fp32 steps.  z (fp32) goes through the residuals' quantiser and
 // replaces the identity coder's codes of the token.
-//
-// Persistent CTAs of 256 threads; the side's three matrices are staged once per CTA in shared
-// memory, transposed (row pitch 130 halves, so the transposing stores are conflict-free).
-// Sixteen tokens per pass: thread j computes hidden unit j, then latent channel j, of eight of
-// them; the quantiser then runs 16 lanes per token.
 constexpr int kLatD = 128;
-constexpr int kLatP = kLatD + 2;          // row pitch of the transposed weights (halves)
-constexpr int kLatTok = 16;
-constexpr int kLatThreads = 256;
-
-struct LatentSmem {
-    uint16_t wgT[kLatD * kLatP];          // [c][j] = Wg[j][c]
-    uint16_t wuT[kLatD * kLatP];
-    uint16_t woT[kLatD * kLatP];          // [j][l] = Wo[l][j]
-    float xs[kLatTok][kLatD];
-    float ms[kLatTok][kLatD];
-    float ds[kLatTok][kLatD];             // h(x) - h(m), then z
-};
+constexpr int kLatTok = 16;               // tokens per tile (one warp's MMA rows)
 
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
 
-template <int SIDE>
-__global__ void __launch_bounds__(kLatThreads, 1) encode_latent_kernel(CacheArgs a, const void* __restrict__ X,
-                                                                       int total_tiles)
-{
-    extern __shared__ __align__(16) unsigned char lat_raw[];
-    LatentSmem& S = *reinterpret_cast<LatentSmem*>(lat_raw);
-    const int tid = threadIdx.x;
-    {
-        const uint16_t* Wg = a.cw[4 * SIDE + 0];
-        const uint16_t* Wu = a.cw[4 * SIDE + 1];
-        const uint16_t* Wo = a.cw[4 * SIDE + 2];
-        for (int i = tid; i < kLatD * kLatD; i += kLatThreads) {
-            const int r = i / kLatD, col = i % kLatD;
-            S.wgT[col * kLatP + r] = Wg[i];
-            S.wuT[col * kLatP + r] = Wu[i];
-            S.woT[col * kLatP + r] = Wo[i];
-        }
-    }
-    const uint16_t* Xb = static_cast<const uint16_t*>(X);
-    const uint16_t* refs = SIDE ? a.ref_V : a.ref_K;
-    uint8_t* codes = SIDE ? a.codes_V : a.codes_K;
-    uint16_t* scales = SIDE ? a.scale_V : a.scale_K;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
-        int u = 0, t0 = tile;
-        while (u < a.n_units) {
-            const int nt = (a.units[u].C + kLatTok - 1) / kLatTok;
-            if (t0 < nt)
-                break;
-            t0 -= nt;
-            ++u;
-        }
-        const UnitMeta um = a.units[u];
-        const int c0 = t0 * kLatTok;
-        __syncthreads();   // the weights are staged / the previous pass is done with the buffers
-        {
-            // token t = tid / 16, channels cc .. cc + 7
-            const int t = tid >> 4, cc = (tid & 15) * 8;
-            const int c = c0 + t;
-            float xv[8], mv[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                xv[i] = mv[i] = 0.0f;
-            if (c < um.C) {
-                const int p = slot_pos(a.ph, c);
-                load_bf16_row<8>(Xb + (static_cast<int64_t>(u) * a.max_len + p) * kLatD + cc, xv);
-                const uint16_t* id = a.idx + (um.cmp_row + c) * a.k;
-                int keff = 0;
-                for (int l = 0; l < a.k; ++l) {
-                    const int o = id[l];
-                    if (o == RKV_IDX_UNUSED || o >= um.R)
-                        break;
-                    float rv[8];
-                    load_bf16_row<8>(refs + (um.ref_row + o) * kLatD + cc, rv);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        mv[i] = (keff == 0) ? rv[i] : __fadd_rn(mv[i], rv[i]);
-                    ++keff;
-                }
-                const float fk = static_cast<float>(max(keff, 1));
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    mv[i] = __fdiv_rn(mv[i], fk);
-            }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                S.xs[t][cc + i] = xv[i];
-                S.ms[t][cc + i] = mv[i];
-            }
-        }
-        __syncthreads();
-        const int j = tid & (kLatD - 1), tb = (tid >> 7) * 8;
-        {
-            // hidden unit j of tokens tb .. tb + 7: h(x) - h(m)
-            float gx[8], ux[8], gm[8], uu[8];
-#pragma unroll
-            for (int t = 0; t < 8; ++t)
-                gx[t] = ux[t] = gm[t] = uu[t] = 0.0f;
-            for (int c = 0; c < kLatD; c += 4) {
-                float wg[4], wu[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    wg[i] = bf16_bits_to_f32(S.wgT[(c + i) * kLatP + j]);
-                    wu[i] = bf16_bits_to_f32(S.wuT[(c + i) * kLatP + j]);
-                }
-#pragma unroll
-                for (int t = 0; t < 8; ++t) {
-                    const float4 x4 = *reinterpret_cast<const float4*>(&S.xs[tb + t][c]);
-                    const float4 m4 = *reinterpret_cast<const float4*>(&S.ms[tb + t][c]);
-                    gx[t] = fmaf(wg[3], x4.w, fmaf(wg[2], x4.z, fmaf(wg[1], x4.y, fmaf(wg[0], x4.x, gx[t]))));
-                    ux[t] = fmaf(wu[3], x4.w, fmaf(wu[2], x4.z, fmaf(wu[1], x4.y, fmaf(wu[0], x4.x, ux[t]))));
-                    gm[t] = fmaf(wg[3], m4.w, fmaf(wg[2], m4.z, fmaf(wg[1], m4.y, fmaf(wg[0], m4.x, gm[t]))));
-                    uu[t] = fmaf(wu[3], m4.w, fmaf(wu[2], m4.z, fmaf(wu[1], m4.y, fmaf(wu[0], m4.x, uu[t]))));
-                }
-            }
-#pragma unroll
-            for (int t = 0; t < 8; ++t)
-                S.ds[tb + t][j] = silu_f(gx[t]) * ux[t] - silu_f(gm[t]) * uu[t];
-        }
-        __syncthreads();
-        float z[8];
-        {
-            // latent channel j: z = Wo (h(x) - h(m))
-#pragma unroll
-            for (int t = 0; t < 8; ++t)
-                z[t] = 0.0f;
-            for (int h = 0; h < kLatD; h += 4) {
-                float wo[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    wo[i] = bf16_bits_to_f32(S.woT[(h + i) * kLatP + j]);
-#pragma unroll
-                for (int t = 0; t < 8; ++t) {
-                    const float4 d4 = *reinterpret_cast<const float4*>(&S.ds[tb + t][h]);
-                    z[t] = fmaf(wo[3], d4.w, fmaf(wo[2], d4.z, fmaf(wo[1], d4.y, fmaf(wo[0], d4.x, z[t]))));
-                }
-            }
-        }
-        __syncthreads();
-#pragma unroll
-        for (int t = 0; t < 8; ++t)
-            S.ds[tb + t][j] = z[t];
-        __syncthreads();
-        {
-            // the residuals' quantiser, 16 lanes per token (warp w: tokens 2w, 2w + 1)
-            const int warp = tid >> 5, lane = tid & 31;
-            const int t = 2 * warp + (lane >> 4), sub = lane & 15;
-            const int c = c0 + t;
-            const bool st = c < um.C;
-            float zz[8], zero[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                zz[i] = S.ds[t][sub * 8 + i];
-                zero[i] = 0.0f;
-            }
-            const int64_t row = um.cmp_row + (st ? c : 0);
-            quantise_store<8>(zz, zero, a.bits, sub, st, codes + row * a.code_bytes, scales + row * a.n_groups, a.err);
-        }
-    }
-}
-
 // ---- learned-coder shapes on the tensor cores --------------------------------------------
-// The same latent residual z = Wo (h(x) - h(m)) as encode_latent_kernel, as warp-level bf16
+// The latent residual z = Wo (h(x) - h(m)) as warp-level bf16
 // MMAs (m16n8k16, fp32 accumulators): one warp takes 16 tokens; the CTA stages the side's three
 // matrices once.  x is bf16 (an exact operand).  The mean enters through e = x - m: the
 // products g(m) = g(x) - We and u(m) = u(x) - Wu e take e, small, as a hi + mid + lo bf16
@@ -1268,7 +1112,7 @@ int encode_latent_tiles(int C) { return (C + kLatTok - 1) / kLatTok; }
 
 cudaError_t launch_encode_latent(const CacheArgs& a, const void* K, const void* V, int total, cudaStream_t st)
 {
-    if (a.D != kLatD || a.in_dtype != RKV_DTYPE_BF16)
+    if (a.D != kLatD || a.in_dtype != RKV_DTYPE_BF16 || a.bits != 4)
         return cudaErrorNotSupported;
     if (total == 0)
         return cudaSuccess;
@@ -1278,33 +1122,19 @@ cudaError_t launch_encode_latent(const CacheArgs& a, const void* K, const void* 
         e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess)
         return e;
-    if (a.bits == 4) {
-        // tensor-core form: 16-token tiles per warp (int4 codes, the coder's requirement)
-        const int tiles = total;   // kLatTok == 16: the same 16-token tiles, one per warp
-        const int want = (tiles + kTcWarps - 1) / kTcWarps;
-        const int grid = want < sms ? want : sms;
-        const size_t smem = sizeof(LatentTcSmem);
-        e = cudaFuncSetAttribute(encode_latent_tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(smem));
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(encode_latent_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     static_cast<int>(smem));
-        if (e != cudaSuccess)
-            return e;
-        encode_latent_tc_kernel<0><<<grid, kTcWarps * 32, smem, st>>>(a, K, tiles);
-        encode_latent_tc_kernel<1><<<grid, kTcWarps * 32, smem, st>>>(a, V, tiles);
-        return cudaGetLastError();
-    }
-    const int grid = total < sms ? total : sms;
-    const size_t smem = sizeof(LatentSmem);
-    e = cudaFuncSetAttribute(encode_latent_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    const int tiles = total;   // 16-token tiles, one per warp
+    const int want = (tiles + kTcWarps - 1) / kTcWarps;
+    const int grid = want < sms ? want : sms;
+    const size_t smem = sizeof(LatentTcSmem);
+    e = cudaFuncSetAttribute(encode_latent_tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(encode_latent_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(encode_latent_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(smem));
     if (e != cudaSuccess)
         return e;
-    encode_latent_kernel<0><<<grid, kLatThreads, smem, st>>>(a, K, total);
-    encode_latent_kernel<1><<<grid, kLatThreads, smem, st>>>(a, V, total);
+    encode_latent_tc_kernel<0><<<grid, kTcWarps * 32, smem, st>>>(a, K, tiles);
+    encode_latent_tc_kernel<1><<<grid, kTcWarps * 32, smem, st>>>(a, V, tiles);
     return cudaGetLastError();
 }
 
