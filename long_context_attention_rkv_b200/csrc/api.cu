@@ -29,9 +29,14 @@ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 rkv_status make_phases(const rkv_config& c, int64_t max_len, Phases& ph)
 {
     std::memset(&ph, 0, sizeof(ph));
+    auto magic = [&](int i) {
+        div_magic(ph.stride[i], ph.m_stride[i], ph.sh_stride[i]);
+        div_magic(ph.stride[i] - 1, ph.m_per[i], ph.sh_per[i]);
+    };
     if (c.refs_per_phase <= 0) {
         ph.n = 1;
         ph.stride[0] = c.stride0;
+        magic(0);
         return RKV_OK;
     }
     int64_t start = 0, stride = c.stride0, ord = 0;
@@ -43,6 +48,7 @@ rkv_status make_phases(const rkv_config& c, int64_t max_len, Phases& ph)
         ph.stride[n] = static_cast<int32_t>(stride);
         ph.first_ord[n] = static_cast<int32_t>(ord);
         ph.first_slot[n] = static_cast<int32_t>(start - ord);
+        magic(n);
         ++n;
         start += static_cast<int64_t>(c.refs_per_phase) * stride;
         ord += c.refs_per_phase;

@@ -24,17 +24,24 @@ __device__ __forceinline__ int phase_of_pos(const Phases& ph, int p)
     return q;
 }
 
+// n / d with the multiplier and shift the host prepared (div_magic); 0 <= n < 2^31.
+__device__ __forceinline__ int div_by(int n, uint64_t m, int sh)
+{
+    return static_cast<int>((static_cast<uint64_t>(static_cast<uint32_t>(n)) * m) >> sh);
+}
+
 // Number of references at positions <= p.
 __device__ __forceinline__ int refs_upto(const Phases& ph, int p)
 {
     const int q = phase_of_pos(ph, p);
-    return ph.first_ord[q] + (p - ph.start[q]) / ph.stride[q] + 1;
+    return ph.first_ord[q] + div_by(p - ph.start[q], ph.m_stride[q], ph.sh_stride[q]) + 1;
 }
 
 __device__ __forceinline__ bool is_ref_pos(const Phases& ph, int p)
 {
     const int q = phase_of_pos(ph, p);
-    return (p - ph.start[q]) % ph.stride[q] == 0;
+    const int o = p - ph.start[q];
+    return o - div_by(o, ph.m_stride[q], ph.sh_stride[q]) * ph.stride[q] == 0;
 }
 
 // Position of the reference with ordinal j.
@@ -54,7 +61,8 @@ __device__ __forceinline__ int slot_pos(const Phases& ph, int c)
         q = (c >= ph.first_slot[i]) ? i : q;
     const int local = c - ph.first_slot[q];
     const int per = ph.stride[q] - 1;
-    return ph.start[q] + (local / per) * ph.stride[q] + local % per + 1;
+    const int blk = div_by(local, ph.m_per[q], ph.sh_per[q]);
+    return ph.start[q] + blk * ph.stride[q] + (local - blk * per) + 1;
 }
 
 // ---- conversions ---------------------------------------------------------------------

@@ -26,7 +26,24 @@ struct Phases {
     int32_t stride[kMaxPhases];
     int32_t first_ord[kMaxPhases];   // ordinal of the phase's first reference
     int32_t first_slot[kMaxPhases];  // compressed slot of the phase's first non-reference position
+    // division by stride and by stride - 1 as a multiply and a shift (div_magic below)
+    uint64_t m_stride[kMaxPhases];
+    uint64_t m_per[kMaxPhases];
+    int32_t sh_stride[kMaxPhases];
+    int32_t sh_per[kMaxPhases];
 };
+
+// n / d for 0 <= n < 2^31 and 1 <= d < 2^31 as (n * m) >> sh, with l = ceil(log2 d),
+// sh = 31 + l and m = floor(2^sh / d) + 1 (Granlund and Montgomery, "Division by invariant
+// integers using multiplication", 1994: exact because m * d - 2^sh <= d <= 2^l).
+inline void div_magic(int64_t d, uint64_t& m, int32_t& sh)
+{
+    int l = 0;
+    while ((int64_t(1) << l) < d)
+        ++l;
+    sh = 31 + l;
+    m = (uint64_t(1) << sh) / static_cast<uint64_t>(d) + 1;
+}
 
 // One (sequence, kv-head) unit.  Device table, 32 bytes.
 struct UnitMeta {
