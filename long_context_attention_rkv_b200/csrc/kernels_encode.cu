@@ -229,7 +229,6 @@ __global__ void __launch_bounds__(kWarps * 32, encode_min_blocks<KC, LPT>()) enc
     constexpr int kTPW = 32 / kLPT;          // tokens per warp
     constexpr int KM = KC - 4;               // largest k served by this candidate width
     __shared__ float xs[kWarps][kTPW][D];
-    __shared__ int sorted[kWarps][kTPW][KM];
 
     const int u = blockIdx.y;
     const UnitMeta um = a.units[u];
@@ -434,41 +433,42 @@ __global__ void __launch_bounds__(kWarps * 32, encode_min_blocks<KC, LPT>()) enc
             }
         }
     }
-    // ascending ordinal order of the chosen set (identical in the 8 lanes of a token)
-    if (sub == 0) {
+    // ascending ordinal order of the chosen set, in every lane of the token (odd-even
+    // transposition network; unused slots sort last)
+    int so[KM];
+#pragma unroll
+    for (int i = 0; i < KM; ++i)
+        so[i] = (i < keff) ? chosen[i] : 0x7fffffff;
+#pragma unroll
+    for (int pass = 0; pass < KM; ++pass)
+#pragma unroll
+        for (int i = pass & 1; i + 1 < KM; i += 2) {
+            const int lo = min(so[i], so[i + 1]), hi = max(so[i], so[i + 1]);
+            so[i] = lo;
+            so[i + 1] = hi;
+        }
+    if (active && sub == 0) {
 #pragma unroll
         for (int i = 0; i < KM; ++i)
-            if (i < keff) {
-                int pos = 0;
-#pragma unroll
-                for (int j2 = 0; j2 < KM; ++j2)
-                    pos += (j2 < keff && chosen[j2] < chosen[i]) ? 1 : 0;
-                sorted[warp][tg][pos] = chosen[i];
-            }
-    }
-    __syncwarp();
-    if (active && sub == 0) {
-        for (int i = 0; i < k; ++i)
-            a.idx[row * k + i] = (i < keff) ? static_cast<uint16_t>(sorted[warp][tg][i])
-                                            : static_cast<uint16_t>(RKV_IDX_UNUSED);
+            if (i < k)
+                a.idx[row * k + i] = (i < keff) ? static_cast<uint16_t>(so[i]) : static_cast<uint16_t>(RKV_IDX_UNUSED);
     }
 
     // ---- 2. mean reference (fp32, ascending ordinals, one division) -------------------
     float mk[CPL], mv[CPL];
-    {
-        const int o = sorted[warp][tg][0];
-        load_ref<CPL, RB>(a, 0, um.ref_row + o, sub * CPL, mk);
-        load_ref<CPL, RB>(a, 1, um.ref_row + o, sub * CPL, mv);
-    }
-    for (int i = 1; i < keff; ++i) {
-        const int o = sorted[warp][tg][i];
-        float rk[CPL], rv[CPL];
-        load_ref<CPL, RB>(a, 0, um.ref_row + o, sub * CPL, rk);
-        load_ref<CPL, RB>(a, 1, um.ref_row + o, sub * CPL, rv);
+    load_ref<CPL, RB>(a, 0, um.ref_row + so[0], sub * CPL, mk);
+    load_ref<CPL, RB>(a, 1, um.ref_row + so[0], sub * CPL, mv);
 #pragma unroll
-        for (int j2 = 0; j2 < CPL; j2 += 2) {
-            add2_rn(mk[j2], mk[j2 + 1], rk[j2], rk[j2 + 1]);
-            add2_rn(mv[j2], mv[j2 + 1], rv[j2], rv[j2 + 1]);
+    for (int i = 1; i < KM; ++i) {
+        if (i < keff) {
+            float rk[CPL], rv[CPL];
+            load_ref<CPL, RB>(a, 0, um.ref_row + so[i], sub * CPL, rk);
+            load_ref<CPL, RB>(a, 1, um.ref_row + so[i], sub * CPL, rv);
+#pragma unroll
+            for (int j2 = 0; j2 < CPL; j2 += 2) {
+                add2_rn(mk[j2], mk[j2 + 1], rk[j2], rk[j2 + 1]);
+                add2_rn(mv[j2], mv[j2 + 1], rv[j2], rv[j2 + 1]);
+            }
         }
     }
     if (keff & (keff - 1)) {
