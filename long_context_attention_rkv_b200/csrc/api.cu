@@ -199,6 +199,7 @@ rkv_status compute_layout(const rkv_config* c, const int32_t* lengths, Desc& d)
     s.scale_V = take(2ull * cmp_rows * d.n_groups);
     s.idx = take(2ull * cmp_rows * c->k);
     s.append = take(append_scratch_bytes(d.n_units));   // per-unit candidate lists of rkv_append
+    s.hn_max = take(4ull * d.n_units);
     s.end = off;
     d.ws_select = align_up(2ull * cmp_rows * d.kc, 256) + align_up(4ull * cmp_rows * d.kc, 256);
     if (r4)
@@ -252,6 +253,7 @@ CacheArgs make_args(const Desc& d)
     a.ref_sK = (a.ref_bits == 4) ? reinterpret_cast<uint16_t*>(base + d.sec.ref_sK) : nullptr;
     a.ref_sV = (a.ref_bits == 4) ? reinterpret_cast<uint16_t*>(base + d.sec.ref_sV) : nullptr;
     a.ref_hn = reinterpret_cast<float*>(base + d.sec.ref_hn);
+    a.ref_hn_max = reinterpret_cast<float*>(base + d.sec.hn_max);
     a.ref_aug = reinterpret_cast<uint16_t*>(base + d.sec.ref_aug);
     a.ref_pos = reinterpret_cast<int32_t*>(base + d.sec.ref_pos);
     a.codes_K = reinterpret_cast<uint8_t*>(base + d.sec.codes_K);
@@ -463,7 +465,12 @@ rkv_status rkv_build_refs(const rkv_cache_desc* desc, const void* K, const void*
     if (!d || !K || !V || !aligned(K, 16) || !aligned(V, 16))
         return RKV_ERR_INVALID_ARG;
     const CacheArgs a = make_args(*d);
-    return cuda_status(launch_refs_copy(a, d->max_R, K, V, static_cast<cudaStream_t>(stream)));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // the units' largest reference half norms are maxima over this call's rows
+    const cudaError_t e = cudaMemsetAsync(a.ref_hn_max, 0, 4ull * d->n_units, st);
+    if (e != cudaSuccess)
+        return RKV_ERR_CUDA;
+    return cuda_status(launch_refs_copy(a, d->max_R, K, V, st));
 }
 
 static rkv_status check_stage_args(const Desc* d, const void* K, const void* V, const void* workspace,

@@ -12,7 +12,8 @@
 //     delta = 2^-16 (|k|^2 + max|r|^2) (four times the worst-case error of a
 //     128-term fp32 dot product, 2^-18 (|k|^2 + |r|^2), and about 25 times the
 //     largest tensor-core vs. CUDA-core difference measured on these inputs): if the (k+1)-th t is more than 2*delta below the k-th, the
-//     first k candidates are the top-k.  Otherwise every candidate within 2*delta
+//     first k candidates are the top-k (max |r|^2 over all the unit's references, so the
+//     bound covers the references outside the list as well).  Otherwise every candidate within 2*delta
 //     of the k-th is re-ranked by its exact-order fp32 distance sum_c (k_c - r_c)^2
 //     (ties to the lower ordinal); if even the last kept candidate is that close,
 //     the list may be incomplete and all candidates are rescanned exactly.
@@ -296,12 +297,7 @@ __global__ void __launch_bounds__(kWarps * 32, encode_min_blocks<KC, LPT>()) enc
     for (int i = 0; i < CPL; ++i)
         xx = fmaf(xk[i], xk[i], xx);
     xx = tsum<kLPT>(xx);
-    float hm = 0.0f;
-#pragma unroll
-    for (int r = 0; r < PER; ++r)
-        if (r * kLPT + sub < nvalid)
-            hm = fmaxf(hm, a.ref_hn[um.ref_row + co[r]]);
-    hm = tmax<kLPT>(hm);
+    const float hm = a.ref_hn_max[u];     // the unit's largest reference half norm
     const float delta = ldexpf(xx + 2.0f * hm, -16);
     const float tk = slot_t(k - 1);
     const float tk1 = slot_t(k);
@@ -687,6 +683,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(CacheArgs a, con
                 const float hn = 0.5f * ss;
                 a.ref_hn[um.ref_row + j] = hn;
                 a.ref_pos[um.ref_row + j] = p;
+                atomicMax(reinterpret_cast<int*>(a.ref_hn_max + u), __float_as_int(hn));
                 const uint16_t hi = f32_to_bf16_bits(hn);
                 const float r1 = hn - bf16_bits_to_f32(hi);
                 const uint16_t mid = f32_to_bf16_bits(r1);

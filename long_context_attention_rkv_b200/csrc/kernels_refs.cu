@@ -14,17 +14,12 @@
 
 namespace rkv {
 
+// Stores reference row j of unit u (this warp; lane owns D/32 channels) and returns its half
+// norm (the same value in every lane).
 template <int NPL, int RB>
-__global__ void __launch_bounds__(256) refs_copy_kernel(CacheArgs a, const void* __restrict__ K,
-                                                        const void* __restrict__ V)
+__device__ __forceinline__ float copy_ref_row(const CacheArgs& a, const UnitMeta& um, int u, int j, int lane,
+                                              const void* __restrict__ K, const void* __restrict__ V)
 {
-    const int u = blockIdx.y;
-    const UnitMeta um = a.units[u];
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const int j = blockIdx.x * (blockDim.x >> 5) + warp;
-    if (j >= um.R)
-        return;
     const int p = ref_pos_of(a.ph, j);
     const int64_t e = (static_cast<int64_t>(u) * a.max_len + p) * a.D + lane * NPL;
     float kx[NPL], vx[NPL];
@@ -61,8 +56,8 @@ __global__ void __launch_bounds__(256) refs_copy_kernel(CacheArgs a, const void*
         }
     }
     ss = warp_sum(ss);
+    const float hn = 0.5f * ss;
     if (lane == 0) {
-        const float hn = 0.5f * ss;
         a.ref_hn[um.ref_row + j] = hn;
         a.ref_pos[um.ref_row + j] = p;
         // -hn split into three bf16 terms (hi + mid + lo = hn to ~2^-24 relative): a 16-wide
@@ -74,6 +69,33 @@ __global__ void __launch_bounds__(256) refs_copy_kernel(CacheArgs a, const void*
         uint4* aug = reinterpret_cast<uint4*>(a.ref_aug + (um.ref_row + j) * 16);
         aug[0] = make_uint4((hi ^ 0x8000u) | ((mid ^ 0x8000u) << 16), lo ^ 0x8000u, 0u, 0u);
         aug[1] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    return hn;
+}
+
+template <int NPL, int RB>
+__global__ void __launch_bounds__(256) refs_copy_kernel(CacheArgs a, const void* __restrict__ K,
+                                                        const void* __restrict__ V)
+{
+    const int u = blockIdx.y;
+    const UnitMeta um = a.units[u];
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int j = blockIdx.x * (blockDim.x >> 5) + warp;
+    __shared__ int hmax[8];   // the warps' half norms (non-negative floats order as ints)
+    hmax[warp] = 0;
+    if (j < um.R) {
+        const float hn = copy_ref_row<NPL, RB>(a, um, u, j, lane, K, V);
+        if (lane == 0)
+            hmax[warp] = __float_as_int(hn);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int m = 0;
+        for (int i = 0; i < 8; ++i)
+            m = max(m, hmax[i]);
+        if (m > 0)
+            atomicMax(reinterpret_cast<int*>(a.ref_hn_max + u), m);
     }
 }
 

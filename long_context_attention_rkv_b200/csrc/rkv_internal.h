@@ -58,7 +58,7 @@ struct UnitMeta {
 // Byte offsets of the cache sections inside the caller's buffer.
 struct Sections {
     uint64_t err, units, tiles, pairs, ref_K, ref_V, ref_sK, ref_sV, ref_hn, ref_aug, ref_pos, codes_K, codes_V,
-        scale_K, scale_V, idx, append, end;
+        scale_K, scale_V, idx, append, hn_max, end;
 };
 
 // Host-side descriptor stored in rkv_cache_desc::opaque.
@@ -108,6 +108,7 @@ struct CacheArgs {
     uint16_t* ref_sK;    // ref_bits 4: binary16 scales [rows][D/32]
     uint16_t* ref_sV;
     float* ref_hn;
+    float* ref_hn_max;   // [units] largest half norm of the unit's references (bits compared as int)
     uint16_t* ref_aug;   // [rows][16] bf16: -hi, -mid, -lo of 0.5|r|^2, then zeros (augmented GEMM column)
     int32_t* ref_pos;
     uint8_t* codes_K;
