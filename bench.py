@@ -382,25 +382,51 @@ def run_ours(args, rank, world, local_rank):
     mean_step = max_over_ranks(statistics.mean(step_ms), world, dev)
     assert L.device_error() == 0
 
-    # end to end through the public API: host inputs copied in, output copied out, every step
-    e2e_ms = []
+    # end to end through the public API: every step copies its inputs in from pinned host memory
+    # and its output back out.  Two input buffers let step i+1's copies (copy stream) run while
+    # step i computes (compute stream); the time is the span of all steps over their number.
     h2d = Kp.numel() * Kp.element_size() + Vp.numel() * Vp.element_size() + qp.numel() * qp.element_size()
     d2h = out.numel() * out.element_size()
-    with torch.cuda.stream(stream):
-        for i in range(max(3, min(args.steps, 50)) + 2):
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            K.copy_(Kp, non_blocking=True)
-            V.copy_(Vp, non_blocking=True)
-            q.copy_(qp, non_blocking=True)
-            for nm in names:
-                stages[nm]()
-            out_h.copy_(out, non_blocking=True)
-            e1.record(stream)
-            e1.synchronize()
-            if i >= 2:
-                e2e_ms.append(e0.elapsed_time(e1))
+    bufs = [(K, V, q), (torch.empty_like(K), torch.empty_like(V), torch.empty_like(q))]
+    cstream = torch.cuda.Stream(device=dev)
+
+    def e2e_step(Kb, Vb, qb):
+        L.build_refs(Kb, Vb)
+        L.search(Kb)
+        L.encode(Kb, Vb)
+        L.decode(qb, out)
+        L.reconstruct(0, 0, rpos, RECON_ROWS, Kr, Vr, rkv.RKV_DTYPE_F32)
+        out_h.copy_(out, non_blocking=True)
+
+    e2e_ms = []
+    n_e2e = max(3, min(args.steps, 50))
+    for rep in range(2):                                  # the first pass warms up
+        copied = [torch.cuda.Event() for _ in range(2)]
+        done = [torch.cuda.Event() for _ in range(2)]
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        cstream.wait_stream(stream)
+        for i in range(n_e2e):
+            b = i % 2
+            Kb, Vb, qb = bufs[b]
+            with torch.cuda.stream(cstream):
+                if i >= 2:
+                    cstream.wait_event(done[b])              # step i-2 is done with this buffer
+                Kb.copy_(Kp, non_blocking=True)
+                Vb.copy_(Vp, non_blocking=True)
+                qb.copy_(qp, non_blocking=True)
+                copied[b].record(cstream)
+            with torch.cuda.stream(stream):
+                stream.wait_event(copied[b])
+                e2e_step(Kb, Vb, qb)
+                done[b].record(stream)
+        e1.record(stream)
+        e1.synchronize()
+        if rep == 1:
+            e2e_ms.append(e0.elapsed_time(e1) / n_e2e)
+    assert L.device_error() == 0
     e2e_step = max_over_ranks(statistics.mean(e2e_ms), world, dev)
 
     # selective decode (outside the step): SPARSE_SEL seeded uniform positions per unit
