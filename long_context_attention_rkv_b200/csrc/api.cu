@@ -204,6 +204,8 @@ rkv_status compute_layout(const rkv_config* c, const int32_t* lengths, Desc& d)
     d.ws_select = align_up(2ull * cmp_rows * d.kc, 256) + align_up(4ull * cmp_rows * d.kc, 256);
     if (r4)
         d.ws_select += align_up(2ull * ref_rows * D, 256);   // the stored keys as bf16 rows (search operand)
+    d.ws_fix_off = d.ws_select;                                // the encoder's deferred-token list
+    d.ws_select += align_up(8ull + 8ull * cmp_rows, 256);
     const int splits = std::max(decode_splits(d.n_units, max_n), sparse_splits_max(d.n_units));
     d.ws_decode = align_up(4ull * d.n_units * splits * G * (D + 2), 256);
     const CacheArgs a = make_args(d);
@@ -538,7 +540,9 @@ rkv_status rkv_encode(const rkv_cache_desc* desc, const void* K, const void* V, 
         return RKV_ERR_INVALID_ARG;
     const CacheArgs a = make_args(*d);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t e = launch_encode(a, d->max_C, K, V, cand_idx_of(d, workspace), cand_t_of(d, workspace), st);
+    int* fix = reinterpret_cast<int*>(static_cast<char*>(workspace) + d->ws_fix_off);
+    cudaError_t e = launch_encode(a, d->max_C, K, V, cand_idx_of(d, workspace), cand_t_of(d, workspace), fix,
+                                  static_cast<int>(d->total_cmp_rows), st);
     if (e == cudaSuccess && a.coder == 1) {
         // the latent residuals replace the codes
         int total = 0;

@@ -219,26 +219,27 @@ __device__ __forceinline__ void quantise_store(const float (&x)[CPL], const floa
 template <int KC, int LPT>
 constexpr int encode_min_blocks() { return (LPT == 16 && KC <= 12) ? 4 : 2; }
 
-template <int CPL, int KC, int LPT, int RB>
-__global__ void __launch_bounds__(kWarps * 32, encode_min_blocks<KC, LPT>()) encode_kernel(CacheArgs a, const void* __restrict__ K,
-                                                             const void* __restrict__ V,
-                                                             const uint16_t* __restrict__ cand_idx,
-                                                             const float* __restrict__ cand_t)
+// One compressed token per group of LPT lanes: final top-k, mean, residual and quantiser.
+// (u, c): the token's unit and compressed slot; inactive groups shadow a valid token and store
+// nothing.  FIX false: tokens whose candidate list does not settle the top-k at once (mode 1
+// or 2 below, about 2 % of them) are not stored but listed in fix (fix[0] = count, then
+// (unit, slot) pairs), so the main pass stays straight-line; FIX true: the exact re-rank and
+// rescan of the listed tokens.
+template <int CPL, int KC, int LPT, int RB, bool FIX>
+__device__ __forceinline__ void encode_group(const CacheArgs& a, const void* __restrict__ K, const void* __restrict__ V,
+                                             const uint16_t* __restrict__ cand_idx, const float* __restrict__ cand_t,
+                                             int* __restrict__ fix, int u, int c, bool active)
 {
     constexpr int D = CPL * LPT;
     constexpr int kLPT = LPT;                // lanes per token
     constexpr int kTPW = 32 / kLPT;          // tokens per warp
     constexpr int KM = KC - 4;               // largest k served by this candidate width
     __shared__ float xs[kWarps][kTPW][D];
-
-    const int u = blockIdx.y;
-    const UnitMeta um = a.units[u];
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int tg = lane / kLPT;              // token slot within the warp
     const int sub = lane % kLPT;             // lane within the token group
-    const int c = (blockIdx.x * kWarps + warp) * kTPW + tg;
-    const bool active = c < um.C;
+    const UnitMeta um = a.units[u];
     if (__all_sync(0xffffffffu, !active))
         return;
     const int k = a.k;
@@ -304,7 +305,17 @@ __global__ void __launch_bounds__(kWarps * 32, encode_min_blocks<KC, LPT>()) enc
     const float tlast = slot_t(KC - 1);
     if (nvalid > k && tk1 >= tk - 2.0f * delta)
         mode = ((nvalid == KC) && (ncand > KC) && (tlast >= tk - 2.0f * delta)) ? 2 : 1;
-    const int any_mode = __reduce_max_sync(0xffffffffu, mode);
+    bool store = active;
+    if constexpr (!FIX) {
+        // defer the token to the exact pass: listed once (by its group's first lane)
+        if (active && mode != 0 && sub == 0) {
+            const int slot = atomicAdd(fix, 1);
+            reinterpret_cast<int2*>(fix + 2)[slot] = make_int2(u, c);
+        }
+        store = active && mode == 0;
+        mode = 0;
+    }
+    const int any_mode = FIX ? __reduce_max_sync(0xffffffffu, mode) : 0;
     if (any_mode == 0) {
 #pragma unroll
         for (int i = 0; i < KM; ++i)
@@ -443,7 +454,7 @@ __global__ void __launch_bounds__(kWarps * 32, encode_min_blocks<KC, LPT>()) enc
             so[i] = lo;
             so[i + 1] = hi;
         }
-    if (active && sub == 0) {
+    if (store && sub == 0) {
 #pragma unroll
         for (int i = 0; i < KM; ++i)
             if (i < k)
@@ -487,10 +498,36 @@ __global__ void __launch_bounds__(kWarps * 32, encode_min_blocks<KC, LPT>()) enc
     // ---- 3. residual and group quantiser ---------------------------------------------
     float xv[CPL];
     load_input_row<CPL>(V, e, a.in_dtype, xv);
-    quantise_store<CPL>(xk, mk, a.bits, sub, active, a.codes_K + row * a.code_bytes, a.scale_K + row * a.n_groups,
+    quantise_store<CPL>(xk, mk, a.bits, sub, store, a.codes_K + row * a.code_bytes, a.scale_K + row * a.n_groups,
                         a.err);
-    quantise_store<CPL>(xv, mv, a.bits, sub, active, a.codes_V + row * a.code_bytes, a.scale_V + row * a.n_groups,
+    quantise_store<CPL>(xv, mv, a.bits, sub, store, a.codes_V + row * a.code_bytes, a.scale_V + row * a.n_groups,
                         a.err);
+}
+
+template <int CPL, int KC, int LPT, int RB, bool FIX>
+__global__ void __launch_bounds__(kWarps * 32, encode_min_blocks<KC, LPT>()) encode_kernel(CacheArgs a, const void* __restrict__ K,
+                                                             const void* __restrict__ V,
+                                                             const uint16_t* __restrict__ cand_idx,
+                                                             const float* __restrict__ cand_t,
+                                                             int* __restrict__ fix)
+{
+    constexpr int kTPW = 32 / LPT;
+    const int warp = threadIdx.x >> 5;
+    const int tg = (threadIdx.x & 31) / LPT;
+    if constexpr (FIX) {
+        // the listed tokens, strided over a grid sized for the device
+        const int n_fix = *reinterpret_cast<volatile int*>(fix);
+        for (int base = blockIdx.x * kWarps * kTPW; base < n_fix; base += gridDim.x * kWarps * kTPW) {
+            const int t = base + warp * kTPW + tg;
+            const bool active = t < n_fix;
+            const int2 uc = active ? reinterpret_cast<const int2*>(fix + 2)[t] : make_int2(0, 0);
+            encode_group<CPL, KC, LPT, RB, true>(a, K, V, cand_idx, cand_t, fix, uc.x, uc.y, active);
+        }
+    } else {
+        const int u = blockIdx.y;
+        const int c = (blockIdx.x * kWarps + warp) * kTPW + tg;
+        encode_group<CPL, KC, LPT, RB, false>(a, K, V, cand_idx, cand_t, fix, u, c, c < a.units[u].C);
+    }
 }
 
 // ---- incremental compression: one new token per unit ----------------------------------
@@ -1081,24 +1118,35 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) encode_latent_tc_kernel(Cach
     }
 }
 
+template <int CPL, int KC, int LPT, int RB>
+void launch_pair(const CacheArgs& a, dim3 grid, const void* K, const void* V, const uint16_t* ci, const float* ct,
+                 int* fix, int fix_grid, cudaStream_t st)
+{
+    encode_kernel<CPL, KC, LPT, RB, false><<<grid, kWarps * 32, 0, st>>>(a, K, V, ci, ct, fix);
+    encode_kernel<CPL, KC, LPT, RB, true><<<fix_grid, kWarps * 32, 0, st>>>(a, K, V, ci, ct, fix);
+}
+
 template <int CPL, int LPT>
 cudaError_t launch_cpl(const CacheArgs& a, int max_C, const void* K, const void* V, const uint16_t* ci,
-                       const float* ct, cudaStream_t st)
+                       const float* ct, int* fix, int fix_cap, int sms, cudaStream_t st)
 {
     const int per_block = kWarps * (32 / LPT);
     const dim3 grid((max_C + per_block - 1) / per_block, a.n_units);
+    // the deferred pass: a few blocks per SM stride over the list (a few percent of the tokens)
+    const int fix_need = (fix_cap + per_block - 1) / per_block;
+    const int fix_grid = fix_need < 4 * sms ? (fix_need > 0 ? fix_need : 1) : 4 * sms;
     if (a.ref_bits == 4) {
         switch (a.kc) {
-        case 8: encode_kernel<CPL, 8, LPT, 4><<<grid, kWarps * 32, 0, st>>>(a, K, V, ci, ct); break;
-        case 12: encode_kernel<CPL, 12, LPT, 4><<<grid, kWarps * 32, 0, st>>>(a, K, V, ci, ct); break;
-        default: encode_kernel<CPL, 20, LPT, 4><<<grid, kWarps * 32, 0, st>>>(a, K, V, ci, ct); break;
+        case 8: launch_pair<CPL, 8, LPT, 4>(a, grid, K, V, ci, ct, fix, fix_grid, st); break;
+        case 12: launch_pair<CPL, 12, LPT, 4>(a, grid, K, V, ci, ct, fix, fix_grid, st); break;
+        default: launch_pair<CPL, 20, LPT, 4>(a, grid, K, V, ci, ct, fix, fix_grid, st); break;
         }
         return cudaGetLastError();
     }
     switch (a.kc) {
-    case 8: encode_kernel<CPL, 8, LPT, 16><<<grid, kWarps * 32, 0, st>>>(a, K, V, ci, ct); break;
-    case 12: encode_kernel<CPL, 12, LPT, 16><<<grid, kWarps * 32, 0, st>>>(a, K, V, ci, ct); break;
-    default: encode_kernel<CPL, 20, LPT, 16><<<grid, kWarps * 32, 0, st>>>(a, K, V, ci, ct); break;
+    case 8: launch_pair<CPL, 8, LPT, 16>(a, grid, K, V, ci, ct, fix, fix_grid, st); break;
+    case 12: launch_pair<CPL, 12, LPT, 16>(a, grid, K, V, ci, ct, fix, fix_grid, st); break;
+    default: launch_pair<CPL, 20, LPT, 16>(a, grid, K, V, ci, ct, fix, fix_grid, st); break;
     }
     return cudaGetLastError();
 }
@@ -1162,12 +1210,21 @@ cudaError_t launch_append(const CacheArgs& a, const void* K_new, const void* V_n
 }
 
 cudaError_t launch_encode(const CacheArgs& a, int max_C, const void* K, const void* V, const uint16_t* cand_idx,
-                          const float* cand_t, cudaStream_t st)
+                          const float* cand_t, int* fix, int fix_cap, cudaStream_t st)
 {
     if (max_C <= 0)
         return cudaSuccess;
-    return (a.D == 128) ? launch_cpl<kCpl128, 128 / kCpl128>(a, max_C, K, V, cand_idx, cand_t, st)
-                        : launch_cpl<8, 8>(a, max_C, K, V, cand_idx, cand_t, st);
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess)
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess)
+        return e;
+    e = cudaMemsetAsync(fix, 0, sizeof(int), st);
+    if (e != cudaSuccess)
+        return e;
+    return (a.D == 128) ? launch_cpl<kCpl128, 128 / kCpl128>(a, max_C, K, V, cand_idx, cand_t, fix, fix_cap, sms, st)
+                        : launch_cpl<8, 8>(a, max_C, K, V, cand_idx, cand_t, fix, fix_cap, sms, st);
 }
 
 }  // namespace rkv

@@ -18,8 +18,11 @@ bool select_tc_supported(const CacheArgs& a);
 cudaError_t launch_select_tc(const CacheArgs& a, const Tile* items, int n_items, const void* K, const uint16_t* refB,
                              int64_t in_rows, int64_t ref_rows, uint16_t* cand_idx, float* cand_t, cudaStream_t st);
 
+// Final top-k, mean and quantiser of every compressed token.  fix: device scratch of
+// 2 + 2 * fix_cap ints (fix_cap >= the compressed tokens of the layer) for the tokens the main
+// pass defers to the exact pass.
 cudaError_t launch_encode(const CacheArgs& a, int max_C, const void* K, const void* V, const uint16_t* cand_idx,
-                          const float* cand_t, cudaStream_t st);
+                          const float* cand_t, int* fix, int fix_cap, cudaStream_t st);
 
 // Incremental compression: one new token ([unit][D] rows) for every unit of the sequences whose
 // bit is set in active (256 bits).
