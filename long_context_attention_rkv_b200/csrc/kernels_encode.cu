@@ -166,23 +166,28 @@ __device__ __forceinline__ void quantise_store(const float (&x)[CPL], const floa
         yv[i + 1] = d[i + 1];
         mul2_rn(yv[i], yv[i + 1], rs, rs);
     }
+    // Round half to even by adding 1.5 * 2^23 (for |y| < 2^22 the sum's last bits are rint(y)):
+    // three adds on the FMA pipe instead of a rounding and a conversion on the slower one.
+    // |y| <= qmax (the scale is rounded up), so no code needs clamping.
+    constexpr float kRound = 12582912.0f;
+    constexpr int kRoundBits = 0x4B400000;
     bool near_half = false;
+    int q[CPL];
 #pragma unroll
     for (int i = 0; i < CPL; ++i) {
-        y[i] = rintf(yv[i]);
+        const float t = __fadd_rn(yv[i], kRound);
+        q[i] = __float_as_int(t) - kRoundBits;
+        y[i] = __fsub_rn(t, kRound);
         near_half |= fabsf(__fsub_rn(yv[i], y[i])) >= 0.5f - 0x1p-14f;
     }
     if (near_half) {
 #pragma unroll
         for (int i = 0; i < CPL; ++i)
-            y[i] = rintf(__fdiv_rn(d[i], s));
+            q[i] = __float_as_int(__fadd_rn(__fdiv_rn(d[i], s), kRound)) - kRoundBits;
     }
-    int q[CPL];
 #pragma unroll
-    for (int i = 0; i < CPL; ++i) {
-        const int c = static_cast<int>(y[i]);
-        q[i] = (amax > 0.0f) ? max(-qmax, min(qmax, c)) : 0;
-    }
+    for (int i = 0; i < CPL; ++i)
+        q[i] = (amax > 0.0f) ? q[i] : 0;
     if (!store)
         return;
     if (bits == 8) {
