@@ -828,301 +828,6 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(CacheArgs a, con
     }
 }
 
-// ---- learned-coder shapes: latent residuals ------------------------------------------------
-// (ResidualKV paper summary page, "DeltaKV Framework Architecture": the residual is taken after
-// the compressor, z = fc(KV) - fc(KV_R); "Improvements for AI systems": fc a SwiGLU block.)
-// fc(v) = Wo h(v) with h(v) = silu(Wg v) * (Wu v), all weights bf16 [128][128]; since Wo is
-// linear, z = Wo (h(x) - h(m)).  m is the encoder's mean reference, formed again here from the
-// stored ordinals with the same fp32 steps.  z (fp32) goes through the residuals' quantiser and
-// replaces the identity coder's codes of the token.
-constexpr int kLatD = 128;
-constexpr int kLatTok = 16;               // tokens per tile (one warp's MMA rows)
-
-__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
-
-// ---- learned-coder shapes on the tensor cores --------------------------------------------
-// The latent residual z = Wo (h(x) - h(m)) as warp-level bf16
-// MMAs (m16n8k16, fp32 accumulators): one warp takes 16 tokens; the CTA stages the side's three
-// matrices once.  x is bf16 (an exact operand).  The mean enters through e = x - m: the
-// products g(m) = g(x) - We and u(m) = u(x) - Wu e take e, small, as a hi + mid + lo bf16
-// triple (the 24 bits of an fp32 value), so the tensor cores' accumulation error in g(x)
-// reaches both h(x) and h(m) alike and cancels in their difference (forming g(m) from m
-// directly moved about 0.3 % of the groups' binary16 scales).  The hidden difference d enters
-// the second product as a triple too.  The
-// hidden layer runs in four chunks of 32 units; a chunk's accumulators are, in the m16n8 C
-// layout of two adjacent 8-column tiles, exactly the A operand of the next product, so d never
-// leaves the registers.
-constexpr int kTcPitch = kLatD + 8;          // smem row pitch (halves): conflict-free ldmatrix
-constexpr int kTcWarps = 6;
-
-struct LatentTcSmem {
-    uint16_t wg[kLatD * kTcPitch];           // [unit][channel]  (the B operand's n x k layout)
-    uint16_t wu[kLatD * kTcPitch];
-    uint16_t wo[kLatD * kTcPitch];           // [latent][unit]
-    uint16_t xt[kTcWarps][16 * kTcPitch];    // per warp: 16 token rows of x (bf16)
-    uint16_t mh[kTcWarps][16 * kTcPitch];    // e = x - mean, hi part
-    uint16_t mm[kTcWarps][16 * kTcPitch];    // e, mid part
-    uint16_t ml[kTcWarps][16 * kTcPitch];    // e, lo part
-};
-
-__device__ __forceinline__ void tc_ldsm_x4(const uint16_t* p, uint32_t (&r)[4])
-{
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))));
-}
-
-__device__ __forceinline__ void tc_ldsm_x2(const uint16_t* p, uint32_t (&r)[2])
-{
-    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
-                 : "=r"(r[0]), "=r"(r[1])
-                 : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))));
-}
-
-__device__ __forceinline__ void tc_mma(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2])
-{
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-        "{%0, %1, %2, %3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-}
-
-// A pair of fp32 values as three bf16 pairs (low half = first): hi = bf16(x), mid =
-// bf16(x - hi), lo = bf16(x - hi - mid); hi + mid + lo == x for normal fp32 values.
-__device__ __forceinline__ void tc_split3(float x0, float x1, uint32_t& hi, uint32_t& mid, uint32_t& lo)
-{
-    const uint32_t h0 = f32_to_bf16_bits(x0), h1 = f32_to_bf16_bits(x1);
-    const float r0 = x0 - bf16_bits_to_f32(h0), r1 = x1 - bf16_bits_to_f32(h1);
-    const uint32_t m0 = f32_to_bf16_bits(r0), m1 = f32_to_bf16_bits(r1);
-    hi = h0 | (h1 << 16);
-    mid = m0 | (m1 << 16);
-    lo = f32_to_bf16_bits(r0 - bf16_bits_to_f32(m0)) | (uint32_t(f32_to_bf16_bits(r1 - bf16_bits_to_f32(m1))) << 16);
-}
-
-template <int SIDE>
-__global__ void __launch_bounds__(kTcWarps * 32, 1) encode_latent_tc_kernel(CacheArgs a, const void* __restrict__ X,
-                                                                            int total_tiles)
-{
-    extern __shared__ __align__(16) unsigned char lat_tc_raw[];
-    LatentTcSmem& S = *reinterpret_cast<LatentTcSmem*>(lat_tc_raw);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int gid = lane >> 2, tq = lane & 3;
-    {
-        const uint4* Wg = reinterpret_cast<const uint4*>(a.cw[4 * SIDE + 0]);
-        const uint4* Wu = reinterpret_cast<const uint4*>(a.cw[4 * SIDE + 1]);
-        const uint4* Wo = reinterpret_cast<const uint4*>(a.cw[4 * SIDE + 2]);
-        for (int i = tid; i < kLatD * kLatD / 8; i += kTcWarps * 32) {
-            const int r = i / (kLatD / 8), c8 = (i % (kLatD / 8)) * 8;
-            *reinterpret_cast<uint4*>(&S.wg[r * kTcPitch + c8]) = Wg[i];
-            *reinterpret_cast<uint4*>(&S.wu[r * kTcPitch + c8]) = Wu[i];
-            *reinterpret_cast<uint4*>(&S.wo[r * kTcPitch + c8]) = Wo[i];
-        }
-    }
-    __syncthreads();
-    const uint16_t* Xb = static_cast<const uint16_t*>(X);
-    const uint16_t* refs = SIDE ? a.ref_V : a.ref_K;
-    uint8_t* codes = SIDE ? a.codes_V : a.codes_K;
-    uint16_t* scales = SIDE ? a.scale_V : a.scale_K;
-    uint16_t* xt = S.xt[warp];
-    uint16_t* mh = S.mh[warp];
-    uint16_t* mm = S.mm[warp];
-    uint16_t* ml = S.ml[warp];
-    for (int tile = blockIdx.x * kTcWarps + warp; tile < total_tiles; tile += gridDim.x * kTcWarps) {
-        int u = 0, t0 = tile;
-        while (u < a.n_units) {
-            const int nt = (a.units[u].C + 15) / 16;
-            if (t0 < nt)
-                break;
-            t0 -= nt;
-            ++u;
-        }
-        const UnitMeta um = a.units[u];
-        const int c0 = t0 * 16;
-        // ---- stage x and e = x - mean of the 16 tokens: four passes of four tokens, eight
-        //      lanes per token (16 channels each); a token's ordinals and reference rows are
-        //      all requested before any is used
-#pragma unroll 1
-        for (int pass = 0; pass < 4; ++pass) {
-            const int t = pass * 4 + (lane >> 3), cb = (lane & 7) * 16;
-            const int c = c0 + t;
-            uint4 xw[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
-            float m[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-                m[i] = 0.0f;
-            if (c < um.C) {
-                const int p = slot_pos(a.ph, c);
-                const uint4* xs = reinterpret_cast<const uint4*>(Xb + (static_cast<int64_t>(u) * a.max_len + p) * kLatD + cb);
-                xw[0] = xs[0];
-                xw[1] = xs[1];
-                const uint16_t* id = a.idx + (um.cmp_row + c) * a.k;
-                int o[8];
-#pragma unroll
-                for (int l = 0; l < 8; ++l)
-                    o[l] = (l < a.k) ? static_cast<int>(id[l]) : RKV_IDX_UNUSED;
-                int keff = 0;
-#pragma unroll
-                for (int l = 0; l < 8; ++l)
-                    keff += (keff == l && o[l] != RKV_IDX_UNUSED && o[l] < um.R) ? 1 : 0;
-                uint4 rw[8][2];
-#pragma unroll
-                for (int l = 0; l < 8; ++l) {
-                    if (l < keff) {
-                        const uint4* rs = reinterpret_cast<const uint4*>(refs + (um.ref_row + o[l]) * kLatD + cb);
-                        rw[l][0] = rs[0];
-                        rw[l][1] = rs[1];
-                    }
-                }
-#pragma unroll
-                for (int l = 0; l < 8; ++l) {
-                    if (l < keff) {
-#pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            const uint32_t ww[4] = {rw[l][h].x, rw[l][h].y, rw[l][h].z, rw[l][h].w};
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                const float r0 = bf16_bits_to_f32(ww[i] & 0xffffu), r1 = bf16_bits_to_f32(ww[i] >> 16);
-                                m[8 * h + 2 * i] = (l == 0) ? r0 : __fadd_rn(m[8 * h + 2 * i], r0);
-                                m[8 * h + 2 * i + 1] = (l == 0) ? r1 : __fadd_rn(m[8 * h + 2 * i + 1], r1);
-                            }
-                        }
-                    }
-                }
-                const float fk = static_cast<float>(max(keff, 1));
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    m[i] = __fdiv_rn(m[i], fk);
-            }
-            uint32_t eh[8], em[8], el[8];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const uint32_t ww[4] = {xw[h].x, xw[h].y, xw[h].z, xw[h].w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float x0 = bf16_bits_to_f32(ww[i] & 0xffffu), x1 = bf16_bits_to_f32(ww[i] >> 16);
-                    tc_split3(__fsub_rn(x0, m[8 * h + 2 * i]), __fsub_rn(x1, m[8 * h + 2 * i + 1]), eh[4 * h + i],
-                              em[4 * h + i], el[4 * h + i]);
-                }
-            }
-            uint16_t* rowx = &xt[t * kTcPitch + cb];
-            *reinterpret_cast<uint4*>(rowx) = xw[0];
-            *reinterpret_cast<uint4*>(rowx + 8) = xw[1];
-            *reinterpret_cast<uint4*>(&mh[t * kTcPitch + cb]) = make_uint4(eh[0], eh[1], eh[2], eh[3]);
-            *reinterpret_cast<uint4*>(&mh[t * kTcPitch + cb + 8]) = make_uint4(eh[4], eh[5], eh[6], eh[7]);
-            *reinterpret_cast<uint4*>(&mm[t * kTcPitch + cb]) = make_uint4(em[0], em[1], em[2], em[3]);
-            *reinterpret_cast<uint4*>(&mm[t * kTcPitch + cb + 8]) = make_uint4(em[4], em[5], em[6], em[7]);
-            *reinterpret_cast<uint4*>(&ml[t * kTcPitch + cb]) = make_uint4(el[0], el[1], el[2], el[3]);
-            *reinterpret_cast<uint4*>(&ml[t * kTcPitch + cb + 8]) = make_uint4(el[4], el[5], el[6], el[7]);
-        }
-        __syncwarp();
-        float z[16][4];
-#pragma unroll
-        for (int n = 0; n < 16; ++n)
-            z[n][0] = z[n][1] = z[n][2] = z[n][3] = 0.0f;
-        const int arow = lane & 15, acol = (lane >> 4) * 8;        // ldmatrix x4 (A) addresses
-        const int brow = lane & 7, bcol = ((lane >> 3) & 1) * 8;   // ldmatrix x2 (B) addresses
-#pragma unroll 1
-        for (int chunk = 0; chunk < 4; ++chunk) {
-            float gx[4][4], ux[4][4], gm[4][4], uu[4][4];   // gm, uu: W e first, then g(m), u(m)
-#pragma unroll
-            for (int n = 0; n < 4; ++n)
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    gx[n][e] = ux[n][e] = gm[n][e] = uu[n][e] = 0.0f;
-#pragma unroll 2
-            for (int ks = 0; ks < kLatD / 16; ++ks) {
-                uint32_t ax[4], ah[4], am[4], al[4];
-                tc_ldsm_x4(&xt[arow * kTcPitch + ks * 16 + acol], ax);
-                tc_ldsm_x4(&mh[arow * kTcPitch + ks * 16 + acol], ah);
-                tc_ldsm_x4(&mm[arow * kTcPitch + ks * 16 + acol], am);
-                tc_ldsm_x4(&ml[arow * kTcPitch + ks * 16 + acol], al);
-#pragma unroll
-                for (int n = 0; n < 4; ++n) {
-                    const int unit = chunk * 32 + n * 8 + brow;
-                    uint32_t bg[2], bu[2];
-                    tc_ldsm_x2(&S.wg[unit * kTcPitch + ks * 16 + bcol], bg);
-                    tc_ldsm_x2(&S.wu[unit * kTcPitch + ks * 16 + bcol], bu);
-                    tc_mma(gx[n], ax, bg);
-                    tc_mma(ux[n], ax, bu);
-                    tc_mma(gm[n], ah, bg);
-                    tc_mma(gm[n], am, bg);
-                    tc_mma(gm[n], al, bg);
-                    tc_mma(uu[n], ah, bu);
-                    tc_mma(uu[n], am, bu);
-                    tc_mma(uu[n], al, bu);
-                }
-            }
-            // d = h(x) - h(m) of this chunk's 32 units, straight into A fragments (hi, mid, lo)
-#pragma unroll
-            for (int kb = 0; kb < 2; ++kb) {
-                float d[2][4];
-#pragma unroll
-                for (int h = 0; h < 2; ++h)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int n = 2 * kb + h;
-                        const float g_m = gx[n][e] - gm[n][e], u_m = ux[n][e] - uu[n][e];
-                        d[h][e] = silu_f(gx[n][e]) * ux[n][e] - silu_f(g_m) * u_m;
-                    }
-                uint32_t dh[4], dm[4], dl[4];
-                tc_split3(d[0][0], d[0][1], dh[0], dm[0], dl[0]);   // rows gid,     units 2tq .. (first tile)
-                tc_split3(d[0][2], d[0][3], dh[1], dm[1], dl[1]);   // rows gid + 8
-                tc_split3(d[1][0], d[1][1], dh[2], dm[2], dl[2]);   // rows gid,     second tile (k + 8)
-                tc_split3(d[1][2], d[1][3], dh[3], dm[3], dl[3]);   // rows gid + 8
-#pragma unroll
-                for (int n = 0; n < 16; ++n) {
-                    uint32_t bo[2];
-                    tc_ldsm_x2(&S.wo[(n * 8 + brow) * kTcPitch + chunk * 32 + kb * 16 + bcol], bo);
-                    tc_mma(z[n], dh, bo);
-                    tc_mma(z[n], dm, bo);
-                    tc_mma(z[n], dl, bo);
-                }
-            }
-        }
-        // ---- the residuals' quantiser on z (C layout: rows gid, gid + 8; channels
-        //      8n + 2tq, 8n + 2tq + 1); a group is four tiles of the quad's four lanes
-        const int qmax = (a.bits == 8) ? 127 : 7;
-#pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-            const int c = c0 + gid + 8 * hr;
-            const bool st = c < um.C;
-            const int64_t row = um.cmp_row + (st ? c : 0);
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-                float amax = 0.0f;
-#pragma unroll
-                for (int n = 4 * g; n < 4 * g + 4; ++n)
-                    amax = fmaxf(amax, fmaxf(fabsf(z[n][2 * hr]), fabsf(z[n][2 * hr + 1])));
-                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-                uint16_t sbits = 0;
-                float sc = 1.0f;
-                if (amax > 0.0f) {
-                    const __half hv = __float2half_ru(__fdiv_rn(amax, static_cast<float>(qmax)));
-                    sbits = __half_as_ushort(hv);
-                    sc = __half2float(hv);
-                    if (st && (sbits & 0x7c00u) == 0x7c00u)
-                        report(a.err, RKV_ERR_UNSUPPORTED);
-                }
-#pragma unroll
-                for (int n = 4 * g; n < 4 * g + 4; ++n) {
-                    int q0 = 0, q1 = 0;
-                    if (amax > 0.0f) {
-                        q0 = max(-qmax, min(qmax, static_cast<int>(rintf(__fdiv_rn(z[n][2 * hr], sc)))));
-                        q1 = max(-qmax, min(qmax, static_cast<int>(rintf(__fdiv_rn(z[n][2 * hr + 1], sc)))));
-                    }
-                    if (st)
-                        codes[row * a.code_bytes + n * 4 + tq] = static_cast<uint8_t>((q0 & 0xf) | ((q1 & 0xf) << 4));
-                }
-                if (st && tq == 0)
-                    scales[row * a.n_groups + g] = sbits;
-            }
-        }
-        __syncwarp();   // the tile buffers are rewritten by the next tile
-    }
-}
-
 template <int CPL, int KC, int LPT, int RB>
 void launch_pair(const CacheArgs& a, dim3 grid, const void* K, const void* V, const uint16_t* ci, const float* ct,
                  int* fix, int fix_grid, cudaStream_t st)
@@ -1157,36 +862,6 @@ cudaError_t launch_cpl(const CacheArgs& a, int max_C, const void* K, const void*
 }
 
 }  // namespace
-
-int encode_latent_tiles(int C) { return (C + kLatTok - 1) / kLatTok; }
-
-cudaError_t launch_encode_latent(const CacheArgs& a, const void* K, const void* V, int total, cudaStream_t st)
-{
-    if (a.D != kLatD || a.in_dtype != RKV_DTYPE_BF16 || a.bits != 4)
-        return cudaErrorNotSupported;
-    if (total == 0)
-        return cudaSuccess;
-    int dev = 0, sms = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e == cudaSuccess)
-        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess)
-        return e;
-    const int tiles = total;   // 16-token tiles, one per warp
-    const int want = (tiles + kTcWarps - 1) / kTcWarps;
-    const int grid = want < sms ? want : sms;
-    const size_t smem = sizeof(LatentTcSmem);
-    e = cudaFuncSetAttribute(encode_latent_tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(encode_latent_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(smem));
-    if (e != cudaSuccess)
-        return e;
-    encode_latent_tc_kernel<0><<<grid, kTcWarps * 32, smem, st>>>(a, K, tiles);
-    encode_latent_tc_kernel<1><<<grid, kTcWarps * 32, smem, st>>>(a, V, tiles);
-    return cudaGetLastError();
-}
 
 uint64_t append_scratch_bytes(int n_units)
 {

@@ -29,10 +29,10 @@ cudaError_t launch_encode(const CacheArgs& a, int max_C, const void* K, const vo
 // Scratch that rkv_append needs inside the cache buffer (per-unit candidate lists).
 uint64_t append_scratch_bytes(int n_units);
 // Learned-coder shapes: latent residual codes z = fc(x) - fc(mean) of every compressed token
-// (after launch_encode has chosen the references), both sides.  total = the sum over units of
-// encode_latent_tiles(compressed tokens of the unit).
+// (after launch_encode has chosen the references), both sides, on the tcgen05 tensor cores in
+// 128-token tiles: total_tiles = the sum over units of encode_latent_tiles(compressed tokens).
 int encode_latent_tiles(int C);
-cudaError_t launch_encode_latent(const CacheArgs& a, const void* K, const void* V, int total, cudaStream_t st);
+cudaError_t launch_encode_latent(const CacheArgs& a, const void* K, const void* V, int total_tiles, cudaStream_t st);
 cudaError_t launch_append(const CacheArgs& a, const void* K_new, const void* V_new, const uint32_t (&active)[8],
                           void* scratch, cudaStream_t st);
 
