@@ -436,48 +436,35 @@ __global__ void __launch_bounds__(32 * kConsWarps * NTEAM, 1)
         fence_mbar_init();
         prefetch_tensormap(&tmK);
         prefetch_tensormap(&tmV);
-        // the ring fills while the scores kernel may still run: codes do not depend on it
-        const int n0 = n_local < nst ? n_local : nst;
-        for (int j = 0; j < n0; ++j)
-            issue(j);
-        *issued = n0;
+        *issued = n_local < nst ? n_local : nst;
     }
     __syncthreads();
+    // the ring fills while the scores kernel may still run (codes do not depend on it): lane j
+    // of warp 0 loads local tile j, so the first stages' copies are issued together
+    if (warp == 0 && lane < min(n_local, nst))
+        issue(lane);
 
     // ---- consumer warps -----------------------------------------------------------------
     const int team = warp / kConsWarps, wi = warp % kConsWarps;
     const int gid = lane >> 2, tq = lane & 3;
     const int G = a.G;
-    grid_dep_wait();   // reference scores, maxima and zeroed accumulators of the scores kernel
-    // The references kernel may be scheduled once every CTA has passed this wait: the scores
-    // kernel has then completed, so the references kernel may read its outputs (through L2)
-    // before waiting for this one.
-    grid_dep_launch();
 
-    // unit of the first tile: the last unit whose rows start at or before it
-    int u = 0;
-    {
-        int lo = 0, hi = a.n_units - 1;
-        const int64_t row = static_cast<int64_t>(t_lo) * kTok;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (a.units[mid].cmp_row <= row)
-                lo = mid;
-            else
-                hi = mid - 1;
-        }
-        u = lo;
-    }
     // segments: the runs of this CTA's tiles that belong to one unit.  Their score tables
     // are bulk-copied into two alternating buffers, the next one while the current is used.
     auto unit_end = [&](int uu) {
         const UnitMeta m = a.units[uu];
         return static_cast<int>((m.cmp_row + ((m.C + kTok - 1) / kTok) * kTok) / kTok);
     };
-    auto unit_at = [&](int uu, int T) {   // first unit from uu whose tiles reach past tile T
-        while (uu < a.n_units && T >= unit_end(uu))
-            ++uu;
-        return uu;
+    // The first unit from u0 on whose tiles reach past tile T (the units' rows are laid out in
+    // order, so their end tiles do not decrease); warp-wide, 32 units per round trip.
+    auto unit_after = [&](int u0, int T) {
+        for (int base = u0; base < a.n_units; base += 32) {
+            const bool past = base + lane < a.n_units && T < unit_end(base + lane);
+            const unsigned bal = __ballot_sync(0xffffffffu, past);
+            if (bal)
+                return base + __ffs(bal) - 1;
+        }
+        return a.n_units;
     };
     int tables_issued[2] = {0, 0};             // (thread 0)
     auto load_table = [&](int buf, int uu) {   // one thread
@@ -488,12 +475,23 @@ __global__ void __launch_bounds__(32 * kConsWarps * NTEAM, 1)
         if (bytes)
             bulk_load(s_buf + buf * s_stride, w.s_tab + m.ref_row * Gp, bytes, &tbar[buf]);
     };
-    u = unit_at(u, t_lo);
-    if (!GT && tid == 0 && t_lo < t_hi) {
-        load_table(0, u);
+    // the units of the first two segments: the unit layout does not depend on the scores kernel
+    int u = unit_after(0, t_lo);
+    int u_second = a.n_units;
+    if (t_lo < t_hi && u < a.n_units) {
         const int t1 = min(t_hi, unit_end(u));
         if (t1 < t_hi)
-            load_table(1, unit_at(u, t1));
+            u_second = unit_after(u, t1);
+    }
+    grid_dep_wait();   // reference scores, maxima and zeroed accumulators of the scores kernel
+    // The references kernel may be scheduled once every CTA has passed this wait: the scores
+    // kernel has then completed, so the references kernel may read its outputs (through L2)
+    // before waiting for this one.
+    grid_dep_launch();
+    if (!GT && tid == 0 && t_lo < t_hi) {
+        load_table(0, u);
+        if (u_second < a.n_units)
+            load_table(1, u_second);
     }
     bool overflow = false, corrupt = false;
     int t = t_lo, i = 0, seg = 0;
@@ -797,12 +795,15 @@ __global__ void __launch_bounds__(32 * kConsWarps * NTEAM, 1)
         }
         consumer_sync(NCT);
         // the table buffer of this segment is free: the segment after next loads into it
-        if (!GT && tid == 0 && seg_end < t_hi) {
-            const int u1 = unit_at(u, seg_end);
+        if (!GT && warp == 0 && seg_end < t_hi) {
+            const int u1 = unit_after(u, seg_end);
             const int t2 = min(t_hi, unit_end(u1));
-            if (t2 < t_hi && !*abort_flag) {
-                fence_proxy_async_smem();
-                load_table(seg & 1, unit_at(u1, t2));
+            if (t2 < t_hi) {
+                const int u2 = unit_after(u1, t2);
+                if (lane == 0 && !*abort_flag) {
+                    fence_proxy_async_smem();
+                    load_table(seg & 1, u2);
+                }
             }
         }
         if (!*abort_flag) {
@@ -817,7 +818,7 @@ __global__ void __launch_bounds__(32 * kConsWarps * NTEAM, 1)
                 atomicAdd(&w.L[u * Gp + tid], l_sm[tid]);
         }
         t = seg_end;
-        u = unit_at(u, t);
+        u = unit_after(u, t);
         ++seg;
     }
     if (__any_sync(0xffffffffu, overflow) && lane == 0)
