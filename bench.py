@@ -113,15 +113,12 @@ def workload_quantities(wl, lengths):
 
 
 class ClockSampler:
-    """Samples SM clock, power and clock-event reasons with NVML in a thread, and adds the
-    driver's own SM-clock samples of the same window (a short timed region may see only a
-    few of the thread's)."""
+    """Samples SM clock, power and clock-event reasons with NVML in a thread."""
 
     def __init__(self, index: int, period_s: float = 0.002):
         self.index = index
         self.period = period_s
         self.samples = []
-        self.driver_mhz = []
         self._stop = threading.Event()
         self._t = None
         self.ok = False
@@ -137,7 +134,6 @@ class ClockSampler:
             self.ok = True
         except Exception:
             return self
-        self.t0_us = int(time.time() * 1e6)
         self._t = threading.Thread(target=self._run, daemon=True)
         self._t.start()
         return self
@@ -153,21 +149,12 @@ class ClockSampler:
                 pass
             time.sleep(self.period)
 
-    def _driver_samples(self):
-        nv = self._nv
-        try:
-            _, smp = nv.nvmlDeviceGetSamples(self._h, nv.NVML_PROCESSOR_CLK_SAMPLES, self.t0_us)
-            return [int(x.sampleValue.uiVal) for x in smp if x.timeStamp >= self.t0_us]
-        except Exception:
-            return []
-
     def stop(self):
         self._stop.set()
         if self._t:
             self._t.join()
         if not self.ok:
             return None
-        self.driver_mhz = self._driver_samples()
         names = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
                  0x80: "hw_power_brake_slowdown"}
         seen = set()
@@ -175,9 +162,9 @@ class ClockSampler:
             for bit, nm in names.items():
                 if r & bit:
                     seen.add(nm)
-        mhz = [m for m, _ in self.samples] + self.driver_mhz
+        mhz = [m for m, _ in self.samples]
         return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(seen), "samples": len(self.samples), "driver_samples": len(self.driver_mhz)}
+                "reasons": sorted(seen), "samples": len(mhz)}
 
 
 def _src_sha(paths):
