@@ -427,6 +427,30 @@ def test_learned_coder_shapes_every_stage(case):
     check_decode(run, synth.gen_query(wl, 0, 0))
 
 
+def test_learned_coder_ragged_batch():
+    """Learned-coder shapes over a ragged batch: one sequence spanning many 128-token tiles, one
+    a tile and a ragged tail, one shorter than a tile, and an empty one (units without tiles
+    between units with tiles); every compressed token checked."""
+    wl = _small("llama3_8b_layer", n_kv_heads=2, n_q_heads=8, batch=4, seq_len=2100)
+    lengths = [2100, 150, 17, 0]
+    K, V = synth.gen_layer(wl, 0, lengths, max_len=2103)
+    coder = _random_coders(wl.head_dim, 13)
+    run = GpuRun(wl, K, V, lengths, coder=coder)
+    stats = {}
+    for b, n in enumerate(lengths):
+        if n == 0:
+            continue
+        for h in range(wl.n_kv_heads):
+            g = run.unit(b, h)
+            Xk, Xv = unit_rows(wl, K, V, b, h, n)
+            check_refs(wl, g, Xk, Xv)
+            check_compress(wl, g, Xk, Xv, stats=stats, coder=coder)
+            check_reconstruct(run, g, b, h)
+    n_cmp = sum(n - len(oracle.schedule(n, wl.stride0, wl.refs_per_phase)) for n in lengths if n)
+    assert stats["tokens"] == wl.n_kv_heads * n_cmp
+    check_decode(run, synth.gen_query(wl, 0, 0))
+
+
 def test_learned_coder_refuses_what_it_does_not_cover():
     wl = _small("llama3_8b_layer", n_kv_heads=1, n_q_heads=4, seq_len=600)
     lengths = [600]
