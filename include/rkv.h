@@ -388,6 +388,18 @@ RKV_API rkv_status rkv_compress_noalloc(const rkv_cache_desc* desc, const void* 
  */
 RKV_API rkv_status rkv_read_device_error(const rkv_cache_desc* desc, void* stream, int32_t* device_status);
 
+/*
+ * Self-test of the kernels' bounded waits (every wait on an mbarrier, a flag or a peer gives up
+ * after 2 s of the GPU's global timer and records RKV_ERR_TIMEOUT instead of hanging).  Queues
+ * one small kernel on `stream` whose thread waits, with that same bounded wait, on an mbarrier
+ * phase that nothing completes; when the wait gives up the kernel writes RKV_ERR_TIMEOUT to
+ * *err_dev (a caller-owned device int32, 4-byte aligned) and returns.  The call returns RKV_OK
+ * once the kernel is queued; the caller synchronises the stream and reads *err_dev.  The kernel
+ * takes about 2 s, and the context stays usable afterwards.  RKV_ERR_INVALID_ARG for a null or
+ * unaligned err_dev.
+ */
+RKV_API rkv_status rkv_selftest_wait_timeout(int32_t* err_dev, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -31,7 +31,7 @@ STATUS_CODE = {v: k for k, v in STATUS.items()}
 EXPORTED = ["rkv_abi_version", "rkv_status_string", "rkv_schedule", "rkv_cache_size", "rkv_cache_bind",
             "rkv_unit_view_get", "rkv_build_refs", "rkv_search", "rkv_encode", "rkv_compress", "rkv_decode_attn", "rkv_reconstruct",
             "rkv_read_device_error", "rkv_compress_noalloc", "rkv_decode_attn_sparse", "rkv_cache_set_lengths",
-            "rkv_append", "rkv_set_coder"]
+            "rkv_append", "rkv_set_coder", "rkv_selftest_wait_timeout"]
 
 
 class RkvError(RuntimeError):
@@ -85,6 +85,7 @@ def lib() -> ctypes.CDLL:
         L.rkv_cache_set_lengths.argtypes = [vp, vp, vp]
         L.rkv_append.argtypes = [vp, vp, vp, vp, vp]
         L.rkv_set_coder.argtypes = [vp, vp]
+        L.rkv_selftest_wait_timeout.argtypes = [vp, vp]
         for name in EXPORTED[2:]:
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -238,6 +239,12 @@ def rkv_read_device_error(desc: CacheDesc, stream=None) -> int:
     v = ctypes.c_int32(0)
     _check(lib().rkv_read_device_error(desc.ptr, _stream(stream), ctypes.byref(v)), "rkv_read_device_error")
     return v.value
+
+
+def rkv_selftest_wait_timeout(err_dev, stream=None):
+    """Queues the bounded-wait self-test; after a stream synchronisation err_dev (a device int32
+    tensor) holds RKV_ERR_TIMEOUT (about 2 s later)."""
+    _check(lib().rkv_selftest_wait_timeout(_ptr(err_dev), _stream(stream)), "rkv_selftest_wait_timeout")
 
 
 # --- buffers ---------------------------------------------------------------------------

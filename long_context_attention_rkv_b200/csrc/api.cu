@@ -721,6 +721,13 @@ rkv_status rkv_reconstruct(const rkv_cache_desc* desc, int32_t seq, int32_t kv_h
                                           out_dtype, static_cast<cudaStream_t>(stream)));
 }
 
+rkv_status rkv_selftest_wait_timeout(int32_t* err_dev, void* stream)
+{
+    if (!err_dev || !aligned(err_dev, 4))
+        return RKV_ERR_INVALID_ARG;
+    return cuda_status(launch_wait_timeout_selftest(err_dev, static_cast<cudaStream_t>(stream)));
+}
+
 rkv_status rkv_read_device_error(const rkv_cache_desc* desc, void* stream, int32_t* device_status)
 {
     const Desc* d = get_desc(desc);

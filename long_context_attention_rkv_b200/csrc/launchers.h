@@ -62,4 +62,7 @@ cudaError_t launch_decode_mma(const CacheArgs& a, int64_t ref_rows, int64_t cmp_
 cudaError_t launch_decode_combine(const CacheArgs& a, int batch, int splits, const float* partials, void* out,
                                   cudaStream_t st);
 
+// Self-test of the bounded waits: records RKV_ERR_TIMEOUT in *err after one wait gives up.
+cudaError_t launch_wait_timeout_selftest(int32_t* err, cudaStream_t st);
+
 }  // namespace rkv

@@ -108,6 +108,11 @@ def test_calls_reject_unbound_handles():
         assert fn(*args) == rkv.STATUS_CODE["RKV_ERR_INVALID_ARG"]
 
 
+def test_wait_selftest_rejects_bad_status_pointers():
+    for ptr in (None, 2):                                     # null, and not 4-byte aligned
+        assert rkv.lib().rkv_selftest_wait_timeout(ptr, None) == rkv.STATUS_CODE["RKV_ERR_INVALID_ARG"]
+
+
 def test_bind_without_usable_device_fails_cleanly():
     import torch
 
