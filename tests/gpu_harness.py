@@ -37,7 +37,7 @@ def config(wl: synth.Workload, lengths, max_len=None, out_dtype=rkv.RKV_DTYPE_F3
                            flags=flags, ref_bits=ref_bits, coder=coder)
 
 
-class GpuRun:
+class DeviceRun:
     """One layer compressed on the GPU through the C ABI."""
 
     def __init__(self, wl: synth.Workload, K: np.ndarray, V: np.ndarray, lengths, out_dtype=rkv.RKV_DTYPE_F32,
@@ -266,7 +266,7 @@ def oracle_decode_on_gpu_cache(wl, g: dict, q_group: np.ndarray, coder=None):
     return oracle.attention(q_group.astype(np.float64), Kh, Vh)
 
 
-def check_decode(run: GpuRun, q: np.ndarray, units=None, threads=8):
+def check_decode(run: DeviceRun, q: np.ndarray, units=None, threads=8):
     """Decode output of every (or the listed) unit against the oracle on the GPU's cache."""
     wl = run.wl
     out = run.decode(q)
@@ -294,7 +294,7 @@ def check_decode(run: GpuRun, q: np.ndarray, units=None, threads=8):
     return worst
 
 
-def check_reconstruct(run: GpuRun, g: dict, b: int, h: int, positions=None):
+def check_reconstruct(run: DeviceRun, g: dict, b: int, h: int, positions=None):
     wl = run.wl
     n = g["n"]
     Kh, Vh = oracle.unit_cache_rows(n, g["pos"], g["refK"], g["refV"], g["idx"], g["codesK"], g["scalesK"],

@@ -7,7 +7,7 @@ import torch
 
 import long_context_attention_rkv_b200 as rkv
 import synth
-from gpu_harness import GpuRun, check_compress, check_decode, check_refs, unit_rows
+from gpu_harness import DeviceRun, check_compress, check_decode, check_refs, unit_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -25,7 +25,7 @@ def test_bounded_wait_gives_up_with_timeout_status_and_context_stays_usable():
     wl = synth.WORKLOADS["tiny"]
     lengths = wl.lengths()
     K, V = synth.gen_layer(wl, 0, lengths)
-    run = GpuRun(wl, K, V, lengths)
+    run = DeviceRun(wl, K, V, lengths)
     for b, n in enumerate(lengths):
         for h in range(wl.n_kv_heads):
             g = run.unit(b, h)

@@ -12,7 +12,7 @@ import torch
 import long_context_attention_rkv_b200 as rkv
 import oracle
 import synth
-from gpu_harness import (GpuRun, check_compress, check_decode, check_reconstruct, check_refs, config, sample_positions,
+from gpu_harness import (DeviceRun, check_compress, check_decode, check_reconstruct, check_refs, config, sample_positions,
                          to_dev, unit_rows)
 
 pytestmark = pytest.mark.gpu
@@ -40,7 +40,7 @@ def test_tiny_workload_every_stage():
     wl = synth.WORKLOADS["tiny"]
     lengths = wl.lengths()
     K, V = synth.gen_layer(wl, 0, lengths)
-    run = GpuRun(wl, K, V, lengths)
+    run = DeviceRun(wl, K, V, lengths)
     stats = _full_unit_checks(run, wl, K, V, lengths)
     assert stats["tokens"] == 1920
     check_decode(run, synth.gen_query(wl, 0, 0))
@@ -51,7 +51,7 @@ def test_bf16_ragged_batch_every_stage(bits):
     wl = _small("llama3_8b_layer", n_kv_heads=2, n_q_heads=8, bits=bits, batch=4, seq_len=5000)
     lengths = [5000, 777, 1, 0]
     K, V = synth.gen_layer(wl, 0, lengths, max_len=5003)
-    run = GpuRun(wl, K, V, lengths)
+    run = DeviceRun(wl, K, V, lengths)
     _full_unit_checks(run, wl, K, V, lengths)
     check_decode(run, synth.gen_query(wl, 0, 0))
 
@@ -61,7 +61,7 @@ def test_dynamic_stride_every_stage():
                 bits=8, seq_len=6000, n_proto=64)
     lengths = [6000]
     K, V = synth.gen_layer(wl, 0, lengths)
-    run = GpuRun(wl, K, V, lengths)
+    run = DeviceRun(wl, K, V, lengths)
     stats = _full_unit_checks(run, wl, K, V, lengths)
     assert stats["tokens"] == 6000 - len(oracle.schedule(6000, 4, 64))
     check_decode(run, synth.gen_query(wl, 0, 0))
@@ -71,7 +71,7 @@ def test_k8_stride32_group7_every_stage():
     wl = _small("qwen2_5_7b_batch", n_kv_heads=2, n_q_heads=14, batch=2, seq_len=3000, ragged=None)
     lengths = [3000, 2500]
     K, V = synth.gen_layer(wl, 0, lengths)
-    run = GpuRun(wl, K, V, lengths)
+    run = DeviceRun(wl, K, V, lengths)
     _full_unit_checks(run, wl, K, V, lengths)
     check_decode(run, synth.gen_query(wl, 0, 0))
 
@@ -80,8 +80,8 @@ def test_simt_search_matches_default_search():
     wl = _small("llama3_8b_layer", n_kv_heads=2, n_q_heads=8, seq_len=4100)
     lengths = [4100]
     K, V = synth.gen_layer(wl, 0, lengths)
-    a = GpuRun(wl, K, V, lengths)
-    b = GpuRun(wl, K, V, lengths, flags=rkv.RKV_FLAG_SELECT_SIMT)
+    a = DeviceRun(wl, K, V, lengths)
+    b = DeviceRun(wl, K, V, lengths, flags=rkv.RKV_FLAG_SELECT_SIMT)
     for h in range(2):
         ga, gb = a.unit(0, h), b.unit(0, h)
         Xk, Xv = unit_rows(wl, K, V, 0, h, 4100)
@@ -99,9 +99,9 @@ def test_decode_sharp_query_and_bf16_output():
     for h in range(2):
         q[0, h * 4:(h + 1) * 4] = synth.sharp_query(wl, Kf[0, h], 1234 + 77 * h, 4)
     qb = oracle.bf16_round(q)                                  # the query is a bf16 input
-    run = GpuRun(wl, K, V, lengths)
+    run = DeviceRun(wl, K, V, lengths)
     check_decode(run, qb)
-    run16 = GpuRun(wl, K, V, lengths, out_dtype=rkv.RKV_DTYPE_BF16)
+    run16 = DeviceRun(wl, K, V, lengths, out_dtype=rkv.RKV_DTYPE_BF16)
     check_decode(run16, qb)
 
 
@@ -109,7 +109,7 @@ def test_reconstruct_position_list():
     wl = _small("llama3_8b_layer", n_kv_heads=1, n_q_heads=4, seq_len=2500)
     lengths = [2500]
     K, V = synth.gen_layer(wl, 0, lengths)
-    run = GpuRun(wl, K, V, lengths)
+    run = DeviceRun(wl, K, V, lengths)
     g = run.unit(0, 0)
     pos = np.array([0, 1, 15, 16, 17, 2499, 1024, 3, 3], dtype=np.int32)
     check_reconstruct(run, g, 0, 0, pos)
@@ -119,7 +119,7 @@ def test_corrupted_cache_is_reported_not_faulted():
     wl = _small("llama3_8b_layer", n_kv_heads=1, n_q_heads=4, seq_len=1000)
     lengths = [1000]
     K, V = synth.gen_layer(wl, 0, lengths)
-    run = GpuRun(wl, K, V, lengths)
+    run = DeviceRun(wl, K, V, lengths)
     v = run.layer.unit(0, 0)
     off = v.idx - run.layer.cache.data_ptr()
     saved = run.layer.cache[off:off + 2].clone()
@@ -147,7 +147,7 @@ def _named(name, layers, steps, n_uniform=2048):
     worst = 0.0
     for layer in layers:
         K, V = synth.gen_layer(wl, layer, lengths)
-        run = GpuRun(wl, K, V, lengths, out_dtype=rkv.RKV_DTYPE_BF16)
+        run = DeviceRun(wl, K, V, lengths, out_dtype=rkv.RKV_DTYPE_BF16)
         stats = {}
         for b, n in enumerate(lengths):
             for h in range(wl.n_kv_heads):
@@ -182,7 +182,7 @@ def test_direct_decode_flag_matches_oracle():
     wl = _small("qwen2_5_7b_batch", n_kv_heads=2, n_q_heads=14, batch=2, seq_len=2100, ragged=None)
     lengths = [2100, 900]
     K, V = synth.gen_layer(wl, 0, lengths)
-    run = GpuRun(wl, K, V, lengths, flags=rkv.RKV_FLAG_DECODE_DIRECT)
+    run = DeviceRun(wl, K, V, lengths, flags=rkv.RKV_FLAG_DECODE_DIRECT)
     check_decode(run, synth.gen_query(wl, 0, 0))
 
 
@@ -190,7 +190,7 @@ def test_simt_decode_flag_matches_oracle():
     wl = _small("llama3_8b_layer", n_kv_heads=2, n_q_heads=8, batch=2, seq_len=3100, ragged=None)
     lengths = [3100, 1500]
     K, V = synth.gen_layer(wl, 0, lengths)
-    run = GpuRun(wl, K, V, lengths, flags=rkv.RKV_FLAG_DECODE_SIMT)
+    run = DeviceRun(wl, K, V, lengths, flags=rkv.RKV_FLAG_DECODE_SIMT)
     check_decode(run, synth.gen_query(wl, 0, 0))
 
 
@@ -201,9 +201,9 @@ def test_decode_many_short_units(n_q_heads):
     wl = _small("llama3_8b_layer", n_kv_heads=2, n_q_heads=n_q_heads, batch=16, seq_len=1700, ragged=None)
     lengths = [1700 - 97 * i for i in range(16)]
     K, V = synth.gen_layer(wl, 0, lengths)
-    run = GpuRun(wl, K, V, lengths)
+    run = DeviceRun(wl, K, V, lengths)
     check_decode(run, synth.gen_query(wl, 0, 0))
-    simt = GpuRun(wl, K, V, lengths, flags=rkv.RKV_FLAG_DECODE_SIMT)
+    simt = DeviceRun(wl, K, V, lengths, flags=rkv.RKV_FLAG_DECODE_SIMT)
     q = synth.gen_query(wl, 0, 0)
     a, b = run.decode(q), simt.decode(q)
     assert np.abs(a - b).max() <= 2e-3
@@ -247,7 +247,7 @@ def test_sparse_decode_matches_oracle_on_listed_rows(name):
                 batch=2, seq_len=3000, ragged=None)
     lengths = [3000, 1700]
     K, V = synth.gen_layer(wl, 0, lengths)
-    run = GpuRun(wl, K, V, lengths)
+    run = DeviceRun(wl, K, V, lengths)
     rng = np.random.default_rng(7)
     sel = []
     for b, n in enumerate(lengths):
@@ -266,7 +266,7 @@ def test_sparse_decode_full_list_equals_dense_decode():
     wl = _small("llama3_8b_layer", n_kv_heads=2, n_q_heads=8, seq_len=2500)
     lengths = [2500]
     K, V = synth.gen_layer(wl, 0, lengths)
-    run = GpuRun(wl, K, V, lengths)
+    run = DeviceRun(wl, K, V, lengths)
     q = synth.gen_query(wl, 0, 0)
     dense = run.decode(q)
     sel = [np.arange(2500) for _ in range(2)]
@@ -283,7 +283,7 @@ def test_sparse_decode_reports_out_of_range_positions():
     wl = _small("llama3_8b_layer", n_kv_heads=1, n_q_heads=4, seq_len=1000)
     lengths = [1000]
     K, V = synth.gen_layer(wl, 0, lengths)
-    run = GpuRun(wl, K, V, lengths)
+    run = DeviceRun(wl, K, V, lengths)
     pos = torch.tensor([[5, 999, 1000, -1]], dtype=torch.int32, device="cuda")   # two outside [0, 1000)
     cnt = torch.tensor([4], dtype=torch.int32, device="cuda")
     out = torch.empty((1, 4, 128), dtype=torch.float32, device="cuda")
@@ -305,7 +305,7 @@ def test_append_equals_compressing_the_whole_sequence(case):
                     bits=8, seq_len=1500, n_proto=64)
         cap, start = [1500], [200]
     K, V = synth.gen_layer(wl, 0, cap)
-    run = GpuRun(wl, K, V, cap, start_lengths=start)
+    run = DeviceRun(wl, K, V, cap, start_lengths=start)
     mid = [min(c, s + 300) for c, s in zip(cap, start)]
     run.append_until(mid)                        # every sequence
     run.append_until(cap)                        # then each up to its own capacity
@@ -344,7 +344,7 @@ def test_int4_reference_store_every_stage(case):
         wl = synth.WORKLOADS["tiny"]
         lengths = wl.lengths()
     K, V = synth.gen_layer(wl, 0, lengths)
-    run = GpuRun(wl, K, V, lengths, ref_bits=4)
+    run = DeviceRun(wl, K, V, lengths, ref_bits=4)
     assert run.unit(0, 0)["ref_bits"] == 4
     stats = _full_unit_checks(run, wl, K, V, lengths)
     assert stats["tokens"] > 0
@@ -368,7 +368,7 @@ def test_int4_reference_store_decode_flags(flags):
     lengths = [2600, 1000]
     K, V = synth.gen_layer(wl, 0, lengths)
     f = rkv.RKV_FLAG_DECODE_SIMT if flags == "simt" else rkv.RKV_FLAG_DECODE_DIRECT
-    run = GpuRun(wl, K, V, lengths, ref_bits=4, flags=f)
+    run = DeviceRun(wl, K, V, lengths, ref_bits=4, flags=f)
     assert run.unit(0, 0)["ref_bits"] == 4
     check_decode(run, synth.gen_query(wl, 0, 0))
 
@@ -377,7 +377,7 @@ def test_int4_reference_store_append():
     wl = _small("llama3_8b_layer", n_kv_heads=2, n_q_heads=8, batch=2, seq_len=2200, ragged=None)
     cap, start = [2200, 1900], [1500, 700]
     K, V = synth.gen_layer(wl, 0, cap)
-    run = GpuRun(wl, K, V, cap, start_lengths=start, ref_bits=4)
+    run = DeviceRun(wl, K, V, cap, start_lengths=start, ref_bits=4)
     run.append_until(cap)
     for b, n in enumerate(cap):
         for h in range(wl.n_kv_heads):
@@ -413,7 +413,7 @@ def test_learned_coder_shapes_every_stage(case):
         lengths = [2600, 2000]
     K, V = synth.gen_layer(wl, 0, lengths)
     coder = _random_coders(wl.head_dim, 11)
-    run = GpuRun(wl, K, V, lengths, coder=coder)
+    run = DeviceRun(wl, K, V, lengths, coder=coder)
     stats = {}
     for b, n in enumerate(lengths):
         for h in range(wl.n_kv_heads):
@@ -435,7 +435,7 @@ def test_learned_coder_ragged_batch():
     lengths = [2100, 150, 17, 0]
     K, V = synth.gen_layer(wl, 0, lengths, max_len=2103)
     coder = _random_coders(wl.head_dim, 13)
-    run = GpuRun(wl, K, V, lengths, coder=coder)
+    run = DeviceRun(wl, K, V, lengths, coder=coder)
     stats = {}
     for b, n in enumerate(lengths):
         if n == 0:
@@ -456,7 +456,7 @@ def test_learned_coder_refuses_what_it_does_not_cover():
     lengths = [600]
     K, V = synth.gen_layer(wl, 0, lengths)
     coder = _random_coders(wl.head_dim, 12)
-    run = GpuRun(wl, K, V, lengths, coder=coder)
+    run = DeviceRun(wl, K, V, lengths, coder=coder)
     q = to_dev(synth.gen_query(wl, 0, 0))
     out = torch.empty((1, 4, 128), dtype=torch.float32, device="cuda")
     pos = torch.zeros((1, 4), dtype=torch.int32, device="cuda")
