@@ -23,7 +23,9 @@
  * Conventions for every call
  *   - Memory: the caller allocates every buffer (inputs, the cache, the
  *     workspace, outputs) and keeps ownership.  The library allocates no
- *     device memory, keeps no global state and never frees caller memory.
+ *     device memory and never frees caller memory.  It keeps no global state,
+ *     with one exception: rkv_compress_noalloc's fixed scratch array (a
+ *     file-scope device array, see that call).
  *   - Streams: `stream` is a cudaStream_t (NULL = legacy default stream).
  *     Device work is enqueued asynchronously on it; calls that only touch
  *     host memory ignore it.  Calls on distinct buffers may run concurrently.
@@ -239,7 +241,9 @@ RKV_API rkv_status rkv_build_refs(const rkv_cache_desc* desc, const void* K, con
  * Framework Architecture": top-k nearest references by L2 distance on the key,
  * mean reference, residual; news page, "How ResidualKV Works": quantized
  * residual codes).  Needs rkv_build_refs on the same K first.  Candidates of
- * position i are the references at positions < i; ranking is by (distance,
+ * position i are the references at positions <= i (for a compressed token,
+ * whose position is never a reference, that is the earlier references); ranking
+ * is by (distance,
  * ordinal); k_eff = min(k, candidates); the mean is an fp32 sum in ascending
  * ordinal order divided by k_eff; per 32-channel group
  * scale = smallest binary16 >= max|delta| / qmax and
@@ -368,11 +372,25 @@ RKV_API rkv_status rkv_reconstruct(const rkv_cache_desc* desc, int32_t seq, int3
  * RKV_NOALLOC_SCRATCH_BYTES inside the library instead of in a workspace.  It
  * allocates nothing; every GPU that loads the library holds the array until
  * the process exits.
- *   - Limit: the candidate lists of one layer (6 bytes per compressed row per
- *     kept candidate, rounded to 256-byte sections) must fit the array;
- *     larger caches get RKV_ERR_WORKSPACE before anything is enqueued.
- *   - Set-up: the first call on a device (with that device current) looks up the
- *     array's device address; make that first call before any stream capture.
+ *   - Limit: the search part of the workspace must fit the array.  With
+ *     A(x) = x rounded up to a multiple of 256, rows = the layer's compressed
+ *     rows (every unit's n - n_ref, padded up to a multiple of 128),
+ *     ref_rows = its reference rows (every unit's n_ref, padded up to a
+ *     multiple of 8) and kc = the search's candidate-list width (k + 4 for
+ *     k <= 4, 12 for k <= 8, 20 for k <= 16), that part is
+ *         A(2 * rows * kc) + A(4 * rows * kc)       candidate ordinals, scores
+ *       + A(8 + 8 * rows)                           the encoder's deferred list
+ *       + A(2 * ref_rows * head_dim)                only with ref_bits 4: the
+ *                                                   stored keys as bf16 rows
+ *     Larger caches get RKV_ERR_WORKSPACE before anything is enqueued.  For
+ *     example, a layer of 8 kv-heads x 32768 tokens at stride 16, k 4 (kc 8)
+ *     needs about 14 MB with bf16 references and 18 MB (too much) with
+ *     ref_bits 4.
+ *   - Set-up: the first call in a CUDA context (with that context current)
+ *     looks up the array's device address, which belongs to the library's
+ *     module in that context; a new context (after cudaDeviceReset, say) gets
+ *     its own look-up.  Make the first call in a context before any stream
+ *     capture.
  *   - Sharing: all calls on a device use the same array and it keeps the last
  *     call's contents; nothing in it needs to start at zero (the search writes
  *     every entry the encoder reads).  Calls that overlap on the GPU race on it:
@@ -383,6 +401,8 @@ RKV_API rkv_status rkv_compress_noalloc(const rkv_cache_desc* desc, const void* 
 
 /*
  * Synchronises `stream`, then reads and clears the cache's device error word.
+ * The word lives in the cache buffer (one per bound layer, so concurrent
+ * layers do not share it), which is why the call takes the cache handle.
  * *device_status gets RKV_OK or the first RKV_ERR_* a kernel recorded since
  * the last read.  Returns RKV_ERR_CUDA if the synchronisation failed.
  */

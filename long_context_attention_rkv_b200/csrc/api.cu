@@ -1,6 +1,8 @@
 // C ABI of librkv: argument validation, cache layout and binding, kernel dispatch.
 // Every entry point returns an rkv_status and never throws; see include/rkv.h.
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <atomic>
@@ -19,6 +21,15 @@
 using namespace rkv;
 
 namespace {
+
+// An NVTX range around one entry point, so a profile of the whole path splits by API call.
+// Costs a few nanoseconds when no profiler is attached.
+struct ApiRange {
+    explicit ApiRange(const char* name) { nvtxRangePushA(name); }
+    ~ApiRange() { nvtxRangePop(); }
+    ApiRange(const ApiRange&) = delete;
+    ApiRange& operator=(const ApiRange&) = delete;
+};
 
 uint64_t align_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
 
@@ -463,6 +474,7 @@ rkv_status rkv_unit_view_get(const rkv_cache_desc* desc, int32_t seq, int32_t kv
 
 rkv_status rkv_build_refs(const rkv_cache_desc* desc, const void* K, const void* V, void* stream)
 {
+    const ApiRange range("rkv_build_refs");
     const Desc* d = get_desc(desc);
     if (!d || !K || !V || !aligned(K, 16) || !aligned(V, 16))
         return RKV_ERR_INVALID_ARG;
@@ -499,6 +511,7 @@ static bool coder_ready(const Desc* d) { return d->cfg.coder == 0 || d->coder_w[
 rkv_status rkv_search(const rkv_cache_desc* desc, const void* K, void* workspace, uint64_t workspace_bytes,
                       void* stream)
 {
+    const ApiRange range("rkv_search");
     const Desc* d = get_desc(desc);
     const rkv_status s = check_stage_args(d, K, nullptr, workspace, workspace_bytes);
     if (s != RKV_OK)
@@ -530,6 +543,7 @@ rkv_status rkv_search(const rkv_cache_desc* desc, const void* K, void* workspace
 rkv_status rkv_encode(const rkv_cache_desc* desc, const void* K, const void* V, void* workspace,
                       uint64_t workspace_bytes, void* stream)
 {
+    const ApiRange range("rkv_encode");
     const Desc* d = get_desc(desc);
     if (!V)
         return RKV_ERR_INVALID_ARG;
@@ -558,6 +572,7 @@ rkv_status rkv_encode(const rkv_cache_desc* desc, const void* K, const void* V, 
 rkv_status rkv_compress(const rkv_cache_desc* desc, const void* K, const void* V, void* workspace,
                         uint64_t workspace_bytes, void* stream)
 {
+    const ApiRange range("rkv_compress");
     if (!V)
         return RKV_ERR_INVALID_ARG;
     const rkv_status s = rkv_search(desc, K, workspace, workspace_bytes, stream);
@@ -567,6 +582,7 @@ rkv_status rkv_compress(const rkv_cache_desc* desc, const void* K, const void* V
 rkv_status rkv_decode_attn(const rkv_cache_desc* desc, const void* q, void* out, void* workspace,
                            uint64_t workspace_bytes, void* stream)
 {
+    const ApiRange range("rkv_decode_attn");
     const Desc* d = get_desc(desc);
     if (!d || !q || !out || !workspace || !aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, 256))
         return RKV_ERR_INVALID_ARG;
@@ -614,6 +630,7 @@ rkv_status rkv_set_coder(rkv_cache_desc* desc, const void* const* w)
 
 rkv_status rkv_cache_set_lengths(rkv_cache_desc* desc, const int32_t* lengths, void* stream)
 {
+    const ApiRange range("rkv_cache_set_lengths");
     const Desc* cd = get_desc(desc);
     if (!cd || !lengths)
         return RKV_ERR_INVALID_ARG;
@@ -647,6 +664,7 @@ rkv_status rkv_cache_set_lengths(rkv_cache_desc* desc, const int32_t* lengths, v
 rkv_status rkv_append(rkv_cache_desc* desc, const void* K_new, const void* V_new, const uint8_t* active,
                       void* stream)
 {
+    const ApiRange range("rkv_append");
     const Desc* cd = get_desc(desc);
     if (!cd || !K_new || !V_new || !aligned(K_new, 16) || !aligned(V_new, 16))
         return RKV_ERR_INVALID_ARG;
@@ -680,6 +698,7 @@ rkv_status rkv_decode_attn_sparse(const rkv_cache_desc* desc, const void* q, con
                                   const int32_t* counts, int32_t max_sel, void* out, void* workspace,
                                   uint64_t workspace_bytes, void* stream)
 {
+    const ApiRange range("rkv_decode_attn_sparse");
     const Desc* d = get_desc(desc);
     if (!d || !q || !out || !positions || !counts || max_sel < 1 || !workspace || !aligned(q, 16) ||
         !aligned(out, 16) || !aligned(workspace, 256) || !aligned(positions, 4) || !aligned(counts, 4))
@@ -701,6 +720,7 @@ rkv_status rkv_decode_attn_sparse(const rkv_cache_desc* desc, const void* q, con
 rkv_status rkv_reconstruct(const rkv_cache_desc* desc, int32_t seq, int32_t kv_head, const int32_t* positions,
                            int64_t n_pos, void* K_out, void* V_out, int32_t out_dtype, void* stream)
 {
+    const ApiRange range("rkv_reconstruct");
     const Desc* d = get_desc(desc);
     if (!d || seq < 0 || seq >= d->cfg.batch || kv_head < 0 || kv_head >= d->cfg.n_kv_heads || n_pos < 0)
         return RKV_ERR_INVALID_ARG;
@@ -730,6 +750,7 @@ rkv_status rkv_selftest_wait_timeout(int32_t* err_dev, void* stream)
 
 rkv_status rkv_read_device_error(const rkv_cache_desc* desc, void* stream, int32_t* device_status)
 {
+    const ApiRange range("rkv_read_device_error");
     const Desc* d = get_desc(desc);
     if (!d || !device_status)
         return RKV_ERR_INVALID_ARG;
@@ -751,7 +772,7 @@ rkv_status rkv_read_device_error(const rkv_cache_desc* desc, void* stream, int32
 // ---- compress without a workspace ------------------------------------------------------
 // For callers that cannot allocate (see rkv_compress_noalloc in rkv.h): the candidate lists
 // live in this file-scope device array.  Host code only ever uses its device address, looked
-// up once per device with cudaGetSymbolAddress while that device is current.
+// up with cudaGetSymbolAddress once per CUDA context, with that context current.
 
 }  // extern "C"
 
@@ -759,28 +780,79 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[RKV_NOALLOC_SCR
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-std::atomic<void*> g_noalloc_addr[kMaxDevices];
+// The array's address belongs to a loaded module, and a module belongs to one CUDA context:
+// after cudaDeviceReset, or with another context current on the same device, the array may
+// sit elsewhere.  So the cached address is keyed by the current context's unique id (never
+// reused within a process, unlike a context handle), not by the device ordinal, and it is
+// looked up again whenever a context without an entry is current.
+constexpr int kMaxContexts = 64;
+struct ScratchAddr {
+    unsigned long long ctx_id;
+    void* ptr;
+};
+ScratchAddr g_noalloc_addr[kMaxContexts];
+int g_noalloc_count = 0;
+int g_noalloc_next = 0;
 std::mutex g_noalloc_mutex;
 
-// Device address of the scratch array on the current device (looked up on first use).
+// The two driver calls, resolved through the runtime (the library does not link the driver).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+template <typename Fn>
+Fn driver_fn(const char* name)
+{
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint(name, &fn, cudaEnableDefault, &qr) != cudaSuccess ||
+        qr != cudaDriverEntryPointSuccess)
+        return nullptr;
+    return reinterpret_cast<Fn>(fn);
+}
+
+rkv_status current_context_id(unsigned long long* id)
+{
+    static const CtxGetCurrentFn cuCtxGetCurrent = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+    static const CtxGetIdFn cuCtxGetId = driver_fn<CtxGetIdFn>("cuCtxGetId");
+    if (!cuCtxGetCurrent || !cuCtxGetId)
+        return RKV_ERR_CUDA;
+    CUcontext ctx = nullptr;
+    if (cuCtxGetCurrent(&ctx) != CUDA_SUCCESS)
+        return RKV_ERR_CUDA;
+    if (!ctx) {
+        // no context on this thread yet: a runtime call that needs one makes the current
+        // device's primary context current (it neither allocates nor launches)
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || cudaSetDevice(dev) != cudaSuccess)
+            return RKV_ERR_CUDA;
+        void* probe = nullptr;
+        if (cudaGetSymbolAddress(&probe, g_noalloc_scratch) != cudaSuccess)
+            return RKV_ERR_CUDA;
+        if (cuCtxGetCurrent(&ctx) != CUDA_SUCCESS || !ctx)
+            return RKV_ERR_CUDA;
+    }
+    return cuCtxGetId(ctx, id) == CUDA_SUCCESS ? RKV_OK : RKV_ERR_CUDA;
+}
+
+// Device address of the scratch array in the current context (looked up on first use).
 rkv_status noalloc_scratch(void** out)
 {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess)
-        return RKV_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices)
-        return RKV_ERR_UNSUPPORTED;
-    void* p = g_noalloc_addr[dev].load(std::memory_order_acquire);
-    if (!p) {
-        std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-        p = g_noalloc_addr[dev].load(std::memory_order_relaxed);
-        if (!p) {
-            if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p)
-                return RKV_ERR_CUDA;
-            g_noalloc_addr[dev].store(p, std::memory_order_release);
+    unsigned long long id = 0;
+    const rkv_status st = current_context_id(&id);
+    if (st != RKV_OK)
+        return st;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    for (int i = 0; i < g_noalloc_count; ++i)
+        if (g_noalloc_addr[i].ctx_id == id) {
+            *out = g_noalloc_addr[i].ptr;
+            return RKV_OK;
         }
-    }
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p)
+        return RKV_ERR_CUDA;
+    // a full table replaces its entries in turn (a context without an entry just looks up again)
+    const int slot = g_noalloc_count < kMaxContexts ? g_noalloc_count++ : g_noalloc_next++ % kMaxContexts;
+    g_noalloc_addr[slot] = ScratchAddr{id, p};
     *out = p;
     return RKV_OK;
 }
@@ -791,6 +863,7 @@ extern "C" {
 
 rkv_status rkv_compress_noalloc(const rkv_cache_desc* desc, const void* K, const void* V, void* stream)
 {
+    const ApiRange range("rkv_compress_noalloc");
     const Desc* d = get_desc(desc);
     if (!d || !V)
         return RKV_ERR_INVALID_ARG;

@@ -17,6 +17,8 @@ from gpu_harness import config, to_dev
 
 pytestmark = pytest.mark.gpu
 
+NOALLOC_SCRATCH_BYTES = 16 << 20     # RKV_NOALLOC_SCRATCH_BYTES in rkv.h
+
 
 def _compressed(layer, wl):
     out = {}
@@ -56,5 +58,23 @@ def test_noalloc_refuses_oversized_cache():
     wl = synth.WORKLOADS["llama3_8b_stack"]          # 8 x 122880 rows x 8 candidates: ~47 MB of lists
     lengths = wl.lengths()
     layer = rkv.Layer(config(wl, lengths), lengths, workspace=False)
+    st = rkv.lib().rkv_compress_noalloc(layer.desc.ptr, 256, 256, None)
+    assert st == rkv.STATUS_CODE["RKV_ERR_WORKSPACE"]
+
+
+def test_noalloc_limit_counts_the_int4_key_copy():
+    # the 32768-token Llama-shaped layer fits the array with bf16 references (13.8 MB of
+    # search workspace) but not with the int4 reference store, whose search also keeps the
+    # stored keys as bf16 rows (4.2 MB more): the header's formula, checked both ways
+    wl = synth.WORKLOADS["llama3_8b_layer"]
+    lengths = wl.lengths()
+    rows, ref_rows, kc, D = 8 * 30720, 8 * 2048, 8, wl.head_dim
+
+    def a256(x):
+        return (x + 255) // 256 * 256
+
+    search16 = a256(2 * rows * kc) + a256(4 * rows * kc) + a256(8 + 8 * rows)
+    assert search16 <= NOALLOC_SCRATCH_BYTES < search16 + a256(2 * ref_rows * D)
+    layer = rkv.Layer(config(wl, lengths, ref_bits=4), lengths, workspace=False)
     st = rkv.lib().rkv_compress_noalloc(layer.desc.ptr, 256, 256, None)
     assert st == rkv.STATUS_CODE["RKV_ERR_WORKSPACE"]
