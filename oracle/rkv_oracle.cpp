@@ -502,7 +502,11 @@ float orc_fp16_value(uint16_t h) { return fp16_value(h); }
 //   fc(x) = Wo (silu(Wg x) * (Wu x)),  Wg, Wu [H][D], Wo [L][H],  silu(a) = a / (1 + e^-a)
 //   fd(z) = Wd z,                      Wd [D][L]
 // Everything in double from the exact inputs.  The latent residual is rounded to fp32 and
-// then quantised by the residuals' group quantiser, as the identity coder's residual is.
+// then quantised by the residuals' group quantiser, with each group's scale rounded up to a
+// power of two (as the int4 reference store's are): the pages fix no format for the coder's
+// codes, and a power-of-two scale keeps the stored codes a reproducible function of a
+// network output whose last bits depend on how it is evaluated (boundaries a factor of 2
+// apart instead of 2^-10).
 // ---------------------------------------------------------------------------
 static void fc_apply(int D, int H, int L, const float* Wg, const float* Wu, const float* Wo, const double* x,
                      double* out)
@@ -537,7 +541,8 @@ void orc_coder_fc(int D, int H, int L, int64_t n, const float* X, const float* W
 
 // Latent residual codes: per token m = mean reference (fp32, as the identity coder forms
 // it), z = fc(x) - fc(m) (double, rounded to fp32), then the group quantiser over the L
-// latent channels.  z_out (optional) gets z in double.  Returns 1 on a binary16 overflow.
+// latent channels with power-of-two scales.  z_out (optional) gets z in double.  Returns 1 on
+// a binary16 overflow.
 int orc_encode_latent(int D, int H, int L, int bits, int group, int64_t n_tok, const float* X, const float* refs,
                       const uint16_t* idx, int k, const float* Wg, const float* Wu, const float* Wo, uint8_t* codes,
                       uint16_t* scales, double* z_out)
@@ -561,7 +566,8 @@ int orc_encode_latent(int D, int H, int L, int bits, int group, int64_t n_tok, c
             zf[l] = static_cast<float>(z);
         }
         if (bits > 0)
-            overflow |= quantize_groups(L, bits, group, zf.data(), codes + t * (L * bits / 8), scales + t * (L / group));
+            overflow |= quantize_groups(L, bits, group, zf.data(), codes + t * (L * bits / 8), scales + t * (L / group),
+                                        true);
     }
     return overflow;
 }

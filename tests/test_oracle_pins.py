@@ -518,11 +518,18 @@ def test_latent_residual_is_fc_difference_and_zero_for_the_mean():
     e = oracle.encode_latent(x, refs, idx, 4, cK)
     np.testing.assert_allclose(e["z"], oracle.coder_fc(x, cK) - oracle.coder_fc(mean, cK), rtol=1e-12, atol=1e-12)
     assert np.all(e["codes"][:5] == 0) and np.all(e["scales"][:5] == 0)
-    # the codes are the residuals' group quantiser applied to z (rounded to fp32)
+    # the codes are the residuals' group quantiser applied to z (rounded to fp32), with every
+    # scale the smallest power of two >= fl32(a / 7) (numpy: a float32 division, then frexp)
     q = _numpy_unpack(e["codes"], D, 4)
     s = np.repeat(e["scales"].view(np.float16).astype(np.float64), 32, axis=1)
-    z32 = e["z"].astype(np.float32).astype(np.float64)
-    assert np.all(np.abs(z32 - q * s) <= s / 2 * (1 + 1e-12))
+    z32 = e["z"].astype(np.float32)
+    assert np.all(np.abs(z32.astype(np.float64) - q * s) <= s / 2 * (1 + 1e-12))
+    a7 = (np.abs(z32).reshape(n, -1, 32).max(axis=2) / np.float32(7)).astype(np.float64)
+    fr, ex = np.frexp(a7)
+    want = np.where(a7 > 0, np.ldexp(1.0, np.where(fr == 0.5, ex - 1, ex)), 0.0)
+    np.testing.assert_array_equal(e["scales"].view(np.float16).astype(np.float64), want)
+    # a power-of-two scale divides exactly: every code is rint(z / s), ties to even
+    np.testing.assert_array_equal(q, np.where(s > 0, np.rint(z32.astype(np.float64) / np.where(s > 0, s, 1)), 0))
 
 
 def test_latent_decode_factorises_through_fd():
