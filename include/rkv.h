@@ -120,8 +120,12 @@ typedef enum rkv_status {
  *                   "Improvements for AI systems": fc a SwiGLU block, fd a bias-free
  *                   linear projection), with weights the caller binds by rkv_set_coder:
  *                   fc(x) = Wo (silu(Wg x) * (Wu x)), fd(z) = Wd z, hidden and latent
- *                   widths equal to head_dim.  The latent residual z is stored with the
- *                   same quantiser and layout as the identity coder's residual.  Decode
+ *                   widths equal to head_dim.  The latent residual z is stored in the
+ *                   identity coder's layout with its group quantiser, except that each
+ *                   group's scale is the smallest power of two >= max|z| / qmax (so the
+ *                   stored codes do not depend on the last bits of how z is evaluated);
+ *                   groups whose scale the tensor-core evaluation cannot settle are
+ *                   recomputed in double by an extra pass.  Decode
  *                   applies fd by linearity: the codes meet Wd^T q, and Wd is applied once
  *                   to the softmax-weighted latent sum.  Requires head_dim 128, bits 4,
  *                   bf16 inputs, ref_bits 16, n_q_heads / n_kv_heads <= 8 and k <= 8; the
@@ -382,6 +386,8 @@ RKV_API rkv_status rkv_reconstruct(const rkv_cache_desc* desc, int32_t seq, int3
  *       + A(8 + 8 * rows)                           the encoder's deferred list
  *       + A(2 * ref_rows * head_dim)                only with ref_bits 4: the
  *                                                   stored keys as bf16 rows
+ *       + A(8 + 64 * rows)                          only with coder 1: the groups
+ *                                                   left to the exact latent pass
  *     Larger caches get RKV_ERR_WORKSPACE before anything is enqueued.  For
  *     example, a layer of 8 kv-heads x 32768 tokens at stride 16, k 4 (kc 8)
  *     needs about 14 MB with bf16 references and 18 MB (too much) with

@@ -217,6 +217,9 @@ rkv_status compute_layout(const rkv_config* c, const int32_t* lengths, Desc& d)
         d.ws_select += align_up(2ull * ref_rows * D, 256);   // the stored keys as bf16 rows (search operand)
     d.ws_fix_off = d.ws_select;                                // the encoder's deferred-token list
     d.ws_select += align_up(8ull + 8ull * cmp_rows, 256);
+    d.ws_latent_off = d.ws_select;                             // the learned coder's exact-pass list
+    if (c->coder == 1)
+        d.ws_select += align_up(encode_latent_list_bytes(cmp_rows), 256);
     const int splits = std::max(decode_splits(d.n_units, max_n), sparse_splits_max(d.n_units));
     d.ws_decode = align_up(4ull * d.n_units * splits * G * (D + 2), 256);
     const CacheArgs a = make_args(d);
@@ -564,7 +567,8 @@ rkv_status rkv_encode(const rkv_cache_desc* desc, const void* K, const void* V, 
             const int n = d->cur_len[b];
             total += d->cfg.n_kv_heads * encode_latent_tiles(n - static_cast<int>(host_ref_count(d->ph, n)));
         }
-        e = launch_encode_latent(a, K, V, total, st);
+        e = launch_encode_latent(a, K, V, total,
+                                 reinterpret_cast<int*>(static_cast<char*>(workspace) + d->ws_latent_off), st);
     }
     return cuda_status(e);
 }

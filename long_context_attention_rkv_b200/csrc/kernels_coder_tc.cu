@@ -17,9 +17,15 @@
 //      read) for the quarter w / 4 of the hidden units, forms d = h(x) - h(m) and writes it as
 //      another bf16 triple over the staging buffers;
 //   4. one thread issues z = Wo d (three MMAs per K step) into the first accumulator;
-//   5. every thread reads one 32-channel group of z of its token and quantises it with the
-//      residuals' quantiser: the whole group sits in one thread, so the group maximum needs no
-//      shuffle.
+//   5. every thread reads one 32-channel group of z of its token and quantises it: the
+//      residuals' quantiser with the scale rounded up to a power of two (the learned coder's
+//      code format); the whole group sits in one thread, so the group maximum needs no
+//      shuffle.  A group whose a/7 lies within 2^-12 (relative) of a power of two, where the
+//      tensor cores' fp32 evaluation of z could round the scale the other way than an exact
+//      one, is listed for the exact pass.
+// The exact pass (encode_latent_exact_kernel) recomputes the listed groups from scratch in
+// double: h(x) and h(m) for all hidden units, then the group's 32 latent channels, rounded to
+// fp32 and quantised; it overwrites the group's codes and scale.
 // Every wait on an mbarrier is bounded; a wait that gives up records RKV_ERR_TIMEOUT and the
 // CTA stops, freeing its TMEM.
 #include <cfloat>
@@ -105,9 +111,35 @@ __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, volatil
     return __syncthreads_and(w ? 1 : 0) != 0;
 }
 
+// Bits of the smallest binary16 power of two >= r (r > 0; 2^-24 at least), its value in *s and
+// its exponent in *e; sets *over when it would exceed 2^15.
+__device__ __forceinline__ uint16_t pow2_scale(float r, float* s, int* e, bool* over)
+{
+    int ex = 0;
+    const float fr = frexpf(r, &ex);            // r = fr * 2^ex, fr in [0.5, 1)
+    int E = (fr == 0.5f) ? ex - 1 : ex;         // smallest E with 2^E >= r
+    E = max(E, -24);
+    *over = E > 15;
+    E = min(E, 15);
+    *e = E;
+    *s = ldexpf(1.0f, E);
+    return (E >= -14) ? static_cast<uint16_t>((E + 15) << 10) : static_cast<uint16_t>(1u << (E + 24));
+}
+
+// Relative half-width of the band around a power of two inside which the exact pass decides a
+// group's scale: far above the relative error of the tensor-core evaluation of a group maximum
+// (a few 1e-6), and wide enough to cover it with margin.
+constexpr float kLatentBand = 1.0f / 4096.0f;
+
+// Entry of the exact pass's list: (unit | side << 24 | group << 28, compressed slot).
+__device__ __forceinline__ int2 latent_entry(int u, int side, int g, int c)
+{
+    return make_int2(u | (side << 24) | (g << 28), c);
+}
+
 template <int SIDE>
 __global__ void __launch_bounds__(kCThreads, 1) encode_latent_tc_kernel(CacheArgs a, const void* __restrict__ X,
-                                                                         int total_tiles)
+                                                                         int total_tiles, int* __restrict__ flist)
 {
     extern __shared__ uint8_t coder_raw[];
     const uint32_t raw_addr = smem_addr(coder_raw);
@@ -323,7 +355,7 @@ __global__ void __launch_bounds__(kCThreads, 1) encode_latent_tc_kernel(CacheArg
         phase ^= 1u;
         tc_fence_after();
 
-        // ---- 5. the residuals' quantiser on the thread's 32-channel group of z -----------------
+        // ---- 5. the quantiser on the thread's 32-channel group of z (power-of-two scale) -------
         {
             const int qmax = (a.bits == 8) ? 127 : 7;
             const int64_t row = um.cmp_row + (valid ? c : 0);
@@ -334,18 +366,27 @@ __global__ void __launch_bounds__(kCThreads, 1) encode_latent_tc_kernel(CacheArg
             for (int i = 0; i < 32; ++i)
                 amax = fmaxf(amax, fabsf(z[i]));
             uint16_t sbits = 0;
-            float sc = 1.0f;
+            float inv = 0.0f;
             if (amax > 0.0f) {
-                const __half hv = __float2half_ru(__fdiv_rn(amax, static_cast<float>(qmax)));
-                sbits = __half_as_ushort(hv);
-                sc = __half2float(hv);
-                if (valid && (sbits & 0x7c00u) == 0x7c00u)
+                const float r = __fdiv_rn(amax, static_cast<float>(qmax));
+                float sc, slo, shi;
+                int e, elo, ehi;
+                bool over, o2;
+                sbits = pow2_scale(r, &sc, &e, &over);
+                pow2_scale(r * (1.0f - kLatentBand), &slo, &elo, &o2);
+                pow2_scale(r * (1.0f + kLatentBand), &shi, &ehi, &o2);
+                if (valid && over)
                     report(a.err, RKV_ERR_UNSUPPORTED);
+                if (valid && elo != ehi) {
+                    // the scale could round the other way in an exact evaluation: the exact pass
+                    // decides this group
+                    const int slot = atomicAdd(flist, 1);
+                    reinterpret_cast<int2*>(flist + 2)[slot] = latent_entry(u, SIDE, cq, c);
+                }
+                inv = ldexpf(1.0f, -e);   // exact: 1 / s for a power of two s
             }
-            // code = rint(z / s): z times the rounded reciprocal of s, rounded half to even by adding
-            // 1.5 * 2^23 (|z / s| <= 7 up to rounding, since s >= amax / 7); the product's error is a
-            // few units of 2^-24 relative, far inside the half step the codes are held to
-            const float inv = amax > 0.0f ? __frcp_rn(sc) : 0.0f;
+            // code = rint(z / s): z times 1/s is exact (a power of two), and the addition of
+            // 1.5 * 2^23 in the same fused operation rounds it half to even
             constexpr float kRound = 12582912.0f;
             constexpr int kRoundBits = 0x4B400000;
             uint32_t w[4] = {0u, 0u, 0u, 0u};
@@ -373,11 +414,111 @@ __global__ void __launch_bounds__(kCThreads, 1) encode_latent_tc_kernel(CacheArg
     }
 }
 
+// The exact pass: one block of 128 threads per listed (token, side, group).  Thread j forms
+// hidden unit j of x and of m in double (g = Wg v, u = Wu v, h = silu(g) u); the first warp then
+// forms the group's 32 latent channels z = Wo h(x) - Wo h(m), rounds them to fp32 and quantises
+// them (power-of-two scale), overwriting the fast pass's codes and scale of the group.  m is the
+// mean reference as the oracle defines it: the fp32 sum in ascending ordinal order, divided by
+// k_eff.  The double evaluation is exact to far below fp32 rounding, so the result equals an
+// exact evaluation's except where z or a/7 sits within about 1e-15 of a rounding boundary.
+constexpr int kExactThreads = 128;
+
+__global__ void __launch_bounds__(kExactThreads) encode_latent_exact_kernel(CacheArgs a, const void* __restrict__ K,
+                                                                             const void* __restrict__ V,
+                                                                             const int* __restrict__ flist)
+{
+    __shared__ double xs[kCD], ms[kCD], hx[kCD], hm[kCD];
+    const int n = *reinterpret_cast<const volatile int*>(flist);
+    const int2* list = reinterpret_cast<const int2*>(flist + 2);
+    const int tid = threadIdx.x;
+    for (int e = blockIdx.x; e < n; e += gridDim.x) {
+        const int2 en = list[e];
+        const int u = en.x & 0xffffff, side = (en.x >> 24) & 1, g = (en.x >> 28) & 3, c = en.y;
+        const UnitMeta um = a.units[u];
+        const int64_t row = um.cmp_row + c;
+        const uint16_t* Xb = static_cast<const uint16_t*>(side ? V : K);
+        const uint16_t* refs = side ? a.ref_V : a.ref_K;
+        const uint16_t* id = a.idx + row * a.k;
+        __syncthreads();   // the previous entry's shared values are consumed
+        {
+            const int ch = tid;   // kExactThreads == kCD: one channel per thread
+            xs[ch] = static_cast<double>(
+                bf16_bits_to_f32(Xb[(static_cast<int64_t>(u) * a.max_len + slot_pos(a.ph, c)) * kCD + ch]));
+            float acc = 0.0f;
+            int keff = 0;
+            for (int l = 0; l < a.k; ++l) {
+                const int o = id[l];
+                if (o == RKV_IDX_UNUSED || o >= um.R)
+                    break;
+                const float r = bf16_bits_to_f32(refs[(um.ref_row + o) * kCD + ch]);
+                acc = (keff == 0) ? r : __fadd_rn(acc, r);
+                ++keff;
+            }
+            ms[ch] = static_cast<double>(keff > 0 ? __fdiv_rn(acc, static_cast<float>(keff)) : 0.0f);
+        }
+        __syncthreads();
+        {
+            const int j = tid;    // hidden unit
+            const uint16_t* Wg = a.cw[4 * side + 0] + j * kCD;
+            const uint16_t* Wu = a.cw[4 * side + 1] + j * kCD;
+            double gx = 0.0, ux = 0.0, gm = 0.0, um2 = 0.0;
+            for (int ch = 0; ch < kCD; ++ch) {
+                const double wg = bf16_bits_to_f32(Wg[ch]), wu = bf16_bits_to_f32(Wu[ch]);
+                gx = fma(wg, xs[ch], gx);
+                ux = fma(wu, xs[ch], ux);
+                gm = fma(wg, ms[ch], gm);
+                um2 = fma(wu, ms[ch], um2);
+            }
+            hx[j] = gx / (1.0 + exp(-gx)) * ux;
+            hm[j] = gm / (1.0 + exp(-gm)) * um2;
+        }
+        __syncthreads();
+        if (tid < 32) {
+            const int l = 32 * g + tid;   // latent channel
+            const uint16_t* Wo = a.cw[4 * side + 2] + l * kCD;
+            double fx = 0.0, fm = 0.0;
+            for (int j = 0; j < kCD; ++j) {
+                const double w = bf16_bits_to_f32(Wo[j]);
+                fx = fma(w, hx[j], fx);
+                fm = fma(w, hm[j], fm);
+            }
+            const float z = static_cast<float>(fx - fm);
+            float amax = fabsf(z);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+            const int qmax = (a.bits == 8) ? 127 : 7;
+            uint16_t sbits = 0;
+            int q = 0;
+            if (amax > 0.0f) {
+                float sc;
+                int ex;
+                bool over;
+                sbits = pow2_scale(__fdiv_rn(amax, static_cast<float>(qmax)), &sc, &ex, &over);
+                if (over)
+                    report(a.err, RKV_ERR_UNSUPPORTED);
+                q = max(-qmax, min(qmax, static_cast<int>(rintf(z * ldexpf(1.0f, -ex)))));
+            }
+            // pack: lane pairs (2i, 2i + 1) form byte i of the group's 16 code bytes
+            const uint32_t nib = static_cast<uint32_t>(q & 0xf);
+            const uint32_t other = __shfl_xor_sync(0xffffffffu, nib, 1);
+            uint8_t* codes = (side ? a.codes_V : a.codes_K) + row * a.code_bytes + 16 * g;
+            if ((tid & 1) == 0)
+                codes[tid >> 1] = static_cast<uint8_t>(nib | (other << 4));
+            if (tid == 0)
+                (side ? a.scale_V : a.scale_K)[row * a.n_groups + g] = sbits;
+        }
+    }
+}
+
 }  // namespace
 
 int encode_latent_tiles(int C) { return (C + kCTile - 1) / kCTile; }
 
-cudaError_t launch_encode_latent(const CacheArgs& a, const void* K, const void* V, int total_tiles, cudaStream_t st)
+uint64_t encode_latent_list_bytes(int64_t cmp_rows) { return 8ull + 8ull * 8ull * static_cast<uint64_t>(cmp_rows); }
+
+cudaError_t launch_encode_latent(const CacheArgs& a, const void* K, const void* V, int total_tiles, int* flist,
+                                 cudaStream_t st)
 {
     if (a.D != kCD || a.in_dtype != RKV_DTYPE_BF16 || a.bits != 4)
         return cudaErrorNotSupported;
@@ -398,8 +539,13 @@ cudaError_t launch_encode_latent(const CacheArgs& a, const void* K, const void* 
                                  static_cast<int>(smem));
     if (e != cudaSuccess)
         return e;
-    encode_latent_tc_kernel<0><<<grid, kCThreads, smem, st>>>(a, K, total_tiles);
-    encode_latent_tc_kernel<1><<<grid, kCThreads, smem, st>>>(a, V, total_tiles);
+    e = cudaMemsetAsync(flist, 0, sizeof(int), st);
+    if (e != cudaSuccess)
+        return e;
+    encode_latent_tc_kernel<0><<<grid, kCThreads, smem, st>>>(a, K, total_tiles, flist);
+    encode_latent_tc_kernel<1><<<grid, kCThreads, smem, st>>>(a, V, total_tiles, flist);
+    // the listed groups (a small share): a few blocks per SM stride over the list
+    encode_latent_exact_kernel<<<4 * sms, kExactThreads, 0, st>>>(a, K, V, flist);
     return cudaGetLastError();
 }
 

@@ -16,7 +16,11 @@
 //     bound covers the references outside the list as well).  Otherwise every candidate within 2*delta
 //     of the k-th is re-ranked by its exact-order fp32 distance sum_c (k_c - r_c)^2
 //     (ties to the lower ordinal); if even the last kept candidate is that close,
-//     the list may be incomplete and all candidates are rescanned exactly.
+//     the list may be incomplete and all candidates are rescanned exactly.  Both
+//     slow cases are deferred: the main pass lists them, a rescan kernel gives each
+//     token of the second kind a whole block (its candidates split over 256 threads)
+//     and rewrites its list as the exact top-k, and a last pass re-ranks and encodes
+//     every listed token.
 //  2. Mean of the chosen rows in ascending ordinal order (fp32, left to right),
 //     one IEEE division by k_eff; residual = x - mean (fp32).
 //  3. Per 32-channel group: a = max|residual|, scale = binary16 rounded up from
@@ -221,19 +225,22 @@ __device__ __forceinline__ void quantise_store(const float (&x)[CPL], const floa
 
 // Resident blocks per SM the register budget is set for: four (64 registers) where the code
 // fits without spills, two otherwise.
-template <int KC, int LPT>
-constexpr int encode_min_blocks() { return (LPT == 16 && KC <= 12) ? 4 : 2; }
+template <int KC, int LPT, bool FIX = false>
+constexpr int encode_min_blocks() { return (!FIX && LPT == 16 && KC <= 12) ? 4 : 2; }
 
 // One compressed token per group of LPT lanes: final top-k, mean, residual and quantiser.
 // (u, c): the token's unit and compressed slot; inactive groups shadow a valid token and store
 // nothing.  FIX false: tokens whose candidate list does not settle the top-k at once (mode 1
-// or 2 below, about 2 % of them) are not stored but listed in fix (fix[0] = count, then
-// (unit, slot) pairs), so the main pass stays straight-line; FIX true: the exact re-rank and
-// rescan of the listed tokens.
+// or 2 below: 2 % of them on a 32768-token layer, 10 % on a 131072-token one) are not stored
+// but listed, so the main pass stays straight-line: fix[0] counts the mode-1 tokens, listed as
+// (unit, slot) pairs from the front of the list, fix[1] the mode-2 tokens, listed from its back
+// (the list has fix_cap entries after the two counts).  FIX true: the exact re-rank of the
+// listed tokens (the mode-2 ones arrive with their lists already rewritten by the rescan
+// kernel as the exact top-k).
 template <int CPL, int KC, int LPT, int RB, bool FIX>
 __device__ __forceinline__ void encode_group(const CacheArgs& a, const void* __restrict__ K, const void* __restrict__ V,
                                              const uint16_t* __restrict__ cand_idx, const float* __restrict__ cand_t,
-                                             int* __restrict__ fix, int u, int c, bool active)
+                                             int* __restrict__ fix, int fix_cap, int u, int c, bool active)
 {
     constexpr int D = CPL * LPT;
     constexpr int kLPT = LPT;                // lanes per token
@@ -312,10 +319,13 @@ __device__ __forceinline__ void encode_group(const CacheArgs& a, const void* __r
         mode = ((nvalid == KC) && (ncand > KC) && (tlast >= tk - 2.0f * delta)) ? 2 : 1;
     bool store = active;
     if constexpr (!FIX) {
-        // defer the token to the exact pass: listed once (by its group's first lane)
+        // defer the token to the exact passes: listed once (by its group's first lane)
         if (active && mode != 0 && sub == 0) {
-            const int slot = atomicAdd(fix, 1);
-            reinterpret_cast<int2*>(fix + 2)[slot] = make_int2(u, c);
+            int2* list = reinterpret_cast<int2*>(fix + 2);
+            if (mode == 1)
+                list[atomicAdd(fix, 1)] = make_int2(u, c);
+            else
+                list[fix_cap - 1 - atomicAdd(fix + 1, 1)] = make_int2(u, c);
         }
         store = active && mode == 0;
         mode = 0;
@@ -334,26 +344,28 @@ __device__ __forceinline__ void encode_group(const CacheArgs& a, const void* __r
             if (i < k)
                 chosen[i] = slot_ord(i);
         if (any_mode >= 1) {
-            // exact distances of the near set: candidates i < k, plus those within 2*delta
+            // exact distances of the near set: candidates i < k, plus those within 2*delta.
+            // Every slot's row is read unconditionally (a listed slot's row, else the first
+            // slot's), so all the gathers are issued together.  A mode-2 token reaches this
+            // pass with its list rewritten as the exact top-k (mode 0); should one still read
+            // as mode 2 it is re-ranked within its list like a mode-1 token.
             float dist[KC];
             int ords[KC];
             bool in[KC];
+            const bool near = mode != 0;
 #pragma unroll
             for (int i = 0; i < KC; ++i) {
                 ords[i] = slot_ord(i);
                 const float ti = slot_t(i);
-                in[i] = (mode == 1) && i < nvalid && (i < k || ti >= tk - 2.0f * delta);
-                const bool need = __any_sync(0xffffffffu, in[i]);
-                float d = 0.0f;
-                if (need) {
-                    const int o = in[i] ? ords[i] : 0;
-                    d = tsum<kLPT>(part_dist<CPL, RB>(a, xk, um.ref_row + o, sub * CPL));
-                }
-                dist[i] = d;
+                in[i] = near && i < nvalid && (i < k || ti >= tk - 2.0f * delta);
             }
-            if (mode == 1) {
+#pragma unroll
+            for (int i = 0; i < KC; ++i) {
+                const int o = (i < nvalid) ? ords[i] : ords[0];
+                dist[i] = tsum<kLPT>(part_dist<CPL, RB>(a, xk, um.ref_row + o, sub * CPL));
+            }
+            if (near) {
                 // rank by (distance, ordinal) within the near set
-                int nch = 0;
 #pragma unroll
                 for (int i = 0; i < KC; ++i) {
                     int rank = 0;
@@ -365,82 +377,7 @@ __device__ __forceinline__ void encode_group(const CacheArgs& a, const void* __r
                         for (int s2 = 0; s2 < KM; ++s2)
                             if (s2 == rank)
                                 chosen[s2] = ords[i];
-                        ++nch;
                     }
-                }
-            }
-        }
-        if (any_mode == 2) {
-            // exhaustive exact scan for tokens whose candidate list may be incomplete:
-            // the lanes of such a token split the candidates; each keeps its own best k
-            const bool ex = (mode == 2);
-#pragma unroll
-            for (int i = 0; i < CPL; ++i)
-                xs[warp][tg][sub * CPL + i] = xk[i];
-            __syncwarp();
-            float bd[KM];
-            int bo[KM];
-#pragma unroll
-            for (int s2 = 0; s2 < KM; ++s2) {
-                bd[s2] = FLT_MAX;
-                bo[s2] = 0x7fffffff;
-            }
-            const int nscan = ex ? ncand : 0;
-            for (int j = sub; j < nscan; j += kLPT) {
-                float d = 0.0f;
-                for (int c2 = 0; c2 < D; c2 += 8) {
-                    float rv[8];
-                    load_ref<8, RB>(a, 0, um.ref_row + j, c2, rv);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const float e0 = __fsub_rn(xs[warp][tg][c2 + i], rv[i]);
-                        d = __fmaf_rn(e0, e0, d);
-                    }
-                }
-                float cv = d;
-                int ci = j;
-#pragma unroll
-                for (int s2 = 0; s2 < KM; ++s2) {
-                    if (s2 < k) {
-                        const bool before = (cv < bd[s2]) || (cv == bd[s2] && ci < bo[s2]);
-                        const float fd = bd[s2];
-                        const int fo = bo[s2];
-                        bd[s2] = before ? cv : fd;
-                        bo[s2] = before ? ci : fo;
-                        cv = before ? fd : cv;
-                        ci = before ? fo : ci;
-                    }
-                }
-            }
-            // merge the 8 lane lists of each token: k rounds of a group-wide minimum
-            int head = 0;
-            for (int r = 0; r < k; ++r) {
-                float hd = FLT_MAX;
-                int ho = 0x7fffffff;
-#pragma unroll
-                for (int s2 = 0; s2 < KM; ++s2)
-                    if (s2 == head) {
-                        hd = bd[s2];
-                        ho = bo[s2];
-                    }
-                float wd = hd;
-                int wo = ho;
-#pragma unroll
-                for (int off = 1; off < kLPT; off <<= 1) {
-                    const float od = __shfl_xor_sync(0xffffffffu, wd, off);
-                    const int oo = __shfl_xor_sync(0xffffffffu, wo, off);
-                    if (od < wd || (od == wd && oo < wo)) {
-                        wd = od;
-                        wo = oo;
-                    }
-                }
-                if (ho == wo && hd == wd)
-                    ++head;
-                if (ex) {
-#pragma unroll
-                    for (int s2 = 0; s2 < KM; ++s2)
-                        if (s2 == r)
-                            chosen[s2] = wo;
                 }
             }
         }
@@ -510,28 +447,162 @@ __device__ __forceinline__ void encode_group(const CacheArgs& a, const void* __r
 }
 
 template <int CPL, int KC, int LPT, int RB, bool FIX>
-__global__ void __launch_bounds__(kWarps * 32, encode_min_blocks<KC, LPT>()) encode_kernel(CacheArgs a, const void* __restrict__ K,
-                                                             const void* __restrict__ V,
-                                                             const uint16_t* __restrict__ cand_idx,
-                                                             const float* __restrict__ cand_t,
-                                                             int* __restrict__ fix)
+__global__ void __launch_bounds__(kWarps * 32, (encode_min_blocks<KC, LPT, FIX>())) encode_kernel(
+    CacheArgs a, const void* __restrict__ K, const void* __restrict__ V, const uint16_t* __restrict__ cand_idx,
+    const float* __restrict__ cand_t, int* __restrict__ fix, int fix_cap)
 {
     constexpr int kTPW = 32 / LPT;
     const int warp = threadIdx.x >> 5;
     const int tg = (threadIdx.x & 31) / LPT;
     if constexpr (FIX) {
-        // the listed tokens, strided over a grid sized for the device
-        const int n_fix = *reinterpret_cast<volatile int*>(fix);
+        // the listed tokens (mode 1 from the front of the list, mode 2 from its back), strided
+        // over a grid sized for the device
+        const int n1 = *reinterpret_cast<volatile int*>(fix);
+        const int n_fix = n1 + *reinterpret_cast<volatile int*>(fix + 1);
+        const int2* list = reinterpret_cast<const int2*>(fix + 2);
         for (int base = blockIdx.x * kWarps * kTPW; base < n_fix; base += gridDim.x * kWarps * kTPW) {
             const int t = base + warp * kTPW + tg;
             const bool active = t < n_fix;
-            const int2 uc = active ? reinterpret_cast<const int2*>(fix + 2)[t] : make_int2(0, 0);
-            encode_group<CPL, KC, LPT, RB, true>(a, K, V, cand_idx, cand_t, fix, uc.x, uc.y, active);
+            const int2 uc = !active ? make_int2(0, 0) : (t < n1) ? list[t] : list[fix_cap - 1 - (t - n1)];
+            encode_group<CPL, KC, LPT, RB, true>(a, K, V, cand_idx, cand_t, fix, fix_cap, uc.x, uc.y, active);
         }
     } else {
         const int u = blockIdx.y;
         const int c = (blockIdx.x * kWarps + warp) * kTPW + tg;
-        encode_group<CPL, KC, LPT, RB, false>(a, K, V, cand_idx, cand_t, fix, u, c, c < a.units[u].C);
+        encode_group<CPL, KC, LPT, RB, false>(a, K, V, cand_idx, cand_t, fix, fix_cap, u, c, c < a.units[u].C);
+    }
+}
+
+// Exhaustive exact rescan of the mode-2 tokens (candidate lists that may miss a reference):
+// one block of 256 threads per listed token, every thread a strided share of the token's
+// candidates, each distance the exact-order fp32 sum_c (k_c - r_c)^2 over the channels in
+// order; the block's k best by (distance, ordinal) are written back as the token's candidate
+// list, with t values that make the last pass take them as they are (slots past k repeat the
+// best ordinal with t = -inf).
+constexpr int kScanThreads = 256;
+constexpr int kScanKM = 16;   // largest k
+
+template <int D, int KC, int RB>
+__global__ void __launch_bounds__(kScanThreads) encode_scan_kernel(CacheArgs a, const void* __restrict__ K,
+                                                                   uint16_t* __restrict__ cand_idx,
+                                                                   float* __restrict__ cand_t,
+                                                                   const int* __restrict__ fix, int fix_cap)
+{
+    constexpr int KM = kScanKM;
+    constexpr int NW = kScanThreads / 32;
+    __shared__ float xs[D];
+    __shared__ float wd[NW][KM];
+    __shared__ int wo[NW][KM];
+    __shared__ int best[KM];
+    const int n2 = *reinterpret_cast<const volatile int*>(fix + 1);
+    const int2* list = reinterpret_cast<const int2*>(fix + 2);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int k = a.k;
+    for (int e = blockIdx.x; e < n2; e += gridDim.x) {
+        const int2 uc = list[fix_cap - 1 - e];
+        const UnitMeta um = a.units[uc.x];
+        const int p = slot_pos(a.ph, uc.y);
+        const int ncand = min(refs_upto(a.ph, p), um.R);
+        const int64_t row = um.cmp_row + uc.y;
+        const int64_t el = (static_cast<int64_t>(uc.x) * a.max_len + p) * D;
+        __syncthreads();   // the previous token's shared state is consumed
+        for (int c = tid; c < D; c += kScanThreads)
+            xs[c] = (a.in_dtype == RKV_DTYPE_F32) ? static_cast<const float*>(K)[el + c]
+                                                  : bf16_bits_to_f32(static_cast<const uint16_t*>(K)[el + c]);
+        __syncthreads();
+        float bd[KM];
+        int bo[KM];
+#pragma unroll
+        for (int s2 = 0; s2 < KM; ++s2) {
+            bd[s2] = FLT_MAX;
+            bo[s2] = 0x7fffffff;
+        }
+        for (int j = tid; j < ncand; j += kScanThreads) {
+            float d = 0.0f;
+#pragma unroll 4
+            for (int c2 = 0; c2 < D; c2 += 8) {
+                float rv[8];
+                load_ref<8, RB>(a, 0, um.ref_row + j, c2, rv);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float e0 = __fsub_rn(xs[c2 + i], rv[i]);
+                    d = __fmaf_rn(e0, e0, d);
+                }
+            }
+            float cv = d;
+            int ci = j;
+#pragma unroll
+            for (int s2 = 0; s2 < KM; ++s2) {
+                if (s2 < k) {
+                    const bool before = (cv < bd[s2]) || (cv == bd[s2] && ci < bo[s2]);
+                    const float fd = bd[s2];
+                    const int fo = bo[s2];
+                    bd[s2] = before ? cv : fd;
+                    bo[s2] = before ? ci : fo;
+                    cv = before ? fd : cv;
+                    ci = before ? fo : ci;
+                }
+            }
+        }
+        // k rounds of a warp-wide minimum over the lanes' sorted lists
+        int head = 0;
+        for (int r = 0; r < k; ++r) {
+            float hd = FLT_MAX;
+            int ho = 0x7fffffff;
+#pragma unroll
+            for (int s2 = 0; s2 < KM; ++s2)
+                if (s2 == head) {
+                    hd = bd[s2];
+                    ho = bo[s2];
+                }
+            float md = hd;
+            int mo = ho;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                const float od = __shfl_xor_sync(0xffffffffu, md, off);
+                const int oo = __shfl_xor_sync(0xffffffffu, mo, off);
+                if (od < md || (od == md && oo < mo)) {
+                    md = od;
+                    mo = oo;
+                }
+            }
+            if (ho == mo && hd == md && ho != 0x7fffffff)
+                ++head;
+            if (lane == 0) {
+                wd[warp][r] = md;
+                wo[warp][r] = mo;
+            }
+        }
+        __syncthreads();
+        // warp 0: the k best of the NW sorted warp lists (k rounds over their heads)
+        if (warp == 0) {
+            int wh = 0;   // lane w < NW: head of warp w's list
+            for (int r = 0; r < k; ++r) {
+                float md = (lane < NW && wh < k) ? wd[lane][wh] : FLT_MAX;
+                int mo = (lane < NW && wh < k) ? wo[lane][wh] : 0x7fffffff;
+                const float hd = md;
+                const int ho = mo;
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    const float od = __shfl_xor_sync(0xffffffffu, md, off);
+                    const int oo = __shfl_xor_sync(0xffffffffu, mo, off);
+                    if (od < md || (od == md && oo < mo)) {
+                        md = od;
+                        mo = oo;
+                    }
+                }
+                if (lane < NW && ho == mo && hd == md && ho != 0x7fffffff)
+                    ++wh;
+                if (lane == 0)
+                    best[r] = mo;
+            }
+        }
+        __syncthreads();
+        if (tid < KC) {
+            const bool in_k = tid < k;
+            cand_idx[row * KC + tid] = static_cast<uint16_t>(in_k ? best[tid] : best[0]);
+            cand_t[row * KC + tid] = in_k ? 0.0f : -FLT_MAX;
+        }
     }
 }
 
@@ -829,34 +900,36 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(CacheArgs a, con
 }
 
 template <int CPL, int KC, int LPT, int RB>
-void launch_pair(const CacheArgs& a, dim3 grid, const void* K, const void* V, const uint16_t* ci, const float* ct,
-                 int* fix, int fix_grid, cudaStream_t st)
+void launch_pair(const CacheArgs& a, dim3 grid, const void* K, const void* V, uint16_t* ci, float* ct, int* fix,
+                 int fix_cap, int fix_grid, int scan_grid, cudaStream_t st)
 {
-    encode_kernel<CPL, KC, LPT, RB, false><<<grid, kWarps * 32, 0, st>>>(a, K, V, ci, ct, fix);
-    encode_kernel<CPL, KC, LPT, RB, true><<<fix_grid, kWarps * 32, 0, st>>>(a, K, V, ci, ct, fix);
+    encode_kernel<CPL, KC, LPT, RB, false><<<grid, kWarps * 32, 0, st>>>(a, K, V, ci, ct, fix, fix_cap);
+    encode_scan_kernel<CPL * LPT, KC, RB><<<scan_grid, kScanThreads, 0, st>>>(a, K, ci, ct, fix, fix_cap);
+    encode_kernel<CPL, KC, LPT, RB, true><<<fix_grid, kWarps * 32, 0, st>>>(a, K, V, ci, ct, fix, fix_cap);
 }
 
 template <int CPL, int LPT>
-cudaError_t launch_cpl(const CacheArgs& a, int max_C, const void* K, const void* V, const uint16_t* ci,
-                       const float* ct, int* fix, int fix_cap, int sms, cudaStream_t st)
+cudaError_t launch_cpl(const CacheArgs& a, int max_C, const void* K, const void* V, uint16_t* ci, float* ct,
+                       int* fix, int fix_cap, int sms, cudaStream_t st)
 {
     const int per_block = kWarps * (32 / LPT);
     const dim3 grid((max_C + per_block - 1) / per_block, a.n_units);
     // the deferred pass: a few blocks per SM stride over the list (a few percent of the tokens)
     const int fix_need = (fix_cap + per_block - 1) / per_block;
     const int fix_grid = fix_need < 4 * sms ? (fix_need > 0 ? fix_need : 1) : 4 * sms;
+    const int scan_grid = 2 * sms;   // blocks of the rescan, striding over the mode-2 list
     if (a.ref_bits == 4) {
         switch (a.kc) {
-        case 8: launch_pair<CPL, 8, LPT, 4>(a, grid, K, V, ci, ct, fix, fix_grid, st); break;
-        case 12: launch_pair<CPL, 12, LPT, 4>(a, grid, K, V, ci, ct, fix, fix_grid, st); break;
-        default: launch_pair<CPL, 20, LPT, 4>(a, grid, K, V, ci, ct, fix, fix_grid, st); break;
+        case 8: launch_pair<CPL, 8, LPT, 4>(a, grid, K, V, ci, ct, fix, fix_cap, fix_grid, scan_grid, st); break;
+        case 12: launch_pair<CPL, 12, LPT, 4>(a, grid, K, V, ci, ct, fix, fix_cap, fix_grid, scan_grid, st); break;
+        default: launch_pair<CPL, 20, LPT, 4>(a, grid, K, V, ci, ct, fix, fix_cap, fix_grid, scan_grid, st); break;
         }
         return cudaGetLastError();
     }
     switch (a.kc) {
-    case 8: launch_pair<CPL, 8, LPT, 16>(a, grid, K, V, ci, ct, fix, fix_grid, st); break;
-    case 12: launch_pair<CPL, 12, LPT, 16>(a, grid, K, V, ci, ct, fix, fix_grid, st); break;
-    default: launch_pair<CPL, 20, LPT, 16>(a, grid, K, V, ci, ct, fix, fix_grid, st); break;
+    case 8: launch_pair<CPL, 8, LPT, 16>(a, grid, K, V, ci, ct, fix, fix_cap, fix_grid, scan_grid, st); break;
+    case 12: launch_pair<CPL, 12, LPT, 16>(a, grid, K, V, ci, ct, fix, fix_cap, fix_grid, scan_grid, st); break;
+    default: launch_pair<CPL, 20, LPT, 16>(a, grid, K, V, ci, ct, fix, fix_cap, fix_grid, scan_grid, st); break;
     }
     return cudaGetLastError();
 }
@@ -889,8 +962,8 @@ cudaError_t launch_append(const CacheArgs& a, const void* K_new, const void* V_n
     return cudaGetLastError();
 }
 
-cudaError_t launch_encode(const CacheArgs& a, int max_C, const void* K, const void* V, const uint16_t* cand_idx,
-                          const float* cand_t, int* fix, int fix_cap, cudaStream_t st)
+cudaError_t launch_encode(const CacheArgs& a, int max_C, const void* K, const void* V, uint16_t* cand_idx,
+                          float* cand_t, int* fix, int fix_cap, cudaStream_t st)
 {
     if (max_C <= 0)
         return cudaSuccess;
@@ -900,7 +973,7 @@ cudaError_t launch_encode(const CacheArgs& a, int max_C, const void* K, const vo
         e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess)
         return e;
-    e = cudaMemsetAsync(fix, 0, sizeof(int), st);
+    e = cudaMemsetAsync(fix, 0, 2 * sizeof(int), st);
     if (e != cudaSuccess)
         return e;
     return (a.D == 128) ? launch_cpl<kCpl128, 128 / kCpl128>(a, max_C, K, V, cand_idx, cand_t, fix, fix_cap, sms, st)

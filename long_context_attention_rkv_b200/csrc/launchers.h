@@ -20,9 +20,10 @@ cudaError_t launch_select_tc(const CacheArgs& a, const Tile* items, int n_items,
 
 // Final top-k, mean and quantiser of every compressed token.  fix: device scratch of
 // 2 + 2 * fix_cap ints (fix_cap >= the compressed tokens of the layer) for the tokens the main
-// pass defers to the exact pass.
-cudaError_t launch_encode(const CacheArgs& a, int max_C, const void* K, const void* V, const uint16_t* cand_idx,
-                          const float* cand_t, int* fix, int fix_cap, cudaStream_t st);
+// pass defers to the exact passes.  The rescan of the tokens whose candidate list may be
+// incomplete rewrites their lists in cand_idx / cand_t.
+cudaError_t launch_encode(const CacheArgs& a, int max_C, const void* K, const void* V, uint16_t* cand_idx,
+                          float* cand_t, int* fix, int fix_cap, cudaStream_t st);
 
 // Incremental compression: one new token ([unit][D] rows) for every unit of the sequences whose
 // bit is set in active (256 bits).
@@ -31,8 +32,12 @@ uint64_t append_scratch_bytes(int n_units);
 // Learned-coder shapes: latent residual codes z = fc(x) - fc(mean) of every compressed token
 // (after launch_encode has chosen the references), both sides, on the tcgen05 tensor cores in
 // 128-token tiles: total_tiles = the sum over units of encode_latent_tiles(compressed tokens).
+// flist: device scratch of encode_latent_list_bytes(compressed rows of the layer): the groups
+// the fast pass leaves to the exact pass (at most 8 per compressed row).
 int encode_latent_tiles(int C);
-cudaError_t launch_encode_latent(const CacheArgs& a, const void* K, const void* V, int total_tiles, cudaStream_t st);
+uint64_t encode_latent_list_bytes(int64_t cmp_rows);
+cudaError_t launch_encode_latent(const CacheArgs& a, const void* K, const void* V, int total_tiles, int* flist,
+                                 cudaStream_t st);
 cudaError_t launch_append(const CacheArgs& a, const void* K_new, const void* V_new, const uint32_t (&active)[8],
                           void* scratch, cudaStream_t st);
 

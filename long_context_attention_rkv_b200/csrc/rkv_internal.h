@@ -83,6 +83,7 @@ struct Desc {
     Phases ph;
     uint64_t ws_select;   // workspace bytes of the search stage
     uint64_t ws_fix_off;  // offset of the encoder's deferred-token list in that workspace
+    uint64_t ws_latent_off;  // offset of the learned coder's exact-pass list (coder 1)
     uint64_t ws_decode;   // workspace bytes of the decode stage
     int32_t len[RKV_MAX_BATCH];
     int32_t R[RKV_MAX_BATCH];

@@ -17,7 +17,6 @@ import synth
 IDX_TIE_BAND = 1e-4         # relative gap between the k-th and (k+1)-th oracle distance
 CODE_LSB_FRACTION = 1e-3    # codes may differ by one step on at most this fraction of elements
 RECON_ABS = 1e-2            # reconstructed K/V
-LATENT_SCALE_FRACTION = 1e-2  # learned-coder shapes: groups whose scale is one binary16 step off
 ATTN_ABS = 2e-3             # decode output (fp32 output; bf16 output adds half a bf16 ulp)
 
 
@@ -223,27 +222,9 @@ def check_compress(wl, g: dict, Xk, Xv, positions=None, stats=None, coder=None):
         ev = oracle.encode(Xv[positions], refV, gidx, wl.bits, wl.group)
     assert ek["overflow"] == 0 and ev["overflow"] == 0
     D = wl.head_dim
-    if coder is not None:
-        # the GPU forms the latent z on the tensor cores (bf16 operands split to the 24 bits of
-        # fp32, fp32 accumulation), the oracle in double: with a relative error eps of z a
-        # group's scale takes the neighbouring binary16 value where a/7 lies within eps of a
-        # binary16 boundary, about eps * 2^10 of the groups (measured 0.3 %, eps ~ 3e-6); every
-        # code still quantises the oracle's z within half a step
-        for name, e in (("K", ek), ("V", ev)):
-            gs = g["scales" + name][slots].view(np.float16).astype(np.float64)
-            os_ = e["scales"].view(np.float16).astype(np.float64)
-            diff = gs != os_
-            assert diff.mean() <= LATENT_SCALE_FRACTION, f"{name} latent scales differ in {diff.mean():.2e} of groups"
-            assert np.all(np.abs(gs - os_) <= os_ * 2.0 ** -9), f"{name} latent scales differ by more than a step"
-            gc = _unpack(g["codes" + name][slots], D, wl.bits)
-            sc = np.repeat(gs, 32, axis=1)
-            amax = np.repeat(np.abs(e["z"]).reshape(len(slots), -1, 32).max(axis=2), 32, axis=1)
-            err = np.abs(e["z"] - gc * sc)
-            assert np.all(err <= sc / 2 + 1e-4 * amax), f"{name} latent codes off by {(err - sc / 2).max()}"
-        if stats is not None:
-            stats["tokens"] = stats.get("tokens", 0) + len(positions)
-            stats["idx_tie_mismatch"] = stats.get("idx_tie_mismatch", 0) + mism
-        return
+    # learned-coder shapes and the identity coder share one contract: scales bit-exact, codes
+    # equal except for one step on at most CODE_LSB_FRACTION of the elements (the latent's
+    # power-of-two scales leave its codes a reproducible function of z)
     for name, e in (("K", ek), ("V", ev)):
         assert np.array_equal(g["scales" + name][slots], e["scales"]), f"{name} scales differ"
         gc = _unpack(g["codes" + name][slots], D, wl.bits)

@@ -56,6 +56,19 @@ def test_bf16_ragged_batch_every_stage(bits):
     check_decode(run, synth.gen_query(wl, 0, 0))
 
 
+def test_near_duplicate_references_every_stage():
+    # four prototypes and almost no noise: most tokens have many references within the
+    # search's error band of their k-th nearest (2354 of 2812 tokens per unit need the
+    # exhaustive exact rescan, 284 the exact re-rank), so both deferred passes of the encoder
+    # carry most of the layer
+    wl = _small("llama3_8b_layer", n_kv_heads=2, n_q_heads=8, seq_len=3000, n_proto=4, sigma=0.001, n_outlier=0)
+    lengths = [3000]
+    K, V = synth.gen_layer(wl, 0, lengths)
+    run = DeviceRun(wl, K, V, lengths)
+    _full_unit_checks(run, wl, K, V, lengths)
+    check_decode(run, synth.gen_query(wl, 0, 0))
+
+
 def test_dynamic_stride_every_stage():
     wl = _small("ultra_long_1m", n_kv_heads=1, n_q_heads=4, head_dim=64, stride0=4, refs_per_phase=64, k=3,
                 bits=8, seq_len=6000, n_proto=64)
