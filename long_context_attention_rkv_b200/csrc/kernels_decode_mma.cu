@@ -40,6 +40,7 @@
 #include <cfloat>
 #include <cmath>
 
+#include "decode_mma.h"
 #include "device_common.cuh"
 #include "launchers.h"
 #include "sm100_ptx.cuh"
@@ -49,9 +50,9 @@ namespace rkv {
 namespace {
 
 using namespace sm100;
+using namespace decode_detail;
 
 constexpr int kTok = 128;            // tokens per pipeline stage (= compressed-row padding)
-constexpr int kRefChunk = 64;        // references per CTA of the scores and refs kernels
 constexpr int kWarpTok = 16;         // tokens per consumer warp and stage
 constexpr int kConsWarps = kTok / kWarpTok;
 constexpr int kCodeRow = 64;         // bytes of one int4 code row at D = 128
@@ -133,18 +134,6 @@ __device__ __forceinline__ void red_global_v4(float* p, float a, float b, float 
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
 }
 
-// Order-preserving map of floats to unsigned keys (0 is below every float) and back.
-__device__ __forceinline__ uint32_t fkey(float f)
-{
-    const uint32_t b = __float_as_uint(f);
-    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-}
-
-__device__ __forceinline__ float fkey_inv(uint32_t k)
-{
-    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
-}
-
 // Bytes offset of (row, 16-byte chunk) in a 64-byte-row tile written by TMA with the 64-byte swizzle.
 __device__ __forceinline__ uint32_t sw64(int row, int chunk)
 {
@@ -152,22 +141,6 @@ __device__ __forceinline__ uint32_t sw64(int row, int chunk)
 }
 
 }  // namespace
-
-// Workspace carve-up of this decode (device pointers); see decode_mma_ws_bytes.
-struct MmaWs {
-    float* s_tab;     // [ref rows][Gp]  reference scores, log2 units
-    float* W;         // [ref rows][Gp]  reference weights sum_i p_i / k_eff
-    float* mpart;     // [units][n_chunk][Gp]  maxima of 64-reference chunks
-    float* O;         // [units][Gp][D]  output numerators
-    float* L;         // [units][Gp]     softmax denominators
-    uint32_t* cnt;    // [units]         finished chunks of the refs kernel
-    float* Olat;      // [units][Gp][D]  learned-coder shapes: latent output numerators
-    uint16_t* qlat;   // [batch][Hq][D]  learned-coder shapes: Wd_K^T q (bf16)
-    int n_chunk;
-    int n_tiles;
-    int n_cta;        // CTAs of the tokens kernel
-    float cK;         // log2(e) / sqrt(D)
-};
 
 namespace {
 
@@ -315,33 +288,6 @@ __global__ void __launch_bounds__(128) mma_scores_kernel(const CacheArgs a, cons
             v = fmaxf(v, wmax[i][tid]);
         w.mpart[(static_cast<int64_t>(u) * w.n_chunk + ch) * Gp + tid] = v;
     }
-}
-
-// Common offset m of a unit's q-heads: the maximum reference score (0 for a unit without
-// references).  All threads of the group load the chunk maxima in parallel and fold them
-// into key[Gp] (shared, zeroed beforehand) with atomic maxima; read back with unit_m.
-template <int Gp>
-__device__ __forceinline__ void unit_max_fold(const MmaWs& w, int u, int R, int tid, int nthreads, uint32_t* key)
-{
-    // entry x holds head x % Gp: lanes 0 .. Gp-1 of each warp fold their lane classes
-    const int n = ((R + kRefChunk - 1) / kRefChunk) * Gp;
-    const float* src = w.mpart + static_cast<int64_t>(u) * w.n_chunk * Gp;
-    for (int base = 0; base < n; base += nthreads) {
-        const int x = base + tid;
-        uint32_t k = (x < n) ? fkey(__ldcg(src + x)) : 0u;
-#pragma unroll
-        for (int o = Gp; o < 32; o <<= 1)
-            k = max(k, __shfl_xor_sync(0xffffffffu, k, o));
-        if ((tid & 31) < Gp && k != 0u)
-            atomicMax(&key[tid % Gp], k);
-    }
-}
-
-__device__ __forceinline__ float unit_m(const uint32_t* key, int h)
-{
-    const uint32_t k = key[h];
-    const float v = fkey_inv(k);
-    return (k == 0u || v == -FLT_MAX) ? 0.0f : v;
 }
 
 // ==== 2. compressed tokens ================================================================
@@ -1136,14 +1082,6 @@ cudaError_t launch_gp(const CacheArgs& a, int64_t cmp_rows, const void* q, void*
     if (e != cudaSuccess)
         return e;
     if (w.n_tiles > 0) {
-        const bool gt = tables_global(a);
-        auto kern = gt ? ((a.k <= 4) ? mma_tokens_kernel<Gp, 4, kTeams, true> : mma_tokens_kernel<Gp, 8, kTeams, true>)
-                       : ((a.k <= 4) ? mma_tokens_kernel<Gp, 4, kTeams, false> : mma_tokens_kernel<Gp, 8, kTeams, false>);
-        const size_t smem = TokLayout(Gp, kConsWarps * kTeams, gt ? 0 : a.max_refs, nst).total + 1024;
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-        if (e != cudaSuccess)
-            return e;
-        const int grid = w.n_cta;
         // learned-coder shapes: the tokens kernel meets the latent codes with q' and sums the
         // latent V side into Olat (the refs kernel applies fd to it)
         MmaWs wt = w;
@@ -1152,7 +1090,7 @@ cudaError_t launch_gp(const CacheArgs& a, int64_t cmp_rows, const void* q, void*
             wt.O = w.Olat;
             qt = w.qlat;
         }
-        e = launch_pdl(kern, dim3(grid), dim3(32 * kConsWarps * kTeams), smem, st, mK, mV, a, qt, wt, nst);
+        e = launch_tokens_tc(a, wt, qt, Gp, st);
         if (e != cudaSuccess)
             return e;
     }
