@@ -786,108 +786,105 @@ __global__ void __launch_bounds__(32 * kConsWarps * NTEAM, 1)
 
 // ==== 3. reference tokens, reference weights, output =========================================
 
+// Chunks of kRefChunk references per CTA of the refs kernel (fewer CTAs, and one set of output
+// reductions per kRefBlock chunks).
+constexpr int kRefBlock = 4;
+
 template <int Gp, int RB, bool LC>
 __global__ void __launch_bounds__(256) mma_refs_kernel(const CacheArgs a, void* __restrict__ out, const MmaWs w)
 {
     constexpr int D = 128;
-    constexpr int RQ = kRefChunk / 4;      // references per thread quarter
+    constexpr int RQ = kRefChunk / 4;      // references per thread quarter and chunk
     __shared__ float wt[kRefChunk][Gp];
     __shared__ float red[4][Gp][D];
     __shared__ float lred[Gp];
     __shared__ uint32_t key[Gp];
     __shared__ int last;
-    const int u = blockIdx.y, ch = blockIdx.x, tid = threadIdx.x;
+    const int u = blockIdx.y, tid = threadIdx.x;
     const UnitMeta um = a.units[u];
     const int R = um.R;
     const int nch = max(1, (R + kRefChunk - 1) / kRefChunk);
-    if (ch >= nch)
+    const int nblk = (nch + kRefBlock - 1) / kRefBlock;
+    if (static_cast<int>(blockIdx.x) >= nblk)
         return;
     const int G = a.G;
     const int kvh = u - um.seq * a.Hkv;
-    const int r0 = ch * kRefChunk, r1 = min(R, r0 + kRefChunk);
     const int cp = tid & 63, qq = tid >> 6;
-    // Before the wait on the tokens kernel: the reference V rows, and what depends only on the
-    // scores kernel (complete once this kernel runs; read through L2): the common offsets,
-    // the reference tokens' own terms p_r and their sum.
-    float rv[RQ][2];
     __shared__ float ssc[RB == 4 ? kRefChunk * (D / 32) : 1];   // int4 store: the chunk's V scales
-    uint32_t cb[RB == 4 ? RQ : 1];
-    if constexpr (RB == 4) {
-        // one code byte (channels 2cp, 2cp+1) per row; the rows' scales staged once per CTA
-        const uint8_t* codes = reinterpret_cast<const uint8_t*>(a.ref_V);
-#pragma unroll
-        for (int rr = 0; rr < RQ; ++rr) {
-            const int r = r0 + qq * RQ + rr;
-            cb[rr] = (r < r1) ? codes[(um.ref_row + r) * (D / 2) + cp] : 0u;
-        }
-        if (tid < kRefChunk * (D / 32)) {
-            const int r = r0 + tid / (D / 32);
-            ssc[tid] = (r < r1) ? __half2float(__ushort_as_half(a.ref_sV[(um.ref_row + r) * (D / 32) + tid % (D / 32)]))
-                                : 0.0f;
-        }
-    } else {
-#pragma unroll
-        for (int rr = 0; rr < RQ; ++rr) {
-            const int r = r0 + qq * RQ + rr;
-            rv[rr][0] = rv[rr][1] = 0.0f;
-            if (r < r1)
-                load_ref<2, RB>(a, 1, um.ref_row + r, 2 * cp, rv[rr]);
-        }
-    }
     if (tid < Gp)
         key[tid] = 0u;
     __syncthreads();
-    if constexpr (RB == 4) {
-#pragma unroll
-        for (int rr = 0; rr < RQ; ++rr) {
-            const float sc = ssc[(qq * RQ + rr) * (D / 32) + cp / 16];
-            rv[rr][0] = __fmul_rn(static_cast<float>(static_cast<int>((cb[rr] & 0xfu) ^ 8u) - 8), sc);
-            rv[rr][1] = __fmul_rn(static_cast<float>(static_cast<int>((cb[rr] >> 4) ^ 8u) - 8), sc);
-        }
-    }
+    // the common offsets depend only on the scores kernel (complete once this kernel runs; read
+    // through L2), so they are folded before the wait on the tokens kernel
     unit_max_fold<Gp>(w, u, R, tid, 256, key);
     __syncthreads();
-    float pj[kRefChunk * Gp / 256 > 0 ? kRefChunk * Gp / 256 : 1];
-    constexpr int PJ = kRefChunk * Gp / 256;
+    float acc[Gp][2];
+#pragma unroll
+    for (int h = 0; h < Gp; ++h)
+        acc[h][0] = acc[h][1] = 0.0f;
     float lsum = 0.0f;
+    constexpr int PJ = kRefChunk * Gp / 256;
+    for (int sc = 0; sc < kRefBlock; ++sc) {
+        const int ch = static_cast<int>(blockIdx.x) * kRefBlock + sc;
+        if (ch >= nch)
+            break;
+        const int r0 = ch * kRefChunk, r1 = min(R, r0 + kRefChunk);
+        // the chunk's reference V rows and the reference tokens' own terms p_r (for the first
+        // chunk before the wait on the tokens kernel)
+        float rv[RQ][2];
+        uint32_t cb[RB == 4 ? RQ : 1];
+        if constexpr (RB == 4) {
+            // one code byte (channels 2cp, 2cp+1) per row; the rows' scales staged once per chunk
+            const uint8_t* codes = reinterpret_cast<const uint8_t*>(a.ref_V);
 #pragma unroll
-    for (int z = 0; z < PJ; ++z) {
-        const int x = tid + 256 * z;
-        const int r = r0 + x / Gp, h = x % Gp;
-        float v = 0.0f;
-        if (r < r1 && h < G)
-            v = exp2f(__ldcg(w.s_tab + (um.ref_row + r) * Gp + h) - unit_m(key, h));
-        pj[z] = v;
-        lsum += v;
-    }
-    // per-head sums: entry x holds head x % Gp (256 % Gp == 0)
+            for (int rr = 0; rr < RQ; ++rr) {
+                const int r = r0 + qq * RQ + rr;
+                cb[rr] = (r < r1) ? codes[(um.ref_row + r) * (D / 2) + cp] : 0u;
+            }
+            if (tid < kRefChunk * (D / 32)) {
+                const int r = r0 + tid / (D / 32);
+                ssc[tid] = (r < r1) ? __half2float(__ushort_as_half(a.ref_sV[(um.ref_row + r) * (D / 32) + tid % (D / 32)]))
+                                    : 0.0f;
+            }
+        } else {
 #pragma unroll
-    for (int o = Gp; o < 32; o <<= 1)
-        lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
-    grid_dep_wait();   // weights and partial sums of the tokens kernel
-    if ((tid & 31) < Gp)
-        (&red[0][0][0])[(tid >> 5) * Gp + (tid & 31)] = lsum;   // scratch: 8 warps x Gp
-    // weight of reference r: its own softmax term p_r plus w_r from the tokens that chose it
+            for (int rr = 0; rr < RQ; ++rr) {
+                const int r = r0 + qq * RQ + rr;
+                rv[rr][0] = rv[rr][1] = 0.0f;
+                if (r < r1)
+                    load_ref<2, RB>(a, 1, um.ref_row + r, 2 * cp, rv[rr]);
+            }
+        }
+        float pj[PJ > 0 ? PJ : 1];
 #pragma unroll
-    for (int z = 0; z < PJ; ++z) {
-        const int x = tid + 256 * z;
-        const int r = r0 + x / Gp, h = x % Gp;
-        wt[x / Gp][h] = (r < r1 && h < G) ? w.W[(um.ref_row + r) * Gp + h] + pj[z] : 0.0f;
-    }
-    __syncthreads();
-    if (tid < Gp) {
-        float v = 0.0f;
-        for (int i = 0; i < 8; ++i)
-            v += red[0][0][i * Gp + tid];
-        lred[tid] = v;
-    }
-    __syncthreads();
-    // sum_r wt[r][h] refV[r][c]: thread (channel pair, quarter of the chunk)
-    {
-        float acc[Gp][2];
+        for (int z = 0; z < PJ; ++z) {
+            const int x = tid + 256 * z;
+            const int r = r0 + x / Gp, h = x % Gp;
+            float v = 0.0f;
+            if (r < r1 && h < G)
+                v = exp2f(__ldcg(w.s_tab + (um.ref_row + r) * Gp + h) - unit_m(key, h));
+            pj[z] = v;
+            lsum += v;
+        }
+        if (sc == 0)
+            grid_dep_wait();   // weights and partial sums of the tokens kernel
+        // weight of reference r: its own softmax term p_r plus w_r from the tokens that chose it
 #pragma unroll
-        for (int h = 0; h < Gp; ++h)
-            acc[h][0] = acc[h][1] = 0.0f;
+        for (int z = 0; z < PJ; ++z) {
+            const int x = tid + 256 * z;
+            const int r = r0 + x / Gp, h = x % Gp;
+            wt[x / Gp][h] = (r < r1 && h < G) ? w.W[(um.ref_row + r) * Gp + h] + pj[z] : 0.0f;
+        }
+        __syncthreads();
+        if constexpr (RB == 4) {
+#pragma unroll
+            for (int rr = 0; rr < RQ; ++rr) {
+                const float scl = ssc[(qq * RQ + rr) * (D / 32) + cp / 16];
+                rv[rr][0] = __fmul_rn(static_cast<float>(static_cast<int>((cb[rr] & 0xfu) ^ 8u) - 8), scl);
+                rv[rr][1] = __fmul_rn(static_cast<float>(static_cast<int>((cb[rr] >> 4) ^ 8u) - 8), scl);
+            }
+        }
+        // sum_r wt[r][h] refV[r][c]: thread (channel pair, quarter of the chunk)
 #pragma unroll
         for (int rr = 0; rr < RQ; ++rr) {
             const float x0 = rv[rr][0], x1 = rv[rr][1];
@@ -898,11 +895,26 @@ __global__ void __launch_bounds__(256) mma_refs_kernel(const CacheArgs a, void* 
                 acc[h][1] = fmaf(wr[h], x1, acc[h][1]);
             }
         }
+        __syncthreads();   // wt and ssc are refilled by the next chunk
+    }
+    // per-head sums: entry x holds head x % Gp (256 % Gp == 0)
 #pragma unroll
-        for (int h = 0; h < Gp; ++h) {
-            red[qq][h][2 * cp] = acc[h][0];
-            red[qq][h][2 * cp + 1] = acc[h][1];
-        }
+    for (int o = Gp; o < 32; o <<= 1)
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+    if ((tid & 31) < Gp)
+        (&red[0][0][0])[(tid >> 5) * Gp + (tid & 31)] = lsum;   // scratch: 8 warps x Gp
+    __syncthreads();
+    if (tid < Gp) {
+        float v = 0.0f;
+        for (int i = 0; i < 8; ++i)
+            v += red[0][0][i * Gp + tid];
+        lred[tid] = v;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < Gp; ++h) {
+        red[qq][h][2 * cp] = acc[h][0];
+        red[qq][h][2 * cp + 1] = acc[h][1];
     }
     __syncthreads();
     for (int x = tid; x < G * D; x += 256) {
@@ -914,7 +926,7 @@ __global__ void __launch_bounds__(256) mma_refs_kernel(const CacheArgs a, void* 
     __threadfence();
     __syncthreads();
     if (tid == 0)
-        last = (atomicAdd(&w.cnt[u], 1u) == static_cast<uint32_t>(nch - 1)) ? 1 : 0;
+        last = (atomicAdd(&w.cnt[u], 1u) == static_cast<uint32_t>(nblk - 1)) ? 1 : 0;
     __syncthreads();
     if (!last)
         return;
@@ -1072,6 +1084,7 @@ cudaError_t launch_gp(const CacheArgs& a, int64_t cmp_rows, const void* q, void*
     if (!code_map(enc, &mK, a.codes_K, cmp_rows) || !code_map(enc, &mV, a.codes_V, cmp_rows))
         return cudaErrorInvalidValue;
     const dim3 rgrid(w.n_chunk, a.n_units);
+    const dim3 fgrid((w.n_chunk + kRefBlock - 1) / kRefBlock, a.n_units);   // refs kernel
     if (a.coder == 1)
         mma_scores_kernel<Gp, 16, true><<<rgrid, 128, 0, st>>>(a, q, w);
     else if (a.ref_bits == 4)
@@ -1095,10 +1108,10 @@ cudaError_t launch_gp(const CacheArgs& a, int64_t cmp_rows, const void* q, void*
             return e;
     }
     if (a.coder == 1)
-        return launch_pdl(mma_refs_kernel<Gp, 16, true>, rgrid, dim3(256), 0, st, a, out, w);
+        return launch_pdl(mma_refs_kernel<Gp, 16, true>, fgrid, dim3(256), 0, st, a, out, w);
     if (a.ref_bits == 4)
-        return launch_pdl(mma_refs_kernel<Gp, 4, false>, rgrid, dim3(256), 0, st, a, out, w);
-    return launch_pdl(mma_refs_kernel<Gp, 16, false>, rgrid, dim3(256), 0, st, a, out, w);
+        return launch_pdl(mma_refs_kernel<Gp, 4, false>, fgrid, dim3(256), 0, st, a, out, w);
+    return launch_pdl(mma_refs_kernel<Gp, 16, false>, fgrid, dim3(256), 0, st, a, out, w);
 }
 
 }  // namespace

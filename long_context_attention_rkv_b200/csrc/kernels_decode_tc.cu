@@ -8,9 +8,10 @@
 //   O      += sum_i p_i sum_g sV_ig codeV_i|g,   W_j += p_i / k_eff (j in S(i)),   L += p_i
 // Persistent, one CTA per SM over a contiguous range of 128-token tiles.  Warps:
 //   0     TMA producer: a tile's int4 codes (K and V, 64-byte swizzle), scales and ordinals
-//         into a 4-stage ring;
-//   1     TMEM allocator and MMA issuer (one thread);
-//   2-9   two teams of four token warps taking alternate tiles; thread = token = TMEM lane.
+//         into a 3-stage ring;
+//   1     TMEM allocator and the K-side MMA issuer (one thread);
+//   2-13  three teams of four token warps taking the tiles in turn; thread = token = TMEM lane;
+//   14    the V-side MMA issuer (one thread).
 // Per tile a team
 //   1. turns its tokens' codes into bf16 (136 + v, exact: the bf16 bit pattern of 128 + the
 //      offset nibble): the K codes straight into TMEM (tcgen05.st, one lane per token), where
@@ -54,16 +55,18 @@ using namespace decode_detail;
 
 constexpr int kD = 128;
 constexpr int kT = 128;                        // tokens per tile (TMEM lanes, MMA M of the K side)
-constexpr int kTeams = 2;
+constexpr int kTeams = 3;
 constexpr int kTokWarps = 4 * kTeams;
-constexpr int kThreads = 64 + 32 * kTokWarps;  // producer, MMA issuer, token warps
+constexpr int kVWarp = 2 + kTokWarps;           // the V-side MMA issuer
+constexpr int kThreads = 96 + 32 * kTokWarps;  // producer, two MMA issuers, token warps
+constexpr int kSyncThreads = 64 + 32 * kTokWarps;   // the issuers and the token warps (named barrier 1)
 constexpr int kCodeRow = 64;                   // bytes of one int4 code row
-constexpr int kNst = 4;                        // ring stages
+constexpr int kNst = 3;                        // ring stages
 constexpr int kStageBytes = 2 * kT * kCodeRow + 2 * kT * 8 + kT * 8 * 2;   // codes, scales, ordinals (k <= 8)
 constexpr uint32_t kNibMask = 0x000F000Fu;
 constexpr uint32_t kNibMagic = 0x43084308u;
 constexpr float kCodeOffset = 136.0f;
-constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kTmemCols = 512;
 
 template <int Gp>
 struct TcLayout {
@@ -92,6 +95,7 @@ struct TcBars {
     uint64_t v_done[kTeams];
     uint64_t dv_full;
     uint64_t done;
+    uint64_t done_v;
     uint32_t tmem_base;
     int abort;
     int issued;
@@ -273,6 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_init(&bars->dv_full, 1);
         mbar_init(&bars->done, 1);
+        mbar_init(&bars->done_v, 1);
         bars->abort = 0;
         bars->issued = 0;
         fence_mbar_init();
@@ -287,9 +292,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
-    const uint32_t tm_ak = tmem;                 // team t: columns 64 t .. 64 t + 63 (K-side A)
-    const uint32_t tm_dk = tmem + 128;           // team t: columns 128 + 32 t (K-side D)
-    const uint32_t tm_dv = tmem + 192;           // V-side D (NV <= 64 columns)
+    const uint32_t tm_ak = tmem;                         // team t: columns 64 t .. 64 t + 63 (K-side A)
+    const uint32_t tm_dk = tmem + 64 * kTeams;           // team t: 32 columns from 64 kTeams + 32 t (K-side D)
+    const uint32_t tm_dv = tmem + 96 * kTeams;           // V-side D (NV <= 64 columns)
 
     if (warp == 0) {
         // ---------------- TMA producer (runs ahead of the scores kernel: codes do not depend on it)
@@ -317,90 +322,67 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         grid_dep_wait();
         grid_dep_launch();
-    } else if (warp == 1) {
-        // ---------------- MMA issuer
+    } else if (warp == 1 || warp == kVWarp) {
+        // ---------------- MMA issuers: warp 1 the K side, warp kVWarp the V side.  Each sleeps on
+        // the barrier of the next tile it serves, so the token warps keep their issue slots.
+        // A tile's K side precedes its V side (the team writes its B operand only after it has
+        // read D_K), and a team converts its next tile only after its previous V side has
+        // completed (v_done); the V sides go in tile order, the first of a unit clearing D_V.
         grid_dep_wait();
         grid_dep_launch();
+        const bool kside = warp == 1;
         constexpr uint32_t idescK = idesc_bf16_f32(kT, NK);
         constexpr uint32_t idescV = idesc_bf16_f32(kT, NV) | (1u << 15) | (1u << 16);   // A and B MN-major
         bool issued_any = false;
-        int t = t_lo, seg = 0;
+        int t = t_lo;
         int u = unit_after(a, 0, t_lo, lane);
         while (t < t_hi && u < a.n_units) {
             const int seg_end = min(t_hi, unit_end_tile(a, u));
-            named_sync(1, 32 + 32 * kTokWarps);   // A: the previous unit is read out
-            named_sync(1, 32 + 32 * kTokWarps);   // B: this unit's query block is in shared memory
+            named_sync(1, kSyncThreads);   // A: the previous unit is read out
+            named_sync(1, kSyncThreads);   // B: this unit's query block is in shared memory
             if (lane == 0) {
-                // Issue whichever side is ready: the K side of the next tile (its team has its
-                // codes in place) or the V side of the oldest tile whose B operand is written, so
-                // that neither team waits on the other's progress.  V sides go in tile order (the
-                // first of the unit clears the accumulator); a tile's K side always precedes its V
-                // side, and a team's next codes come only after its previous V side (v_done), so
-                // every wait below is on work that is already issued or under way.
                 const uint32_t bkb = smem_addr(sm + L::bk);
-                int kq = t, vq = t;
-                uint64_t t0 = 0;
-                uint32_t polls = 0;
-                while (vq < seg_end && !*abort) {
-                    bool did = false;
-                    if (kq < seg_end) {
-                        const int li = kq - t_lo, tm = li & 1;
-                        if (mbar_try_wait(&bars->a_ready[tm], (li >> 1) & 1)) {
-                            tc_fence_after();
-#pragma unroll
-                            for (int kk = 0; kk < kD / 16; ++kk)
-                                mma_f16_ts(tm_dk + 32 * tm, tm_ak + 64 * tm + 8 * kk,
-                                           smem_desc_sw128(bkb + (kk / 4) * (NK * 128) + (kk % 4) * 32), idescK,
-                                           kk > 0 ? 1u : 0u);
-                            mma_commit(&bars->k_done[tm]);
-                            issued_any = true;
-                            ++kq;
-                            did = true;
-                        }
-                    }
-                    if (vq < kq) {
-                        const int li = vq - t_lo, tm = li & 1;
-                        if (mbar_try_wait(&bars->p_ready[tm], (li >> 1) & 1)) {
-                            tc_fence_after();
-                            const uint32_t av = smem_addr(sm + L::vtile + tm * 32768);
-                            const uint32_t bvb = smem_addr(sm + L::bv + tm * (kT * NV * 2));
-#pragma unroll
-                            for (int kk = 0; kk < kT / 16; ++kk)
-                                mma_f16(tm_dv, smem_desc(av + kk * 2048, 16384, 1024, 2),
-                                        smem_desc(bvb + kk * 256, 128, 2048, 0), idescV,
-                                        (vq > t || kk > 0) ? 1u : 0u);
-                            mma_commit(&bars->v_done[tm]);
-                            ++vq;
-                            did = true;
-                        }
-                    }
-                    if (did) {
-                        t0 = 0;
-                        polls = 0;
-                    } else if ((++polls & 255u) == 0) {
-                        // bounded: a pipeline that makes no progress for 2 s gives up
-                        const uint64_t now = global_ns();
-                        if (t0 == 0) {
-                            t0 = now;
-                        } else if (now - t0 > kWaitNs) {
+                for (int i = t; i < seg_end && !*abort; ++i) {
+                    const int li = i - t_lo, tm = li % kTeams;
+                    uint64_t* bar = kside ? &bars->a_ready[tm] : &bars->p_ready[tm];
+                    if (!mbar_wait_sleep(bar, (li / kTeams) & 1, abort)) {
+                        if (!*abort)
                             report(a.err, RKV_ERR_TIMEOUT);
-                            *abort = 1;
-                        }
+                        *abort = 1;
+                        break;
                     }
+                    tc_fence_after();
+                    if (kside) {
+#pragma unroll
+                        for (int kk = 0; kk < kD / 16; ++kk)
+                            mma_f16_ts(tm_dk + 32 * tm, tm_ak + 64 * tm + 8 * kk,
+                                       smem_desc_sw128(bkb + (kk / 4) * (NK * 128) + (kk % 4) * 32), idescK,
+                                       kk > 0 ? 1u : 0u);
+                        mma_commit(&bars->k_done[tm]);
+                    } else {
+                        const uint32_t av = smem_addr(sm + L::vtile + tm * 32768);
+                        const uint32_t bvb = smem_addr(sm + L::bv + tm * (kT * NV * 2));
+#pragma unroll
+                        for (int kk = 0; kk < kT / 16; ++kk)
+                            mma_f16(tm_dv, smem_desc(av + kk * 2048, 16384, 1024, 2),
+                                    smem_desc(bvb + kk * 256, 128, 2048, 0), idescV, (i > t || kk > 0) ? 1u : 0u);
+                        mma_commit(&bars->v_done[tm]);
+                    }
+                    issued_any = true;
                 }
-                if (!*abort)
+                if (!kside && !*abort)
                     mma_commit(&bars->dv_full);
             }
             __syncwarp();
             t = seg_end;
             u = unit_after(a, u, t, lane);
-            ++seg;
         }
         if (lane == 0 && issued_any) {
-            // every MMA of this CTA has completed before TMEM is released
+            // every MMA this thread issued has completed before TMEM is released
             volatile int never = 0;
-            mma_commit(&bars->done);
-            mbar_wait(&bars->done, 0, &never);
+            uint64_t* done = kside ? &bars->done : &bars->done_v;
+            mma_commit(done);
+            mbar_wait(done, 0, &never);
         }
     } else {
         // ---------------- token warps: thread = token of the tile = TMEM lane
@@ -420,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const UnitMeta um = a.units[u];
             const int seg_end = min(t_hi, unit_end_tile(a, u));
             const int kvh = u - um.seq * a.Hkv;
-            named_sync(1, 32 + 32 * kTokWarps);   // A
+            named_sync(1, kSyncThreads);   // A
             // ---- unit setup: query, query block (K-major, 128-byte swizzle), offsets
             if (tt < Gp)
                 key_sm[tt] = 0u;
@@ -463,7 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             named_sync(2, 32 * kTokWarps);
             if (tt < Gp)
                 m_sm[tt] = unit_m(key_sm, tt);
-            named_sync(1, 32 + 32 * kTokWarps);   // B
+            named_sync(1, kSyncThreads);   // B
             float qc[NK], mh[Gp], lsum[Gp];
 #pragma unroll
             for (int n = 0; n < NK; ++n)
@@ -478,8 +460,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int R = um.R;
 
             // ---- this team's tiles of the unit
-            for (int i = t + ((t - t_lo) & 1 ? (tm ^ 1) : tm); i < seg_end; i += kTeams) {
-                const int li = i - t_lo, s = li % kNst, use = li >> 1;
+            for (int i = t + (tm - (t - t_lo) % kTeams + kTeams) % kTeams; i < seg_end; i += kTeams) {
+                const int li = i - t_lo, s = li % kNst, use = li / kTeams;
                 bool ok = !*abort;
                 if (ok && use > 0 && !mbar_wait_sleep(&bars->v_done[tm], (use - 1) & 1, abort))
                     ok = false;
