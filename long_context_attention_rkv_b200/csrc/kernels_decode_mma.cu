@@ -786,12 +786,13 @@ __global__ void __launch_bounds__(32 * kConsWarps * NTEAM, 1)
 
 // ==== 3. reference tokens, reference weights, output =========================================
 
-// Chunks of kRefChunk references per CTA of the refs kernel (fewer CTAs, and one set of output
-// reductions per kRefBlock chunks).
-constexpr int kRefBlock = 4;
+// Chunks of kRefChunk references per CTA of the refs kernel.  One: the kernel is bound by the
+// latency of each CTA's chain of dependent loads, so more CTAs in flight beat fewer, longer ones
+// (four chunks per CTA measured slower on every workload).
+constexpr int kRefBlock = 1;
 
 template <int Gp, int RB, bool LC>
-__global__ void __launch_bounds__(256) mma_refs_kernel(const CacheArgs a, void* __restrict__ out, const MmaWs w)
+__global__ void __launch_bounds__(256, 4) mma_refs_kernel(const CacheArgs a, void* __restrict__ out, const MmaWs w)
 {
     constexpr int D = 128;
     constexpr int RQ = kRefChunk / 4;      // references per thread quarter and chunk

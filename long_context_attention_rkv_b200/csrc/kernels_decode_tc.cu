@@ -519,6 +519,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     convert_half(st, tok, hf, wk);
                     tmem_st32(tm_ak + 64 * tm + 32 * hf + lane_off, wk);
                 }
+                // the K side can start: its A operand is in TMEM
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(&bars->a_ready[tm]);
+                // V codes while the K-side MMAs run (made visible to the tensor cores by the fence
+                // before p_ready)
                 // V: pair words 32 hf .. 32 hf + 31 are MMA slots 64 hf .. 64 hf + 63, the
                 // 64-slot MN block hf of the tile (eight 16-byte chunks of this token's row)
                 unsigned char* vt = sm + L::vtile + tm * 32768 + (tok >> 3) * 1024 + (tok & 7) * 128;
@@ -540,10 +546,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 const uint2 skw = *reinterpret_cast<const uint2*>(st + 2 * kT * kCodeRow + tok * 8);
                 const uint2 svw = *reinterpret_cast<const uint2*>(st + 2 * kT * kCodeRow + kT * 8 + tok * 8);
-                fence_proxy_async_smem();
-                tmem_st_wait();
-                tc_fence_before();
-                mbar_arrive(&bars->a_ready[tm]);
                 mbar_arrive(&bars->empty[s]);
 
                 // 2. the mean reference score of each head
