@@ -179,6 +179,12 @@ class ClockSampler:
                 "reasons": sorted(seen), "samples": len(mhz)}
 
 
+DECODE_SRC = ["long_context_attention_rkv_b200/csrc/kernels_decode_mma.cu",
+              "long_context_attention_rkv_b200/csrc/kernels_decode_tc.cu",
+              "long_context_attention_rkv_b200/csrc/decode_mma.h"]
+ENCODE_SRC = ["long_context_attention_rkv_b200/csrc/kernels_encode.cu"]
+
+
 def _src_sha(paths):
     h = hashlib.sha256()
     for p in paths:
@@ -188,15 +194,15 @@ def _src_sha(paths):
 
 
 def _traffic(kernel: str, src: list[str], workload: str):
-    """Per-launch DRAM bytes of a kernel from a committed ncu summary, if it was captured on
-    this workload and on the current source."""
+    """Per-launch DRAM bytes of a kernel on a workload from the committed ncu summary, if
+    they were captured (or scaled from a capture) on the current source."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         t = json.load(f)
-    e = t.get(kernel)
-    if not e or e.get("src_sha") != _src_sha(src) or e.get("workload") != workload:
+    e = t.get(kernel, {}).get(workload)
+    if not e or e.get("src_sha") != _src_sha(src):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -911,10 +917,10 @@ def run_ours(args, rank, world, local_rank):
         traffic = _traffic(kern, ["long_context_attention_rkv_b200/csrc/kernels_%s.cu" % kern], wl.name)
     elif dominant == "encode":
         peak, bound, unit, ach = peaks["hbm"], "hbm", "GB/s", head["encode_gbs"]
-        traffic = _traffic("encode", ["long_context_attention_rkv_b200/csrc/kernels_encode.cu"], wl.name)
+        traffic = _traffic("encode", ENCODE_SRC, wl.name)
     else:
         peak, bound, unit, ach = peaks["hbm"], "hbm", "GB/s", head["decode_hbm_gbs"]
-        traffic = _traffic("decode", ["long_context_attention_rkv_b200/csrc/kernels_decode_mma.cu"], wl.name)
+        traffic = _traffic("decode", DECODE_SRC, wl.name)
     roofline = {"kernel": dominant, "bound": bound, "achieved": ach, "peak": peak, "unit": unit, "frac": ach / peak,
                 "traffic": traffic, "peak_source": peaks["source"] + (" sustained" if bound == "tensor" else ""),
                 "frac_of_burst_peak": (ach / peaks["bf16"]) if bound == "tensor" else None,

@@ -18,11 +18,12 @@
 //
 // Persistent kernel, one CTA per SM, warp-specialised:
 //   warp 0      TMA producer (no multicast): both position tiles of an item
-//               (128-byte swizzle) and a 3-stage ring of reference tiles plus their
+//               (128-byte swizzle) and a 2-stage ring of reference tiles plus their
 //               augmented block (32-byte swizzle); L2 prefetch of the next item
 //   warp 1      TMEM allocator and MMA issuer (one thread)
-//   warps 2-9   epilogue: warp (quarter q, tile a) owns TMEM lanes 32q..32q+31 of
-//               tile a, one position per thread
+//   warps 2-17  epilogue: warps (quarter q, tile a, half h) read TMEM lanes 32q..32q+31
+//               of tile a, columns 64h .. 64h+63 of every reference tile: two threads
+//               per position
 // Two accumulator sets (2 tiles x 128 columns each) let the MMAs of the next
 // reference tile overlap the epilogue of the previous one.
 //
@@ -36,7 +37,8 @@
 //
 // Every wait is bounded; a wait that gives up records RKV_ERR_TIMEOUT, the CTA
 // winds down (waiting, again bounded, for its own copies and MMAs) and frees its
-// TMEM.
+// TMEM.  The pipeline waits sleep in the barrier (a suspend-time hint) instead of
+// polling, so a waiting role leaves its scheduler's issue slots to the epilogue.
 #include <cudaTypedefs.h>
 
 #include <cfloat>
@@ -54,12 +56,15 @@ using namespace sm100;
 constexpr int kM = 128;           // positions per tile = TMEM lanes
 constexpr int kTiles = 2;         // position tiles per work item
 constexpr int kN = 128;           // references per stage = TMEM columns per accumulator
-constexpr int kStagesB = 3;
+constexpr int kStagesB = 2;
 constexpr int kAcc = 2;           // accumulator sets (each kTiles x kN columns)
-constexpr int kEpiWarps = 4 * kTiles;
+constexpr int kHalves = 2;        // column halves of a reference tile (a position's two threads)
+constexpr int kHalfCols = kN / kHalves;
+constexpr int kEpiWarps = 4 * kTiles * kHalves;
 constexpr int kEpiThreads = 32 * kEpiWarps;
+constexpr int kPairs = kEpiWarps / kHalves;   // warp pairs sharing a set of positions
 constexpr int kThreads = 64 + kEpiThreads;
-constexpr int kQC = 24;           // queue entries per epilogue thread
+constexpr int kQC = 20;           // queue entries per epilogue thread (>= 16 + 4, and >= KC)
 constexpr uint32_t kTmemCols = kAcc * kTiles * kN;  // 512
 
 template <int D>
@@ -71,7 +76,8 @@ struct Layout {
     static constexpr uint32_t b_off = a_off + kTiles * a_tile;
     static constexpr uint32_t aaug_off = b_off + kStagesB * b_stage;
     static constexpr uint32_t q_off = aaug_off + kM * 32;
-    static constexpr uint32_t bar_off = q_off + kQC * kEpiThreads * 8;
+    static constexpr uint32_t thr_off = q_off + kQC * kEpiThreads * 8;       // [kHalves][kTiles * kM]
+    static constexpr uint32_t bar_off = thr_off + kHalves * kTiles * kM * 4;
     static constexpr uint32_t total = bar_off + 256;
     static constexpr uint32_t alloc = total + 1024;  // slack for 1024-byte alignment
     static_assert(b_stage % 1024 == 0 && a_tile % 1024 == 0, "stage alignment");
@@ -85,6 +91,7 @@ struct Bars {
     uint64_t acc_full[kAcc];
     uint64_t acc_empty[kAcc];
     uint64_t done;
+    uint64_t pair[kPairs];
     uint32_t tmem_base;
     int abort;
 };
@@ -173,6 +180,30 @@ __device__ __forceinline__ void block_maxima(uint32_t col, int j0, int ncand, fl
     }
 }
 
+// Maxima of the kHalfCols / 16 blocks of 16 columns starting at TMEM column col (this thread's
+// row); columns j0 + c at or past ncand count as -inf.
+__device__ __forceinline__ void half_maxima(uint32_t col, int j0, int ncand, float* mx)
+{
+#pragma unroll
+    for (int c0 = 0; c0 < kHalfCols; c0 += 32) {
+        float v[32];
+        tmem_ld32(col + c0, v);
+        if (j0 + c0 + 32 > ncand) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                v[i] = (j0 + c0 + i < ncand) ? v[i] : -FLT_MAX;
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const float* b = v + 16 * h;
+            const float m0 = fmax3(b[0], b[1], b[2]), m1 = fmax3(b[3], b[4], b[5]);
+            const float m2 = fmax3(b[6], b[7], b[8]), m3 = fmax3(b[9], b[10], b[11]);
+            const float m4 = fmax3(b[12], b[13], b[14]);
+            mx[c0 / 16 + h] = fmax3(fmax3(m0, m1, m2), fmax3(m3, m4, b[15]), -FLT_MAX);
+        }
+    }
+}
+
 // Sorts 16 values in descending order (bitonic network).
 __device__ __forceinline__ void sort16_desc(float (&x)[16])
 {
@@ -219,6 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* sB = smem + L::b_off;
     uint8_t* sAaug = smem + L::aaug_off;
     float2* sQ = reinterpret_cast<float2*>(smem + L::q_off);
+    float* sThr = reinterpret_cast<float*>(smem + L::thr_off);
     Bars* bars = reinterpret_cast<Bars*>(smem + L::bar_off);
     volatile int* abort = &bars->abort;
 
@@ -237,6 +269,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bars->acc_empty[s], kEpiThreads);
         }
         mbar_init(&bars->done, 1);
+        for (int s = 0; s < kPairs; ++s)
+            mbar_init(&bars->pair[s], 64);
         bars->abort = 0;
         fence_mbar_init();
         prefetch_tensormap(&tmA);
@@ -269,14 +303,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             uint32_t it_b = 0, ni = 0;
             int last_a = -1;
-            int last_b[kStagesB] = {-1, -1, -1};
+            int last_b[kStagesB];
+            for (int s = 0; s < kStagesB; ++s)
+                last_b[s] = -1;
             bool ok = true;
             for (int rnd = 0, w = item_of(0); w < n_items && ok; w = item_of(++rnd)) {
                 const Tile it = items[w];
                 const UnitMeta um = a.units[it.unit];
                 const int p0 = it.tile * kTiles * kM;
                 const int nrt = (item_candidates(a, um, p0) + kN - 1) / kN;
-                if (!(ok = mbar_wait(&bars->empty_a, (ni & 1) ^ 1, abort)))
+                if (!(ok = mbar_wait_sleep(&bars->empty_a, (ni & 1) ^ 1, abort)))
                     break;
                 mbar_arrive_expect_tx(&bars->full_a, kTiles * L::a_tile);
                 const int row0 = it.unit * a.max_len + p0;
@@ -299,7 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 for (int r = 0; r < nrt; ++r) {
                     const int sb = it_b % kStagesB;
-                    if (!(ok = mbar_wait(&bars->empty_b[sb], ((it_b / kStagesB) & 1) ^ 1, abort)))
+                    if (!(ok = mbar_wait_sleep(&bars->empty_b[sb], ((it_b / kStagesB) & 1) ^ 1, abort)))
                         break;
                     mbar_arrive_expect_tx(&bars->full_b[sb], L::b_stage);
                     const int rrow = static_cast<int>(um.ref_row) + r * kN;
@@ -336,16 +372,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const Tile it = items[w];
                 const UnitMeta um = a.units[it.unit];
                 const int nrt = (item_candidates(a, um, it.tile * kTiles * kM) + kN - 1) / kN;
-                if (!(ok = mbar_wait(&bars->full_a, ni & 1, abort)))
+                if (!(ok = mbar_wait_sleep(&bars->full_a, ni & 1, abort)))
                     break;
                 tc_fence_after();
                 const uint32_t a_base = smem_addr(sA);
                 for (int r = 0; r < nrt; ++r) {
                     const int sb = it_b % kStagesB;
                     const int acc = it_c % kAcc;
-                    if (!(ok = mbar_wait(&bars->full_b[sb], (it_b / kStagesB) & 1, abort)))
+                    if (!(ok = mbar_wait_sleep(&bars->full_b[sb], (it_b / kStagesB) & 1, abort)))
                         break;
-                    if (!(ok = mbar_wait(&bars->acc_empty[acc], ((it_c / kAcc) & 1) ^ 1, abort)))
+                    if (!(ok = mbar_wait_sleep(&bars->acc_empty[acc], ((it_c / kAcc) & 1) ^ 1, abort)))
                         break;
                     tc_fence_after();
                     const uint32_t b_base = smem_addr(sB + sb * L::b_stage);
@@ -386,17 +422,38 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else {
-        // ---------------- epilogue: one position per thread ----------------
+        // ---------------- epilogue: a position per pair of threads ----------------
+        // Warps e and e + kPairs read the same TMEM lanes (positions) of the same tile, the first
+        // columns 0 .. 63 of every reference tile, the second 64 .. 127.  Each keeps its own
+        // sorted list and queue; they share a threshold (the larger of their kc-th best values
+        // is a lower bound of the position's kc-th best, so either may filter with it), combine
+        // their seeds, and merge their lists at the end of the item.  Pairs synchronise on an
+        // mbarrier of their own (bounded waits).
         const int e = warp - 2;                  // 0 .. kEpiWarps-1
         const int q = warp & 3;                  // TMEM lane quarter this warp may access
-        const int t = e >> 2;                    // position tile of the item
+        const int pi = e % kPairs;               // pair
+        const int hf = e / kPairs;               // column half
+        const int t = pi >> 2;                   // position tile of the item
         const int row = q * 32 + lane;
+        const int trow = t * kM + row;
         const int qi = e * 32 + lane;            // queue column of this thread
         float2* myq = sQ + qi;
+        const float2* otherq = sQ + ((e ^ kPairs) * 32 + lane);   // the partner's queue column
+        volatile float* thr_own = sThr + hf * (kTiles * kM) + trow;
+        volatile float* thr_oth = sThr + (hf ^ 1) * (kTiles * kM) + trow;
+        const int cb = hf * kHalfCols;           // first column of this thread's half
         const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-        uint32_t it_c = 0;
+        uint32_t it_c = 0, pph = 0;
         bool ok = true;
-        for (int rnd = 0, w = item_of(0); w < n_items && ok; w = item_of(++rnd)) {
+        auto pair_sync = [&]() {
+            mbar_arrive(&bars->pair[pi]);
+            if (!mbar_wait_sleep(&bars->pair[pi], pph & 1, abort))
+                ok = false;
+            ++pph;
+        };
+        // (no early exit from the item loop: after a wait gives up every later wait returns at
+        // once, and both threads of a pair still take the same synchronisations)
+        for (int rnd = 0, w = item_of(0); w < n_items; w = item_of(++rnd)) {
             const Tile it = items[w];
             const UnitMeta um = a.units[it.unit];
             const int p0 = it.tile * kTiles * kM;
@@ -413,64 +470,54 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ti[s] = 0x7fffffff;
             }
             int cnt = 0;
-            float seed = -FLT_MAX;   // lower bound of the kc-th best t (from sub-block maxima)
             float seed_lo = -FLT_MAX;
+            *thr_own = -FLT_MAX;
+            pair_sync();   // both halves start the item with no threshold
             for (int r = 0; r < nrt; ++r) {
                 const int acc = it_c % kAcc;
                 // one lane waits, the warp follows: the TMEM loads below are warp-collective
                 int got = 1;
                 if (lane == 0)
-                    got = mbar_wait(&bars->acc_full[acc], (it_c / kAcc) & 1, abort) ? 1 : 0;
+                    got = (ok && mbar_wait_sleep(&bars->acc_full[acc], (it_c / kAcc) & 1, abort)) ? 1 : 0;
                 ok = __shfl_sync(0xffffffffu, got, 0) != 0;
-                if (!ok)
-                    break;
                 tc_fence_after();
-                const int j0 = r * kN;
-                const uint32_t col0 = lane_base + (acc * kTiles + t) * kN;
+                const int j0 = r * kN + cb;
+                const uint32_t col0 = lane_base + (acc * kTiles + t) * kN + cb;
                 if (r == 0 && nrt >= 2 && KC <= 16) {
                     // the KC-th largest of the sixteen block maxima of the first two reference
-                    // tiles (distinct elements) bounds the kc-th best t from below; the first
-                    // tile stays in TMEM while the second is read, and is scanned after
+                    // tiles (distinct elements; eight from each half) bounds the kc-th best t
+                    // from below; the first tile stays in TMEM while the second is read
                     float mx[16];
-                    block_maxima(col0, 0, ncand, mx);
                     const int acc1 = (it_c + 1) % kAcc;
                     int got1 = 1;
                     if (lane == 0)
-                        got1 = mbar_wait(&bars->acc_full[acc1], ((it_c + 1) / kAcc) & 1, abort) ? 1 : 0;
+                        got1 = (ok && mbar_wait_sleep(&bars->acc_full[acc1], ((it_c + 1) / kAcc) & 1, abort)) ? 1 : 0;
                     ok = __shfl_sync(0xffffffffu, got1, 0) != 0;
-                    if (!ok)
-                        break;
                     tc_fence_after();
-                    block_maxima(lane_base + (acc1 * kTiles + t) * kN, kN, ncand, mx + 8);
-                    sort16_desc(mx);
-                    seed = mx[KC - 1];
-                    seed_lo = (seed > -FLT_MAX) ? nextafterf(seed, -FLT_MAX) : -FLT_MAX;
-                } else if (r == 0 && nc_max >= kN && KC <= kN / 16) {
-                    // the kc largest of kN/16 sub-block maxima are distinct elements, so the
-                    // smallest of them bounds the kc-th best t from below
-                    float mxs[kN / 16];
+                    if (ok) {
+                        half_maxima(col0, j0, ncand, mx);
+                        half_maxima(lane_base + (acc1 * kTiles + t) * kN + cb, j0 + kN, ncand, mx + 4);
+                    } else {
 #pragma unroll
-                    for (int c0 = 0; c0 < kN; c0 += 32) {
-                        float v[32];
-                        tmem_ld32(col0 + c0, v);
-#pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            float m = -FLT_MAX;
-#pragma unroll
-                            for (int i = 0; i < 16; ++i)
-                                m = fmaxf(m, (c0 + h * 16 + i < ncand) ? v[h * 16 + i] : -FLT_MAX);
-                            mxs[c0 / 16 + h] = m;
-                        }
+                        for (int i = 0; i < 8; ++i)
+                            mx[i] = -FLT_MAX;
                     }
-                    // kc-th largest of the maxima (kc <= 8 = kN/16: the minimum when kc == 8)
-                    float lo = FLT_MAX;
 #pragma unroll
-                    for (int i = 0; i < kN / 16; ++i)
-                        lo = fminf(lo, mxs[i]);
-                    seed = (KC == kN / 16) ? lo : -FLT_MAX;
+                    for (int i = 0; i < 4; ++i)
+                        myq[i * kEpiThreads] = make_float2(mx[2 * i], mx[2 * i + 1]);
+                    pair_sync();
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float2 o = otherq[i * kEpiThreads];
+                        mx[8 + 2 * i] = o.x;
+                        mx[8 + 2 * i + 1] = o.y;
+                    }
+                    pair_sync();   // the partner has read this thread's maxima (the queue is reused)
+                    sort16_desc(mx);
+                    const float seed = mx[KC - 1];
                     seed_lo = (seed > -FLT_MAX) ? nextafterf(seed, -FLT_MAX) : -FLT_MAX;
                 }
-                for (int c0 = 0; c0 < kN && j0 + c0 < nc_max; c0 += 32) {
+                for (int c0 = 0; ok && c0 < kHalfCols && j0 + c0 < nc_max; c0 += 32) {
                     float v[32];
                     tmem_ld32(col0 + c0, v);
                     if (j0 + c0 + 32 > ncand) {
@@ -483,10 +530,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (__any_sync(0xffffffffu, cnt > kQC - 16)) {
                             drain<KC>(myq, cnt, tv, ti);
                             cnt = 0;
+                            *thr_own = tv[KC - 1];
                         }
                         // one compare per element: seed_lo is just below the seed, so the element
-                        // that defines the seed is still appended
-                        const float thr = fmaxf(tv[KC - 1], seed_lo);
+                        // that defines the seed is still appended; the partner's kc-th best
+                        // bounds this position's kc-th best as well
+                        const float thr = fmax3(tv[KC - 1], seed_lo, *thr_oth);
                         int o = cnt * kEpiThreads;
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
@@ -500,23 +549,36 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_before();
                 mbar_arrive(&bars->acc_empty[acc]);
                 ++it_c;
-                // (queues drain only when one could overflow, and at the end of the item:
-                // draining at every reference-tile boundary as well measured slower)
             }
-            if (!ok)
-                break;
-            drain<KC>(myq, cnt, tv, ti);
-            order_ties<KC>(tv, ti);
-            if (valid) {
-                const int64_t orow = um.cmp_row + (p - ncand);
-                const int nv = min(KC, ncand);
+            if (ok)
+                drain<KC>(myq, cnt, tv, ti);
+            // merge: the second half hands its list over through its queue column (KC <= kQC)
+            if (hf == 1) {
+#pragma unroll
+                for (int s = 0; s < KC; ++s)
+                    myq[s * kEpiThreads] = make_float2(tv[s], __int_as_float(ti[s]));
+            }
+            pair_sync();
+            if (hf == 0) {
 #pragma unroll
                 for (int s = 0; s < KC; ++s) {
-                    cand_idx[orow * KC + s] = (s < nv) ? static_cast<uint16_t>(ti[s])
-                                                       : static_cast<uint16_t>(RKV_IDX_UNUSED);
-                    cand_t[orow * KC + s] = (s < nv) ? tv[s] : -FLT_MAX;
+                    const float2 x = otherq[s * kEpiThreads];
+                    if (x.x > tv[KC - 1])
+                        topk_insert<KC>(tv, ti, x.x, __float_as_int(x.y));
+                }
+                order_ties<KC>(tv, ti);
+                if (valid && ok) {
+                    const int64_t orow = um.cmp_row + (p - ncand);
+                    const int nv = min(KC, ncand);
+#pragma unroll
+                    for (int s = 0; s < KC; ++s) {
+                        cand_idx[orow * KC + s] = (s < nv) ? static_cast<uint16_t>(ti[s])
+                                                           : static_cast<uint16_t>(RKV_IDX_UNUSED);
+                        cand_t[orow * KC + s] = (s < nv) ? tv[s] : -FLT_MAX;
+                    }
                 }
             }
+            pair_sync();   // the second half's column is free again
         }
         if (!ok) {
             *abort = 1;
