@@ -25,6 +25,7 @@ struct MmaWs {
     int n_chunk;
     int n_tiles;
     int n_cta;        // CTAs of the tokens kernel
+    int ref_blk;      // 64-reference chunks per CTA of the refs kernel
     float cK;         // log2(e) / sqrt(D)
 };
 

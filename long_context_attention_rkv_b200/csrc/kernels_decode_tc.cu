@@ -15,8 +15,9 @@
 // Per tile a team
 //   1. turns its tokens' codes into bf16 (136 + v, exact: the bf16 bit pattern of 128 + the
 //      offset nibble): the K codes straight into TMEM (tcgen05.st, one lane per token), where
-//      they are the A operand of the K-side product, the V codes into shared memory as the
-//      MN-major A operand of the V side;
+//      they are the A operand of the K-side product, then, once its previous tile's V-side
+//      MMAs have completed (at Gp 8 the team waits for them before the K codes), the V codes
+//      into shared memory as the MN-major A operand of the V side;
 //   2. the MMA thread forms D_K[token][(head, group)] = codes x qblock, M 128, N 4 Gp, K 128,
 //      with qblock the query split by scale group (block-diagonal, bf16, exact);
 //   3. each thread turns its D_K row into the logits, p, the reference weights (vector
@@ -242,6 +243,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 {
     using L = TcLayout<Gp>;
     constexpr int NK = L::NK, NV = L::NV;
+    // K conversion of a tile before the wait for the team's previous V side (Gp 4; at Gp 8 the
+    // values it keeps live across that wait spill)
+    constexpr bool kEarlyK = Gp == 4;
     extern __shared__ unsigned char tc_smem_raw[];
     const uint32_t raw_addr = smem_addr(tc_smem_raw);
     unsigned char* sm = tc_smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
@@ -463,7 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = t + (tm - (t - t_lo) % kTeams + kTeams) % kTeams; i < seg_end; i += kTeams) {
                 const int li = i - t_lo, s = li % kNst, use = li / kTeams;
                 bool ok = !*abort;
-                if (ok && use > 0 && !mbar_wait_sleep(&bars->v_done[tm], (use - 1) & 1, abort))
+                if (!kEarlyK && ok && use > 0 && !mbar_wait_sleep(&bars->v_done[tm], (use - 1) & 1, abort))
                     ok = false;
                 if (ok && !mbar_wait_sleep(&bars->full[s], (li / kNst) & 1, abort))
                     ok = false;
@@ -523,6 +527,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(&bars->a_ready[tm]);
+                // the team's previous V-side MMAs read its V tile and B operand: they complete
+                // before either is rewritten (with kEarlyK the K side above overlapped them)
+                if constexpr (kEarlyK) {
+                    const bool vd = use == 0 || mbar_wait_sleep(&bars->v_done[tm], (use - 1) & 1, abort);
+                    if (!vd) {
+                        if (!*abort)
+                            report(a.err, RKV_ERR_TIMEOUT);
+                        *abort = 1;
+                    }
+                    if (!__all_sync(0xffffffffu, vd))
+                        continue;
+                }
                 // V codes while the K-side MMAs run (made visible to the tensor cores by the fence
                 // before p_ready)
                 // V: pair words 32 hf .. 32 hf + 31 are MMA slots 64 hf .. 64 hf + 63, the

@@ -27,13 +27,12 @@
 // Two accumulator sets (2 tiles x 128 columns each) let the MMAs of the next
 // reference tile overlap the epilogue of the previous one.
 //
-// Top-kc per position (ties to the lower ordinal): each thread appends, without
-// branching, every t above its current threshold to a private queue in shared
-// memory; when any lane's queue could overflow, and at the end of an item, the warp
-// drains all queues in lockstep into the sorted per-thread lists, which raises the
-// thresholds.  This
-// keeps the per-element cost at a compare and a store, and the sorted
-// insertions coherent across the warp.
+// Top-kc per position (ties to the lower ordinal): per 32 columns a thread forms the bit
+// mask of the t above its threshold (one subtraction and one funnel shift per element: the
+// sign bit of threshold - t), and only the set bits are inserted, in column order, into its
+// sorted list in registers (the chunk's values parked in the thread's own shared-memory
+// slots so that a set bit can fetch its value).  Most chunks of a row hold no t above the
+// threshold, so the per-element cost is the two instructions of the mask.
 //
 // Every wait is bounded; a wait that gives up records RKV_ERR_TIMEOUT, the CTA
 // winds down (waiting, again bounded, for its own copies and MMAs) and frees its
@@ -64,7 +63,7 @@ constexpr int kEpiWarps = 4 * kTiles * kHalves;
 constexpr int kEpiThreads = 32 * kEpiWarps;
 constexpr int kPairs = kEpiWarps / kHalves;   // warp pairs sharing a set of positions
 constexpr int kThreads = 64 + kEpiThreads;
-constexpr int kQC = 20;           // queue entries per epilogue thread (>= 16 + 4, and >= KC)
+constexpr int kSlots = 10;        // 16-byte shared-memory slots per epilogue thread (>= 8, >= KC / 2)
 constexpr uint32_t kTmemCols = kAcc * kTiles * kN;  // 512
 
 template <int D>
@@ -76,12 +75,13 @@ struct Layout {
     static constexpr uint32_t b_off = a_off + kTiles * a_tile;
     static constexpr uint32_t aaug_off = b_off + kStagesB * b_stage;
     static constexpr uint32_t q_off = aaug_off + kM * 32;
-    static constexpr uint32_t thr_off = q_off + kQC * kEpiThreads * 8;       // [kHalves][kTiles * kM]
+    static constexpr uint32_t thr_off = q_off + kSlots * kEpiThreads * 16;   // [kHalves][kTiles * kM]
     static constexpr uint32_t bar_off = thr_off + kHalves * kTiles * kM * 4;
     static constexpr uint32_t total = bar_off + 256;
     static constexpr uint32_t alloc = total + 1024;  // slack for 1024-byte alignment
     static_assert(b_stage % 1024 == 0 && a_tile % 1024 == 0, "stage alignment");
 };
+static_assert(2 * kSlots >= 20, "the merge hands over up to 20 (t, ordinal) pairs");
 
 struct Bars {
     uint64_t full_a;
@@ -223,18 +223,6 @@ __device__ __forceinline__ void sort16_desc(float (&x)[16])
             }
 }
 
-// Drains this thread's queue (entries [0, cnt)) into its sorted list, in lockstep with the warp.
-template <int KC>
-__device__ __forceinline__ void drain(const float2* q, int cnt, float (&tv)[KC], int (&ti)[KC])
-{
-    const int m = static_cast<int>(__reduce_max_sync(0xffffffffu, static_cast<unsigned>(cnt)));
-    for (int e = 0; e < m; ++e) {
-        const float2 x = q[e * kEpiThreads];
-        if (e < cnt && x.x > tv[KC - 1])
-            topk_insert<KC>(tv, ti, x.x, __float_as_int(x.y));
-    }
-}
-
 template <int D, int KC>
 __global__ void __launch_bounds__(kThreads, 1)
     select_tc_kernel(const CacheArgs a, const Tile* __restrict__ items, int n_items,
@@ -249,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* sA = smem + L::a_off;
     uint8_t* sB = smem + L::b_off;
     uint8_t* sAaug = smem + L::aaug_off;
-    float2* sQ = reinterpret_cast<float2*>(smem + L::q_off);
+    float4* sQ = reinterpret_cast<float4*>(smem + L::q_off);   // [kSlots][kEpiThreads]
     float* sThr = reinterpret_cast<float*>(smem + L::thr_off);
     Bars* bars = reinterpret_cast<Bars*>(smem + L::bar_off);
     volatile int* abort = &bars->abort;
@@ -425,10 +413,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---------------- epilogue: a position per pair of threads ----------------
         // Warps e and e + kPairs read the same TMEM lanes (positions) of the same tile, the first
         // columns 0 .. 63 of every reference tile, the second 64 .. 127.  Each keeps its own
-        // sorted list and queue; they share a threshold (the larger of their kc-th best values
-        // is a lower bound of the position's kc-th best, so either may filter with it), combine
-        // their seeds, and merge their lists at the end of the item.  Pairs synchronise on an
-        // mbarrier of their own (bounded waits).
+        // sorted list and shared-memory slots; they share a threshold (the larger of their
+        // kc-th best values is a lower bound of the position's kc-th best, so either may filter
+        // with it), combine their seeds, and merge their lists at the end of the item.  Pairs
+        // synchronise on an mbarrier of their own (bounded waits).
         const int e = warp - 2;                  // 0 .. kEpiWarps-1
         const int q = warp & 3;                  // TMEM lane quarter this warp may access
         const int pi = e % kPairs;               // pair
@@ -436,9 +424,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int t = pi >> 2;                   // position tile of the item
         const int row = q * 32 + lane;
         const int trow = t * kM + row;
-        const int qi = e * 32 + lane;            // queue column of this thread
-        float2* myq = sQ + qi;
-        const float2* otherq = sQ + ((e ^ kPairs) * 32 + lane);   // the partner's queue column
+        const int qi = e * 32 + lane;            // slot column of this thread
+        float4* myq = sQ + qi;                                     // this thread's slots
+        const float4* otherq = sQ + ((e ^ kPairs) * 32 + lane);   // the partner's slots
         volatile float* thr_own = sThr + hf * (kTiles * kM) + trow;
         volatile float* thr_oth = sThr + (hf ^ 1) * (kTiles * kM) + trow;
         const int cb = hf * kHalfCols;           // first column of this thread's half
@@ -469,7 +457,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tv[s] = -FLT_MAX;
                 ti[s] = 0x7fffffff;
             }
-            int cnt = 0;
             float seed_lo = -FLT_MAX;
             *thr_own = -FLT_MAX;
             pair_sync();   // both halves start the item with no threshold
@@ -503,16 +490,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                             mx[i] = -FLT_MAX;
                     }
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        myq[i * kEpiThreads] = make_float2(mx[2 * i], mx[2 * i + 1]);
+                    for (int i = 0; i < 2; ++i)
+                        myq[i * kEpiThreads] = make_float4(mx[4 * i], mx[4 * i + 1], mx[4 * i + 2], mx[4 * i + 3]);
                     pair_sync();
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float2 o = otherq[i * kEpiThreads];
-                        mx[8 + 2 * i] = o.x;
-                        mx[8 + 2 * i + 1] = o.y;
+                    for (int i = 0; i < 2; ++i) {
+                        const float4 o = otherq[i * kEpiThreads];
+                        mx[8 + 4 * i] = o.x;
+                        mx[8 + 4 * i + 1] = o.y;
+                        mx[8 + 4 * i + 2] = o.z;
+                        mx[8 + 4 * i + 3] = o.w;
                     }
-                    pair_sync();   // the partner has read this thread's maxima (the queue is reused)
+                    pair_sync();   // the partner has read this thread's maxima (the slots are reused)
                     sort16_desc(mx);
                     const float seed = mx[KC - 1];
                     seed_lo = (seed > -FLT_MAX) ? nextafterf(seed, -FLT_MAX) : -FLT_MAX;
@@ -525,46 +514,51 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int i = 0; i < 32; ++i)
                             v[i] = (j0 + c0 + i < ncand) ? v[i] : -FLT_MAX;
                     }
+                    // one compare per element: seed_lo is just below the seed, so the element that
+                    // defines the seed still passes; the partner's kc-th best bounds this
+                    // position's kc-th best as well
+                    // (+0 turns a threshold of -0 into +0: the sign of thr - t is then set exactly
+                    // when t > thr)
+                    const float thr = __fadd_rn(fmax3(tv[KC - 1], seed_lo, *thr_oth), 0.0f);
+                    uint32_t hit = 0u;   // bit 31 - k: column c0 + k is above thr
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        if (__any_sync(0xffffffffu, cnt > kQC - 16)) {
-                            drain<KC>(myq, cnt, tv, ti);
-                            cnt = 0;
-                            *thr_own = tv[KC - 1];
-                        }
-                        // one compare per element: seed_lo is just below the seed, so the element
-                        // that defines the seed is still appended; the partner's kc-th best
-                        // bounds this position's kc-th best as well
-                        const float thr = fmax3(tv[KC - 1], seed_lo, *thr_oth);
-                        int o = cnt * kEpiThreads;
+                    for (int k = 0; k < 32; ++k)
+                        hit = __funnelshift_l(__float_as_uint(__fsub_rn(thr, v[k])), hit, 1);
+                    if (hit != 0u) {
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const int k = h * 16 + i;
-                            myq[o] = make_float2(v[k], __int_as_float(j0 + c0 + k));
-                            o += (v[k] > thr) ? kEpiThreads : 0;
-                        }
-                        cnt = o / kEpiThreads;
+                        for (int i = 0; i < 8; ++i)
+                            myq[i * kEpiThreads] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                        const float* mine = reinterpret_cast<const float*>(myq);
+                        do {
+                            const int k = __clz(hit);
+                            hit ^= 0x80000000u >> k;
+                            const float x = mine[(k >> 2) * (4 * kEpiThreads) + (k & 3)];
+                            if (x > tv[KC - 1])
+                                topk_insert<KC>(tv, ti, x, j0 + c0 + k);
+                        } while (hit != 0u);
+                        *thr_own = tv[KC - 1];
                     }
                 }
                 tc_fence_before();
                 mbar_arrive(&bars->acc_empty[acc]);
                 ++it_c;
             }
-            if (ok)
-                drain<KC>(myq, cnt, tv, ti);
-            // merge: the second half hands its list over through its queue column (KC <= kQC)
+            // merge: the second half hands its list over through its slots (KC <= 2 kSlots)
             if (hf == 1) {
 #pragma unroll
-                for (int s = 0; s < KC; ++s)
-                    myq[s * kEpiThreads] = make_float2(tv[s], __int_as_float(ti[s]));
+                for (int s = 0; s < KC; s += 2)
+                    myq[(s / 2) * kEpiThreads] =
+                        make_float4(tv[s], __int_as_float(ti[s]), tv[s + 1], __int_as_float(ti[s + 1]));
             }
             pair_sync();
             if (hf == 0) {
 #pragma unroll
-                for (int s = 0; s < KC; ++s) {
-                    const float2 x = otherq[s * kEpiThreads];
+                for (int s = 0; s < KC; s += 2) {
+                    const float4 x = otherq[(s / 2) * kEpiThreads];
                     if (x.x > tv[KC - 1])
                         topk_insert<KC>(tv, ti, x.x, __float_as_int(x.y));
+                    if (x.z > tv[KC - 1])
+                        topk_insert<KC>(tv, ti, x.z, __float_as_int(x.w));
                 }
                 order_ties<KC>(tv, ti);
                 if (valid && ok) {
