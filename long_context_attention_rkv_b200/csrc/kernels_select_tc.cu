@@ -204,6 +204,14 @@ __device__ __forceinline__ void half_maxima(uint32_t col, int j0, int ncand, flo
     }
 }
 
+// (m << 1) | sign bit of x: one funnel shift.
+__device__ __forceinline__ uint32_t shl_sign(uint32_t m, float x)
+{
+    uint32_t r;
+    asm("shf.l.wrap.b32 %0, %1, %2, 1;" : "=r"(r) : "r"(__float_as_uint(x)), "r"(m));
+    return r;
+}
+
 // Sorts 16 values in descending order (bitonic network).
 __device__ __forceinline__ void sort16_desc(float (&x)[16])
 {
@@ -509,11 +517,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c0 = 0; ok && c0 < kHalfCols && j0 + c0 < nc_max; c0 += 32) {
                     float v[32];
                     tmem_ld32(col0 + c0, v);
-                    if (j0 + c0 + 32 > ncand) {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            v[i] = (j0 + c0 + i < ncand) ? v[i] : -FLT_MAX;
-                    }
                     // one compare per element: seed_lo is just below the seed, so the element that
                     // defines the seed still passes; the partner's kc-th best bounds this
                     // position's kc-th best as well
@@ -523,7 +526,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint32_t hit = 0u;   // bit 31 - k: column c0 + k is above thr
 #pragma unroll
                     for (int k = 0; k < 32; ++k)
-                        hit = __funnelshift_l(__float_as_uint(__fsub_rn(thr, v[k])), hit, 1);
+                        hit = shl_sign(hit, __fsub_rn(thr, v[k]));
+                    // columns at or past this row's own candidate count are not candidates
+                    const int nvalid = ncand - (j0 + c0);
+                    if (nvalid < 32)
+                        hit = (nvalid <= 0) ? 0u : (hit & ~(0xffffffffu >> nvalid));
                     if (hit != 0u) {
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
