@@ -262,6 +262,12 @@ __device__ __forceinline__ void encode_group(const CacheArgs& a, const void* __r
     const int64_t e = (static_cast<int64_t>(u) * a.max_len + p) * D + sub * CPL;
     float xk[CPL];
     load_input_row<CPL>(K, e, a.in_dtype, xk);
+    {
+        // the V row is read only at the end (step 3): its lines start towards L2 now, so that
+        // read does not add a third memory round trip after the candidates and the gathers
+        const char* pv = static_cast<const char*>(V) + e * (a.in_dtype == RKV_DTYPE_F32 ? 4 : 2);
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(pv));
+    }
 
     // ---- 1. final top-k -------------------------------------------------------------
     const int nvalid = min(KC, ncand);
