@@ -462,12 +462,22 @@ __global__ void __launch_bounds__(kExactThreads) encode_latent_exact_kernel(Cach
             const uint16_t* Wg = a.cw[4 * side + 0] + j * kCD;
             const uint16_t* Wu = a.cw[4 * side + 1] + j * kCD;
             double gx = 0.0, ux = 0.0, gm = 0.0, um2 = 0.0;
-            for (int ch = 0; ch < kCD; ++ch) {
-                const double wg = bf16_bits_to_f32(Wg[ch]), wu = bf16_bits_to_f32(Wu[ch]);
-                gx = fma(wg, xs[ch], gx);
-                ux = fma(wu, xs[ch], ux);
-                gm = fma(wg, ms[ch], gm);
-                um2 = fma(wu, ms[ch], um2);
+            // the thread's rows of Wg and Wu, eight weights per 16-byte load (the lanes read
+            // different rows); the products are summed in channel order as before
+            for (int c8 = 0; c8 < kCD; c8 += 8) {
+                const uint4 g8 = *reinterpret_cast<const uint4*>(Wg + c8);
+                const uint4 u8 = *reinterpret_cast<const uint4*>(Wu + c8);
+                const uint32_t gw[4] = {g8.x, g8.y, g8.z, g8.w}, uw[4] = {u8.x, u8.y, u8.z, u8.w};
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int ch = c8 + i;
+                    const double wg = bf16_bits_to_f32((i & 1) ? (gw[i >> 1] >> 16) : (gw[i >> 1] & 0xffffu));
+                    const double wu = bf16_bits_to_f32((i & 1) ? (uw[i >> 1] >> 16) : (uw[i >> 1] & 0xffffu));
+                    gx = fma(wg, xs[ch], gx);
+                    ux = fma(wu, xs[ch], ux);
+                    gm = fma(wg, ms[ch], gm);
+                    um2 = fma(wu, ms[ch], um2);
+                }
             }
             hx[j] = gx / (1.0 + exp(-gx)) * ux;
             hm[j] = gm / (1.0 + exp(-gm)) * um2;
@@ -477,10 +487,15 @@ __global__ void __launch_bounds__(kExactThreads) encode_latent_exact_kernel(Cach
             const int l = 32 * g + tid;   // latent channel
             const uint16_t* Wo = a.cw[4 * side + 2] + l * kCD;
             double fx = 0.0, fm = 0.0;
-            for (int j = 0; j < kCD; ++j) {
-                const double w = bf16_bits_to_f32(Wo[j]);
-                fx = fma(w, hx[j], fx);
-                fm = fma(w, hm[j], fm);
+            for (int j8 = 0; j8 < kCD; j8 += 8) {
+                const uint4 o8 = *reinterpret_cast<const uint4*>(Wo + j8);
+                const uint32_t ow[4] = {o8.x, o8.y, o8.z, o8.w};
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const double w = bf16_bits_to_f32((i & 1) ? (ow[i >> 1] >> 16) : (ow[i >> 1] & 0xffffu));
+                    fx = fma(w, hx[j8 + i], fx);
+                    fm = fma(w, hm[j8 + i], fm);
+                }
             }
             const float z = static_cast<float>(fx - fm);
             float amax = fabsf(z);
