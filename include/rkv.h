@@ -368,10 +368,9 @@ RKV_API rkv_status rkv_reconstruct(const rkv_cache_desc* desc, int32_t seq, int3
  * rkv_compress without a caller-provided workspace (no counterpart on the
  * pages; this is an interface convenience of this library).
  *
- * Some callers cannot call cudaMalloc or lend a workspace: code that runs
- * while a stream is being captured into a CUDA graph (allocation calls are not
- * allowed there), or an engine that has handed all device memory to its own
- * fixed pool.  This entry point does the same work as rkv_compress, with the
+ * Some callers cannot call cudaMalloc or lend a workspace, for instance an
+ * engine that has handed all device memory to its own fixed pool.  This entry
+ * point does the same work as rkv_compress, with the
  * search -> encoder candidate lists kept in a file-scope device array of
  * RKV_NOALLOC_SCRATCH_BYTES inside the library instead of in a workspace.  It
  * allocates nothing; every GPU that loads the library holds the array until
@@ -395,8 +394,7 @@ RKV_API rkv_status rkv_reconstruct(const rkv_cache_desc* desc, int32_t seq, int3
  *   - Set-up: the first call in a CUDA context (with that context current)
  *     looks up the array's device address, which belongs to the library's
  *     module in that context; a new context (after cudaDeviceReset, say) gets
- *     its own look-up.  Make the first call in a context before any stream
- *     capture.
+ *     its own look-up.
  *   - Sharing: all calls on a device use the same array and it keeps the last
  *     call's contents; nothing in it needs to start at zero (the search writes
  *     every entry the encoder reads).  Calls that overlap on the GPU race on it:

@@ -1,7 +1,6 @@
 """rkv_compress_noalloc: compression for callers that cannot allocate device memory.
 
-Such callers (code running under CUDA-graph stream capture, where allocation calls
-are not allowed, or engines whose whole device memory is a fixed pool) get the
+Such callers (an engine whose whole device memory is a fixed pool, say) get the
 search -> encoder scratch from a fixed array inside the library instead of a
 workspace.  Its result must equal rkv_compress's on the same inputs, on two calls in
 a row (the array keeps the previous call's contents), and a cache whose scratch
