@@ -244,12 +244,8 @@ __device__ __forceinline__ void encode_group(const CacheArgs& a, const void* __r
 {
     constexpr int D = CPL * LPT;
     constexpr int kLPT = LPT;                // lanes per token
-    constexpr int kTPW = 32 / kLPT;          // tokens per warp
     constexpr int KM = KC - 4;               // largest k served by this candidate width
-    __shared__ float xs[kWarps][kTPW][D];
-    const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int tg = lane / kLPT;              // token slot within the warp
     const int sub = lane % kLPT;             // lane within the token group
     const UnitMeta um = a.units[u];
     if (__all_sync(0xffffffffu, !active))

@@ -156,30 +156,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c)
     return r;
 }
 
-// Maxima of the eight 16-column blocks of one accumulator tile (this thread's row); columns
-// j0 + c at or past ncand count as -inf.
-__device__ __forceinline__ void block_maxima(uint32_t col, int j0, int ncand, float* mx)
-{
-#pragma unroll
-    for (int c0 = 0; c0 < kN; c0 += 32) {
-        float v[32];
-        tmem_ld32(col + c0, v);
-        if (j0 + c0 + 32 > ncand) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-                v[i] = (j0 + c0 + i < ncand) ? v[i] : -FLT_MAX;
-        }
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const float* b = v + 16 * h;
-            const float m0 = fmax3(b[0], b[1], b[2]), m1 = fmax3(b[3], b[4], b[5]);
-            const float m2 = fmax3(b[6], b[7], b[8]), m3 = fmax3(b[9], b[10], b[11]);
-            const float m4 = fmax3(b[12], b[13], b[14]);
-            mx[c0 / 16 + h] = fmax3(fmax3(m0, m1, m2), fmax3(m3, m4, b[15]), -FLT_MAX);
-        }
-    }
-}
-
 // Maxima of the kHalfCols / 16 blocks of 16 columns starting at TMEM column col (this thread's
 // row); columns j0 + c at or past ncand count as -inf.
 __device__ __forceinline__ void half_maxima(uint32_t col, int j0, int ncand, float* mx)
