@@ -114,6 +114,19 @@ __global__ void __launch_bounds__(128) mma_scores_kernel(const CacheArgs a, cons
         for (int x = 0; x < 4; ++x)
             bq[x] = (gid < a.G) ? src[x] : make_uint4(0u, 0u, 0u, 0u);
     }
+    float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    auto word = [](const uint4 (&v)[4], int i) {
+        const uint4 x = v[i >> 2];
+        return (i & 3) == 0 ? x.x : (i & 3) == 1 ? x.y : (i & 3) == 2 ? x.z : x.w;
+    };
+#pragma unroll
+    for (int kb = 0; kb < 8; ++kb)
+        mma_bf16(d, word(ar[0], 2 * kb), word(ar[1], 2 * kb), word(ar[0], 2 * kb + 1), word(ar[1], 2 * kb + 1),
+                 word(bq, 2 * kb), word(bq, 2 * kb + 1));
+    // everything above only reads (the cache's reference keys and the query); the writes below
+    // reuse the workspace of the previous decode on this stream, which may still be running
+    // (this kernel is its programmatic dependent): wait for it here
+    grid_dep_wait();
     if (ch == 0) {
         for (int i = tid; i < Gp * D; i += 128)
             w.O[static_cast<int64_t>(u) * Gp * D + i] = 0.0f;
@@ -158,15 +171,7 @@ __global__ void __launch_bounds__(128) mma_scores_kernel(const CacheArgs a, cons
     }
     for (int i = tid; i < (r1 - r0) * Gp; i += 128)
         w.W[(um.ref_row + r0) * Gp + i] = 0.0f;
-    float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    auto word = [](const uint4 (&v)[4], int i) {
-        const uint4 x = v[i >> 2];
-        return (i & 3) == 0 ? x.x : (i & 3) == 1 ? x.y : (i & 3) == 2 ? x.z : x.w;
-    };
-#pragma unroll
-    for (int kb = 0; kb < 8; ++kb)
-        mma_bf16(d, word(ar[0], 2 * kb), word(ar[1], 2 * kb), word(ar[0], 2 * kb + 1), word(ar[1], 2 * kb + 1),
-                 word(bq, 2 * kb), word(bq, 2 * kb + 1));
+
     // d: rows gid / gid + 8, heads 2tq / 2tq + 1
     float mloc[2] = {-FLT_MAX, -FLT_MAX};
 #pragma unroll
@@ -218,6 +223,7 @@ __global__ void __launch_bounds__(256, kRefsPerSm) mma_refs_kernel(const CacheAr
     __shared__ float lred[Gp];
     __shared__ uint32_t key[Gp];
     __shared__ int last;
+    grid_dep_launch();   // the next decode's scores kernel may start its loads
     const int u = blockIdx.y, tid = threadIdx.x;
     const UnitMeta um = a.units[u];
     const int R = um.R;
@@ -461,13 +467,11 @@ cudaError_t launch_gp(const CacheArgs& a, const void* q, void* out, const MmaWs&
 {
     const dim3 rgrid(w.n_chunk, a.n_units);
     const dim3 fgrid((w.n_chunk + w.ref_blk - 1) / w.ref_blk, a.n_units);   // refs kernel
-    if (a.coder == 1)
-        mma_scores_kernel<Gp, 16, true><<<rgrid, 128, 0, st>>>(a, q, w);
-    else if (a.ref_bits == 4)
-        mma_scores_kernel<Gp, 4, false><<<rgrid, 128, 0, st>>>(a, q, w);
-    else
-        mma_scores_kernel<Gp, 16, false><<<rgrid, 128, 0, st>>>(a, q, w);
-    cudaError_t e = cudaGetLastError();
+    // the scores kernel loads and multiplies while the previous decode on the stream finishes
+    // (it waits for it before its first write)
+    cudaError_t e = (a.coder == 1)      ? launch_pdl(mma_scores_kernel<Gp, 16, true>, rgrid, dim3(128), 0, st, a, q, w)
+                    : (a.ref_bits == 4) ? launch_pdl(mma_scores_kernel<Gp, 4, false>, rgrid, dim3(128), 0, st, a, q, w)
+                                        : launch_pdl(mma_scores_kernel<Gp, 16, false>, rgrid, dim3(128), 0, st, a, q, w);
     if (e != cudaSuccess)
         return e;
     if (w.n_tiles > 0) {
