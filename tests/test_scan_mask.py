@@ -20,6 +20,7 @@ def _cases():
     vals = [0.0, -0.0, 1.0, -1.0, TINY, -TINY, 2 * TINY, np.float32(1e-38), np.float32(-1e-38), 1e30, -1e30,
             F32_MAX, -F32_MAX, np.float32(300.25), np.float32(-300.25)]
     out = []
+    np_err = np.seterr(over="ignore")                 # the neighbours of +-FLT_MAX are +-inf (skipped)
     for a in vals:
         a = np.float32(a)
         for b in vals:
@@ -27,6 +28,7 @@ def _cases():
         out.append((a, np.nextafter(a, np.float32(np.inf), dtype=np.float32)))
         out.append((a, np.nextafter(a, np.float32(-np.inf), dtype=np.float32)))
         out.append((np.nextafter(a, np.float32(np.inf), dtype=np.float32), a))
+    np.seterr(**np_err)
     return out
 
 
