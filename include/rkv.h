@@ -287,6 +287,10 @@ RKV_API rkv_status rkv_encode(const rkv_cache_desc* desc, const void* K, const v
  * streams need different workspaces.  With bf16 inputs, head_dim 128, int4
  * codes, k <= 8 and at most 8 query heads per kv-head the per-token dot
  * products run on the tensor cores (flag RKV_FLAG_DECODE_SIMT turns that off).
+ * That form starts reading q and the reference keys while the previous
+ * rkv_decode_attn on the same stream is still finishing (it waits for it only
+ * before its first write), so q must not be that call's out or lie in its
+ * workspace; work of any other kind queued in between is waited for as usual.
  */
 RKV_API rkv_status rkv_decode_attn(const rkv_cache_desc* desc, const void* q, void* out, void* workspace,
                            uint64_t workspace_bytes, void* stream);
